@@ -1,0 +1,430 @@
+#!/usr/bin/env python
+"""Benchmark of the batched multi-agent decode-and-verify step on B200.
+
+One step = one pass of the whole hot path over one packed batch: 4 agents x
+(next token + 2 drafts) = 12 rows through a 64-layer synthetic Q4_K/Q6_K
+decoder stack (hidden 5120, intermediate 17408, 48 query / 8 KV heads of 128),
+each layer's quantized weights streamed once for all 12 rows, each agent's
+rows attending over its own bf16 KV cache. Inputs are synthetic and seeded
+(weights, caches and rows drawn in device memory); the step streams ~13.7 GB
+of weights, far more than the 126 MB L2, so no L2 flush is needed between
+steps.
+
+Metric: decode-step ms and weight-stream GB/s at 12 rows. ``value`` is the
+weight-stream rate: quantized weight bytes per step x GPUs / step time.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...   # the fp64 CPU oracle on the host cores
+
+Multi-GPU: replicas only (every GPU holds the whole stack and serves its own
+agents; nothing is exchanged between GPUs), launched one process per GPU.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "decode-step ms and weight-stream GB/s at M=12 vs B200 HBM peak (1 GPU)"
+SEED = 20261202
+
+# name -> (description, layers, rows per agent, agents, cached tokens per agent)
+WORKLOADS = {
+    "stack12_ctx1k": ("64-layer Q4_K stack (hidden 5120, inter 17408, down Q6_K), 12 rows = 4 agents x 3, "
+                      "1024 cached tokens per agent", 64, 3, 4, 1024),
+    "stack12_ctx23k": ("64-layer Q4_K stack, 12 rows = 4 agents x 3, 23000 cached tokens per agent "
+                       "(GQA 48/8 heads, bf16 KV)", 64, 3, 4, 23000),
+}
+for _m in (1, 2, 3, 4, 6, 8, 12, 16):
+    WORKLOADS[f"stack_m{_m}"] = (f"64-layer Q4_K stack, {_m} rows (row-count sweep), 1024 cached tokens",
+                                 64, _m, 1, 1024)
+
+
+class Workload:
+    """A synthetic stack, its KV caches and one packed batch, all in device memory."""
+
+    def __init__(self, name, device="cuda", seed=SEED, n_layers=None, shape=None, rows_per_agent=None,
+                 n_agents=None, ctx=None):
+        import quantized_agent_decode_b200 as q
+        desc, L, rpa, na, cl = WORKLOADS.get(name, ("custom", 64, 3, 4, 1024))
+        self.name, self.desc = name, desc
+        self.seed, self.device = seed, device
+        L = n_layers or L
+        rpa = rows_per_agent or rpa
+        na = n_agents or na
+        cl = ctx if ctx is not None else cl
+        sh = shape or synth.StackShape(n_layers=L)
+        sh.n_layers = L
+        self.shape, self.rows_per_agent, self.n_agents, self.ctx = sh, rpa, na, cl
+        self.M = rpa * na
+        self.kv_cap = cl + rpa
+        g = synth.torch_gen(seed, device, 0)
+        H, I, hd = sh.hidden, sh.inter, sh.head_dim
+        nq, nkv = sh.n_qh * hd, sh.n_kvh * hd
+        self.w_qkv, self.w_o, self.w_gu, self.w_down, self.kc, self.vc = [], [], [], [], [], []
+        for layer in range(L):
+            gl = synth.torch_gen(seed, device, synth.layer_weight_tag(layer, 0))
+            self.w_qkv.append(torch.cat([synth.q4k_matrix_torch(gl, nq, H, device),
+                                         synth.q4k_matrix_torch(gl, nkv, H, device),
+                                         synth.q4k_matrix_torch(gl, nkv, H, device)]))
+            self.w_o.append(synth.q4k_matrix_torch(gl, H, nq, device))
+            self.w_gu.append(torch.cat([synth.q4k_matrix_torch(gl, I, H, device),
+                                        synth.q4k_matrix_torch(gl, I, H, device)]))
+            self.w_down.append(q.q6k_pack(synth.q6k_matrix_torch(gl, H, I, device), H, I))
+            self.kc.append(synth.bf16_normal_torch(gl, (na, sh.n_kvh, self.kv_cap, hd), device))
+            self.vc.append(synth.bf16_normal_torch(gl, (na, sh.n_kvh, self.kv_cap, hd), device))
+        self.model = q.Model(hidden=H, inter=I, n_qh=sh.n_qh, n_kvh=sh.n_kvh, head_dim=hd, max_agents=na,
+                             kv_cap=self.kv_cap, w_qkv=self.w_qkv, w_o=self.w_o, w_gu=self.w_gu,
+                             w_down=self.w_down, k_cache=self.kc, v_cache=self.vc)
+        self.X = synth.bf16_normal_torch(g, (self.M, H), device)
+        self.ars = torch.arange(0, self.M + 1, rpa, dtype=torch.int32, device=device)
+        self.lens = torch.full((na,), cl, dtype=torch.int32, device=device)
+        self.H_out = torch.empty(self.M, H, dtype=torch.float32, device=device)
+        self.ws = q.alloc_ws(self.model.ws_bytes(self.M), device)
+        self.weight_bytes = sum(t.numel() for ts in (self.w_qkv, self.w_o, self.w_gu, self.w_down) for t in ts)
+        # (the packed down projection carries each block's 210 bytes plus up to 14 bytes of row padding)
+        self.kv_bytes = 2 * L * na * sh.n_kvh * (cl + rpa) * hd * 2  # keys read per step (incl. new rows)
+        self.act_bytes = L * self.M * (2 * H * 4 + 2 * I * 4 + (nq + 2 * nkv) * 4)  # fp32 outputs/residual
+
+    def down_gguf(self, layer):
+        """The GGUF-layout bytes of a layer's down projection, redrawn from its seed."""
+        sh = self.shape
+        H, I, hd = sh.hidden, sh.inter, sh.head_dim
+        nq, nkv = sh.n_qh * hd, sh.n_kvh * hd
+        gl = synth.torch_gen(self.seed, self.device, synth.layer_weight_tag(layer, 0))
+        for n, k in ((nq, H), (nkv, H), (nkv, H), (H, nq), (I, H), (I, H)):  # same draw order as __init__
+            synth.q4k_matrix_torch(gl, n, k, self.device)
+        return synth.q6k_matrix_torch(gl, H, I, self.device)
+
+    def step(self, stream=None):
+        self.model.decode_step(self.X, self.M, self.ars, self.n_agents, self.rows_per_agent, self.lens,
+                               self.H_out, self.ws, stream)
+
+    def graph(self, stream):
+        return self.model.graph(self.X, self.M, self.ars, self.n_agents, self.rows_per_agent, self.lens,
+                                self.H_out, self.ws, stream)
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi samples during the timed region (SM clock, throttle reasons)."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index, self.rows, self.proc = index, [], None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except FileNotFoundError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append([x.strip() for x in line.split(",")])
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in self.rows if len(r) > 2 and r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if len(r) > 2 and r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4)
+                          if len(r) > 5 + i and r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.rows)}
+
+
+# ------------------------------------------------------------------ helpers
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d.get("hbm_gbs", 6650.0), "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_traffic(kernel_file: str, record: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on the
+    current source of the kernel (else None)."""
+    p = os.path.join(ROOT, "profiles", record)
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    src = os.path.join(ROOT, "quantized_agent_decode_b200", "csrc", kernel_file)
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    return d.get("dram_bytes_per_launch") if d.get("source_sha") == h else None
+
+
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return ws, rank, local
+
+
+def max_over_ranks(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------------ CPU oracle (baseline and reference arm)
+
+_SAMPLE_CACHE = {}
+
+
+def oracle_layer_sample(seed=SEED, ctx=1024, rows_per_agent=3, n_agents=4, threads=0):
+    """One decoder layer of the same stack through the fp64 CPU oracle (inputs
+    drawn once and reused). Returns (seconds, weight bytes of the layer, threads used)."""
+    import oracle
+    key = (seed, ctx, rows_per_agent, n_agents)
+    if key not in _SAMPLE_CACHE:
+        _SAMPLE_CACHE[key] = _oracle_layer_inputs(seed, ctx, rows_per_agent, n_agents)
+    Wqkv, Wo, Wgu, Wd, Kc0, Vc0, h0, ars, lens, cap = _SAMPLE_CACHE[key]
+    sh = synth.StackShape(n_layers=1)
+    Kc, Vc, h = Kc0.copy(), Vc0.copy(), h0.copy()
+    nth = threads or oracle.max_threads()
+    t0 = time.perf_counter()
+    oracle.decode_layer(Wqkv, Wo, Wgu, Wd, sh.hidden, sh.inter, sh.n_qh, sh.n_kvh, sh.head_dim, h, ars, lens,
+                        Kc, Vc, cap, nthreads=nth)
+    dt = time.perf_counter() - t0
+    wbytes = Wqkv.size + Wo.size + Wgu.size + Wd.size
+    return dt, wbytes, nth
+
+
+def _oracle_layer_inputs(seed, ctx, rows_per_agent, n_agents):
+    import oracle
+    sh = synth.StackShape(n_layers=1)
+    H, I, hd = sh.hidden, sh.inter, sh.head_dim
+    nq, nkv = sh.n_qh * hd, sh.n_kvh * hd
+    Wqkv = np.concatenate([synth.q4k_matrix_np(seed, 1, nq, H), synth.q4k_matrix_np(seed, 2, nkv, H),
+                           synth.q4k_matrix_np(seed, 3, nkv, H)])
+    Wo = synth.q4k_matrix_np(seed, 4, H, nq)
+    Wgu = np.concatenate([synth.q4k_matrix_np(seed, 5, I, H), synth.q4k_matrix_np(seed, 6, I, H)])
+    Wd = synth.q6k_matrix_np(seed, 7, H, I)
+    cap = ctx + rows_per_agent
+    Kc = synth.bf16_normal_np(seed, 8, (n_agents, sh.n_kvh, cap, hd))
+    Vc = synth.bf16_normal_np(seed, 9, (n_agents, sh.n_kvh, cap, hd))
+    M = rows_per_agent * n_agents
+    h = oracle.bf16_array_to_f64(synth.bf16_normal_np(seed, 10, (M, H)))
+    ars = np.arange(0, M + 1, rows_per_agent, dtype=np.int32)
+    lens = np.full(n_agents, ctx, np.int32)
+    return Wqkv, Wo, Wgu, Wd, Kc, Vc, h, ars, lens, cap
+
+
+def run_reference(args, ws, rank):
+    """The oracle, as it stands, on the host cores: each step one decoder layer of
+    the workload (1/64 of a decode step), extrapolated to the full step."""
+    if rank != 0:
+        return 0
+    desc, L, rpa, na, cl = WORKLOADS[args.workload]
+    for _ in range(args.warmup):
+        oracle_layer_sample(ctx=cl, rows_per_agent=rpa, n_agents=na)
+    times = []
+    for _ in range(args.steps):
+        dt, wb, nth = oracle_layer_sample(ctx=cl, rows_per_agent=rpa, n_agents=na)
+        times.append(dt)
+    t = statistics.median(times)
+    step_s = t * L
+    val = wb * L / step_s / 1e9
+    line = {"metric": METRIC, "value": val, "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)", "impl": "reference",
+            "config": {"workload": desc, "rows": rpa * na, "layers": L, "cached_tokens": cl,
+                       "parallelism": f"replicas{args.gpus}"},
+            "cpu_baseline": {"value": val, "unit": "GB/s", "cores": nth, "kind": "oracle",
+                             "sample": f"one decoder layer per step (1/{L} of a decode step), median of "
+                                       f"{args.steps}, extrapolated x{L}"},
+            "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def run_gpu(args, ws, rank, local):
+    import quantized_agent_decode_b200 as q
+    from quantized_agent_decode_b200 import build
+    if rank == 0 or not os.path.exists(q.LIB_PATH):
+        build.build()
+    barrier(ws)
+    w = Workload(args.workload)
+    stream = torch.cuda.Stream()
+    torch.cuda.synchronize()
+
+    # per-kernel durations (eager, event-bracketed launches) for the roofline
+    w.model.set_profile(True)
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            w.step(stream)
+            stream.synchronize()
+            w.model.profile_read()
+        w.model.set_profile(True)  # reset totals after warm-up
+        for _ in range(3):
+            w.step(stream)
+            stream.synchronize()
+            prof = w.model.profile_read()
+    w.model.set_profile(False)
+
+    # graph-replayed timed region
+    g = w.graph(stream)
+    for _ in range(args.warmup):
+        g.launch(stream)
+    stream.synchronize()
+    barrier(ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        time.sleep(0.3)
+        e0.record(stream)
+        for _ in range(args.steps):
+            g.launch(stream)
+        e1.record(stream)
+        stream.synchronize()
+        time.sleep(0.2)
+    barrier(ws)
+    torch.cuda.synchronize()
+    ms_step = max_over_ranks(e0.elapsed_time(e1) / args.steps, ws)
+    status = q.device_status(reset=True)
+
+    # end to end through the host-buffer entry point (pinned host in/out, copies timed)
+    Xh = w.X.cpu().pin_memory()
+    arsh = w.ars.cpu().pin_memory()
+    lensh = w.lens.cpu().pin_memory()
+    Hh = torch.empty(w.M, w.shape.hidden, dtype=torch.float32).pin_memory()
+    for _ in range(max(1, args.warmup)):
+        w.model.decode_step_host(Xh, w.M, arsh, w.n_agents, w.rows_per_agent, lensh, Hh, w.ws, stream)
+    barrier(ws)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        w.model.decode_step_host(Xh, w.M, arsh, w.n_agents, w.rows_per_agent, lensh, Hh, w.ws, stream)
+    e2e_ms = max_over_ranks((time.perf_counter() - t0) * 1e3 / args.steps, ws)
+    h2d = Xh.numel() * 2 + arsh.numel() * 4 + lensh.numel() * 4
+    d2h = Hh.numel() * 4
+    g.close()
+
+    if rank != 0:
+        return 0
+    peak, peak_kind = measured_peaks()
+    L = w.shape.n_layers
+    # dominant kernel: the gate|up Q4_K GEMM (largest weight matrix of the layer)
+    gu_ms, gu_n = prof["gemm_gate_up"]
+    gu_bytes = (w.w_gu[0].numel() + w.M * w.shape.hidden * 2 + w.M * 2 * w.shape.inter * 4)
+    gu_avg_s = gu_ms / max(gu_n, 1) / 1e3
+    achieved = gu_bytes / gu_avg_s / 1e9
+    prof_total = sum(v[0] for v in prof.values())
+    shares = {k: round(v[0] / prof_total, 4) for k, v in prof.items()}
+    per_kernel = {k: {"avg_us": round(v[0] / max(v[1], 1) * 1e3, 2), "launches_per_step": v[1] // 3}
+                  for k, v in prof.items()}
+    value = w.weight_bytes * ws / (ms_step / 1e3) / 1e9
+    cpu = {}
+    if ws == 1 and not args.no_cpu_baseline:
+        dt, wb, nth = oracle_layer_sample(ctx=w.ctx, rows_per_agent=w.rows_per_agent, n_agents=w.n_agents)
+        cpu = {"value": wb / dt / 1e9, "unit": "GB/s", "cores": nth, "kind": "oracle",
+               "sample": f"one decoder layer (1/{L} of a decode step) of the same stack, fp64, "
+                         f"{dt:.1f} s; the full step extrapolates to {dt * L * 1e3:.0f} ms"}
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16xf16->f32 (tensor-core operands exact), bf16 KV/activations",
+        "data": "synthetic (seeded, drawn in device memory)",
+        "config": {"workload": w.desc, "rows": w.M, "agents": w.n_agents, "layers": L,
+                   "cached_tokens": w.ctx, "weight_bytes_per_step": w.weight_bytes,
+                   "kv_bytes_per_step": w.kv_bytes, "parallelism": f"replicas{ws}",
+                   "l2": "inputs larger than L2 (13.7 GB of weights per step), no flush"},
+        "roofline": {"bound": "hbm", "kernel": "q4k gate|up GEMM (N=34816, K=5120)",
+                     "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "peak_kind": peak_kind,
+                     "traffic": kernel_traffic("gemm.cu", "q4k_gemm_gate_up_traffic.json"),
+                     "duration_us": gu_avg_s * 1e6, "bytes_per_launch": gu_bytes,
+                     "timing": "CUDA events around each launch, eager profiled steps"},
+        "step_stream_gbs": (w.weight_bytes + w.kv_bytes) / (ms_step / 1e3) / 1e9,
+        "kernel_shares": shares, "kernels": per_kernel,
+        "e2e": {"value": w.weight_bytes * ws / (e2e_ms / 1e3) / 1e9, "unit": "GB/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": w.model.launches() * args.steps,
+        "clocks": clk.summary(),
+        "device_status": status,
+    }
+    if cpu:
+        line["cpu_baseline"] = cpu
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="stack12_ctx1k", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    ws, rank, local = (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+                       int(os.environ.get("LOCAL_RANK", "0")))
+    if args.impl == "reference":
+        return run_reference(args, ws, rank)
+    ws, rank, local = dist_setup()
+    try:
+        return run_gpu(args, ws, rank, local)
+    finally:
+        if ws > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,254 @@
+/*
+ * qad.h -- C ABI of the B200 (sm_100a) multi-agent quantized decode step.
+ *
+ * One batched decode-and-verify step for several coding agents that share one
+ * Q4_K-quantized model: every active agent contributes its next token plus its
+ * draft tokens, all rows are stacked into one batch, the quantized weights are
+ * streamed from HBM once per step and each weight is used for every row, and
+ * each agent's rows attend over that agent's own KV cache.
+ *
+ * Citations name the page and its section:
+ *   [OpenJet page] rebasdaily.com, 2026-10-29, "OpenJet ... Qwen3.8-27B
+ *   multi-agent serving": intro (four coding agents, one GPU, Q4_K_M weights);
+ *   section 只搬一次权重 ("move the weights once": 4 agents x (next token +
+ *   2 drafts) = 12 rows, one pass over the weights for all rows, drafts
+ *   verified in the same pass, each agent reads its own KV cache).
+ *   [P3 page] rebasdaily.com, 2026-09-10, dual-4090 llama.cpp agent
+ *   concurrency, section 真正昂贵的是“同时记住” (KV cache per agent).
+ *
+ * Conventions for every entry point:
+ *   - Pointers named d_* or documented "device" are device pointers owned by
+ *     the caller; the library never frees or retains them past the call
+ *     (except the model handle, which keeps the pointers it was given).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL = legacy default stream) unless stated otherwise. Nothing here
+ *     allocates device memory on the hot path: scratch space is a caller
+ *     workspace whose size a *_ws_bytes() query returns.
+ *   - bf16 values are passed as uint16_t bit patterns.
+ *   - Row-major layouts. Quantized matrices are [N rows][K/256 blocks]:
+ *     row n's blocks are contiguous, rows follow each other.
+ *   - Return 0 on success, or a negative QAD_ERR_* code; the thread-local
+ *     text of the last error is available from qad_last_error(). Arguments
+ *     are checked on the host before any launch; a failed check launches
+ *     nothing.
+ */
+#ifndef QAD_H
+#define QAD_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define QAD_OK 0
+#define QAD_ERR_INVALID (-1)     /* null pointer, negative size, inconsistent sizes */
+#define QAD_ERR_UNSUPPORTED (-2) /* shape outside the supported range (e.g. M > 16, K % 256) */
+#define QAD_ERR_WORKSPACE (-3)   /* workspace smaller than the *_ws_bytes() query */
+#define QAD_ERR_CUDA (-4)        /* a CUDA runtime call or launch failed */
+
+#define QAD_MAX_ROWS 16          /* rows of one step (skinny path) */
+#define QAD_QK 256               /* weights per quantized block */
+#define QAD_Q4K_BLOCK_BYTES 144
+#define QAD_Q6K_BLOCK_BYTES 210
+
+/* Text of the last error on this thread ("" if none). */
+const char *qad_last_error(void);
+
+/* ABI version (major*100 + minor). */
+int qad_version(void);
+
+/* ---------------------------------------------------------------- codecs
+ * Q4_K super-block (the "Q4_K_M" weights of [OpenJet page], intro; block
+ * layout per the GGUF Q4_K convention): 144 bytes = d fp16, dmin fp16,
+ * 12 bytes of packed 6-bit sub-block scales/mins, 128 bytes of 4-bit quants;
+ * weight i = d*sc_{i/32}*q_i - dmin*m_{i/32}.
+ *
+ * qad_q4k_unpack: decodes n_blocks device blocks at W into
+ *   q [n_blocks][256] (0..15), sc [n_blocks][8], m [n_blocks][8] (0..63),
+ *   d [n_blocks], dmin [n_blocks] (fp16 bit patterns). All device pointers.
+ *   Bit-exact. Used by tests and diagnostics.
+ * qad_q6k_unpack: Q6_K-like block (210 bytes: ql[128], qh[64], int8
+ *   scales[16], d fp16); weight i = d*scales_{i/16}*(q_i - 32).
+ *   q [n_blocks][256] (0..63), sc [n_blocks][16] (int8), d [n_blocks]. */
+int qad_q4k_unpack(const void *W, long long n_blocks, uint8_t *q, uint8_t *sc, uint8_t *m,
+                   uint16_t *d, uint16_t *dmin, void *stream);
+int qad_q6k_unpack(const void *W, long long n_blocks, uint8_t *q, int8_t *sc, uint16_t *d,
+                   void *stream);
+
+/* ---------------------------------------------------------------- skinny GEMM
+ * Y[r][n] = sum_k w[n][k] * X[r][k] for r < M, n < N: the shared weight pass
+ * of [OpenJet page], section 只搬一次权重 -- each quantized block is read from
+ * HBM once and used for all M rows.
+ *   W  device, 16-byte aligned: Q4_K [N][K/256 blocks] (q4k), or Q6_K-like in
+ *      the packed layout of qad_q6k_pack (q6k)
+ *   X  device bf16 [M][K]
+ *   Y  device fp32 [M][N]; overwritten, or accumulated into (Y += X W^T) when
+ *      `accumulate` is non-zero
+ *   ws device workspace of at least qad_gemm_ws_bytes(K, M) bytes, 256-byte
+ *      aligned; its contents are scratch
+ * 1 <= M <= 16, K % 256 == 0, K <= 65536, N >= 1. Results are fp32-accumulated
+ * products of exact operands (the tensor-core operand of X is fp16 with a
+ * per-row power-of-two scale, see the design notes); the result is not
+ * bit-reproducible across launches because partial sums are combined with
+ * atomic adds. */
+size_t qad_gemm_ws_bytes(int K, int M);
+
+/* Q6_K-like weights are streamed from a packed device layout that keeps every
+ * field 16-byte aligned (a 210-byte block cannot be addressed by the tensor
+ * memory accelerator): plane A [N][K/256][208] holds the first 208 bytes of
+ * each block (ql, qh, int8 scales, unchanged), followed by plane D
+ * [N][ceil8(K/256)] holding each block's fp16 d (rows padded with zeros to a
+ * multiple of 8 blocks). Same bytes per block as the GGUF layout, plus the
+ * padding. qad_q6k_pack converts N x K GGUF-layout blocks W (device) into
+ * W_packed (device, 16-byte aligned, qad_q6k_packed_bytes(N, K) bytes); it is
+ * a one-time load step, not part of the decode step. */
+size_t qad_q6k_packed_bytes(long long N, int K);
+int qad_q6k_pack(const void *W, int N, int K, void *W_packed, void *stream);
+
+/* Device status word of the GEMM pipelines on the current device: 0 if every
+ * shared-memory pipeline wait completed; non-zero if a wait gave up after its
+ * bounded number of polls (the kernel then returned early and its outputs are
+ * incomplete). Synchronous (reads device memory); reset != 0 clears it.
+ * Returns the status (>= 0) or a negative QAD_ERR_* code. */
+int qad_device_status(int reset);
+int qad_q4k_gemm(const void *W, int N, int K, const uint16_t *X, int M, float *Y, int accumulate,
+                 void *ws, size_t ws_bytes, void *stream);
+int qad_q6k_gemm(const void *W, int N, int K, const uint16_t *X, int M, float *Y, int accumulate,
+                 void *ws, size_t ws_bytes, void *stream);
+
+/* ---------------------------------------------------------------- attention
+ * Grouped-query decode attention of each agent's rows over that agent's own
+ * bf16 KV cache ([OpenJet page], section 只搬一次权重; [P3 page]).
+ * Agent a owns rows r = agent_row_start[a] .. agent_row_start[a+1]-1; row
+ * j = r - agent_row_start[a] sits at position lens[a] + j and attends over
+ * keys t = 0 .. lens[a] + j (cached context plus the agent's new rows up to
+ * itself: the draft rows see exactly what one-at-a-time decoding would).
+ * q-head h reads kv-head h * n_kvh / n_qh.
+ *   Q      device bf16 [M][n_qh][hd]
+ *   Kc, Vc device bf16 [n_agents][n_kvh][kv_cap][hd]; positions
+ *          lens[a] .. lens[a]+n_rows-1 must already hold the new rows' keys
+ *          and values (qad_decode_step writes them itself)
+ *   lens, agent_row_start  device int32 [n_agents], [n_agents+1]
+ *   O      device bf16 [M][n_qh][hd]
+ *   ws     device workspace of qad_decode_attn_ws_bytes(...) bytes
+ * hd == 128, n_qh % n_kvh == 0, rows per agent * (n_qh/n_kvh) <= 96,
+ * lens[a] + rows <= kv_cap (entries beyond kv_cap are skipped on the device).
+ * scale is the softmax temperature (1/sqrt(hd) for standard attention). */
+size_t qad_decode_attn_ws_bytes(int n_agents, int n_qh, int n_kvh, int kv_cap, int max_rows_per_agent);
+int qad_decode_attn(const uint16_t *Q, const uint16_t *Kc, const uint16_t *Vc, const int *lens,
+                    const int *agent_row_start, int n_agents, int max_rows_per_agent, int kv_cap,
+                    int n_qh, int n_kvh, int hd, float scale, uint16_t *O, void *ws, size_t ws_bytes,
+                    void *stream);
+
+/* ---------------------------------------------------------------- row packer
+ * Host-only. Stacks every agent's rows (next token + drafts) agent-major into
+ * one batch ([OpenJet page], section 只搬一次权重). An agent paused for a tool
+ * call passes n_rows = 0.
+ *   agents[a].rows   host bf16 [n_rows][hidden]
+ *   agents[a].len    cached tokens before the step
+ * Writes X [M][hidden], row_agent[M], row_pos[M] (= len + j) and
+ * agent_row_start[n_agents+1] (host arrays of capacity max_rows rows).
+ * Returns M >= 0, or a negative QAD_ERR_* code (M > max_rows, n_rows < 0 ...). */
+typedef struct {
+    const uint16_t *rows;
+    int n_rows;
+    int len;
+} qad_agent_rows;
+
+int qad_pack_rows(const qad_agent_rows *agents, int n_agents, int hidden, int max_rows, uint16_t *X,
+                  int *row_agent, int *row_pos, int *agent_row_start);
+
+/* ---------------------------------------------------------------- decode step
+ * A model is a stack of decoder layers whose weights and KV caches the caller
+ * owns. Per layer (device pointers):
+ *   w_qkv  Q4_K [(n_qh + 2 n_kvh) hd][hidden]   rows: q heads, k heads, v heads
+ *   w_o    Q4_K [hidden][n_qh hd]
+ *   w_gu   Q4_K [2 inter][hidden]               rows: gate, then up
+ *   w_down Q6_K-like [hidden][inter], packed by qad_q6k_pack
+ *   k_cache, v_cache bf16 [max_agents][n_kvh][kv_cap][hd]
+ * The descriptor's pointer arrays are host arrays of n_layers entries and are
+ * copied by qad_model_create. */
+typedef struct {
+    int n_layers, hidden, inter, n_qh, n_kvh, head_dim;
+    int max_agents, kv_cap;
+    float rms_eps;
+    const void *const *w_qkv;
+    const void *const *w_o;
+    const void *const *w_gu;
+    const void *const *w_down;
+    uint16_t *const *k_cache;
+    uint16_t *const *v_cache;
+} qad_model_desc;
+
+typedef struct qad_model qad_model;
+
+int qad_model_create(const qad_model_desc *desc, qad_model **out);
+void qad_model_destroy(qad_model *model);
+
+/* One decode-and-verify forward step for the packed batch, per layer:
+ *   x1 = bf16(rmsnorm(h)); qkv = x1 Wqkv^T; Q = bf16(q); append bf16 k, v of
+ *   every row at its position; o = attention; h += bf16(o) Wo^T;
+ *   x2 = bf16(rmsnorm(h)); gu = x2 Wgu^T; h += bf16(silu(gate)*up) Wdown^T.
+ *   X        device bf16 [M][hidden] (the rows' input hidden states)
+ *   agent_row_start, lens  device int32 [n_agents+1], [n_agents]; lens are
+ *            the cached lengths before the step (the caller commits accepted
+ *            tokens afterwards; rejected slots are overwritten next step)
+ *   H_out    device fp32 [M][hidden]: the residual stream after the last layer
+ *   ws       device workspace of qad_decode_step_ws_bytes(model, M) bytes
+ * 1 <= M <= 16, n_agents <= max_agents. */
+size_t qad_decode_step_ws_bytes(const qad_model *model, int M);
+int qad_decode_step(qad_model *model, const uint16_t *X, int M, const int *agent_row_start,
+                    int n_agents, int max_rows_per_agent, const int *lens, float *H_out, void *ws,
+                    size_t ws_bytes, void *stream);
+
+/* The same step with HOST inputs and output: copies X, agent_row_start and
+ * lens into the workspace, runs the step (replaying a CUDA graph captured on
+ * the first call for this (model, M, n_agents, workspace)), copies H_out back
+ * and synchronises the stream. Host buffers should be pinned for speed. */
+int qad_decode_step_host(qad_model *model, const uint16_t *X_host, int M,
+                         const int *agent_row_start_host, int n_agents, int max_rows_per_agent,
+                         const int *lens_host, float *H_out_host, void *ws, size_t ws_bytes,
+                         void *stream);
+
+/* CUDA-graph form of qad_decode_step: capture once, replay each step. The
+ * graph records the given device pointers; refresh their contents between
+ * replays. */
+typedef struct qad_step_graph qad_step_graph;
+int qad_step_graph_create(qad_model *model, const uint16_t *X, int M, const int *agent_row_start,
+                          int n_agents, int max_rows_per_agent, const int *lens, float *H_out,
+                          void *ws, size_t ws_bytes, void *stream, qad_step_graph **out);
+int qad_step_graph_launch(qad_step_graph *g, void *stream);
+void qad_step_graph_destroy(qad_step_graph *g);
+
+/* Number of kernel launches one qad_decode_step issues (for accounting). */
+int qad_decode_step_launches(const qad_model *model);
+
+/* Teacher-forced checking aid. When a debug buffer of
+ * qad_decode_step_debug_bytes(model, M) bytes is attached, every following
+ * qad_decode_step also copies, per layer l, the intermediates x1 (bf16
+ * [M][hidden]), qkv (fp32 [M][(n_qh+2 n_kvh) hd]), attention output (bf16
+ * [M][n_qh hd]), h after the o projection (fp32 [M][hidden]), x2 (bf16),
+ * gate|up (fp32 [M][2 inter]), silu(gate)*up (bf16 [M][inter]) and h after
+ * the layer (fp32), each at a 256-byte aligned offset in that order, into
+ * layer l's slice. Pass dbg = NULL to detach. Graph capture refuses a model
+ * with a debug buffer attached. */
+size_t qad_decode_step_debug_bytes(const qad_model *model, int M);
+int qad_model_set_debug(qad_model *model, void *dbg, size_t bytes);
+
+/* Per-launch event profiler. While enabled, every eager qad_decode_step records
+ * a CUDA event before and after each of its launches (which serialises the
+ * launch chain) and qad_model_profile_read() accumulates the elapsed times per
+ * kernel class into ms[k], count[k] (k: 0 init, 1 prep, 2 qkv GEMM, 3 qkv
+ * split/append, 4 attention + combine, 5 o GEMM, 6 gate|up GEMM, 7 down GEMM;
+ * n_kinds >= 8) and returns the number of classes. Read after every profiled
+ * step (a step not read before the next one is dropped). Enabling resets the
+ * totals. Graph capture refuses a model with the profiler on. */
+int qad_model_set_profile(qad_model *model, int enable);
+int qad_model_profile_read(qad_model *model, double *ms, long long *count, int n_kinds);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* QAD_H */

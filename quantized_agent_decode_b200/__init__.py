@@ -1,0 +1,349 @@
+"""Python binding of libqad.so (include/qad.h): argument marshalling only.
+
+Every step of the decode path runs in the CUDA library; this module converts
+torch tensors to pointers and return codes to exceptions. There is no CPU
+fallback: importing works without a GPU (for the C-ABI export checks), but any
+compute call raises if the library or a CUDA device is missing.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqad.so")
+_lib = None
+
+QAD_MAX_ROWS = 16
+Q4K_BLOCK_BYTES = 144
+Q6K_BLOCK_BYTES = 210
+
+
+class QadError(RuntimeError):
+    pass
+
+
+class ModelDesc(C.Structure):
+    _fields_ = [("n_layers", C.c_int), ("hidden", C.c_int), ("inter", C.c_int), ("n_qh", C.c_int),
+                ("n_kvh", C.c_int), ("head_dim", C.c_int), ("max_agents", C.c_int), ("kv_cap", C.c_int),
+                ("rms_eps", C.c_float), ("w_qkv", C.POINTER(C.c_void_p)), ("w_o", C.POINTER(C.c_void_p)),
+                ("w_gu", C.POINTER(C.c_void_p)), ("w_down", C.POINTER(C.c_void_p)),
+                ("k_cache", C.POINTER(C.c_void_p)), ("v_cache", C.POINTER(C.c_void_p))]
+
+
+class AgentRows(C.Structure):
+    _fields_ = [("rows", C.c_void_p), ("n_rows", C.c_int), ("len", C.c_int)]
+
+
+# name -> (restype, argtypes)
+SIGNATURES = {
+    "qad_last_error": (C.c_char_p, []),
+    "qad_version": (C.c_int, []),
+    "qad_q4k_unpack": (C.c_int, [C.c_void_p, C.c_longlong] + [C.c_void_p] * 5 + [C.c_void_p]),
+    "qad_q6k_unpack": (C.c_int, [C.c_void_p, C.c_longlong] + [C.c_void_p] * 3 + [C.c_void_p]),
+    "qad_gemm_ws_bytes": (C.c_size_t, [C.c_int, C.c_int]),
+    "qad_device_status": (C.c_int, [C.c_int]),
+    "qad_q6k_packed_bytes": (C.c_size_t, [C.c_longlong, C.c_int]),
+    "qad_q6k_pack": (C.c_int, [C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_void_p]),
+    "qad_q4k_gemm": (C.c_int, [C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_int, C.c_void_p, C.c_int,
+                               C.c_void_p, C.c_size_t, C.c_void_p]),
+    "qad_q6k_gemm": (C.c_int, [C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_int, C.c_void_p, C.c_int,
+                               C.c_void_p, C.c_size_t, C.c_void_p]),
+    "qad_decode_attn_ws_bytes": (C.c_size_t, [C.c_int] * 5),
+    "qad_decode_attn": (C.c_int, [C.c_void_p] * 5 + [C.c_int] * 6 + [C.c_float, C.c_void_p, C.c_void_p,
+                                                                     C.c_size_t, C.c_void_p]),
+    "qad_pack_rows": (C.c_int, [C.POINTER(AgentRows), C.c_int, C.c_int, C.c_int, C.c_void_p, C.c_void_p,
+                                C.c_void_p, C.c_void_p]),
+    "qad_model_create": (C.c_int, [C.POINTER(ModelDesc), C.POINTER(C.c_void_p)]),
+    "qad_model_destroy": (None, [C.c_void_p]),
+    "qad_decode_step_ws_bytes": (C.c_size_t, [C.c_void_p, C.c_int]),
+    "qad_decode_step": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int, C.c_void_p, C.c_int, C.c_int, C.c_void_p,
+                                  C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p]),
+    "qad_decode_step_host": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int, C.c_void_p, C.c_int, C.c_int,
+                                       C.c_void_p, C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p]),
+    "qad_step_graph_create": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int, C.c_void_p, C.c_int, C.c_int,
+                                        C.c_void_p, C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p,
+                                        C.POINTER(C.c_void_p)]),
+    "qad_step_graph_launch": (C.c_int, [C.c_void_p, C.c_void_p]),
+    "qad_step_graph_destroy": (None, [C.c_void_p]),
+    "qad_decode_step_launches": (C.c_int, [C.c_void_p]),
+    "qad_decode_step_debug_bytes": (C.c_size_t, [C.c_void_p, C.c_int]),
+    "qad_model_set_debug": (C.c_int, [C.c_void_p, C.c_void_p, C.c_size_t]),
+    "qad_model_set_profile": (C.c_int, [C.c_void_p, C.c_int]),
+    "qad_model_profile_read": (C.c_int, [C.c_void_p, C.POINTER(C.c_double), C.POINTER(C.c_longlong), C.c_int]),
+}
+
+PROFILE_KINDS = ["init", "prep", "gemm_qkv", "qkv_post", "attn", "gemm_o", "gemm_gate_up", "gemm_down"]
+
+
+def lib():
+    """Load libqad.so (built in-tree by build.py). Raises if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise QadError(f"CUDA library not built: {LIB_PATH} (run __graft_entry__.build())")
+        L = C.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(rc: int, what: str):
+    if rc < 0:
+        raise QadError(f"{what} failed ({rc}): {lib().qad_last_error().decode()}")
+    return rc
+
+
+def _dev(t: torch.Tensor, name: str):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise QadError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise QadError(f"{name} must be contiguous")
+    return C.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return C.c_void_p(stream.cuda_stream)
+
+
+def _require_gpu():
+    if not torch.cuda.is_available():
+        raise QadError("no CUDA device: the decode path has no CPU fallback")
+
+
+def alloc_ws(nbytes: int, device="cuda") -> torch.Tensor:
+    """A 256-byte aligned device workspace (torch allocations are)."""
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def device_status(reset: bool = True) -> int:
+    """0 if every GEMM pipeline wait on this device completed since the last reset."""
+    return _check(lib().qad_device_status(int(reset)), "qad_device_status")
+
+
+# ------------------------------------------------------------------ codecs
+
+def q4k_unpack(W: torch.Tensor, n_blocks: int, stream=None):
+    _require_gpu()
+    dev = W.device
+    q = torch.empty(n_blocks, 256, dtype=torch.uint8, device=dev)
+    sc = torch.empty(n_blocks, 8, dtype=torch.uint8, device=dev)
+    m = torch.empty(n_blocks, 8, dtype=torch.uint8, device=dev)
+    d = torch.empty(n_blocks, dtype=torch.int16, device=dev)
+    dmin = torch.empty(n_blocks, dtype=torch.int16, device=dev)
+    _check(lib().qad_q4k_unpack(_dev(W, "W"), n_blocks, _dev(q, "q"), _dev(sc, "sc"), _dev(m, "m"),
+                                _dev(d, "d"), _dev(dmin, "dmin"), _stream(stream)), "qad_q4k_unpack")
+    return q, sc, m, d, dmin
+
+
+def q6k_unpack(W: torch.Tensor, n_blocks: int, stream=None):
+    _require_gpu()
+    dev = W.device
+    q = torch.empty(n_blocks, 256, dtype=torch.uint8, device=dev)
+    sc = torch.empty(n_blocks, 16, dtype=torch.int8, device=dev)
+    d = torch.empty(n_blocks, dtype=torch.int16, device=dev)
+    _check(lib().qad_q6k_unpack(_dev(W, "W"), n_blocks, _dev(q, "q"), _dev(sc, "sc"), _dev(d, "d"),
+                                _stream(stream)), "qad_q6k_unpack")
+    return q, sc, d
+
+
+# ------------------------------------------------------------------ GEMM
+
+def gemm_ws_bytes(K: int, M: int) -> int:
+    return int(lib().qad_gemm_ws_bytes(K, M))
+
+
+def _gemm(fn, W, N, K, X, M, Y, accumulate, ws, stream):
+    _require_gpu()
+    if ws is None:
+        ws = alloc_ws(gemm_ws_bytes(K, M), X.device)
+    _check(getattr(lib(), fn)(_dev(W, "W"), N, K, _dev(X, "X"), M, _dev(Y, "Y"), int(bool(accumulate)),
+                              _dev(ws, "ws"), ws.numel() * ws.element_size(), _stream(stream)), fn)
+    return Y
+
+
+def q4k_gemm(W, N, K, X, M, Y, accumulate=False, ws=None, stream=None):
+    """Y[M,N] (fp32) = X[M,K] (bf16) @ W^T with W a Q4_K [N, K/256*144] uint8 tensor."""
+    return _gemm("qad_q4k_gemm", W, N, K, X, M, Y, accumulate, ws, stream)
+
+
+def q6k_gemm(W, N, K, X, M, Y, accumulate=False, ws=None, stream=None):
+    """Y[M,N] (fp32) = X[M,K] (bf16) @ W^T with W a Q6_K-like matrix in the packed layout (q6k_pack)."""
+    return _gemm("qad_q6k_gemm", W, N, K, X, M, Y, accumulate, ws, stream)
+
+
+def q6k_packed_bytes(N: int, K: int) -> int:
+    return int(lib().qad_q6k_packed_bytes(N, K))
+
+
+def q6k_pack(W, N, K, out=None, stream=None):
+    """GGUF-layout Q6_K-like blocks (uint8 CUDA tensor [N, K/256*210]) -> packed device layout."""
+    _require_gpu()
+    if out is None:
+        out = torch.empty(q6k_packed_bytes(N, K), dtype=torch.uint8, device=W.device)
+    _check(lib().qad_q6k_pack(_dev(W, "W"), N, K, _dev(out, "out"), _stream(stream)), "qad_q6k_pack")
+    return out
+
+
+# ------------------------------------------------------------------ attention
+
+def decode_attn_ws_bytes(n_agents, n_qh, n_kvh, kv_cap, max_rows_per_agent) -> int:
+    return int(lib().qad_decode_attn_ws_bytes(n_agents, n_qh, n_kvh, kv_cap, max_rows_per_agent))
+
+
+def decode_attn(Q, Kc, Vc, lens, agent_row_start, n_agents, max_rows_per_agent, kv_cap, n_qh, n_kvh, hd, O,
+                scale=None, ws=None, stream=None):
+    _require_gpu()
+    if scale is None:
+        scale = hd ** -0.5
+    if ws is None:
+        ws = alloc_ws(decode_attn_ws_bytes(n_agents, n_qh, n_kvh, kv_cap, max_rows_per_agent), Q.device)
+    _check(lib().qad_decode_attn(_dev(Q, "Q"), _dev(Kc, "Kc"), _dev(Vc, "Vc"), _dev(lens, "lens"),
+                                 _dev(agent_row_start, "agent_row_start"), n_agents, max_rows_per_agent, kv_cap,
+                                 n_qh, n_kvh, hd, float(scale), _dev(O, "O"), _dev(ws, "ws"),
+                                 ws.numel() * ws.element_size(), _stream(stream)), "qad_decode_attn")
+    return O
+
+
+# ------------------------------------------------------------------ row packer (host)
+
+def pack_rows(agent_rows, lens, hidden: int, max_rows: int = QAD_MAX_ROWS):
+    """agent_rows: list of CPU bf16 tensors [n_a, hidden] (n_a may be 0).
+    Returns (X [M, hidden] bf16, row_agent, row_pos, agent_row_start) as CPU tensors."""
+    n = len(agent_rows)
+    keep = [r.contiguous() for r in agent_rows]
+    arr = (AgentRows * max(n, 1))()
+    for a, r in enumerate(keep):
+        arr[a].rows = r.data_ptr() if r.numel() else None
+        arr[a].n_rows = int(r.shape[0])
+        arr[a].len = int(lens[a])
+    X = torch.empty(max(max_rows, 1), hidden, dtype=torch.bfloat16)
+    ra = torch.empty(max(max_rows, 1), dtype=torch.int32)
+    rp = torch.empty(max(max_rows, 1), dtype=torch.int32)
+    ars = torch.empty(n + 1, dtype=torch.int32)
+    M = _check(lib().qad_pack_rows(arr, n, hidden, max_rows, C.c_void_p(X.data_ptr()),
+                                   C.c_void_p(ra.data_ptr()), C.c_void_p(rp.data_ptr()),
+                                   C.c_void_p(ars.data_ptr())), "qad_pack_rows")
+    return X[:M], ra[:M], rp[:M], ars
+
+
+# ------------------------------------------------------------------ model / decode step
+
+class Model:
+    """A decoder stack whose weights and KV caches live in caller-owned device tensors."""
+
+    def __init__(self, *, hidden, inter, n_qh, n_kvh, head_dim, max_agents, kv_cap, w_qkv, w_o, w_gu, w_down,
+                 k_cache, v_cache, rms_eps=1e-6):
+        _require_gpu()
+        L = len(w_qkv)
+        self._keep = (w_qkv, w_o, w_gu, w_down, k_cache, v_cache)
+        arrs = []
+        for name, ts in zip(("w_qkv", "w_o", "w_gu", "w_down", "k_cache", "v_cache"), self._keep):
+            assert len(ts) == L, name
+            arrs.append((C.c_void_p * L)(*[_dev(t, name).value for t in ts]))
+        self._arrs = arrs
+        d = ModelDesc(L, hidden, inter, n_qh, n_kvh, head_dim, max_agents, kv_cap, rms_eps, *arrs)
+        h = C.c_void_p()
+        _check(lib().qad_model_create(C.byref(d), C.byref(h)), "qad_model_create")
+        self.handle = h
+        self.n_layers, self.hidden, self.inter = L, hidden, inter
+        self.n_qh, self.n_kvh, self.head_dim, self.max_agents, self.kv_cap = n_qh, n_kvh, head_dim, max_agents, kv_cap
+        self._dbg = None
+
+    def close(self):
+        if getattr(self, "handle", None):
+            lib().qad_model_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def ws_bytes(self, M: int) -> int:
+        return int(lib().qad_decode_step_ws_bytes(self.handle, M))
+
+    def launches(self) -> int:
+        return int(lib().qad_decode_step_launches(self.handle))
+
+    def set_debug(self, M: int | None):
+        """Attach (M rows) or detach (None) a per-layer intermediates buffer."""
+        if M is None:
+            self._dbg = None
+            _check(lib().qad_model_set_debug(self.handle, None, 0), "qad_model_set_debug")
+            return None
+        n = int(lib().qad_decode_step_debug_bytes(self.handle, M))
+        self._dbg = alloc_ws(n)
+        _check(lib().qad_model_set_debug(self.handle, _dev(self._dbg, "dbg"), n), "qad_model_set_debug")
+        return self._dbg
+
+    def set_profile(self, enable: bool):
+        _check(lib().qad_model_set_profile(self.handle, int(bool(enable))), "qad_model_set_profile")
+
+    def profile_read(self):
+        """{kind: (total_ms, launches)} accumulated since the profiler was enabled."""
+        n = len(PROFILE_KINDS)
+        ms = (C.c_double * n)()
+        cnt = (C.c_longlong * n)()
+        _check(lib().qad_model_profile_read(self.handle, ms, cnt, n), "qad_model_profile_read")
+        return {k: (ms[i], cnt[i]) for i, k in enumerate(PROFILE_KINDS)}
+
+    def decode_step(self, X, M, agent_row_start, n_agents, max_rows_per_agent, lens, H_out, ws, stream=None):
+        _check(lib().qad_decode_step(self.handle, _dev(X, "X"), M, _dev(agent_row_start, "agent_row_start"),
+                                     n_agents, max_rows_per_agent, _dev(lens, "lens"), _dev(H_out, "H_out"),
+                                     _dev(ws, "ws"), ws.numel() * ws.element_size(), _stream(stream)),
+               "qad_decode_step")
+        return H_out
+
+    def decode_step_host(self, X_host, M, agent_row_start_host, n_agents, max_rows_per_agent, lens_host, H_host,
+                         ws, stream=None):
+        """Host tensors in and out (pinned for speed); copies happen inside the call."""
+        for t, n in ((X_host, "X"), (agent_row_start_host, "agent_row_start"), (lens_host, "lens"),
+                     (H_host, "H_out")):
+            if t.is_cuda or not t.is_contiguous():
+                raise QadError(f"{n} must be a contiguous host tensor")
+        _check(lib().qad_decode_step_host(self.handle, C.c_void_p(X_host.data_ptr()), M,
+                                          C.c_void_p(agent_row_start_host.data_ptr()), n_agents,
+                                          max_rows_per_agent, C.c_void_p(lens_host.data_ptr()),
+                                          C.c_void_p(H_host.data_ptr()), _dev(ws, "ws"),
+                                          ws.numel() * ws.element_size(), _stream(stream)), "qad_decode_step_host")
+        return H_host
+
+    def graph(self, X, M, agent_row_start, n_agents, max_rows_per_agent, lens, H_out, ws, stream):
+        return StepGraph(self, X, M, agent_row_start, n_agents, max_rows_per_agent, lens, H_out, ws, stream)
+
+
+class StepGraph:
+    """A captured decode step (CUDA graph); replay with launch()."""
+
+    def __init__(self, model, X, M, ars, n_agents, max_rows, lens, H_out, ws, stream):
+        self.model = model
+        self._keep = (X, ars, lens, H_out, ws)
+        g = C.c_void_p()
+        _check(lib().qad_step_graph_create(model.handle, _dev(X, "X"), M, _dev(ars, "ars"), n_agents, max_rows,
+                                           _dev(lens, "lens"), _dev(H_out, "H_out"), _dev(ws, "ws"),
+                                           ws.numel() * ws.element_size(), _stream(stream), C.byref(g)),
+               "qad_step_graph_create")
+        self.handle = g
+
+    def launch(self, stream=None):
+        _check(lib().qad_step_graph_launch(self.handle, _stream(stream)), "qad_step_graph_launch")
+
+    def close(self):
+        if getattr(self, "handle", None):
+            lib().qad_step_graph_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,403 @@
+// attn.cu -- grouped-query decode attention of each agent's rows over that
+// agent's own bf16 KV cache, split along the keys (flash-decoding style), then
+// a log-sum-exp combine of the splits.
+//
+// [OpenJet page] = rebasdaily.com 2026-10-29, "OpenJet ... multi-agent
+// serving", section 只搬一次权重: every agent reads its own KV cache, and the
+// two draft rows are checked in the same pass as the next-token row. Row j of
+// an agent sits at position len + j and sees keys 0..len+j, which is exactly
+// what decoding the rows one at a time would see.
+//
+// Design (sm_100a): one CTA = (split of the agent's keys, group of up to 24
+// query vectors, agent, kv-head). The query vectors of one kv-head are all of
+// the agent's rows times the q-heads that share it (3 rows x 6 heads = 18).
+// The products run on the tensor cores with keys in the MMA's M dimension:
+//   S^T[key][q] = K Q^T      (A = K tile via ldmatrix, B = Q^T in registers)
+//   O^T[d][q]  += V^T P^T    (A = V^T tile via ldmatrix.trans, B = P^T via movmatrix)
+// so 18 query vectors pad to 24 (three n=8 tiles) instead of 32. Keys and
+// values stream HBM -> shared memory with cp.async (3 stages per warp, XOR
+// swizzled 16-byte chunks so ldmatrix is bank-conflict free). The softmax is
+// online in fp32 (exp2 with the scale folded in); P enters the bf16 MMA as a
+// hi + lo pair of bf16 values, so its rounding error is ~2^-17 relative.
+#include "attn.cuh"
+
+namespace qad {
+
+constexpr int QG = 24;          // query vectors per CTA
+constexpr int KT = 16;          // keys per tile (one MMA M tile)
+constexpr int ATT_WARPS = 4;
+constexpr int ATT_STAGES = 3;
+constexpr int TILE_BYTES = KT * 128 * 2;  // 4 KB (K) ; V follows
+constexpr int PART_FLOATS = QG * 128 + 2 * QG;
+
+struct AttnArgs {
+    const uint16_t *Q, *Kc, *Vc;
+    const int *lens, *ars;
+    int n_kvh, kv_cap, n_qh, G, CH, n_rg, max_splits;
+    float scale_log2;
+    float *part;
+};
+
+__device__ __forceinline__ int swz(int key, int chunk) { return key * 256 + ((chunk ^ (key & 7)) << 4); }
+
+__global__ void __launch_bounds__(128, 2) k_decode_attn(AttnArgs p)
+{
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int sp = blockIdx.x, rg = blockIdx.y, ag = blockIdx.z;
+    const int a = ag / p.n_kvh, g = ag - a * p.n_kvh;
+    const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31, gq = lane >> 2, c = lane & 3;
+    pdl_trigger();
+    pdl_wait();
+    const int r0 = p.ars[a], na = p.ars[a + 1] - r0;
+    const int len = p.lens[a];
+    const int R = na * p.G;
+    const int q0 = rg * QG;
+    if (q0 >= R)
+        return;
+    const int L = min(len + na, p.kv_cap);
+    const int kbeg = sp * p.CH;
+    if (kbeg >= L)
+        return;
+    const int kend = min(L, kbeg + p.CH);
+    const size_t head_off = ((size_t)a * p.n_kvh + g) * (size_t)p.kv_cap * 128;
+    const uint16_t *Kh = p.Kc + head_off, *Vh = p.Vc + head_off;
+
+    // Q^T fragments: b0 = Q[q][16ks+2c..], b1 = Q[q][16ks+8+2c..] for q = q0 + 8nt + gq
+    uint32_t qf[3][8][2];
+    int qpos[3][2];  // last visible key of the two query columns this lane owns (per nt)
+#pragma unroll
+    for (int nt = 0; nt < 3; ++nt) {
+        const int qi = q0 + 8 * nt + gq;
+        const bool ok = qi < R;
+        const int j = ok ? qi / p.G : 0, hl = ok ? qi - j * p.G : 0;
+        const uint16_t *qrow = p.Q + ((size_t)(r0 + j) * p.n_qh + g * p.G + hl) * 128;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            qf[nt][ks][0] = ok ? *reinterpret_cast<const uint32_t *>(qrow + 16 * ks + 2 * c) : 0u;
+            qf[nt][ks][1] = ok ? *reinterpret_cast<const uint32_t *>(qrow + 16 * ks + 8 + 2 * c) : 0u;
+        }
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int qc = q0 + 8 * nt + 2 * c + e;
+            qpos[nt][e] = qc < R ? len + qc / p.G : -1;
+        }
+    }
+
+    float o[8][3][4];
+#pragma unroll
+    for (int dt = 0; dt < 8; ++dt)
+#pragma unroll
+        for (int nt = 0; nt < 3; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                o[dt][nt][e] = 0.f;
+    float m[3][2], l[3][2];
+#pragma unroll
+    for (int nt = 0; nt < 3; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            m[nt][e] = -INFINITY;
+            l[nt][e] = 0.f;
+        }
+
+    const int ntiles = (kend - kbeg + KT - 1) / KT;
+    const int my = ntiles > w ? (ntiles - w + ATT_WARPS - 1) / ATT_WARPS : 0;
+    uint8_t *wbuf = smem + (size_t)w * ATT_STAGES * 2 * TILE_BYTES;
+
+    auto issue = [&](int it) {
+        const int kb = kbeg + KT * (w + ATT_WARPS * it);
+        uint8_t *st = wbuf + (size_t)(it % ATT_STAGES) * 2 * TILE_BYTES;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int idx = lane + 32 * i, kk = idx >> 4, ch = idx & 15;
+            const bool ok = kb + kk < kend;
+            const size_t src = (size_t)(ok ? kb + kk : 0) * 128 + ch * 8;
+            cp_async16_zfill(st + swz(kk, ch), Kh + src, ok);
+            cp_async16_zfill(st + TILE_BYTES + swz(kk, ch), Vh + src, ok);
+        }
+    };
+    if (my > 0)
+        issue(0);
+    cp_async_commit();
+    if (my > 1)
+        issue(1);
+    cp_async_commit();
+
+    for (int it = 0; it < my; ++it) {
+        if (it + 2 < my)
+            issue(it + 2);
+        cp_async_commit();
+        cp_async_wait<2>();
+        __syncwarp();
+        const uint8_t *Ks = wbuf + (size_t)(it % ATT_STAGES) * 2 * TILE_BYTES;
+        const uint8_t *Vs = Ks + TILE_BYTES;
+        const int kb = kbeg + KT * (w + ATT_WARPS * it);
+
+        float s[3][4];
+#pragma unroll
+        for (int nt = 0; nt < 3; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                s[nt][e] = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            uint32_t a0, a1, a2, a3;
+            const int key = (lane & 7) + 8 * ((lane >> 3) & 1), ch = 2 * ks + (lane >> 4);
+            ldsm_x4(a0, a1, a2, a3, Ks + swz(key, ch));
+#pragma unroll
+            for (int nt = 0; nt < 3; ++nt)
+                mma_bf16(s[nt], a0, a1, a2, a3, qf[nt][ks][0], qf[nt][ks][1]);
+        }
+        // online softmax per query column (keys gq and gq+8 of this lane)
+        uint32_t bh[3][2], bl[3][2];
+#pragma unroll
+        for (int nt = 0; nt < 3; ++nt) {
+            float pv[4];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int k0 = kb + gq, k1 = kb + gq + 8;
+                const float v0 = (k0 < kend && k0 <= qpos[nt][e]) ? s[nt][e] * p.scale_log2 : -INFINITY;
+                const float v1 = (k1 < kend && k1 <= qpos[nt][e]) ? s[nt][e + 2] * p.scale_log2 : -INFINITY;
+                float mx = fmaxf(v0, v1);
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+                const float mn = fmaxf(m[nt][e], mx);
+                float corr, p0, p1;
+                if (mn == -INFINITY) {
+                    corr = 1.f;
+                    p0 = p1 = 0.f;
+                } else {
+                    corr = exp2f(m[nt][e] - mn);
+                    p0 = exp2f(v0 - mn);
+                    p1 = exp2f(v1 - mn);
+                }
+                m[nt][e] = mn;
+                l[nt][e] = l[nt][e] * corr + p0 + p1;
+                pv[e] = p0;
+                pv[e + 2] = p1;
+#pragma unroll
+                for (int dt = 0; dt < 8; ++dt) {
+                    o[dt][nt][e] *= corr;
+                    o[dt][nt][e + 2] *= corr;
+                }
+            }
+            // P^T fragment (keys x queries) via an in-register transpose, as bf16 hi + lo
+            const uint32_t h0 = pack_bf162(pv[0], pv[1]), h1 = pack_bf162(pv[2], pv[3]);
+            const uint32_t l0 = pack_bf162(pv[0] - bf16_to_f((uint16_t)(h0 & 0xFFFF)),
+                                           pv[1] - bf16_to_f((uint16_t)(h0 >> 16)));
+            const uint32_t l1 = pack_bf162(pv[2] - bf16_to_f((uint16_t)(h1 & 0xFFFF)),
+                                           pv[3] - bf16_to_f((uint16_t)(h1 >> 16)));
+            bh[nt][0] = movmatrix_t(h0);
+            bh[nt][1] = movmatrix_t(h1);
+            bl[nt][0] = movmatrix_t(l0);
+            bl[nt][1] = movmatrix_t(l1);
+        }
+#pragma unroll
+        for (int dt = 0; dt < 8; ++dt) {
+            uint32_t a0, a1, a2, a3;
+            const int key = (lane & 7) + 8 * (lane >> 4), ch = 2 * dt + ((lane >> 3) & 1);
+            ldsm_x4_t(a0, a1, a2, a3, Vs + swz(key, ch));
+#pragma unroll
+            for (int nt = 0; nt < 3; ++nt) {
+                mma_bf16(o[dt][nt], a0, a1, a2, a3, bh[nt][0], bh[nt][1]);
+                mma_bf16(o[dt][nt], a0, a1, a2, a3, bl[nt][0], bl[nt][1]);
+            }
+        }
+        __syncwarp();
+    }
+    cp_async_wait<0>();
+
+    // row sums over the 8 lanes sharing a query column
+#pragma unroll
+    for (int nt = 0; nt < 3; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            float v = l[nt][e];
+            v += __shfl_xor_sync(0xffffffffu, v, 4);
+            v += __shfl_xor_sync(0xffffffffu, v, 8);
+            v += __shfl_xor_sync(0xffffffffu, v, 16);
+            l[nt][e] = v;
+        }
+    __syncthreads();  // all warps done with their stages: reuse shared memory
+    float *sO = reinterpret_cast<float *>(smem);          // [4][QG][128]
+    float *sM = sO + ATT_WARPS * QG * 128;                // [4][QG]
+    float *sL = sM + ATT_WARPS * QG;                      // [4][QG]
+#pragma unroll
+    for (int dt = 0; dt < 8; ++dt)
+#pragma unroll
+        for (int nt = 0; nt < 3; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int d = 16 * dt + gq + 8 * (e >> 1), q = 8 * nt + 2 * c + (e & 1);
+                sO[((size_t)w * QG + q) * 128 + d] = o[dt][nt][e];
+            }
+    if (gq == 0) {
+#pragma unroll
+        for (int nt = 0; nt < 3; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                sM[w * QG + 8 * nt + 2 * c + e] = m[nt][e];
+                sL[w * QG + 8 * nt + 2 * c + e] = l[nt][e];
+            }
+    }
+    __syncthreads();
+    const size_t pidx = (((size_t)a * p.n_kvh + g) * p.n_rg + rg) * p.max_splits + sp;
+    float *out = p.part + pidx * PART_FLOATS;
+    for (int idx = tid; idx < QG * 128; idx += blockDim.x) {
+        const int q = idx >> 7;
+        float M = -INFINITY;
+#pragma unroll
+        for (int ww = 0; ww < ATT_WARPS; ++ww)
+            M = fmaxf(M, sM[ww * QG + q]);
+        float acc = 0.f;
+        if (M != -INFINITY)
+#pragma unroll
+            for (int ww = 0; ww < ATT_WARPS; ++ww)
+                acc += exp2f(sM[ww * QG + q] - M) * sO[((size_t)ww * QG + q) * 128 + (idx & 127)];
+        out[idx] = acc;
+    }
+    if (tid < QG) {
+        float M = -INFINITY, Lsum = 0.f;
+        for (int ww = 0; ww < ATT_WARPS; ++ww)
+            M = fmaxf(M, sM[ww * QG + tid]);
+        if (M != -INFINITY)
+            for (int ww = 0; ww < ATT_WARPS; ++ww)
+                Lsum += exp2f(sM[ww * QG + tid] - M) * sL[ww * QG + tid];
+        out[QG * 128 + tid] = M;
+        out[QG * 128 + QG + tid] = Lsum;
+    }
+}
+
+// One CTA per (query vector, row group, agent*kv-head); thread = dimension.
+__global__ void __launch_bounds__(128) k_attn_combine(AttnArgs p, uint16_t *O)
+{
+    const int q = blockIdx.x, rg = blockIdx.y, ag = blockIdx.z;
+    const int a = ag / p.n_kvh, g = ag - a * p.n_kvh;
+    const int d = threadIdx.x;
+    pdl_trigger();
+    pdl_wait();
+    const int r0 = p.ars[a], na = p.ars[a + 1] - r0;
+    const int R = na * p.G;
+    const int qi = rg * QG + q;
+    if (qi >= R)
+        return;
+    const int L = min(p.lens[a] + na, p.kv_cap);
+    const int nsp = (L + p.CH - 1) / p.CH;
+    const size_t base = (((size_t)a * p.n_kvh + g) * p.n_rg + rg) * p.max_splits;
+    float M = -INFINITY;
+    for (int s = 0; s < nsp; ++s)
+        M = fmaxf(M, p.part[(base + s) * PART_FLOATS + QG * 128 + q]);
+    float acc = 0.f, Ls = 0.f;
+    if (M != -INFINITY)
+        for (int s = 0; s < nsp; ++s) {
+            const float *pp = p.part + (base + s) * PART_FLOATS;
+            const float wgt = exp2f(pp[QG * 128 + q] - M);
+            acc += wgt * pp[q * 128 + d];
+            Ls += wgt * pp[QG * 128 + QG + q];
+        }
+    const int j = qi / p.G, hl = qi - j * p.G;
+    O[((size_t)(r0 + j) * p.n_qh + g * p.G + hl) * 128 + d] = f_to_bf16(Ls > 0.f ? acc / Ls : 0.f);
+}
+
+// ------------------------------------------------------------- host side
+
+AttnPlan attn_plan(int n_agents, int n_qh, int n_kvh, int kv_cap, int max_rows_per_agent)
+{
+    AttnPlan pl;
+    pl.G = n_qh / n_kvh;
+    pl.n_rg = (max_rows_per_agent * pl.G + QG - 1) / QG;
+    // one wave: two resident CTAs per SM (registers and shared memory allow two)
+    const int pairs = n_agents * n_kvh * pl.n_rg;
+    const int target = 2 * num_sms();
+    int splits = target / pairs;
+    if (splits < 1)
+        splits = 1;
+    int ch = (kv_cap + splits - 1) / splits;
+    ch = ((ch + 63) / 64) * 64;
+    if (ch < 64)
+        ch = 64;
+    pl.CH = ch;
+    pl.max_splits = (kv_cap + ch - 1) / ch;
+    pl.part_bytes = (size_t)n_agents * n_kvh * pl.n_rg * pl.max_splits * PART_FLOATS * sizeof(float);
+    return pl;
+}
+
+size_t attn_smem_bytes()
+{
+    const size_t stages = (size_t)ATT_WARPS * ATT_STAGES * 2 * TILE_BYTES;
+    const size_t merge = ((size_t)ATT_WARPS * QG * 128 + 2 * ATT_WARPS * QG) * sizeof(float);
+    return stages > merge ? stages : merge;
+}
+
+int launch_attn(const AttnPlan &pl, const uint16_t *Q, const uint16_t *Kc, const uint16_t *Vc, const int *lens,
+                const int *ars, int n_agents, int kv_cap, int n_qh, int n_kvh, float scale, uint16_t *O, float *part,
+                cudaStream_t s, bool pdl)
+{
+    AttnArgs p;
+    p.Q = Q;
+    p.Kc = Kc;
+    p.Vc = Vc;
+    p.lens = lens;
+    p.ars = ars;
+    p.n_kvh = n_kvh;
+    p.kv_cap = kv_cap;
+    p.n_qh = n_qh;
+    p.G = pl.G;
+    p.CH = pl.CH;
+    p.n_rg = pl.n_rg;
+    p.max_splits = pl.max_splits;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.part = part;
+    const size_t smem = attn_smem_bytes();
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+        int rc = cuda_check(cudaFuncSetAttribute(k_decode_attn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem),
+                            "cudaFuncSetAttribute(attn)");
+        if (rc)
+            return rc;
+        if (dev >= 0 && dev < 64)
+            attr_set[dev] = true;
+    }
+    dim3 grid(pl.max_splits, pl.n_rg, n_agents * n_kvh);
+    cudaError_t e = pdl ? launch_pdl(k_decode_attn, grid, dim3(128), smem, s, p)
+                        : (k_decode_attn<<<grid, 128, smem, s>>>(p), cudaGetLastError());
+    if (e != cudaSuccess)
+        return cuda_check(e, "attn launch");
+    dim3 g2(QG, pl.n_rg, n_agents * n_kvh);
+    e = pdl ? launch_pdl(k_attn_combine, g2, dim3(128), 0, s, p, O)
+            : (k_attn_combine<<<g2, 128, 0, s>>>(p, O), cudaGetLastError());
+    return cuda_check(e, "attn combine launch");
+}
+
+}  // namespace qad
+
+extern "C" size_t qad_decode_attn_ws_bytes(int n_agents, int n_qh, int n_kvh, int kv_cap, int max_rows_per_agent)
+{
+    if (n_agents <= 0 || n_kvh <= 0 || n_qh <= 0 || n_qh % n_kvh || kv_cap <= 0 || max_rows_per_agent <= 0)
+        return 0;
+    return qad::attn_plan(n_agents, n_qh, n_kvh, kv_cap, max_rows_per_agent).part_bytes;
+}
+
+extern "C" int qad_decode_attn(const uint16_t *Q, const uint16_t *Kc, const uint16_t *Vc, const int *lens,
+                               const int *agent_row_start, int n_agents, int max_rows_per_agent, int kv_cap, int n_qh,
+                               int n_kvh, int hd, float scale, uint16_t *O, void *ws, size_t ws_bytes, void *stream)
+{
+    if (!Q || !Kc || !Vc || !lens || !agent_row_start || !O || !ws || n_agents <= 0 || kv_cap <= 0 || n_qh <= 0 ||
+        n_kvh <= 0 || max_rows_per_agent <= 0)
+        return qad::fail(QAD_ERR_INVALID, "qad_decode_attn: null pointer or non-positive size");
+    if (hd != 128 || n_qh % n_kvh || max_rows_per_agent * (n_qh / n_kvh) > 96 || max_rows_per_agent > QAD_MAX_ROWS)
+        return qad::fail(QAD_ERR_UNSUPPORTED,
+                         "qad_decode_attn: need hd == 128, n_qh %% n_kvh == 0, rows*group <= 96 (hd=%d n_qh=%d n_kvh=%d "
+                         "rows=%d)",
+                         hd, n_qh, n_kvh, max_rows_per_agent);
+    if (((uintptr_t)Kc | (uintptr_t)Vc) & 15)
+        return qad::fail(QAD_ERR_INVALID, "qad_decode_attn: caches must be 16-byte aligned");
+    qad::AttnPlan pl = qad::attn_plan(n_agents, n_qh, n_kvh, kv_cap, max_rows_per_agent);
+    if (ws_bytes < pl.part_bytes)
+        return qad::fail(QAD_ERR_WORKSPACE, "qad_decode_attn: workspace %zu < %zu bytes", ws_bytes, pl.part_bytes);
+    return qad::launch_attn(pl, Q, Kc, Vc, lens, agent_row_start, n_agents, kv_cap, n_qh, n_kvh, scale, O,
+                            (float *)ws, (cudaStream_t)stream, false);
+}

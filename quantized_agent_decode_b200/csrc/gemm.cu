@@ -1,0 +1,817 @@
+// gemm.cu -- the shared weight pass: skinny (M <= 16) dequant-GEMM over Q4_K
+// and Q6_K-like weights, Y[r][n] = sum_k w[n][k] x[r][k].
+//
+// [OpenJet page] = rebasdaily.com 2026-10-29, "OpenJet ... multi-agent
+// serving", section 只搬一次权重 (move the weights once): the rows of all
+// active agents are stacked into one batch, the quantized weights are read
+// from memory once per step and every weight just read is used for all rows.
+// The page's own cost model is that weight read (16.7 GB / 936 GB/s ~ 18 ms
+// on its GPU), so this kernel is an HBM stream with the decode and the
+// multiply-accumulate hidden under it.
+//
+// Design (sm_100a):
+//  * Each quantized byte is loaded exactly once, by one thread, with 16-byte
+//    streaming loads (Q4_K blocks are 16-byte aligned; the 210-byte Q6_K-like
+//    blocks are read as 4-byte words and realigned with funnel shifts).
+//  * The block is decoded in registers into fp16 tensor-core operands that are
+//    EXACT: for Q4_K, A = sc_j * q (<= 945) and the mins enter through a second
+//    small MMA against per-sub-block activation sums; for Q6_K, A = sc * (q-32)
+//    (|.| <= 2048 for |sc| <= 64). The fp16 values come from the "1024 + q"
+//    exponent trick (OR of the nibble into the mantissa of 1024.0) followed by
+//    one fused multiply-add that applies the scale.
+//  * M = 12 rows need ~16 multiply-adds per weight, four times what the FP32
+//    pipes deliver at the HBM rate, so the product runs on the tensor cores as
+//    m16n8k16 warp MMAs (weights = A, the 16 padded activation rows = B).
+//  * The activations are prepared once per GEMM (k_prep) into fp16 B
+//    fragments in exactly the register order each lane consumes, with a
+//    per-row power-of-two scale so fp16's range always holds them.
+//  * Work is split stream-K style over all warps of a persistent grid (one CTA
+//    per SM): unit = (tile of 16*MT weight rows, one 256-wide block); each warp
+//    takes a contiguous run of units, accumulates in registers, and adds its
+//    partial tile sums into Y with fp32 atomics when its run leaves a tile.
+//  * Programmatic dependent launch: the first unit's weights are requested
+//    before griddepcontrol.wait, so the weight stream starts while the
+//    producer of the activations is still finishing.
+#include <cuda.h>
+
+#include "gemm.cuh"
+
+namespace qad {
+
+// Set by a GEMM whose pipeline wait timed out (1: a consumer, 2: the producer);
+// read and cleared by qad_device_status().
+__device__ int g_gemm_status;
+
+// ------------------------------------------------------------- fragment layout
+// Activation rows r = 8*nt + g (nt < NT, g < 8); blocks b < nblk; k-steps
+// s < 16; lane quad c < 4. Block-major, so one block's fragments are one
+// contiguous bulk copy and a warp's 32 lanes read 32 consecutive entries.
+//   XP (uint2 units): [b][s][g][c][nt] = {b0, b1}: the two B registers of the
+//       m16n8k16 fragment: b0 = (x[k0], x[k0+2]), b1 = (x[k0+1], x[k0+3]) with
+//       k0 = 256 b + frag_k0(s, c), as fp16 of x * 2^e_r.
+//   SP (uint2 units): [b][g][c][nt] = {(Shi_2c, Shi_2c+1), (Slo_2c, Slo_2c+1)}
+//       with S_j the sum of the 32 fp16 activations of Q4_K sub-block j split
+//       into two fp16 parts (Q4_K only).
+//   RS: 16 floats, 2^-e_r (0 for rows >= M).
+static inline size_t xp_words(int nblk, int nt) { return (size_t)8 * nblk * 16 * 4 * nt * 2; }
+static inline size_t sp_words(int nblk, int nt) { return (size_t)8 * nblk * 4 * nt * 2; }
+static inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+size_t frag_bytes(int K, int nt)
+{
+    int nblk = K / 256;
+    return align256(xp_words(nblk, nt) * 4) + align256(sp_words(nblk, nt) * 4) + 256;
+}
+
+FragBuf frag_carve(void *ws, int K, int nt)
+{
+    int nblk = K / 256;
+    char *p = (char *)ws;
+    FragBuf f;
+    f.xp = (uint32_t *)p;
+    p += align256(xp_words(nblk, nt) * 4);
+    f.sp = (uint32_t *)p;
+    p += align256(sp_words(nblk, nt) * 4);
+    f.rs = (float *)p;
+    return f;
+}
+
+// Which activation column feeds logical k-slot (s, c). The weight-side decode
+// below produces, for lane quad c and k-step s, the weights at within-block
+// positions k0, k0+2 (first B register) and k0+1, k0+3 (second).
+template <int FMT>
+__device__ __forceinline__ int frag_k0(int s, int c)
+{
+    if (FMT == 4)  // quant bytes 32c..32c+31: word s>>1, low (s even) or high (s odd) nibbles
+        return 64 * c + 4 * (s >> 1) + 32 * (s & 1);
+    else           // half c>>1, l-range 16*(c&1); word s>>2; t = s&3 selects the 32-weight quarter
+        return 128 * (c >> 1) + 16 * (c & 1) + 4 * (s >> 2) + 32 * (s & 3);
+}
+
+// ------------------------------------------------------------- prep kernel
+
+struct PrepArgs {
+    PrepSrc src;
+    int K, M;
+    FragBuf fb;
+};
+
+__device__ __forceinline__ float warp_sum(float v)
+{
+#pragma unroll
+    for (int o = 16; o; o >>= 1)
+        v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+__device__ __forceinline__ float warp_max(float v)
+{
+#pragma unroll
+    for (int o = 16; o; o >>= 1)
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+__device__ float block_sum(float v, float *red)
+{
+    v = warp_sum(v);
+    int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+    __syncthreads();
+    if (l == 0)
+        red[w] = v;
+    __syncthreads();
+    v = (l < (int)(blockDim.x >> 5)) ? red[l] : 0.f;
+    return warp_sum(v);
+}
+__device__ float block_max(float v, float *red)
+{
+    v = warp_max(v);
+    int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+    __syncthreads();
+    if (l == 0)
+        red[w] = v;
+    __syncthreads();
+    v = (l < (int)(blockDim.x >> 5)) ? red[l] : 0.f;
+    return warp_max(v);
+}
+__device__ __forceinline__ float round_half(float v) { return __half2float(__float2half_rn(v)); }
+
+// One CTA per activation row r < 8*NT (rows >= M write zero fragments).
+// Phase 1 forms the row exactly as the GEMM must see it (bf16 values: the
+// input itself, RMSNorm of the fp32 residual, or silu(gate)*up), phase 2 picks
+// the power-of-two scale that puts max|x| in [512, 1024) and writes the row's
+// fragments and sub-block sums.
+template <int FMT, int NT>
+__global__ void __launch_bounds__(512) k_prep(PrepArgs a)
+{
+    extern __shared__ uint16_t sxb[];  // the row as bf16 bits
+    __shared__ float red[32];
+    const int r = blockIdx.x, tid = threadIdx.x, nth = blockDim.x;
+    const int K = a.K, nblk = K >> 8;
+    const PrepSrc &S = a.src;
+    pdl_trigger();
+    pdl_wait();
+    if (S.zero) {
+        long long per = (S.zero_n + gridDim.x - 1) / gridDim.x;
+        long long z0 = (long long)r * per, z1 = min(S.zero_n, z0 + per);
+        for (long long i = z0 + tid; i < z1; i += nth)
+            S.zero[i] = 0.f;
+    }
+    const bool live = r < a.M;
+    float mx = 0.f;
+    if (live) {
+        if (S.kind == PREP_BF16) {
+            const uint16_t *x = S.xb + (size_t)r * S.ldx;
+            for (int k = tid; k < K; k += nth) {
+                const uint16_t v = x[k];
+                sxb[k] = v;
+                mx = fmaxf(mx, fabsf(bf16_to_f(v)));
+            }
+        } else if (S.kind == PREP_RMSNORM) {
+            const float *h = S.xf + (size_t)r * S.ldx;
+            float ss = 0.f;
+            for (int k = tid; k < K; k += nth) {
+                float v = h[k];
+                ss = fmaf(v, v, ss);
+            }
+            ss = block_sum(ss, red);
+            const float inv = 1.f / sqrtf(ss / (float)K + S.eps);
+            for (int k = tid; k < K; k += nth) {
+                const uint16_t v = f_to_bf16(h[k] * inv);
+                sxb[k] = v;
+                mx = fmaxf(mx, fabsf(bf16_to_f(v)));
+            }
+        } else {
+            const float *gp = S.xf + (size_t)r * S.ldx;
+            for (int k = tid; k < K; k += nth) {
+                const float gg = gp[k], uu = gp[K + k];
+                float r;
+                if (gg >= -80.f) {
+                    r = gg / (1.f + expf(-gg)) * uu;
+                } else {
+                    // 1 + e^-g == e^-g in fp32 here; e^-g would overflow below -88, so
+                    // form g*u*e^g in the log domain (exact zero stays zero)
+                    const float p = gg * uu;
+                    r = p == 0.f ? p : copysignf(expf(gg + logf(fabsf(p))), p);
+                }
+                const uint16_t v = f_to_bf16(r);
+                sxb[k] = v;
+                mx = fmaxf(mx, fabsf(bf16_to_f(v)));
+            }
+        }
+        if (S.dbg)
+            for (int k = tid; k < K; k += nth)
+                S.dbg[(size_t)r * S.ld_dbg + k] = sxb[k];
+    }
+    mx = block_max(mx, red);
+    int e = 0;
+    if (mx > 0.f) {
+        int E;
+        frexpf(mx, &E);  // mx in [2^(E-1), 2^E)
+        e = min(126, max(-126, 10 - E));
+    }
+    const float sc = ldexpf(1.f, e);
+    if (tid == 0)
+        a.fb.rs[r] = live ? ldexpf(1.f, -e) : 0.f;
+    __syncthreads();
+    const int g = r & 7, nt = r >> 3;
+    uint2 *xp = reinterpret_cast<uint2 *>(a.fb.xp);
+    for (int it = tid; it < nblk * 64; it += nth) {
+        const int b = it >> 6, s = (it >> 2) & 15, c = it & 3;
+        uint2 v = make_uint2(0u, 0u);
+        if (live) {
+            const int k = 256 * b + frag_k0<FMT>(s, c);
+            v.x = pack_half2(bf16_to_f(sxb[k]) * sc, bf16_to_f(sxb[k + 2]) * sc);
+            v.y = pack_half2(bf16_to_f(sxb[k + 1]) * sc, bf16_to_f(sxb[k + 3]) * sc);
+        }
+        xp[((((size_t)b * 16 + s) * 8 + g) * 4 + c) * NT + nt] = v;
+    }
+    if (FMT == 4) {
+        uint2 *sp = reinterpret_cast<uint2 *>(a.fb.sp);
+        for (int it = tid; it < nblk * 4; it += nth) {
+            const int b = it >> 2, c = it & 3;
+            uint2 v = make_uint2(0u, 0u);
+            if (live) {
+                const uint16_t *x0 = sxb + 256 * b + 64 * c;
+                float s0 = 0.f, s1 = 0.f;
+                for (int k = 0; k < 32; ++k) {
+                    s0 += round_half(bf16_to_f(x0[k]) * sc);
+                    s1 += round_half(bf16_to_f(x0[32 + k]) * sc);
+                }
+                const float h0 = round_half(s0), h1 = round_half(s1);
+                v.x = pack_half2(h0, h1);
+                v.y = pack_half2(s0 - h0, s1 - h1);
+            }
+            sp[(((size_t)b * 8 + g) * 4 + c) * NT + nt] = v;
+        }
+    }
+}
+
+// ------------------------------------------------------------- GEMM kernels
+//
+// One CTA per SM: 8 consumer warps + 1 producer warp. A CTA unit is a tile of
+// 128 weight rows x one 256-wide block. Units are numbered tile-major with the
+// block fastest, and each CTA takes a contiguous run of them (stream-K). For
+// each unit the producer issues ONE 2-D tensor-map load (TMA) of the 128
+// row-blocks (plus the d plane for Q6_K) and one bulk copy of the block's
+// activation fragments into a ring of shared-memory stages, completing on a
+// "full" mbarrier; the consumer warps (16 rows each) decode their rows from
+// shared memory, run the MMAs and release the stage on an "empty" mbarrier.
+// Every wait is bounded: on timeout the warp records a status code and returns.
+//
+// Q6_K-like weights use the packed device layout of qad_q6k_pack(): plane A
+// [N][nblk][208] (ql, qh, int8 scales: the first 208 bytes of each GGUF block,
+// so every field is 16-byte aligned) followed by plane D [N][ceil8(nblk)] fp16
+// d. 210-byte GGUF blocks cannot be addressed by TMA (16-byte start rule).
+
+constexpr int GW = 8;                // consumer warps per CTA
+constexpr int TILE_ROWS = 16 * GW;   // weight rows per CTA unit
+constexpr int Q6A_BYTES = 208;       // plane A bytes per Q6_K block
+
+template <int FMT, int NT>
+struct Stage {
+    static constexpr int W_BYTES = TILE_ROWS * (FMT == 4 ? 144 : Q6A_BYTES);
+    static constexpr int D_BYTES = FMT == 4 ? 0 : TILE_ROWS * 16;   // 8 fp16 d per row (aligned group of 8 blocks)
+    static constexpr int X_BYTES = 4096 * NT;                       // [s 16][g 8][c 4][nt][2 words]
+    static constexpr int S_BYTES = FMT == 4 ? 256 * NT : 0;         // [g 8][c 4][nt][2 words]
+    static constexpr int BYTES = W_BYTES + D_BYTES + X_BYTES + S_BYTES;
+};
+
+template <int FMT>
+struct Stages {
+    static constexpr int N = FMT == 4 ? 6 : 5;
+};
+
+template <int FMT, int NT>
+constexpr size_t gemm_smem_bytes()
+{
+    return (size_t)Stages<FMT>::N * Stage<FMT, NT>::BYTES + 2 * Stages<FMT>::N * sizeof(uint64_t);
+}
+
+struct WeightMaps {
+    CUtensorMap w;  // Q4_K matrix, or Q6_K plane A
+    CUtensorMap d;  // Q6_K plane D (unused for Q4_K)
+};
+
+struct GemmArgs {
+    int N, nblk, M, ldy, units;
+    const uint32_t *xp, *sp;
+    const float *rs;
+    float *Y;
+};
+
+enum { ERR_FULL_TIMEOUT = 1, ERR_EMPTY_TIMEOUT = 2 };
+
+template <int NT>
+__device__ __forceinline__ void flush_rows(float (&tot)[NT][4], const GemmArgs &a, int n0, int g, int c)
+{
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int n = n0 + g + 8 * (e >> 1);
+            const int r = 8 * nt + 2 * c + (e & 1);
+            if (n < a.N && r < a.M)
+                atomicAdd(a.Y + (size_t)r * a.ldy + n, a.rs[r] * tot[nt][e]);
+            tot[nt][e] = 0.f;
+        }
+}
+
+template <int NT>
+__device__ __forceinline__ void lds_b(const uint8_t *p, uint32_t (&b)[NT][2])
+{
+    if (NT == 2) {
+        const uint4 v = lds_v4(p);
+        b[0][0] = v.x;
+        b[0][1] = v.y;
+        b[NT - 1][0] = v.z;
+        b[NT - 1][1] = v.w;
+    } else {
+        const uint2 v = lds_v2(p);
+        b[0][0] = v.x;
+        b[0][1] = v.y;
+    }
+}
+
+__device__ __forceinline__ uint32_t u4w(const uint4 &v, int i)
+{
+    return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
+
+// One Q4_K block of this warp's 16 rows against all activation rows.
+// W16: the warp's first row in the stage; XS/SS: the block's fragments.
+template <int NT>
+__device__ __forceinline__ void q4_block(const uint8_t *W16, const uint8_t *XS, const uint8_t *SS, int g, int c,
+                                         uint32_t selT, bool hib, float (&tot)[NT][4])
+{
+    uint4 hdr[2], q0[2], q1[2];
+#pragma unroll
+    for (int rh = 0; rh < 2; ++rh) {
+        const uint8_t *row = W16 + (g + 8 * rh) * 144;
+        hdr[rh] = lds_v4(row);
+        q0[rh] = lds_v4(row + 16 + 32 * c);
+        q1[rh] = lds_v4(row + 32 + 32 * c);
+    }
+    uint32_t SCl[2], NGl[2], SCh[2], NGh[2], AM[2];
+    float dd[2], dm[2];
+#pragma unroll
+    for (int rh = 0; rh < 2; ++rh) {
+        const uint4 h = hdr[rh];
+        // scales/mins of sub-blocks 2c and 2c+1 (bytes (2c)&3, +1 of the packed words)
+        const uint32_t scA = h.y & 0x3F3F3F3Fu, mA = h.z & 0x3F3F3F3Fu;
+        const uint32_t scB = (h.w & 0x0F0F0F0Fu) | ((h.y >> 2) & 0x30303030u);
+        const uint32_t mB = ((h.w >> 4) & 0x0F0F0F0Fu) | ((h.z >> 2) & 0x30303030u);
+        const uint32_t T = prmt(hib ? scB : scA, hib ? mB : mA, selT);  // [sc_lo, sc_hi, m_lo, m_hi]
+        const uint32_t Tl = prmt(T, 0x64u, 0x4040u);                     // 1024 + sc_lo (x2)
+        const uint32_t Th = prmt(T, 0x64u, 0x4141u);                     // 1024 + sc_hi (x2)
+        const uint32_t Tm = prmt(T, 0x64u, 0x4342u);                     // 1024 + (m_lo, m_hi)
+        SCl[rh] = hsub2(Tl, H2_1024);                                    // sc_lo
+        NGl[rh] = hmul2(SCl[rh], H2_NEG1024);                            // -1024 sc_lo
+        SCh[rh] = hfma2(Th, H2_SIXTEENTH, H2_NEG64);                     // sc_hi / 16
+        NGh[rh] = hmul2(SCh[rh], H2_NEG1024);                            // -64 sc_hi
+        AM[rh] = hsub2(Tm, H2_1024);                                     // (m_lo, m_hi)
+        dd[rh] = half_lo(h.x);
+        dm[rh] = half_hi(h.x);
+    }
+    float acc[NT][4];
+    const uint8_t *xl = XS + (g * 4 + c) * 8 * NT;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        uint32_t blo[NT][2], bhi[NT][2];
+        lds_b<NT>(xl + (2 * i) * 256 * NT, blo);
+        lds_b<NT>(xl + (2 * i + 1) * 256 * NT, bhi);
+        const uint32_t w0 = i < 4 ? u4w(q0[0], i) : u4w(q1[0], i - 4);
+        const uint32_t w1 = i < 4 ? u4w(q0[1], i) : u4w(q1[1], i - 4);
+        const uint32_t w0s = w0 >> 8, w1s = w1 >> 8;
+        // low nibbles: sub-block 2c, k-step 2i
+        const uint32_t a0 = hfma2(and_or(w0, 0x000F000Fu, H2_1024), SCl[0], NGl[0]);
+        const uint32_t a1 = hfma2(and_or(w1, 0x000F000Fu, H2_1024), SCl[1], NGl[1]);
+        const uint32_t a2 = hfma2(and_or(w0s, 0x000F000Fu, H2_1024), SCl[0], NGl[0]);
+        const uint32_t a3 = hfma2(and_or(w1s, 0x000F000Fu, H2_1024), SCl[1], NGl[1]);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            if (i == 0)
+                mma_f16_zero(acc[nt], a0, a1, a2, a3, blo[nt][0], blo[nt][1]);
+            else
+                mma_f16(acc[nt], a0, a1, a2, a3, blo[nt][0], blo[nt][1]);
+        }
+        // high nibbles: sub-block 2c+1, k-step 2i+1
+        const uint32_t c0 = hfma2(and_or(w0, 0x00F000F0u, H2_1024), SCh[0], NGh[0]);
+        const uint32_t c1 = hfma2(and_or(w1, 0x00F000F0u, H2_1024), SCh[1], NGh[1]);
+        const uint32_t c2 = hfma2(and_or(w0s, 0x00F000F0u, H2_1024), SCh[0], NGh[0]);
+        const uint32_t c3 = hfma2(and_or(w1s, 0x00F000F0u, H2_1024), SCh[1], NGh[1]);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+            mma_f16(acc[nt], c0, c1, c2, c3, bhi[nt][0], bhi[nt][1]);
+    }
+    // mins: sum_j m_j * S_j, S split into two fp16 parts along k
+    uint32_t sb[NT][2];
+    lds_b<NT>(SS + (g * 4 + c) * 8 * NT, sb);
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        float accm[4];
+        mma_f16_zero(accm, AM[0], AM[1], AM[0], AM[1], sb[nt][0], sb[nt][1]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int rh = e >> 1;
+            tot[nt][e] = fmaf(dd[rh], acc[nt][e], tot[nt][e]);
+            tot[nt][e] = fmaf(-dm[rh], accm[e], tot[nt][e]);
+        }
+    }
+}
+
+constexpr uint32_t H2_1152 = 0x64806480u;  // 1152.0
+
+// One Q6_K-like block (packed layout) of this warp's 16 rows. A16: the warp's
+// first row in plane A of the stage; D16: its first row of the d tile.
+template <int NT>
+__device__ __forceinline__ void q6_block(const uint8_t *A16, const uint8_t *D16, int bsub, const uint8_t *XS, int g,
+                                         int c, float (&tot)[NT][4])
+{
+    uint4 QL0[2], QL1[2], QH[2];
+    uint32_t SC[2][4];
+    float dd[2];
+    const int h = c >> 1, lq = 16 * (c & 1);
+#pragma unroll
+    for (int rh = 0; rh < 2; ++rh) {
+        const uint8_t *blk = A16 + (g + 8 * rh) * Q6A_BYTES;
+        QL0[rh] = lds_v4(blk + 64 * h + lq);
+        QL1[rh] = lds_v4(blk + 64 * h + 32 + lq);
+        QH[rh] = lds_v4(blk + 128 + 32 * h + lq);
+        // int8 scales of sub-blocks 8h + 2t + (c&1): bytes (c&1) + 2t of the 8 scale bytes
+        const uint2 sw = lds_v2(blk + 192 + 8 * h);
+        const uint32_t s0 = sw.x ^ 0x80808080u, s1 = sw.y ^ 0x80808080u;
+        const uint32_t j = (uint32_t)(c & 1);
+        const uint32_t sel0 = j | 0x40u | (j << 8) | 0x4000u, sel1 = (j + 2) | 0x40u | ((j + 2) << 8) | 0x4000u;
+        // (sc + 128) + 1024 - 1152 = sc, exact in fp16
+        SC[rh][0] = hsub2(prmt(s0, 0x64u, sel0), H2_1152);
+        SC[rh][1] = hsub2(prmt(s0, 0x64u, sel1), H2_1152);
+        SC[rh][2] = hsub2(prmt(s1, 0x64u, sel0), H2_1152);
+        SC[rh][3] = hsub2(prmt(s1, 0x64u, sel1), H2_1152);
+        const uint32_t dw = lds_u32(D16 + (g + 8 * rh) * 16 + (bsub & 6) * 2);
+        dd[rh] = __half2float(__ushort_as_half((unsigned short)(dw >> ((bsub & 1) * 16))));
+    }
+    float acc[NT][4];
+    const uint8_t *xl = XS + (g * 4 + c) * 8 * NT;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint32_t qt[2][4];
+#pragma unroll
+        for (int rh = 0; rh < 2; ++rh) {
+            const uint32_t l0 = u4w(QL0[rh], i), l1 = u4w(QL1[rh], i), hh = u4w(QH[rh], i);
+            qt[rh][0] = (l0 & 0x0F0F0F0Fu) | ((hh << 4) & 0x30303030u);
+            qt[rh][1] = (l1 & 0x0F0F0F0Fu) | ((hh << 2) & 0x30303030u);
+            qt[rh][2] = ((l0 >> 4) & 0x0F0F0F0Fu) | (hh & 0x30303030u);
+            qt[rh][3] = ((l1 >> 4) & 0x0F0F0F0Fu) | ((hh >> 2) & 0x30303030u);
+        }
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            const int s = 4 * i + t;
+            uint32_t bf[NT][2];
+            lds_b<NT>(xl + s * 256 * NT, bf);
+            // pairs (bytes 0,2) and (bytes 1,3) -> 1024 + q -> q - 32 -> sc*(q-32)
+            const uint32_t a0 = hmul2(hsub2(prmt(qt[0][t], 0x64u, 0x4240u), H2_1056), SC[0][t]);
+            const uint32_t a1 = hmul2(hsub2(prmt(qt[1][t], 0x64u, 0x4240u), H2_1056), SC[1][t]);
+            const uint32_t a2 = hmul2(hsub2(prmt(qt[0][t], 0x64u, 0x4341u), H2_1056), SC[0][t]);
+            const uint32_t a3 = hmul2(hsub2(prmt(qt[1][t], 0x64u, 0x4341u), H2_1056), SC[1][t]);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                if (s == 0)
+                    mma_f16_zero(acc[nt], a0, a1, a2, a3, bf[nt][0], bf[nt][1]);
+                else
+                    mma_f16(acc[nt], a0, a1, a2, a3, bf[nt][0], bf[nt][1]);
+            }
+        }
+    }
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            tot[nt][e] = fmaf(dd[e >> 1], acc[nt][e], tot[nt][e]);
+}
+
+template <int FMT, int NT>
+__global__ void __launch_bounds__(32 * (GW + 1), 1) k_qgemm(const __grid_constant__ WeightMaps maps, GemmArgs a)
+{
+    extern __shared__ __align__(128) uint8_t smem[];
+    using St = Stage<FMT, NT>;
+    constexpr int S = Stages<FMT>::N;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + (size_t)S * St::BYTES);
+    uint64_t *empty = full + S;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int u0 = (int)((long long)blockIdx.x * a.units / gridDim.x);
+    const int u1 = (int)((long long)(blockIdx.x + 1) * a.units / gridDim.x);
+    const int n_units = u1 - u0;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < S; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], GW);
+        }
+        mbar_fence_init();
+    }
+    __syncthreads();
+    pdl_trigger();
+
+    if (warp == GW) {
+        // ------------------------------------------------ producer warp (lane 0 issues)
+        if (lane != 0) {
+            pdl_wait();
+            return;
+        }
+        auto issue_weights = [&](int i) {
+            const int u = u0 + i, t = u / a.nblk, b = u - t * a.nblk;
+            uint8_t *st = smem + (size_t)(i % S) * St::BYTES;
+            uint64_t *bar = &full[i % S];
+            mbar_arrive_expect_tx(bar, (uint32_t)St::BYTES);
+            tma_load_2d(st, &maps.w, b * (FMT == 4 ? 144 : Q6A_BYTES), t * TILE_ROWS, bar);
+            if (FMT == 6)
+                tma_load_2d(st + St::W_BYTES, &maps.d, b & ~7, t * TILE_ROWS, bar);
+        };
+        auto issue_frags = [&](int i) {
+            const int u = u0 + i, t = u / a.nblk, b = u - t * a.nblk;
+            (void)t;
+            uint8_t *st = smem + (size_t)(i % S) * St::BYTES + St::W_BYTES + St::D_BYTES;
+            uint64_t *bar = &full[i % S];
+            bulk_g2s(st, reinterpret_cast<const uint8_t *>(a.xp) + (size_t)b * St::X_BYTES, St::X_BYTES, bar);
+            if (FMT == 4)
+                bulk_g2s(st + St::X_BYTES, reinterpret_cast<const uint8_t *>(a.sp) + (size_t)b * St::S_BYTES,
+                         St::S_BYTES, bar);
+        };
+        const int pre = min(S, n_units);
+        for (int i = 0; i < pre; ++i)
+            issue_weights(i);  // weights do not depend on the previous kernel
+        pdl_wait();
+        for (int i = 0; i < pre; ++i)
+            issue_frags(i);
+        for (int i = S; i < n_units; ++i) {
+            if (!mbar_wait(&empty[i % S], ((i / S) - 1) & 1)) {
+                atomicExch(&g_gemm_status, ERR_EMPTY_TIMEOUT);
+                return;
+            }
+            issue_weights(i);
+            issue_frags(i);
+        }
+        return;
+    }
+
+    // ---------------------------------------------------- consumer warps
+    const int g = lane >> 2, c = lane & 3;
+    const int jj = 2 * (c & 1);
+    const uint32_t selT = (uint32_t)(jj | ((jj + 1) << 4) | ((jj + 4) << 8) | ((jj + 5) << 12));
+    const bool hib = c >= 2;
+    pdl_wait();
+    float tot[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            tot[nt][e] = 0.f;
+    int t = n_units > 0 ? u0 / a.nblk : 0, b = u0 - t * a.nblk;
+    for (int i = 0; i < n_units; ++i) {
+        const uint8_t *st = smem + (size_t)(i % S) * St::BYTES;
+        if (!mbar_wait(&full[i % S], (i / S) & 1)) {
+            if (lane == 0)
+                atomicExch(&g_gemm_status, ERR_FULL_TIMEOUT);
+            return;
+        }
+        const uint8_t *XS = st + St::W_BYTES + St::D_BYTES;
+        if (FMT == 4)
+            q4_block<NT>(st + (size_t)(16 * warp) * 144, XS, XS + St::X_BYTES, g, c, selT, hib, tot);
+        else
+            q6_block<NT>(st + (size_t)(16 * warp) * Q6A_BYTES, st + St::W_BYTES + (size_t)(16 * warp) * 16, b & 7, XS,
+                         g, c, tot);
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(&empty[i % S]);
+        if (b == a.nblk - 1 || i == n_units - 1)
+            flush_rows<NT>(tot, a, t * TILE_ROWS + 16 * warp, g, c);
+        if (++b == a.nblk) {
+            b = 0;
+            ++t;
+        }
+    }
+}
+
+// Q6_K-like GGUF blocks -> packed device layout (plane A: first 208 bytes of
+// each block; plane D: d, rows padded to a multiple of 8 blocks with zeros).
+__global__ void k_q6k_pack(const uint8_t *__restrict__ W, int N, int nblk, uint8_t *__restrict__ P)
+{
+    const int nblk8 = (nblk + 7) & ~7;
+    uint8_t *A = P;
+    uint16_t *D = reinterpret_cast<uint16_t *>(P + (size_t)N * nblk * Q6A_BYTES);
+    const long long total = (long long)N * nblk;
+    for (long long blk = blockIdx.x * (long long)(blockDim.x / 32) + threadIdx.x / 32; blk < total;
+         blk += (long long)gridDim.x * (blockDim.x / 32)) {
+        const uint8_t *src = W + blk * 210;
+        uint8_t *dst = A + blk * Q6A_BYTES;
+        for (int i = threadIdx.x & 31; i < Q6A_BYTES; i += 32)
+            dst[i] = src[i];
+        if ((threadIdx.x & 31) == 0) {
+            const long long n = blk / nblk, b = blk - n * nblk;
+            D[n * nblk8 + b] = (uint16_t)(src[208] | src[209] << 8);
+            if (b == nblk - 1)
+                for (int p = nblk; p < nblk8; ++p)
+                    D[n * nblk8 + p] = 0;
+        }
+    }
+}
+
+size_t q6k_packed_bytes(long long N, int K)
+{
+    const int nblk = K / 256, nblk8 = (nblk + 7) & ~7;
+    return (size_t)N * nblk * Q6A_BYTES + (size_t)N * nblk8 * 2;
+}
+
+// ------------------------------------------------------------- launchers
+
+template <typename K>
+static int set_smem(K kernel, size_t bytes)
+{
+    return cuda_check(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes),
+                      "cudaFuncSetAttribute");
+}
+
+int launch_prep(int fmt, int K, int M, const PrepSrc &src, const FragBuf &fb, cudaStream_t s, bool pdl)
+{
+    const int nt = M <= 8 ? 1 : 2;
+    PrepArgs a{src, K, M, fb};
+    const size_t smem = (size_t)K * sizeof(uint16_t);
+    void (*kern)(PrepArgs);
+    if (fmt == 4)
+        kern = nt == 1 ? k_prep<4, 1> : k_prep<4, 2>;
+    else
+        kern = nt == 1 ? k_prep<6, 1> : k_prep<6, 2>;
+    if (smem > 48 * 1024) {
+        // once per (device, kernel variant): room for the longest row (K <= 65536)
+        static bool done[64][4] = {};
+        int dev = 0;
+        cudaGetDevice(&dev);
+        const int v = (fmt == 4 ? 0 : 2) + (nt - 1);
+        if (dev < 0 || dev >= 64 || !done[dev][v]) {
+            int rc = set_smem(kern, (size_t)65536 * sizeof(uint16_t));
+            if (rc)
+                return rc;
+            if (dev >= 0 && dev < 64)
+                done[dev][v] = true;
+        }
+    }
+    cudaError_t e = pdl ? launch_pdl(kern, dim3(8 * nt), dim3(512), smem, s, a)
+                        : (kern<<<8 * nt, 512, smem, s>>>(a), cudaGetLastError());
+    return cuda_check(e, "prep launch");
+}
+
+int make_weight_maps(int fmt, const void *W, int N, int K, WeightMapsBlob *out)
+{
+    static_assert(sizeof(WeightMapsBlob) >= sizeof(WeightMaps), "blob too small");
+    WeightMaps *m = reinterpret_cast<WeightMaps *>(out);
+    const int nblk = K / 256;
+    if (fmt == 4)
+        return encode_tmap_2d(&m->w, W, 1, (uint64_t)nblk * 144, (uint64_t)N, (uint64_t)nblk * 144, 144, TILE_ROWS);
+    int rc = encode_tmap_2d(&m->w, W, 1, (uint64_t)nblk * Q6A_BYTES, (uint64_t)N, (uint64_t)nblk * Q6A_BYTES,
+                            Q6A_BYTES, TILE_ROWS);
+    if (rc)
+        return rc;
+    const int nblk8 = (nblk + 7) & ~7;
+    const uint8_t *D = (const uint8_t *)W + (size_t)N * nblk * Q6A_BYTES;
+    return encode_tmap_2d(&m->d, D, 2, (uint64_t)nblk8, (uint64_t)N, (uint64_t)nblk8 * 2, 8, TILE_ROWS);
+}
+
+int launch_gemm(int fmt, const WeightMapsBlob &maps_blob, int N, int K, int M, const FragBuf &fb, float *Y, int ldy,
+                cudaStream_t s, bool pdl)
+{
+    const int nt = M <= 8 ? 1 : 2;
+    const WeightMaps &maps = reinterpret_cast<const WeightMaps &>(maps_blob);
+    GemmArgs a;
+    a.N = N;
+    a.nblk = K / 256;
+    a.M = M;
+    a.ldy = ldy;
+    a.units = ((N + TILE_ROWS - 1) / TILE_ROWS) * a.nblk;
+    a.xp = fb.xp;
+    a.sp = fb.sp;
+    a.rs = fb.rs;
+    a.Y = Y;
+    void (*kern)(const WeightMaps, GemmArgs);
+    size_t smem;
+    if (fmt == 4) {
+        kern = nt == 1 ? k_qgemm<4, 1> : k_qgemm<4, 2>;
+        smem = nt == 1 ? gemm_smem_bytes<4, 1>() : gemm_smem_bytes<4, 2>();
+    } else {
+        kern = nt == 1 ? k_qgemm<6, 1> : k_qgemm<6, 2>;
+        smem = nt == 1 ? gemm_smem_bytes<6, 1>() : gemm_smem_bytes<6, 2>();
+    }
+    static bool done[64][4] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const int v = (fmt == 4 ? 0 : 2) + (nt - 1);
+    if (dev < 0 || dev >= 64 || !done[dev][v]) {
+        int rc = set_smem(kern, smem);
+        if (rc)
+            return rc;
+        if (dev >= 0 && dev < 64)
+            done[dev][v] = true;
+    }
+    const int grid = num_sms();
+    cudaError_t e = pdl ? launch_pdl(kern, dim3(grid), dim3(32 * (GW + 1)), smem, s, maps, a)
+                        : (kern<<<grid, 32 * (GW + 1), smem, s>>>(maps, a), cudaGetLastError());
+    return cuda_check(e, "gemm launch");
+}
+
+int launch_q6k_pack(const void *W, int N, int K, void *P, cudaStream_t s)
+{
+    const long long blocks = (long long)N * (K / 256);
+    long long grid = (blocks + 7) / 8;
+    if (grid > 65535LL * 16)
+        grid = 65535LL * 16;
+    k_q6k_pack<<<(unsigned)grid, 256, 0, s>>>((const uint8_t *)W, N, K / 256, (uint8_t *)P);
+    return cuda_check(cudaGetLastError(), "q6k pack launch");
+}
+
+}  // namespace qad
+
+// ------------------------------------------------------------- C ABI
+
+extern "C" int qad_device_status(int reset)
+{
+    int v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, qad::g_gemm_status, sizeof(int));
+    if (e != cudaSuccess)
+        return qad::cuda_check(e, "qad_device_status");
+    if (reset && v) {
+        const int z = 0;
+        e = cudaMemcpyToSymbol(qad::g_gemm_status, &z, sizeof(int));
+        if (e != cudaSuccess)
+            return qad::cuda_check(e, "qad_device_status reset");
+    }
+    return v;
+}
+
+extern "C" size_t qad_gemm_ws_bytes(int K, int M)
+{
+    if (K <= 0 || K % 256 || M < 1 || M > QAD_MAX_ROWS)
+        return 0;
+    return qad::frag_bytes(K, M <= 8 ? 1 : 2);
+}
+
+extern "C" size_t qad_q6k_packed_bytes(long long N, int K)
+{
+    if (N <= 0 || K <= 0 || K % 256)
+        return 0;
+    return qad::q6k_packed_bytes(N, K);
+}
+
+extern "C" int qad_q6k_pack(const void *W, int N, int K, void *W_packed, void *stream)
+{
+    if (!W || !W_packed || N <= 0 || K <= 0)
+        return qad::fail(QAD_ERR_INVALID, "qad_q6k_pack: null pointer or non-positive size");
+    if (K % 256)
+        return qad::fail(QAD_ERR_UNSUPPORTED, "qad_q6k_pack: K %% 256 != 0");
+    if ((uintptr_t)W_packed & 15)
+        return qad::fail(QAD_ERR_INVALID, "qad_q6k_pack: packed weights must be 16-byte aligned");
+    return qad::launch_q6k_pack(W, N, K, W_packed, (cudaStream_t)stream);
+}
+
+static int gemm_entry(int fmt, const void *W, int N, int K, const uint16_t *X, int M, float *Y, int accumulate,
+                      void *ws, size_t ws_bytes, void *stream)
+{
+    const char *name = fmt == 4 ? "qad_q4k_gemm" : "qad_q6k_gemm";
+    if (!W || !X || !Y || !ws || N <= 0 || K <= 0 || M <= 0)
+        return qad::fail(QAD_ERR_INVALID, "%s: null pointer or non-positive size (N=%d K=%d M=%d)", name, N, K, M);
+    if (M > QAD_MAX_ROWS || K % 256 || K > 65536)
+        return qad::fail(QAD_ERR_UNSUPPORTED, "%s: need 1 <= M <= 16 and K %% 256 == 0, K <= 65536 (M=%d K=%d)",
+                         name, M, K);
+    if ((uintptr_t)ws & 255)
+        return qad::fail(QAD_ERR_INVALID, "%s: workspace must be 256-byte aligned", name);
+    if ((uintptr_t)W & 15)
+        return qad::fail(QAD_ERR_INVALID, "%s: weights must be 16-byte aligned", name);
+    if (ws_bytes < qad_gemm_ws_bytes(K, M))
+        return qad::fail(QAD_ERR_WORKSPACE, "%s: workspace %zu < %zu bytes", name, ws_bytes, qad_gemm_ws_bytes(K, M));
+    qad::WeightMapsBlob maps;
+    int rc = qad::make_weight_maps(fmt, W, N, K, &maps);
+    if (rc)
+        return rc;
+    cudaStream_t s = (cudaStream_t)stream;
+    qad::FragBuf fb = qad::frag_carve(ws, K, M <= 8 ? 1 : 2);
+    qad::PrepSrc src = {};
+    src.kind = qad::PREP_BF16;
+    src.xb = X;
+    src.ldx = K;
+    if (!accumulate) {
+        src.zero = Y;
+        src.zero_n = (long long)M * N;
+    }
+    rc = qad::launch_prep(fmt, K, M, src, fb, s, false);
+    if (rc)
+        return rc;
+    return qad::launch_gemm(fmt, maps, N, K, M, fb, Y, N, s, true);
+}
+
+extern "C" int qad_q4k_gemm(const void *W, int N, int K, const uint16_t *X, int M, float *Y, int accumulate, void *ws,
+                            size_t ws_bytes, void *stream)
+{
+    return gemm_entry(4, W, N, K, X, M, Y, accumulate, ws, ws_bytes, stream);
+}
+
+extern "C" int qad_q6k_gemm(const void *W, int N, int K, const uint16_t *X, int M, float *Y, int accumulate, void *ws,
+                            size_t ws_bytes, void *stream)
+{
+    return gemm_entry(6, W, N, K, X, M, Y, accumulate, ws, ws_bytes, stream);
+}

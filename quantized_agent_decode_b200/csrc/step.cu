@@ -1,0 +1,602 @@
+// step.cu -- one batched decode-and-verify step through the whole synthetic
+// decoder stack, the model handle, CUDA-graph capture and the host-buffer
+// entry point.
+//
+// [OpenJet page] = rebasdaily.com 2026-10-29, "OpenJet ... multi-agent
+// serving", section 只搬一次权重: per step all active agents' rows (next
+// token + two drafts each) form one batch, the weights stream once for the
+// whole batch and each agent reads its own KV cache; the drafts are checked in
+// the same forward pass. The page runs this as one persistent megakernel on an
+// RTX 3090; here the step is a chain of sm_100a kernels linked by
+// programmatic dependent launch (each GEMM starts streaming its weights while
+// its producer drains) and replayed as one CUDA graph.
+//
+// Per layer (rounding points as in the layer definition of qad.h):
+//   prep(rmsnorm h)          -> fp16 fragments; zeroes the qkv buffer
+//   q4k_gemm(Wqkv)           -> qkv fp32 (atomic partial sums)
+//   qkv_post                 -> Q bf16; k, v bf16 appended at each row's position
+//   decode_attn + combine    -> O bf16
+//   prep(O)                  -> fragments
+//   q4k_gemm(Wo)             -> h += ...
+//   prep(rmsnorm h)          -> fragments; zeroes the gate|up buffer
+//   q4k_gemm(Wgu)            -> gate|up fp32
+//   prep(silu(gate) * up)    -> fragments (Q6_K order)
+//   q6k_gemm(Wdown)          -> h += ...
+#include <vector>
+
+#include "attn.cuh"
+#include "gemm.cuh"
+
+struct qad_step_graph {
+    cudaGraph_t graph = nullptr;
+    cudaGraphExec_t exec = nullptr;
+};
+
+// Kernel classes timed by the optional per-launch event profiler.
+enum ProfKind {
+    PK_INIT = 0, PK_PREP, PK_GEMM_QKV, PK_QKV_POST, PK_ATTN, PK_GEMM_O, PK_GEMM_GU, PK_GEMM_DOWN, PK_COUNT
+};
+
+struct qad_model {
+    qad_model_desc d;
+    // per-launch event profiler (eager steps only)
+    bool prof = false;
+    std::vector<cudaEvent_t> prof_ev;
+    std::vector<int> prof_kind;
+    double prof_ms[PK_COUNT] = {};
+    long long prof_n[PK_COUNT] = {};
+    size_t prof_used = 0;
+    bool prof_pending = false;
+    std::vector<const void *> wqkv, wo, wgu, wdown;
+    std::vector<qad::WeightMapsBlob> mqkv, mo, mgu, mdown;  // TMA descriptors, built once
+    std::vector<uint16_t *> kc, vc;
+    void *dbg = nullptr;
+    size_t dbg_bytes = 0;
+    // graph cache of the host-buffer entry point
+    qad_step_graph *hg = nullptr;
+    int hg_M = -1, hg_agents = -1, hg_rows = -1;
+    void *hg_ws = nullptr;
+    cudaStream_t hg_stream = nullptr;
+};
+
+namespace qad {
+
+static inline size_t a256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+struct StepLayout {
+    size_t qkv, qb, ob, gu, frag, part, x_in, ars_in, lens_in, h_out, total;
+    AttnPlan plan;
+};
+
+// Largest attention-partials footprint over the launch shapes a step of M
+// rows can take (n_agents <= max_agents, rows per agent <= M).
+static size_t max_part_bytes(const qad_model_desc &d, int M)
+{
+    size_t best = 0;
+    for (int na = 1; na <= d.max_agents; ++na)
+        for (int rows = 1; rows <= M; ++rows) {
+            size_t b = attn_plan(na, d.n_qh, d.n_kvh, d.kv_cap, rows).part_bytes;
+            if (b > best)
+                best = b;
+        }
+    return best;
+}
+
+static StepLayout step_layout(const qad_model_desc &d, int M)
+{
+    StepLayout L;
+    const int nq = d.n_qh * d.head_dim, nqkv = (d.n_qh + 2 * d.n_kvh) * d.head_dim;
+    const int nt = M <= 8 ? 1 : 2;
+    size_t off = 0;
+    L.qkv = off;
+    off += a256((size_t)M * nqkv * 4);
+    L.qb = off;
+    off += a256((size_t)M * nq * 2);
+    L.ob = off;
+    off += a256((size_t)M * nq * 2);
+    L.gu = off;
+    off += a256((size_t)M * 2 * d.inter * 4);
+    L.frag = off;
+    size_t fb = frag_bytes(d.hidden, nt);
+    if (frag_bytes(nq, nt) > fb)
+        fb = frag_bytes(nq, nt);
+    if (frag_bytes(d.inter, nt) > fb)
+        fb = frag_bytes(d.inter, nt);
+    off += a256(fb);
+    L.part = off;
+    off += a256(max_part_bytes(d, M));
+    L.x_in = off;
+    off += a256((size_t)M * d.hidden * 2);
+    L.ars_in = off;
+    off += a256((size_t)(d.max_agents + 1) * 4);
+    L.lens_in = off;
+    off += a256((size_t)d.max_agents * 4);
+    L.h_out = off;
+    off += a256((size_t)M * d.hidden * 4);
+    L.total = off;
+    return L;
+}
+
+// Debug intermediates of one layer (teacher-forced parity checks).
+struct DbgLayout {
+    size_t x1, qkv, attn, hmid, x2, gu, act, hout, per_layer;
+};
+static DbgLayout dbg_layout(const qad_model_desc &d, int M)
+{
+    DbgLayout L;
+    const int nq = d.n_qh * d.head_dim, nqkv = (d.n_qh + 2 * d.n_kvh) * d.head_dim;
+    size_t off = 0;
+    L.x1 = off;
+    off += a256((size_t)M * d.hidden * 2);
+    L.qkv = off;
+    off += a256((size_t)M * nqkv * 4);
+    L.attn = off;
+    off += a256((size_t)M * nq * 2);
+    L.hmid = off;
+    off += a256((size_t)M * d.hidden * 4);
+    L.x2 = off;
+    off += a256((size_t)M * d.hidden * 2);
+    L.gu = off;
+    off += a256((size_t)M * 2 * d.inter * 4);
+    L.act = off;
+    off += a256((size_t)M * d.inter * 2);
+    L.hout = off;
+    off += a256((size_t)M * d.hidden * 4);
+    L.per_layer = off;
+    return L;
+}
+
+// h[r][k] = X[r][k] (bf16 -> fp32): the residual stream starts at the input rows.
+__global__ void k_init_h(const uint16_t *__restrict__ X, float *__restrict__ h, int n)
+{
+    pdl_trigger();
+    pdl_wait();
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x)
+        h[i] = bf16_to_f(X[i]);
+}
+
+// Split the fused q|k|v projection of row r: Q as bf16 for attention, and the
+// row's k and v as bf16 appended to its agent's cache at position len + j.
+__global__ void k_qkv_post(const float *__restrict__ qkv, uint16_t *__restrict__ Qb, uint16_t *__restrict__ Kc,
+                           uint16_t *__restrict__ Vc, const int *__restrict__ ars, const int *__restrict__ lens,
+                           int n_agents, int nq, int nkv, int n_kvh, int hd, int kv_cap)
+{
+    const int r = blockIdx.x;
+    pdl_trigger();
+    pdl_wait();
+    int a = 0;
+    while (a < n_agents && !(ars[a] <= r && r < ars[a + 1]))
+        ++a;
+    if (a == n_agents)
+        return;
+    const int pos = lens[a] + (r - ars[a]);
+    const float *src = qkv + (size_t)r * (nq + 2 * nkv);
+    for (int i = threadIdx.x; i < nq; i += blockDim.x)
+        Qb[(size_t)r * nq + i] = f_to_bf16(src[i]);
+    if (pos < 0 || pos >= kv_cap)
+        return;
+    for (int i = threadIdx.x; i < nkv; i += blockDim.x) {
+        const int g = i / hd, dd = i - g * hd;
+        const size_t dst = (((size_t)a * n_kvh + g) * kv_cap + pos) * hd + dd;
+        Kc[dst] = f_to_bf16(src[nq + i]);
+        Vc[dst] = f_to_bf16(src[nq + nkv + i]);
+    }
+}
+
+// Profiler: events around each launch (serialises the chain; eager steps only).
+struct Prof {
+    qad_model *m;
+    cudaStream_t s;
+    size_t next = 0;
+    int begin(int kind)
+    {
+        if (!m->prof)
+            return QAD_OK;
+        if (next + 2 > m->prof_ev.size()) {
+            for (int i = 0; i < 64; ++i) {
+                cudaEvent_t e;
+                int rc = cuda_check(cudaEventCreate(&e), "profiler event");
+                if (rc)
+                    return rc;
+                m->prof_ev.push_back(e);
+            }
+        }
+        if (m->prof_kind.size() < m->prof_ev.size() / 2)
+            m->prof_kind.resize(m->prof_ev.size() / 2);
+        m->prof_kind[next / 2] = kind;
+        return cuda_check(cudaEventRecord(m->prof_ev[next++], s), "profiler record");
+    }
+    int end()
+    {
+        if (!m->prof)
+            return QAD_OK;
+        return cuda_check(cudaEventRecord(m->prof_ev[next++], s), "profiler record");
+    }
+};
+
+static int copy_d2d(void *dst, const void *src, size_t n, cudaStream_t s)
+{
+    return cuda_check(cudaMemcpyAsync(dst, src, n, cudaMemcpyDeviceToDevice, s), "debug copy");
+}
+
+static int run_step(qad_model *m, const uint16_t *X, int M, const int *ars, int n_agents, int max_rows,
+                    const int *lens, float *h, char *ws, cudaStream_t s)
+{
+    const qad_model_desc &d = m->d;
+    const int H = d.hidden, I = d.inter, hd = d.head_dim;
+    const int nq = d.n_qh * hd, nkv = d.n_kvh * hd, nqkv = nq + 2 * nkv;
+    const StepLayout L = step_layout(d, M);
+    const int nt = M <= 8 ? 1 : 2;
+    float *qkv = (float *)(ws + L.qkv), *gu = (float *)(ws + L.gu);
+    uint16_t *Qb = (uint16_t *)(ws + L.qb), *Ob = (uint16_t *)(ws + L.ob);
+    float *part = (float *)(ws + L.part);
+    const AttnPlan plan = attn_plan(n_agents, d.n_qh, d.n_kvh, d.kv_cap, max_rows);
+    const float scale = 1.0f / sqrtf((float)hd);
+    const DbgLayout DL = dbg_layout(d, M);
+    int rc;
+
+    Prof P{m, s};
+    if (m->prof && !m->prof_ev.empty() && m->prof_pending) {
+        m->prof_pending = false;  // a previous profiled step was never read: drop it
+    }
+#define QAD_PROF(kind, launch_expr)                     \
+    do {                                                \
+        if ((rc = P.begin(kind)))                       \
+            return rc;                                  \
+        if ((rc = (launch_expr)))                       \
+            return rc;                                  \
+        if ((rc = P.end()))                             \
+            return rc;                                  \
+    } while (0)
+    QAD_PROF(PK_INIT, (k_init_h<<<(M * H + 255) / 256, 256, 0, s>>>(X, h, M * H),
+                       cuda_check(cudaGetLastError(), "init launch")));
+    for (int l = 0; l < d.n_layers; ++l) {
+        char *dbg = m->dbg ? (char *)m->dbg + (size_t)l * DL.per_layer : nullptr;
+        PrepSrc src = {};
+        // x1 = bf16(rmsnorm(h)) -> qkv
+        FragBuf fb = frag_carve(ws + L.frag, H, nt);
+        src.kind = PREP_RMSNORM;
+        src.xf = h;
+        src.ldx = H;
+        src.eps = d.rms_eps;
+        src.zero = qkv;
+        src.zero_n = (long long)M * nqkv;
+        src.dbg = dbg ? (uint16_t *)(dbg + DL.x1) : nullptr;
+        src.ld_dbg = H;
+        QAD_PROF(PK_PREP, launch_prep(4, H, M, src, fb, s, true));
+        QAD_PROF(PK_GEMM_QKV, launch_gemm(4, m->mqkv[l], nqkv, H, M, fb, qkv, nqkv, s, true));
+        if (dbg && (rc = copy_d2d(dbg + DL.qkv, qkv, (size_t)M * nqkv * 4, s)))
+            return rc;
+        // Q, and k/v appended to the caches
+        QAD_PROF(PK_QKV_POST, cuda_check(launch_pdl(k_qkv_post, dim3(M), dim3(256), 0, s, (const float *)qkv, Qb,
+                                                     m->kc[l], m->vc[l], ars, lens, n_agents, nq, nkv, d.n_kvh, hd,
+                                                     d.kv_cap),
+                                          "qkv_post launch"));
+        // attention over each agent's cache
+        QAD_PROF(PK_ATTN, launch_attn(plan, Qb, m->kc[l], m->vc[l], lens, ars, n_agents, d.kv_cap, d.n_qh, d.n_kvh,
+                                      scale, Ob, part, s, true));
+        if (dbg && (rc = copy_d2d(dbg + DL.attn, Ob, (size_t)M * nq * 2, s)))
+            return rc;
+        // h += O Wo^T
+        fb = frag_carve(ws + L.frag, nq, nt);
+        src = PrepSrc{};
+        src.kind = PREP_BF16;
+        src.xb = Ob;
+        src.ldx = nq;
+        QAD_PROF(PK_PREP, launch_prep(4, nq, M, src, fb, s, true));
+        QAD_PROF(PK_GEMM_O, launch_gemm(4, m->mo[l], H, nq, M, fb, h, H, s, true));
+        if (dbg && (rc = copy_d2d(dbg + DL.hmid, h, (size_t)M * H * 4, s)))
+            return rc;
+        // x2 = bf16(rmsnorm(h)) -> gate | up
+        fb = frag_carve(ws + L.frag, H, nt);
+        src = PrepSrc{};
+        src.kind = PREP_RMSNORM;
+        src.xf = h;
+        src.ldx = H;
+        src.eps = d.rms_eps;
+        src.zero = gu;
+        src.zero_n = (long long)M * 2 * I;
+        src.dbg = dbg ? (uint16_t *)(dbg + DL.x2) : nullptr;
+        src.ld_dbg = H;
+        QAD_PROF(PK_PREP, launch_prep(4, H, M, src, fb, s, true));
+        QAD_PROF(PK_GEMM_GU, launch_gemm(4, m->mgu[l], 2 * I, H, M, fb, gu, 2 * I, s, true));
+        if (dbg && (rc = copy_d2d(dbg + DL.gu, gu, (size_t)M * 2 * I * 4, s)))
+            return rc;
+        // h += bf16(silu(gate) * up) Wdown^T
+        fb = frag_carve(ws + L.frag, I, nt);
+        src = PrepSrc{};
+        src.kind = PREP_SILU;
+        src.xf = gu;
+        src.ldx = 2 * I;
+        src.dbg = dbg ? (uint16_t *)(dbg + DL.act) : nullptr;
+        src.ld_dbg = I;
+        QAD_PROF(PK_PREP, launch_prep(6, I, M, src, fb, s, true));
+        QAD_PROF(PK_GEMM_DOWN, launch_gemm(6, m->mdown[l], H, I, M, fb, h, H, s, true));
+        if (dbg && (rc = copy_d2d(dbg + DL.hout, h, (size_t)M * H * 4, s)))
+            return rc;
+    }
+#undef QAD_PROF
+    if (m->prof) {
+        m->prof_used = P.next;
+        m->prof_pending = true;
+    }
+    return QAD_OK;
+}
+
+static int check_step_args(const qad_model *m, const void *X, int M, const void *ars, int n_agents, int max_rows,
+                           const void *lens, const void *H_out, const void *ws, size_t ws_bytes)
+{
+    if (!m || !X || !ars || !lens || !H_out || !ws || M <= 0 || n_agents <= 0 || max_rows <= 0)
+        return fail(QAD_ERR_INVALID, "decode_step: null pointer or non-positive size");
+    if (M > QAD_MAX_ROWS || n_agents > m->d.max_agents || max_rows > M)
+        return fail(QAD_ERR_UNSUPPORTED, "decode_step: need M <= 16, n_agents <= %d, max_rows_per_agent <= M",
+                    m->d.max_agents);
+    if (max_rows * (m->d.n_qh / m->d.n_kvh) > 96)
+        return fail(QAD_ERR_UNSUPPORTED, "decode_step: rows per agent x group exceeds 96");
+    if ((uintptr_t)ws & 255)
+        return fail(QAD_ERR_INVALID, "decode_step: workspace must be 256-byte aligned");
+    if (ws_bytes < step_layout(m->d, M).total)
+        return fail(QAD_ERR_WORKSPACE, "decode_step: workspace %zu < %zu bytes", ws_bytes, step_layout(m->d, M).total);
+    return QAD_OK;
+}
+
+}  // namespace qad
+
+extern "C" int qad_model_create(const qad_model_desc *desc, qad_model **out)
+{
+    if (!desc || !out)
+        return qad::fail(QAD_ERR_INVALID, "qad_model_create: null argument");
+    const qad_model_desc &d = *desc;
+    if (d.n_layers <= 0 || d.hidden <= 0 || d.inter <= 0 || d.n_qh <= 0 || d.n_kvh <= 0 || d.max_agents <= 0 ||
+        d.kv_cap <= 0 || !(d.rms_eps >= 0.f) || !d.w_qkv || !d.w_o || !d.w_gu || !d.w_down || !d.k_cache ||
+        !d.v_cache)
+        return qad::fail(QAD_ERR_INVALID, "qad_model_create: invalid descriptor");
+    if (d.head_dim != 128 || d.n_qh % d.n_kvh || d.hidden % 256 || d.inter % 256 || (d.n_qh * d.head_dim) % 256 ||
+        d.hidden > 65536 || d.inter > 65536)
+        return qad::fail(QAD_ERR_UNSUPPORTED,
+                         "qad_model_create: need head_dim 128, n_qh %% n_kvh == 0, hidden/inter/n_qh*hd multiples "
+                         "of 256 and <= 65536");
+    qad_model *m = new qad_model();
+    m->d = d;
+    for (int l = 0; l < d.n_layers; ++l) {
+        if (!d.w_qkv[l] || !d.w_o[l] || !d.w_gu[l] || !d.w_down[l] || !d.k_cache[l] || !d.v_cache[l] ||
+            (((uintptr_t)d.w_qkv[l] | (uintptr_t)d.w_o[l] | (uintptr_t)d.w_gu[l] | (uintptr_t)d.w_down[l] |
+              (uintptr_t)d.k_cache[l] | (uintptr_t)d.v_cache[l]) & 15)) {
+            delete m;
+            return qad::fail(QAD_ERR_INVALID, "qad_model_create: null or misaligned pointer in layer %d", l);
+        }
+        qad::WeightMapsBlob mb[4];
+        const int nqkv = (d.n_qh + 2 * d.n_kvh) * d.head_dim, nq = d.n_qh * d.head_dim;
+        int rc = qad::make_weight_maps(4, d.w_qkv[l], nqkv, d.hidden, &mb[0]);
+        if (!rc)
+            rc = qad::make_weight_maps(4, d.w_o[l], d.hidden, nq, &mb[1]);
+        if (!rc)
+            rc = qad::make_weight_maps(4, d.w_gu[l], 2 * d.inter, d.hidden, &mb[2]);
+        if (!rc)
+            rc = qad::make_weight_maps(6, d.w_down[l], d.hidden, d.inter, &mb[3]);
+        if (rc) {
+            delete m;
+            return rc;
+        }
+        m->mqkv.push_back(mb[0]);
+        m->mo.push_back(mb[1]);
+        m->mgu.push_back(mb[2]);
+        m->mdown.push_back(mb[3]);
+        m->wqkv.push_back(d.w_qkv[l]);
+        m->wo.push_back(d.w_o[l]);
+        m->wgu.push_back(d.w_gu[l]);
+        m->wdown.push_back(d.w_down[l]);
+        m->kc.push_back(d.k_cache[l]);
+        m->vc.push_back(d.v_cache[l]);
+    }
+    m->d.w_qkv = m->wqkv.data();
+    m->d.w_o = m->wo.data();
+    m->d.w_gu = m->wgu.data();
+    m->d.w_down = m->wdown.data();
+    m->d.k_cache = m->kc.data();
+    m->d.v_cache = m->vc.data();
+    *out = m;
+    return QAD_OK;
+}
+
+extern "C" void qad_model_destroy(qad_model *m)
+{
+    if (!m)
+        return;
+    qad_step_graph_destroy(m->hg);
+    for (cudaEvent_t e : m->prof_ev)
+        cudaEventDestroy(e);
+    delete m;
+}
+
+extern "C" size_t qad_decode_step_ws_bytes(const qad_model *m, int M)
+{
+    if (!m || M <= 0 || M > QAD_MAX_ROWS)
+        return 0;
+    return qad::step_layout(m->d, M).total;
+}
+
+extern "C" size_t qad_decode_step_debug_bytes(const qad_model *m, int M)
+{
+    if (!m || M <= 0 || M > QAD_MAX_ROWS)
+        return 0;
+    return qad::dbg_layout(m->d, M).per_layer * m->d.n_layers;
+}
+
+extern "C" int qad_model_set_debug(qad_model *m, void *dbg, size_t bytes)
+{
+    if (!m)
+        return qad::fail(QAD_ERR_INVALID, "qad_model_set_debug: null model");
+    m->dbg = dbg;
+    m->dbg_bytes = bytes;
+    return QAD_OK;
+}
+
+extern "C" int qad_decode_step(qad_model *m, const uint16_t *X, int M, const int *agent_row_start, int n_agents,
+                               int max_rows_per_agent, const int *lens, float *H_out, void *ws, size_t ws_bytes,
+                               void *stream)
+{
+    int rc = qad::check_step_args(m, X, M, agent_row_start, n_agents, max_rows_per_agent, lens, H_out, ws, ws_bytes);
+    if (rc)
+        return rc;
+    if (m->dbg && m->dbg_bytes < qad_decode_step_debug_bytes(m, M))
+        return qad::fail(QAD_ERR_WORKSPACE, "decode_step: debug buffer too small");
+    return qad::run_step(m, X, M, agent_row_start, n_agents, max_rows_per_agent, lens, H_out, (char *)ws,
+                         (cudaStream_t)stream);
+}
+
+extern "C" int qad_decode_step_launches(const qad_model *m)
+{
+    if (!m)
+        return 0;
+    return 1 + 11 * m->d.n_layers;
+}
+
+extern "C" int qad_step_graph_create(qad_model *m, const uint16_t *X, int M, const int *agent_row_start, int n_agents,
+                                     int max_rows_per_agent, const int *lens, float *H_out, void *ws, size_t ws_bytes,
+                                     void *stream, qad_step_graph **out)
+{
+    if (!out)
+        return qad::fail(QAD_ERR_INVALID, "qad_step_graph_create: null output");
+    int rc = qad::check_step_args(m, X, M, agent_row_start, n_agents, max_rows_per_agent, lens, H_out, ws, ws_bytes);
+    if (rc)
+        return rc;
+    if (m->dbg || m->prof)
+        return qad::fail(QAD_ERR_UNSUPPORTED,
+                         "qad_step_graph_create: a model with a debug buffer or the profiler on is not captured");
+    cudaStream_t s = (cudaStream_t)stream;
+    if (!s)
+        return qad::fail(QAD_ERR_INVALID, "qad_step_graph_create: needs a non-default stream");
+    if ((rc = qad::cuda_check(cudaStreamBeginCapture(s, cudaStreamCaptureModeThreadLocal), "begin capture")))
+        return rc;
+    rc = qad::run_step(m, X, M, agent_row_start, n_agents, max_rows_per_agent, lens, H_out, (char *)ws, s);
+    cudaGraph_t graph = nullptr;
+    cudaError_t e = cudaStreamEndCapture(s, &graph);
+    if (rc) {
+        if (graph)
+            cudaGraphDestroy(graph);
+        return rc;
+    }
+    if ((rc = qad::cuda_check(e, "end capture")))
+        return rc;
+    qad_step_graph *g = new qad_step_graph();
+    g->graph = graph;
+    if ((rc = qad::cuda_check(cudaGraphInstantiate(&g->exec, graph, 0), "graph instantiate"))) {
+        cudaGraphDestroy(graph);
+        delete g;
+        return rc;
+    }
+    *out = g;
+    return QAD_OK;
+}
+
+extern "C" int qad_step_graph_launch(qad_step_graph *g, void *stream)
+{
+    if (!g || !g->exec)
+        return qad::fail(QAD_ERR_INVALID, "qad_step_graph_launch: null graph");
+    return qad::cuda_check(cudaGraphLaunch(g->exec, (cudaStream_t)stream), "graph launch");
+}
+
+extern "C" void qad_step_graph_destroy(qad_step_graph *g)
+{
+    if (!g)
+        return;
+    if (g->exec)
+        cudaGraphExecDestroy(g->exec);
+    if (g->graph)
+        cudaGraphDestroy(g->graph);
+    delete g;
+}
+
+extern "C" int qad_decode_step_host(qad_model *m, const uint16_t *X_host, int M, const int *agent_row_start_host,
+                                    int n_agents, int max_rows_per_agent, const int *lens_host, float *H_out_host,
+                                    void *ws, size_t ws_bytes, void *stream)
+{
+    if (!X_host || !agent_row_start_host || !lens_host || !H_out_host)
+        return qad::fail(QAD_ERR_INVALID, "qad_decode_step_host: null host pointer");
+    int rc = qad::check_step_args(m, X_host, M, agent_row_start_host, n_agents, max_rows_per_agent, lens_host,
+                                  H_out_host, ws, ws_bytes);
+    if (rc)
+        return rc;
+    for (int a = 0; a < n_agents; ++a)
+        if (agent_row_start_host[a] > agent_row_start_host[a + 1] || lens_host[a] < 0 ||
+            lens_host[a] + (agent_row_start_host[a + 1] - agent_row_start_host[a]) > m->d.kv_cap)
+            return qad::fail(QAD_ERR_INVALID, "qad_decode_step_host: agent %d rows/len out of range", a);
+    if (agent_row_start_host[0] != 0 || agent_row_start_host[n_agents] != M)
+        return qad::fail(QAD_ERR_INVALID, "qad_decode_step_host: agent_row_start must span 0..M");
+    cudaStream_t s = (cudaStream_t)stream;
+    const qad::StepLayout L = qad::step_layout(m->d, M);
+    char *w = (char *)ws;
+    uint16_t *X = (uint16_t *)(w + L.x_in);
+    int *ars = (int *)(w + L.ars_in), *lens = (int *)(w + L.lens_in);
+    float *H = (float *)(w + L.h_out);
+    if ((rc = qad::cuda_check(cudaMemcpyAsync(X, X_host, (size_t)M * m->d.hidden * 2, cudaMemcpyHostToDevice, s),
+                              "H2D X")) ||
+        (rc = qad::cuda_check(cudaMemcpyAsync(ars, agent_row_start_host, (size_t)(n_agents + 1) * 4,
+                                              cudaMemcpyHostToDevice, s),
+                              "H2D agent_row_start")) ||
+        (rc = qad::cuda_check(cudaMemcpyAsync(lens, lens_host, (size_t)n_agents * 4, cudaMemcpyHostToDevice, s),
+                              "H2D lens")))
+        return rc;
+    if (s && !m->dbg && !m->prof) {
+        if (!m->hg || m->hg_M != M || m->hg_agents != n_agents || m->hg_rows != max_rows_per_agent || m->hg_ws != ws ||
+            m->hg_stream != s) {
+            qad_step_graph_destroy(m->hg);
+            m->hg = nullptr;
+            if ((rc = qad_step_graph_create(m, X, M, ars, n_agents, max_rows_per_agent, lens, H, ws, ws_bytes, stream,
+                                            &m->hg)))
+                return rc;
+            m->hg_M = M;
+            m->hg_agents = n_agents;
+            m->hg_rows = max_rows_per_agent;
+            m->hg_ws = ws;
+            m->hg_stream = s;
+        }
+        if ((rc = qad_step_graph_launch(m->hg, stream)))
+            return rc;
+    } else if ((rc = qad::run_step(m, X, M, ars, n_agents, max_rows_per_agent, lens, H, w, s))) {
+        return rc;
+    }
+    if ((rc = qad::cuda_check(cudaMemcpyAsync(H_out_host, H, (size_t)M * m->d.hidden * 4, cudaMemcpyDeviceToHost, s),
+                              "D2H H")))
+        return rc;
+    return qad::cuda_check(cudaStreamSynchronize(s), "step sync");
+}
+
+extern "C" int qad_model_set_profile(qad_model *m, int enable)
+{
+    if (!m)
+        return qad::fail(QAD_ERR_INVALID, "qad_model_set_profile: null model");
+    m->prof = enable != 0;
+    for (int k = 0; k < PK_COUNT; ++k) {
+        m->prof_ms[k] = 0;
+        m->prof_n[k] = 0;
+    }
+    m->prof_pending = false;
+    return QAD_OK;
+}
+
+extern "C" int qad_model_profile_read(qad_model *m, double *ms, long long *count, int n_kinds)
+{
+    if (!m || !ms || !count || n_kinds < PK_COUNT)
+        return qad::fail(QAD_ERR_INVALID, "qad_model_profile_read: invalid arguments");
+    if (m->prof_pending) {
+        int rc = qad::cuda_check(cudaEventSynchronize(m->prof_ev[m->prof_used - 1]), "profiler sync");
+        if (rc)
+            return rc;
+        for (size_t i = 0; i + 1 < m->prof_used; i += 2) {
+            float t = 0.f;
+            rc = qad::cuda_check(cudaEventElapsedTime(&t, m->prof_ev[i], m->prof_ev[i + 1]), "profiler elapsed");
+            if (rc)
+                return rc;
+            m->prof_ms[m->prof_kind[i / 2]] += t;
+            m->prof_n[m->prof_kind[i / 2]] += 1;
+        }
+        m->prof_pending = false;
+    }
+    for (int k = 0; k < PK_COUNT; ++k) {
+        ms[k] = m->prof_ms[k];
+        count[k] = m->prof_n[k];
+    }
+    return PK_COUNT;
+}

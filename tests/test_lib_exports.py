@@ -1,0 +1,95 @@
+"""The C-ABI library builds for sm_100a, loads without a GPU and exports every
+symbol include/qad.h declares; host-only entry points run here (CPU only)."""
+import ctypes as C
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from conftest import ROOT, SEED, golden
+
+
+@pytest.fixture(scope="module")
+def qlib():
+    from quantized_agent_decode_b200 import build
+    build.build()
+    import quantized_agent_decode_b200 as q
+    return q
+
+
+def _declared_functions():
+    names = set()
+    inc = os.path.join(ROOT, "include")
+    for fn in os.listdir(inc):
+        if not fn.endswith(".h"):
+            continue
+        text = open(os.path.join(inc, fn)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"\b(qad_[a-z0-9_]+)\s*\(", text):
+            names.add(m.group(1))
+    return names
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for need in ("qad_q4k_gemm", "qad_q6k_gemm", "qad_decode_attn", "qad_decode_step", "qad_pack_rows",
+                 "qad_q4k_unpack", "qad_model_create", "qad_decode_step_host"):
+        assert need in names
+
+
+def test_every_declared_symbol_is_exported(qlib):
+    L = C.CDLL(qlib.LIB_PATH)
+    missing = [n for n in _declared_functions() if not hasattr(L, n)]
+    assert not missing, missing
+    # and the binding declares a signature for each of them
+    assert not (_declared_functions() - set(qlib.SIGNATURES)), _declared_functions() - set(qlib.SIGNATURES)
+
+
+def test_build_targets_sm100a_only():
+    from quantized_agent_decode_b200 import build
+    assert build.ARCH == ["-gencode", "arch=compute_100a,code=sm_100a"]
+
+
+def test_version_and_error_text(qlib):
+    L = qlib.lib()
+    assert L.qad_version() >= 100
+    # a host-side argument check fails without touching the GPU
+    rc = L.qad_q4k_gemm(None, 1, 256, None, 1, None, 0, None, 0, None)
+    assert rc == -1 and b"qad_q4k_gemm" in L.qad_last_error()
+    assert L.qad_gemm_ws_bytes(255, 1) == 0 and L.qad_gemm_ws_bytes(256, 17) == 0
+    assert L.qad_gemm_ws_bytes(5120, 12) > 0
+
+
+def test_pack_rows_matches_oracle(qlib, orc):
+    gd = golden("pack_rows.json")
+    H = 64
+    rows_np = [synth.bf16_normal_np(SEED, 60 + a, (n, H)) for a, n in enumerate(gd["n_rows"])]
+    rows_t = [torch.from_numpy(r.view(np.int16)).view(torch.bfloat16) for r in rows_np]
+    X, ra, rp, ars = qlib.pack_rows(rows_t, gd["lens"], H)
+    oX, ora, orp, oars = orc.pack_rows(rows_np, gd["lens"], H)
+    assert np.array_equal(X.view(torch.int16).numpy().view(np.uint16), oX)
+    assert ra.tolist() == ora.tolist() == gd["row_agent"]
+    assert rp.tolist() == orp.tolist() == gd["row_pos"]
+    assert ars.tolist() == oars.tolist() == gd["agent_row_start"]
+
+
+def test_pack_rows_rejects_overflow_and_negative(qlib):
+    H = 8
+    rows = [torch.zeros(9, H, dtype=torch.bfloat16), torch.zeros(9, H, dtype=torch.bfloat16)]
+    with pytest.raises(qlib.QadError):
+        qlib.pack_rows(rows, [0, 0], H, max_rows=16)
+    with pytest.raises(qlib.QadError):
+        qlib.pack_rows([torch.zeros(1, H, dtype=torch.bfloat16)], [-1], H)
+    X, ra, rp, ars = qlib.pack_rows([torch.zeros(0, H, dtype=torch.bfloat16)] * 3, [1, 2, 3], H)
+    assert X.shape[0] == 0 and ars.tolist() == [0, 0, 0, 0]
+
+
+def test_compute_calls_fail_loudly_without_gpu(qlib):
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    with pytest.raises(qlib.QadError):
+        qlib.q4k_gemm(torch.zeros(1, 144, dtype=torch.uint8), 1, 256, torch.zeros(1, 256, dtype=torch.bfloat16),
+                      1, torch.zeros(1, 1))
