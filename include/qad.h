@@ -107,6 +107,28 @@ size_t qad_gemm_ws_bytes(int K, int M);
 size_t qad_q6k_packed_bytes(long long N, int K);
 int qad_q6k_pack(const void *W, int N, int K, void *W_packed, void *stream);
 
+/* qad_q4k_gemm for callers that cannot allocate device memory at call time
+ * (the pages have no counterpart: this is a library-integration entry point).
+ * Such callers include servers that reserve all of HBM for weights and
+ * KV-cache pools at start-up and forbid later allocations, code that must not
+ * trigger the device-wide synchronisation cudaFree can cause while other
+ * streams are decoding, and plain C integrations that only hold pointers to
+ * buffers owned elsewhere. Arguments and result are those of qad_q4k_gemm
+ * without the workspace: the scratch is a fixed array of
+ * qad_q4k_gemm_noalloc_scratch_bytes() bytes (1 MiB; enough for K <= 30720 at
+ * 16 rows) in device memory that every GPU loading this library holds until
+ * the process exits. Calls that need more scratch fail with
+ * QAD_ERR_UNSUPPORTED before any launch. The first call on each device looks
+ * up the array's device address (cudaGetSymbolAddress); make that first call
+ * before any stream capture. All calls on a device share the one array, and
+ * each call rewrites the parts it reads, so calls that overlap on the GPU
+ * (different streams, or different host threads without ordering) race and
+ * must be serialised by the caller. Nothing here calls cudaMalloc, cudaFree
+ * or any allocating routine. */
+size_t qad_q4k_gemm_noalloc_scratch_bytes(void);
+int qad_q4k_gemm_noalloc(const void *W, int N, int K, const uint16_t *X, int M, float *Y, int accumulate,
+                         void *stream);
+
 /* Device status word of the GEMM pipelines on the current device: 0 if every
  * shared-memory pipeline wait completed; non-zero if a wait gave up after its
  * bounded number of polls (the kernel then returned early and its outputs are

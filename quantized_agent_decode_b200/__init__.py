@@ -47,6 +47,9 @@ SIGNATURES = {
     "qad_device_status": (C.c_int, [C.c_int]),
     "qad_q6k_packed_bytes": (C.c_size_t, [C.c_longlong, C.c_int]),
     "qad_q6k_pack": (C.c_int, [C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_void_p]),
+    "qad_q4k_gemm_noalloc_scratch_bytes": (C.c_size_t, []),
+    "qad_q4k_gemm_noalloc": (C.c_int, [C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_int, C.c_void_p, C.c_int,
+                                       C.c_void_p]),
     "qad_q4k_gemm": (C.c_int, [C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_int, C.c_void_p, C.c_int,
                                C.c_void_p, C.c_size_t, C.c_void_p]),
     "qad_q6k_gemm": (C.c_int, [C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_int, C.c_void_p, C.c_int,
@@ -177,6 +180,15 @@ def q4k_gemm(W, N, K, X, M, Y, accumulate=False, ws=None, stream=None):
 def q6k_gemm(W, N, K, X, M, Y, accumulate=False, ws=None, stream=None):
     """Y[M,N] (fp32) = X[M,K] (bf16) @ W^T with W a Q6_K-like matrix in the packed layout (q6k_pack)."""
     return _gemm("qad_q6k_gemm", W, N, K, X, M, Y, accumulate, ws, stream)
+
+
+def q4k_gemm_noalloc(W, N, K, X, M, Y, accumulate=False, stream=None):
+    """q4k_gemm without a workspace: the scratch is the library's fixed device
+    array (see qad_q4k_gemm_noalloc in include/qad.h); overlapping calls race."""
+    _require_gpu()
+    _check(lib().qad_q4k_gemm_noalloc(_dev(W, "W"), N, K, _dev(X, "X"), M, _dev(Y, "Y"), int(bool(accumulate)),
+                                      _stream(stream)), "qad_q4k_gemm_noalloc")
+    return Y
 
 
 def q6k_packed_bytes(N: int, K: int) -> int:

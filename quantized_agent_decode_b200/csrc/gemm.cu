@@ -34,6 +34,8 @@
 //    producer of the activations is still finishing.
 #include <cuda.h>
 
+#include <mutex>
+
 #include "gemm.cuh"
 
 namespace qad {
@@ -814,4 +816,70 @@ extern "C" int qad_q6k_gemm(const void *W, int N, int K, const uint16_t *X, int 
                             size_t ws_bytes, void *stream)
 {
     return gemm_entry(6, W, N, K, X, M, Y, accumulate, ws, ws_bytes, stream);
+}
+
+// ------------------------------------------------------------- allocation-free variant
+//
+// Some callers cannot allocate device memory when they run this GEMM: servers
+// that reserve all of HBM for weights and KV-cache pools at start-up and
+// forbid later allocations, code that must not trigger the device-wide
+// synchronisation cudaFree can cause while other streams are decoding, and
+// plain C integrations that only hold pointers to buffers owned elsewhere.
+// For them the activation-fragment scratch lives in a fixed array of device
+// memory that every GPU loading this library keeps until the process exits.
+
+static constexpr size_t NOALLOC_SCRATCH_BYTES = (size_t)1 << 20;  // 1 MiB: K <= 30720 at 16 rows
+static __device__ __align__(256) unsigned char g_noalloc_scratch[NOALLOC_SCRATCH_BYTES];
+
+// The array's host-side name is not a device address: resolve it once per
+// device (with that device current) and reuse the address.
+static void *noalloc_scratch_address(int *rc)
+{
+    static void *addr[64] = {};
+    static std::mutex mu;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) {
+        *rc = qad::cuda_check(e, "qad_q4k_gemm_noalloc: cudaGetDevice");
+        return nullptr;
+    }
+    if (dev < 0 || dev >= 64) {
+        *rc = qad::fail(QAD_ERR_UNSUPPORTED, "qad_q4k_gemm_noalloc: device ordinal %d >= 64", dev);
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) {
+            *rc = qad::cuda_check(e, "qad_q4k_gemm_noalloc: cudaGetSymbolAddress");
+            return nullptr;
+        }
+        addr[dev] = p;
+    }
+    *rc = QAD_OK;
+    return addr[dev];
+}
+
+extern "C" size_t qad_q4k_gemm_noalloc_scratch_bytes(void) { return NOALLOC_SCRATCH_BYTES; }
+
+extern "C" int qad_q4k_gemm_noalloc(const void *W, int N, int K, const uint16_t *X, int M, float *Y, int accumulate,
+                                    void *stream)
+{
+    if (!W || !X || !Y || N <= 0 || K <= 0 || M <= 0)
+        return qad::fail(QAD_ERR_INVALID, "qad_q4k_gemm_noalloc: null pointer or non-positive size (N=%d K=%d M=%d)",
+                         N, K, M);
+    if (M > QAD_MAX_ROWS || K % 256)
+        return qad::fail(QAD_ERR_UNSUPPORTED, "qad_q4k_gemm_noalloc: need 1 <= M <= 16 and K %% 256 == 0");
+    const size_t need = qad_gemm_ws_bytes(K, M);
+    if (need > NOALLOC_SCRATCH_BYTES)
+        return qad::fail(QAD_ERR_UNSUPPORTED,
+                         "qad_q4k_gemm_noalloc: K=%d with M=%d needs %zu bytes of scratch; the fixed array holds %zu "
+                         "(use qad_q4k_gemm with a workspace)",
+                         K, M, need, NOALLOC_SCRATCH_BYTES);
+    int rc = QAD_OK;
+    void *scratch = noalloc_scratch_address(&rc);
+    if (!scratch)
+        return rc;
+    return gemm_entry(4, W, N, K, X, M, Y, accumulate, scratch, NOALLOC_SCRATCH_BYTES, stream);
 }
