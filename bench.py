@@ -206,12 +206,20 @@ def dist_setup():
 
 
 def max_over_ranks(x: float, ws: int) -> float:
+    """The slowest rank's time: every rank calls this with its own measurement."""
     if ws == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def weight_stream_gbs(weight_bytes_per_gpu: int, n_gpus: int, ms_per_step: float) -> float:
+    """Whole-job weight-stream rate: every replica streams its own copy of the
+    weights once per step, in the slowest rank's step time."""
+    return weight_bytes_per_gpu * n_gpus / (ms_per_step / 1e3) / 1e9
 
 
 def barrier(ws):
@@ -368,7 +376,7 @@ def run_gpu(args, ws, rank, local):
     shares = {k: round(v[0] / prof_total, 4) for k, v in prof.items()}
     per_kernel = {k: {"avg_us": round(v[0] / max(v[1], 1) * 1e3, 2), "launches_per_step": v[1] // 3}
                   for k, v in prof.items()}
-    value = w.weight_bytes * ws / (ms_step / 1e3) / 1e9
+    value = weight_stream_gbs(w.weight_bytes, ws, ms_step)
     cpu = {}
     if ws == 1 and not args.no_cpu_baseline:
         dt, wb, nth = oracle_layer_sample(ctx=w.ctx, rows_per_agent=w.rows_per_agent, n_agents=w.n_agents)
@@ -392,7 +400,7 @@ def run_gpu(args, ws, rank, local):
                      "timing": "CUDA events around each launch, eager profiled steps"},
         "step_stream_gbs": (w.weight_bytes + w.kv_bytes) / (ms_step / 1e3) / 1e9,
         "kernel_shares": shares, "kernels": per_kernel,
-        "e2e": {"value": w.weight_bytes * ws / (e2e_ms / 1e3) / 1e9, "unit": "GB/s", "ms_per_step": e2e_ms,
+        "e2e": {"value": weight_stream_gbs(w.weight_bytes, ws, e2e_ms), "unit": "GB/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": w.model.launches() * args.steps,
         "clocks": clk.summary(),

@@ -15,6 +15,7 @@ struct FragBuf {
 };
 
 size_t frag_bytes(int K, int nt);
+int frag_nt(int M);  // fragment layout used for M rows by the active GEMM backend
 FragBuf frag_carve(void *ws, int K, int nt);
 
 struct PrepSrc {

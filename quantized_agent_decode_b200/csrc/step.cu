@@ -86,7 +86,7 @@ static StepLayout step_layout(const qad_model_desc &d, int M)
 {
     StepLayout L;
     const int nq = d.n_qh * d.head_dim, nqkv = (d.n_qh + 2 * d.n_kvh) * d.head_dim;
-    const int nt = M <= 8 ? 1 : 2;
+    const int nt = 2;  // the larger fragment layout serves every backend and row count
     size_t off = 0;
     L.qkv = off;
     off += a256((size_t)M * nqkv * 4);
@@ -226,7 +226,7 @@ static int run_step(qad_model *m, const uint16_t *X, int M, const int *ars, int 
     const int H = d.hidden, I = d.inter, hd = d.head_dim;
     const int nq = d.n_qh * hd, nkv = d.n_kvh * hd, nqkv = nq + 2 * nkv;
     const StepLayout L = step_layout(d, M);
-    const int nt = M <= 8 ? 1 : 2;
+    const int nt = frag_nt(M);
     float *qkv = (float *)(ws + L.qkv), *gu = (float *)(ws + L.gu);
     uint16_t *Qb = (uint16_t *)(ws + L.qb), *Ob = (uint16_t *)(ws + L.ob);
     float *part = (float *)(ws + L.part);
