@@ -412,6 +412,58 @@ def run_gpu(args, ws, rank, local):
     return 0
 
 
+KERNELS = {  # single-kernel cases for profiler captures: (format, N, K)
+    "qkv": (4, 8192, 5120), "o": (4, 5120, 6144), "gate_up": (4, 34816, 5120), "down": (6, 5120, 17408),
+}
+
+
+def run_kernel(args):
+    """Time one matrix of the stack through the public GEMM entry point (prep +
+    GEMM per call), rotating 8 weight copies so every call streams from HBM."""
+    import quantized_agent_decode_b200 as q
+    from quantized_agent_decode_b200 import build
+    build.build()
+    g = synth.torch_gen(SEED, "cuda", 77)
+    if args.kernel == "attn23k":
+        A, L, n_qh, n_kvh = 4, 23000, 48, 8
+        cap = L + 3
+        Kd = synth.bf16_normal_torch(g, (A, n_kvh, cap, 128), "cuda")
+        Vd = synth.bf16_normal_torch(g, (A, n_kvh, cap, 128), "cuda")
+        Qd = synth.bf16_normal_torch(g, (12, n_qh, 128), "cuda")
+        lens = torch.full((A,), L, dtype=torch.int32, device="cuda")
+        ars = torch.arange(0, 13, 3, dtype=torch.int32, device="cuda")
+        O = torch.zeros(12, n_qh, 128, dtype=torch.bfloat16, device="cuda")
+        ws = q.alloc_ws(q.decode_attn_ws_bytes(A, n_qh, n_kvh, cap, 3))
+        fn = lambda i: q.decode_attn(Qd, Kd, Vd, lens, ars, A, 3, cap, n_qh, n_kvh, 128, O, ws=ws)  # noqa: E731
+        nbytes = 2 * A * n_kvh * cap * 128 * 2
+    else:
+        fmt, N, K = KERNELS[args.kernel]
+        mk = synth.q4k_matrix_torch if fmt == 4 else synth.q6k_matrix_torch
+        Ws = [mk(g, N, K, "cuda") for _ in range(8)]
+        if fmt == 6:
+            Ws = [q.q6k_pack(w, N, K) for w in Ws]
+        M = args.rows
+        X = synth.bf16_normal_torch(g, (M, K), "cuda")
+        Y = torch.zeros(M, N, device="cuda")
+        ws = q.alloc_ws(q.gemm_ws_bytes(K, M))
+        gemm = q.q4k_gemm if fmt == 4 else q.q6k_gemm
+        fn = lambda i: gemm(Ws[i % 8], N, K, X, M, Y, ws=ws)  # noqa: E731
+        nbytes = Ws[0].numel()
+    for i in range(args.warmup):
+        fn(i)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(args.steps):
+        fn(i)
+    e1.record()
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) / args.steps * 1e3
+    print(json.dumps({"kernel": args.kernel, "rows": args.rows, "us_per_call": us,
+                      "gbs": nbytes / us / 1e3, "bytes": nbytes, "device_status": q.device_status()}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -420,7 +472,12 @@ def main():
     ap.add_argument("--workload", default="stack12_ctx1k", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel", choices=sorted(list(KERNELS) + ["attn23k"]),
+                    help="time one kernel of the step instead (profiler captures)")
+    ap.add_argument("--rows", type=int, default=12)
     args = ap.parse_args()
+    if args.kernel:
+        return run_kernel(args)
     ws, rank, local = (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
                        int(os.environ.get("LOCAL_RANK", "0")))
     if args.impl == "reference":

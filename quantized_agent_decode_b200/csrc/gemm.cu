@@ -141,26 +141,7 @@ __device__ __forceinline__ float round_half(float v) { return __half2float(__flo
 // input itself, RMSNorm of the fp32 residual, or silu(gate)*up), phase 2 picks
 // the power-of-two scale that puts max|x| in [512, 1024) and writes the row's
 // fragments and sub-block sums.
-// Within-block position of the weight behind logical k-pair `col`, half `v`, in
-// the tensor-core (tcgen05) operand order produced by the decoder threads.
-template <int FMT>
-__device__ __forceinline__ int tc_phys(int col, int v)
-{
-    if (FMT == 4) {  // column 4i+t of quant word i: t = lo0, lo1, hi0, hi1 of bytes (0,2), (1,3)
-        const int i = col >> 2, t = col & 3;
-        return 64 * (i >> 3) + 32 * (t >> 1) + 4 * (i & 7) + (t & 1) + 2 * v;
-    } else {         // column (8h + ci)*8 + 2t + u: quarter t, bytes (u, u+2) of 4-chunk ci of half h
-        const int grp = col >> 3, t = (col & 7) >> 1, u = col & 1;
-        return 128 * (grp >> 3) + 32 * t + 4 * (grp & 7) + u + 2 * v;
-    }
-}
-
-// LAYOUT 0: m16n8k16 B fragments (XP/SP above). LAYOUT 1: tcgen05 B tiles: per
-// block 16 k-steps x 512 bytes in the K-major, non-swizzled canonical layout
-// (core matrices of 8 rows x 16 bytes; +128 bytes for k 8..15 of the step,
-// +256 bytes for rows 8..15), logical k ordered as tc_phys; plus a 512-byte
-// tile of the sub-block sums (k 0..7: Shi_j, k 8..15: Slo_j) for Q4_K.
-template <int FMT, int NT, int LAYOUT = 0>
+template <int FMT, int NT>
 __global__ void __launch_bounds__(512) k_prep(PrepArgs a)
 {
     extern __shared__ uint16_t sxb[];  // the row as bf16 bits
@@ -233,48 +214,6 @@ __global__ void __launch_bounds__(512) k_prep(PrepArgs a)
     if (tid == 0)
         a.fb.rs[r] = live ? ldexpf(1.f, -e) : 0.f;
     __syncthreads();
-    if (LAYOUT == 1) {
-        uint8_t *xt = reinterpret_cast<uint8_t *>(a.fb.xp);
-        const size_t rowoff = (size_t)(r >> 3) * 256 + (r & 7) * 16;
-        for (int it = tid; it < nblk * 32; it += nth) {
-            const int b = it >> 5, ks = (it >> 1) & 15, kg = it & 1;
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (live) {
-                uint32_t w[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int col = 8 * ks + 4 * kg + e;  // k = 16 ks + 8 kg + 2 e + {0, 1}
-                    const float lo = bf16_to_f(sxb[256 * b + tc_phys<FMT>(col, 0)]) * sc;
-                    const float hi = bf16_to_f(sxb[256 * b + tc_phys<FMT>(col, 1)]) * sc;
-                    w[e] = pack_half2(lo, hi);
-                }
-                v = make_uint4(w[0], w[1], w[2], w[3]);
-            }
-            *reinterpret_cast<uint4 *>(xt + (size_t)b * 8192 + ks * 512 + kg * 128 + rowoff) = v;
-        }
-        if (FMT == 4) {
-            uint8_t *stile = reinterpret_cast<uint8_t *>(a.fb.sp);
-            for (int b = tid; b < nblk; b += nth) {
-                float hs[8], ls[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    float S = 0.f;
-                    if (live)
-                        for (int k = 0; k < 32; ++k)
-                            S += round_half(bf16_to_f(sxb[256 * b + 32 * j + k]) * sc);
-                    hs[j] = round_half(S);
-                    ls[j] = S - hs[j];
-                }
-                *reinterpret_cast<uint4 *>(stile + (size_t)b * 512 + rowoff) =
-                    make_uint4(pack_half2(hs[0], hs[1]), pack_half2(hs[2], hs[3]), pack_half2(hs[4], hs[5]),
-                               pack_half2(hs[6], hs[7]));
-                *reinterpret_cast<uint4 *>(stile + (size_t)b * 512 + 128 + rowoff) =
-                    make_uint4(pack_half2(ls[0], ls[1]), pack_half2(ls[2], ls[3]), pack_half2(ls[4], ls[5]),
-                               pack_half2(ls[6], ls[7]));
-            }
-        }
-        return;
-    }
     const int g = r & 7, nt = r >> 3;
     uint2 *xp = reinterpret_cast<uint2 *>(a.fb.xp);
     for (int it = tid; it < nblk * 64; it += nth) {
@@ -325,7 +264,8 @@ __global__ void __launch_bounds__(512) k_prep(PrepArgs a)
 // so every field is 16-byte aligned) followed by plane D [N][ceil8(nblk)] fp16
 // d. 210-byte GGUF blocks cannot be addressed by TMA (16-byte start rule).
 
-constexpr int GW = 8;                // consumer warps per CTA
+constexpr int GW = 8;                // consumer warps per group (16 rows each)
+constexpr int CG = 2;                // consumer groups, taking alternate units
 constexpr int TILE_ROWS = 16 * GW;   // weight rows per CTA unit
 constexpr int Q6A_BYTES = 208;       // plane A bytes per Q6_K block
 
@@ -434,7 +374,7 @@ __device__ __forceinline__ void q4_block(const uint8_t *W16, const uint8_t *XS, 
         dd[rh] = half_lo(h.x);
         dm[rh] = half_hi(h.x);
     }
-    float acc[NT][4];
+    float acc[NT][4], acc2[NT][4];  // two independent chains: low and high nibbles
     const uint8_t *xl = XS + (g * 4 + c) * 8 * NT;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -462,9 +402,18 @@ __device__ __forceinline__ void q4_block(const uint8_t *W16, const uint8_t *XS, 
         const uint32_t c2 = hfma2(and_or(w0s, 0x00F000F0u, H2_1024), SCh[0], NGh[0]);
         const uint32_t c3 = hfma2(and_or(w1s, 0x00F000F0u, H2_1024), SCh[1], NGh[1]);
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-            mma_f16(acc[nt], c0, c1, c2, c3, bhi[nt][0], bhi[nt][1]);
+        for (int nt = 0; nt < NT; ++nt) {
+            if (i == 0)
+                mma_f16_zero(acc2[nt], c0, c1, c2, c3, bhi[nt][0], bhi[nt][1]);
+            else
+                mma_f16(acc2[nt], c0, c1, c2, c3, bhi[nt][0], bhi[nt][1]);
+        }
     }
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            acc[nt][e] += acc2[nt][e];
     // mins: sum_j m_j * S_j, S split into two fp16 parts along k
     uint32_t sb[NT][2];
     lds_b<NT>(SS + (g * 4 + c) * 8 * NT, sb);
@@ -552,7 +501,7 @@ __device__ __forceinline__ void q6_block(const uint8_t *A16, const uint8_t *D16,
 }
 
 template <int FMT, int NT>
-__global__ void __launch_bounds__(32 * (GW + 1), 1) k_qgemm(const __grid_constant__ WeightMaps maps, GemmArgs a)
+__global__ void __launch_bounds__(32 * (CG * GW + 1), 1) k_qgemm(const __grid_constant__ WeightMaps maps, GemmArgs a)
 {
     extern __shared__ __align__(128) uint8_t smem[];
     using St = Stage<FMT, NT>;
@@ -566,56 +515,74 @@ __global__ void __launch_bounds__(32 * (GW + 1), 1) k_qgemm(const __grid_constan
     if (threadIdx.x == 0) {
         for (int i = 0; i < S; ++i) {
             mbar_init(&full[i], 1);
-            mbar_init(&empty[i], GW);
+            mbar_init(&empty[i], GW);  // the 8 warps of the consumer group that used the stage
         }
         mbar_fence_init();
     }
     __syncthreads();
     pdl_trigger();
 
-    if (warp == GW) {
+    if (warp == CG * GW) {
         // ------------------------------------------------ producer warp (lane 0 issues)
         if (lane != 0) {
             pdl_wait();
             return;
         }
-        auto issue_weights = [&](int i) {
-            const int u = u0 + i, t = u / a.nblk, b = u - t * a.nblk;
+        auto issue = [&](int i, int t, int b, bool weights, bool frags) {
             uint8_t *st = smem + (size_t)(i % S) * St::BYTES;
             uint64_t *bar = &full[i % S];
-            mbar_arrive_expect_tx(bar, (uint32_t)St::BYTES);
-            tma_load_2d(st, &maps.w, b * (FMT == 4 ? 144 : Q6A_BYTES), t * TILE_ROWS, bar);
-            if (FMT == 6)
-                tma_load_2d(st + St::W_BYTES, &maps.d, b & ~7, t * TILE_ROWS, bar);
-        };
-        auto issue_frags = [&](int i) {
-            const int u = u0 + i, t = u / a.nblk, b = u - t * a.nblk;
-            (void)t;
-            uint8_t *st = smem + (size_t)(i % S) * St::BYTES + St::W_BYTES + St::D_BYTES;
-            uint64_t *bar = &full[i % S];
-            bulk_g2s(st, reinterpret_cast<const uint8_t *>(a.xp) + (size_t)b * St::X_BYTES, St::X_BYTES, bar);
-            if (FMT == 4)
-                bulk_g2s(st + St::X_BYTES, reinterpret_cast<const uint8_t *>(a.sp) + (size_t)b * St::S_BYTES,
-                         St::S_BYTES, bar);
+            if (weights) {
+                mbar_arrive_expect_tx(bar, (uint32_t)St::BYTES);
+                tma_load_2d(st, &maps.w, b * (FMT == 4 ? 144 : Q6A_BYTES), t * TILE_ROWS, bar);
+                if (FMT == 6)
+                    tma_load_2d(st + St::W_BYTES, &maps.d, b & ~7, t * TILE_ROWS, bar);
+            }
+            if (frags) {
+                uint8_t *xs = st + St::W_BYTES + St::D_BYTES;
+                bulk_g2s(xs, reinterpret_cast<const uint8_t *>(a.xp) + (size_t)b * St::X_BYTES, St::X_BYTES, bar);
+                if (FMT == 4)
+                    bulk_g2s(xs + St::X_BYTES, reinterpret_cast<const uint8_t *>(a.sp) + (size_t)b * St::S_BYTES,
+                             St::S_BYTES, bar);
+            }
         };
         const int pre = min(S, n_units);
-        for (int i = 0; i < pre; ++i)
-            issue_weights(i);  // weights do not depend on the previous kernel
+        int t = n_units > 0 ? u0 / a.nblk : 0, b = u0 - t * a.nblk;
+        for (int i = 0, tt = t, bb = b; i < pre; ++i) {
+            issue(i, tt, bb, true, false);  // weights do not depend on the previous kernel
+            if (++bb == a.nblk) {
+                bb = 0;
+                ++tt;
+            }
+        }
         pdl_wait();
-        for (int i = 0; i < pre; ++i)
-            issue_frags(i);
-        for (int i = S; i < n_units; ++i) {
+        int i = 0;
+        for (; i < pre; ++i) {
+            issue(i, t, b, false, true);
+            if (++b == a.nblk) {
+                b = 0;
+                ++t;
+            }
+        }
+        for (; i < n_units; ++i) {
             if (!mbar_wait(&empty[i % S], ((i / S) - 1) & 1)) {
                 atomicExch(&g_gemm_status, ERR_EMPTY_TIMEOUT);
-                return;
+                break;
             }
-            issue_weights(i);
-            issue_frags(i);
+            issue(i, t, b, true, true);
+            if (++b == a.nblk) {
+                b = 0;
+                ++t;
+            }
         }
+        // every issued copy lands before this CTA may exit
+        for (int k = max(0, i - S); k < i; ++k)
+            if (!mbar_wait(&full[k % S], (k / S) & 1, 20000))
+                atomicExch(&g_gemm_status, ERR_FULL_TIMEOUT);
         return;
     }
 
-    // ---------------------------------------------------- consumer warps
+    // ---------------------------------------------------- consumer groups (alternate units)
+    const int grp = warp / GW, wi = warp % GW;
     const int g = lane >> 2, c = lane & 3;
     const int jj = 2 * (c & 1);
     const uint32_t selT = (uint32_t)(jj | ((jj + 1) << 4) | ((jj + 4) << 8) | ((jj + 5) << 12));
@@ -627,8 +594,12 @@ __global__ void __launch_bounds__(32 * (GW + 1), 1) k_qgemm(const __grid_constan
 #pragma unroll
         for (int e = 0; e < 4; ++e)
             tot[nt][e] = 0.f;
-    int t = n_units > 0 ? u0 / a.nblk : 0, b = u0 - t * a.nblk;
-    for (int i = 0; i < n_units; ++i) {
+    int t = 0, b = 0;
+    if (grp < n_units) {
+        t = (u0 + grp) / a.nblk;
+        b = (u0 + grp) - t * a.nblk;
+    }
+    for (int i = grp; i < n_units; i += CG) {
         const uint8_t *st = smem + (size_t)(i % S) * St::BYTES;
         if (!mbar_wait(&full[i % S], (i / S) & 1)) {
             if (lane == 0)
@@ -637,319 +608,23 @@ __global__ void __launch_bounds__(32 * (GW + 1), 1) k_qgemm(const __grid_constan
         }
         const uint8_t *XS = st + St::W_BYTES + St::D_BYTES;
         if (FMT == 4)
-            q4_block<NT>(st + (size_t)(16 * warp) * 144, XS, XS + St::X_BYTES, g, c, selT, hib, tot);
+            q4_block<NT>(st + (size_t)(16 * wi) * 144, XS, XS + St::X_BYTES, g, c, selT, hib, tot);
         else
-            q6_block<NT>(st + (size_t)(16 * warp) * Q6A_BYTES, st + St::W_BYTES + (size_t)(16 * warp) * 16, b & 7, XS,
-                         g, c, tot);
+            q6_block<NT>(st + (size_t)(16 * wi) * Q6A_BYTES, st + St::W_BYTES + (size_t)(16 * wi) * 16, b & 7, XS, g,
+                         c, tot);
         __syncwarp();
         if (lane == 0)
             mbar_arrive(&empty[i % S]);
-        if (b == a.nblk - 1 || i == n_units - 1)
-            flush_rows<NT>(tot, a, t * TILE_ROWS + 16 * warp, g, c);
-        if (++b == a.nblk) {
-            b = 0;
-            ++t;
+        // next unit of this group: CG blocks further along
+        int tn = t, bn = b + CG;
+        while (bn >= a.nblk) {
+            bn -= a.nblk;
+            ++tn;
         }
-    }
-}
-
-// ------------------------------------------------------------- tcgen05 GEMM
-//
-// Same unit split and TMA producer as k_qgemm, but the multiply runs on the
-// 5th-generation tensor cores: M = 128 weight rows (one per TMEM lane) x N = 16
-// activation rows x K = 16 per tcgen05.mma, A (the decoded weights) in TMEM and
-// B (the activation tile) in shared memory, the fp32 accumulator in TMEM.
-// Warps: 0 = TMA producer, 1 = TMEM allocator, 2..13 = three decoder
-// warpgroups that take units round-robin (while one waits for its MMAs the
-// other two decode). A decoder thread owns one weight row: it reads
-// the row's block from shared memory, writes the exact fp16 operands
-// (sc*q for Q4_K, sc*(q-32) for Q6_K) into its TMEM lane, one elected thread
-// of the warpgroup issues the block's 16 MMAs (+1 for the Q4_K mins) and
-// commits them to an mbarrier, and every thread then reads its row's 16
-// accumulators back and folds in the block's d (and dmin) in fp32.
-//
-// TMEM columns: D_g [16 g, 16 g + 16), D_mins_g [48 + 16 g, ...), and per
-// warpgroup g an A region at 96 + 136 g: weights [0,128), mins [128,136).
-
-constexpr int TC_WG = 3;
-constexpr int TC_THREADS = 32 * (2 + 4 * TC_WG);
-
-template <int FMT>
-struct StageTC {
-    static constexpr int W_BYTES = TILE_ROWS * (FMT == 4 ? 144 : Q6A_BYTES);
-    static constexpr int D_BYTES = FMT == 4 ? 0 : TILE_ROWS * 16;
-    static constexpr int X_BYTES = 8192;
-    static constexpr int S_BYTES = FMT == 4 ? 512 : 0;
-    static constexpr int BYTES = W_BYTES + D_BYTES + X_BYTES + S_BYTES;
-};
-
-template <int FMT>
-constexpr size_t gemm_tc_smem_bytes()
-{
-    return (size_t)Stages<FMT>::N * StageTC<FMT>::BYTES + (2 * Stages<FMT>::N + TC_WG) * sizeof(uint64_t) +
-           16;  // + tmem base, abort flag
-}
-
-// Decode this thread's Q4_K row-block into TMEM: columns [0,128) = sc*q pairs in
-// tc_phys order, [128,136) = the mins (m_0..m_7 twice) for the min MMA.
-__device__ __forceinline__ void tc_decode_q4(const uint8_t *rowp, uint32_t tA, float &dd, float &dm)
-{
-    const uint4 h = lds_v4(rowp);
-    const uint32_t scA = h.y & 0x3F3F3F3Fu, mA = h.z & 0x3F3F3F3Fu;
-    const uint32_t scB = (h.w & 0x0F0F0F0Fu) | ((h.y >> 2) & 0x30303030u);
-    const uint32_t mB = ((h.w >> 4) & 0x0F0F0F0Fu) | ((h.z >> 2) & 0x30303030u);
-    dd = half_lo(h.x);
-    dm = half_hi(h.x);
-#pragma unroll
-    for (int p = 0; p < 4; ++p) {
-        const uint32_t scw = p < 2 ? scA : scB;
-        const uint32_t blo = 2 * (p & 1);  // byte of sub-block 2p in scw
-        const uint32_t SCl = hsub2(prmt(scw, 0x64u, blo | 0x40u | (blo << 8) | 0x4000u), H2_1024);
-        const uint32_t NGl = hmul2(SCl, H2_NEG1024);
-        const uint32_t SCh = hfma2(prmt(scw, 0x64u, (blo + 1) | 0x40u | ((blo + 1) << 8) | 0x4000u), H2_SIXTEENTH,
-                                   H2_NEG64);
-        const uint32_t NGh = hmul2(SCh, H2_NEG1024);
-        const uint4 qa = lds_v4(rowp + 16 + 32 * p), qb = lds_v4(rowp + 32 + 32 * p);
-        uint32_t v[32];
-#pragma unroll
-        for (int w8 = 0; w8 < 8; ++w8) {
-            const uint32_t wd = w8 < 4 ? u4w(qa, w8) : u4w(qb, w8 - 4);
-            const uint32_t ws = wd >> 8;
-            v[4 * w8 + 0] = hfma2(and_or(wd, 0x000F000Fu, H2_1024), SCl, NGl);
-            v[4 * w8 + 1] = hfma2(and_or(ws, 0x000F000Fu, H2_1024), SCl, NGl);
-            v[4 * w8 + 2] = hfma2(and_or(wd, 0x00F000F0u, H2_1024), SCh, NGh);
-            v[4 * w8 + 3] = hfma2(and_or(ws, 0x00F000F0u, H2_1024), SCh, NGh);
-        }
-        tmem_st_x32(tA + 32 * p, v);
-    }
-    uint32_t m8[8];
-    m8[0] = hsub2(prmt(mA, 0x64u, 0x4140u), H2_1024);
-    m8[1] = hsub2(prmt(mA, 0x64u, 0x4342u), H2_1024);
-    m8[2] = hsub2(prmt(mB, 0x64u, 0x4140u), H2_1024);
-    m8[3] = hsub2(prmt(mB, 0x64u, 0x4342u), H2_1024);
-    m8[4] = m8[0];
-    m8[5] = m8[1];
-    m8[6] = m8[2];
-    m8[7] = m8[3];
-    tmem_st_x8(tA + 128, m8);
-}
-
-// Decode this thread's Q6_K-like row-block (packed plane A + d) into TMEM
-// columns [0,128) = sc*(q-32) pairs in tc_phys order.
-__device__ __forceinline__ void tc_decode_q6(const uint8_t *rowA, const uint8_t *dtile_row, int bsub, uint32_t tA,
-                                             float &dd)
-{
-    const uint4 sw = lds_v4(rowA + 192);
-    const uint32_t dw = lds_u32(dtile_row + (bsub & 6) * 2);
-    dd = __half2float(__ushort_as_half((unsigned short)(dw >> ((bsub & 1) * 16))));
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-#pragma unroll
-        for (int cq = 0; cq < 2; ++cq) {
-            const uint4 L0 = lds_v4(rowA + 64 * h + 16 * cq);
-            const uint4 L1 = lds_v4(rowA + 64 * h + 32 + 16 * cq);
-            const uint4 QH = lds_v4(rowA + 128 + 32 * h + 16 * cq);
-            // int8 scales of sub-blocks 8h + 2t + cq -> (sc + 128) + 1024 - 1152 = sc
-            uint32_t SC[4];
-#pragma unroll
-            for (int t = 0; t < 4; ++t) {
-                const int j = 8 * h + 2 * t + cq;
-                const uint32_t wj = u4w(sw, j >> 2) ^ 0x80808080u;
-                const uint32_t bj = (uint32_t)(j & 3);
-                SC[t] = hsub2(prmt(wj, 0x64u, bj | 0x40u | (bj << 8) | 0x4000u), H2_1152);
-            }
-            uint32_t v[32];
-#pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                const uint32_t l0 = u4w(L0, cc), l1 = u4w(L1, cc), hh = u4w(QH, cc);
-                uint32_t qt[4];
-                qt[0] = (l0 & 0x0F0F0F0Fu) | ((hh << 4) & 0x30303030u);
-                qt[1] = (l1 & 0x0F0F0F0Fu) | ((hh << 2) & 0x30303030u);
-                qt[2] = ((l0 >> 4) & 0x0F0F0F0Fu) | (hh & 0x30303030u);
-                qt[3] = ((l1 >> 4) & 0x0F0F0F0Fu) | ((hh >> 2) & 0x30303030u);
-#pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    v[8 * cc + 2 * t + 0] = hmul2(hsub2(prmt(qt[t], 0x64u, 0x4240u), H2_1056), SC[t]);
-                    v[8 * cc + 2 * t + 1] = hmul2(hsub2(prmt(qt[t], 0x64u, 0x4341u), H2_1056), SC[t]);
-                }
-            }
-            // chunks ci = 4 cq + cc of half h -> columns (8h + ci) * 8 + ...
-            tmem_st_x32(tA + (8 * h + 4 * cq) * 8, v);
-        }
-    }
-}
-
-template <int FMT>
-__global__ void __launch_bounds__(TC_THREADS, 1) k_qgemm_tc(const __grid_constant__ WeightMaps maps, GemmArgs a)
-{
-    extern __shared__ __align__(128) uint8_t smem[];
-    using St = StageTC<FMT>;
-    constexpr int S = Stages<FMT>::N;
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + (size_t)S * St::BYTES);
-    uint64_t *empty = full + S;
-    uint64_t *mma_done = empty + S;  // [TC_WG], one per decoder warpgroup
-    uint32_t *tmem_base_sh = reinterpret_cast<uint32_t *>(mma_done + TC_WG);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int u0 = (int)((long long)blockIdx.x * a.units / gridDim.x);
-    const int u1 = (int)((long long)(blockIdx.x + 1) * a.units / gridDim.x);
-    const int n_units = u1 - u0;
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < S; ++i) {
-            mbar_init(&full[i], 1);
-            mbar_init(&empty[i], 4);  // the 4 warps of the decoder warpgroup that used the stage
-        }
-        for (int gg = 0; gg < TC_WG; ++gg)
-            mbar_init(&mma_done[gg], 1);
-        mbar_fence_init();
-    }
-    if (warp == 1) {
-        tmem_alloc(tmem_base_sh, 512);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_base_sh;
-    pdl_trigger();
-
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_base_sh + 1);
-    if (threadIdx.x == 0)
-        *abort_flag = 0;
-    __syncthreads();
-
-    if (warp == 0) {
-        // ------------------------------------------------ TMA producer (lane 0)
-        if (lane == 0) {
-            auto issue = [&](int i, bool weights, bool frags) {
-                const int u = u0 + i, t = u / a.nblk, b = u - t * a.nblk;
-                uint8_t *st = smem + (size_t)(i % S) * St::BYTES;
-                uint64_t *bar = &full[i % S];
-                if (weights) {
-                    mbar_arrive_expect_tx(bar, (uint32_t)St::BYTES);
-                    tma_load_2d(st, &maps.w, b * (FMT == 4 ? 144 : Q6A_BYTES), t * TILE_ROWS, bar);
-                    if (FMT == 6)
-                        tma_load_2d(st + St::W_BYTES, &maps.d, b & ~7, t * TILE_ROWS, bar);
-                }
-                if (frags) {
-                    uint8_t *xs = st + St::W_BYTES + St::D_BYTES;
-                    bulk_g2s(xs, reinterpret_cast<const uint8_t *>(a.xp) + (size_t)b * St::X_BYTES, St::X_BYTES,
-                             bar);
-                    if (FMT == 4)
-                        bulk_g2s(xs + St::X_BYTES, reinterpret_cast<const uint8_t *>(a.sp) + (size_t)b * St::S_BYTES,
-                                 St::S_BYTES, bar);
-                }
-            };
-            const int pre = min(S, n_units);
-            for (int i = 0; i < pre; ++i)
-                issue(i, true, false);  // weights do not depend on the previous kernel
-            pdl_wait();
-            for (int i = 0; i < pre; ++i)
-                issue(i, false, true);
-            int i = S;
-            for (; i < n_units; ++i) {
-                if (!mbar_wait(&empty[i % S], ((i / S) - 1) & 1)) {
-                    atomicExch(&g_gemm_status, ERR_EMPTY_TIMEOUT);
-                    break;
-                }
-                issue(i, true, true);
-            }
-            // every issued copy must land before the CTA may exit
-            for (int k = max(0, min(i, n_units) - S); k < min(i, n_units); ++k)
-                if (!mbar_wait(&full[k % S], (k / S) & 1, 20000))
-                    atomicExch(&g_gemm_status, ERR_FULL_TIMEOUT);
-        } else {
-            pdl_wait();
-        }
-    } else if (warp >= 2) {
-        // ------------------------------------------------ decoder warpgroups
-        const int g = (warp - 2) >> 2;
-        const int row = 32 * (warp & 3) + lane;  // TMEM lane = weight row within the tile
-        const uint32_t lane_bits = (uint32_t)(32 * (warp & 3)) << 16;
-        const uint32_t a_col = 96 + 136 * g, d_col = 16 * g, dm_col = 48 + 16 * g;
-        const uint32_t tA = tmem + a_col + lane_bits;
-        const uint32_t tD = tmem + d_col + lane_bits, tDm = tmem + dm_col + lane_bits;
-        const uint32_t idesc = umma_idesc_f16(128, 16);
-        const bool leader = (warp == 2 + 4 * g) && lane == 0;
-        pdl_wait();
-        float tot[16];
-#pragma unroll
-        for (int c = 0; c < 16; ++c)
-            tot[c] = 0.f;
-        int k_local = 0;
-        for (int i = g; i < n_units; i += TC_WG, ++k_local) {
-            const int u = u0 + i, t = u / a.nblk, b = u - t * a.nblk;
-            const uint8_t *st = smem + (size_t)(i % S) * St::BYTES;
-            // every thread of the warpgroup takes the same path: an abort is
-            // decided only right after a named barrier, from a shared flag
-            float dd = 0.f, dm = 0.f;
-            if (mbar_wait(&full[i % S], (i / S) & 1)) {
-                if (FMT == 4)
-                    tc_decode_q4(st + row * 144, tA, dd, dm);
-                else
-                    tc_decode_q6(st + row * Q6A_BYTES, st + St::W_BYTES + row * 16, b & 7, tA, dd);
-                tmem_wait_st();
-            } else {
-                *abort_flag = 1;
-                atomicExch(&g_gemm_status, ERR_FULL_TIMEOUT);
-            }
-            tc_fence_before();
-            named_bar_sync(1 + g, 128);
-            if (*abort_flag)
-                break;
-            if (leader) {
-                tc_fence_after();
-                const uint32_t xs = smem_u32(st + St::W_BYTES + St::D_BYTES);
-                const uint32_t a_base = tmem + a_col, d_base = tmem + d_col;
-#pragma unroll
-                for (int ks = 0; ks < 16; ++ks)
-                    umma_f16_ts(d_base, a_base + 8 * ks, umma_desc_k_noswz(xs + 512 * ks, 128, 256), idesc, ks > 0);
-                if (FMT == 4)
-                    umma_f16_ts(tmem + dm_col, a_base + 128, umma_desc_k_noswz(xs + St::X_BYTES, 128, 256), idesc, 0);
-                umma_commit(&mma_done[g]);
-            }
-            if (!mbar_wait(&mma_done[g], k_local & 1)) {
-                *abort_flag = 1;
-                atomicExch(&g_gemm_status, ERR_FULL_TIMEOUT);
-            }
-            named_bar_sync(1 + g, 128);
-            if (*abort_flag)
-                break;
-            tc_fence_after();
-            uint32_t dv[16], dmv[16];
-            tmem_ld_x16(tD, dv);
-            if (FMT == 4)
-                tmem_ld_x16(tDm, dmv);
-            tmem_wait_ld();
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(&empty[i % S]);
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-                tot[c] = fmaf(dd, __uint_as_float(dv[c]), tot[c]);
-                if (FMT == 4)
-                    tot[c] = fmaf(-dm, __uint_as_float(dmv[c]), tot[c]);
-            }
-            // flush when this warpgroup's next unit belongs to another tile (or there is none)
-            if (i + TC_WG >= n_units || (u + TC_WG) / a.nblk != t) {
-                const int n = t * TILE_ROWS + row;
-                if (n < a.N)
-#pragma unroll
-                    for (int c = 0; c < 16; ++c)
-                        if (c < a.M)
-                            atomicAdd(a.Y + (size_t)c * a.ldy + n, a.rs[c] * tot[c]);
-#pragma unroll
-                for (int c = 0; c < 16; ++c)
-                    tot[c] = 0.f;
-            }
-        }
-    } else {
-        pdl_wait();
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 1) {
-        tc_fence_after();
-        tmem_dealloc(tmem, 512);
+        if (tn != t || i + CG >= n_units)
+            flush_rows<NT>(tot, a, t * TILE_ROWS + 16 * wi, g, c);
+        t = tn;
+        b = bn;
     }
 }
 
@@ -992,38 +667,24 @@ static int set_smem(K kernel, size_t bytes)
                       "cudaFuncSetAttribute");
 }
 
-// GEMM backend: tcgen05 (default) or the legacy warp-MMA kernel (QAD_GEMM_BACKEND=mma).
-static bool use_tc()
-{
-    static int v = -1;
-    if (v < 0) {
-        const char *e = getenv("QAD_GEMM_BACKEND");
-        v = (e && e[0] == 'm') ? 0 : 1;
-    }
-    return v == 1;
-}
-
-int frag_nt(int M) { return (M <= 8 && !use_tc()) ? 1 : 2; }
+int frag_nt(int M) { return M <= 8 ? 1 : 2; }
 
 int launch_prep(int fmt, int K, int M, const PrepSrc &src, const FragBuf &fb, cudaStream_t s, bool pdl)
 {
-    const bool tc = use_tc();
     const int nt = frag_nt(M);
     PrepArgs a{src, K, M, fb};
     const size_t smem = (size_t)K * sizeof(uint16_t);
     void (*kern)(PrepArgs);
-    if (tc)
-        kern = fmt == 4 ? k_prep<4, 2, 1> : k_prep<6, 2, 1>;
-    else if (fmt == 4)
+    if (fmt == 4)
         kern = nt == 1 ? k_prep<4, 1> : k_prep<4, 2>;
     else
         kern = nt == 1 ? k_prep<6, 1> : k_prep<6, 2>;
     if (smem > 48 * 1024) {
         // once per (device, kernel variant): room for the longest row (K <= 65536)
-        static bool done[64][6] = {};
+        static bool done[64][4] = {};
         int dev = 0;
         cudaGetDevice(&dev);
-        const int v = tc ? (fmt == 4 ? 4 : 5) : (fmt == 4 ? 0 : 2) + (nt - 1);
+        const int v = (fmt == 4 ? 0 : 2) + (nt - 1);
         if (dev < 0 || dev >= 64 || !done[dev][v]) {
             int rc = set_smem(kern, (size_t)65536 * sizeof(uint16_t));
             if (rc)
@@ -1053,26 +714,6 @@ int make_weight_maps(int fmt, const void *W, int N, int K, WeightMapsBlob *out)
     return encode_tmap_2d(&m->d, D, 2, (uint64_t)nblk8, (uint64_t)N, (uint64_t)nblk8 * 2, 8, TILE_ROWS);
 }
 
-static int launch_gemm_tc(int fmt, const WeightMaps &maps, const GemmArgs &a, cudaStream_t s, bool pdl)
-{
-    void (*kern)(const WeightMaps, GemmArgs) = fmt == 4 ? k_qgemm_tc<4> : k_qgemm_tc<6>;
-    const size_t smem = fmt == 4 ? gemm_tc_smem_bytes<4>() : gemm_tc_smem_bytes<6>();
-    static bool done[64][2] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64 || !done[dev][fmt == 4 ? 0 : 1]) {
-        int rc = set_smem(kern, smem);
-        if (rc)
-            return rc;
-        if (dev >= 0 && dev < 64)
-            done[dev][fmt == 4 ? 0 : 1] = true;
-    }
-    const int grid = num_sms();
-    cudaError_t e = pdl ? launch_pdl(kern, dim3(grid), dim3(TC_THREADS), smem, s, maps, a)
-                        : (kern<<<grid, TC_THREADS, smem, s>>>(maps, a), cudaGetLastError());
-    return cuda_check(e, "gemm(tc) launch");
-}
-
 int launch_gemm(int fmt, const WeightMapsBlob &maps_blob, int N, int K, int M, const FragBuf &fb, float *Y, int ldy,
                 cudaStream_t s, bool pdl)
 {
@@ -1088,8 +729,6 @@ int launch_gemm(int fmt, const WeightMapsBlob &maps_blob, int N, int K, int M, c
     a.sp = fb.sp;
     a.rs = fb.rs;
     a.Y = Y;
-    if (use_tc())
-        return launch_gemm_tc(fmt, maps, a, s, pdl);
     void (*kern)(const WeightMaps, GemmArgs);
     size_t smem;
     if (fmt == 4) {
@@ -1111,8 +750,8 @@ int launch_gemm(int fmt, const WeightMapsBlob &maps_blob, int N, int K, int M, c
             done[dev][v] = true;
     }
     const int grid = num_sms();
-    cudaError_t e = pdl ? launch_pdl(kern, dim3(grid), dim3(32 * (GW + 1)), smem, s, maps, a)
-                        : (kern<<<grid, 32 * (GW + 1), smem, s>>>(maps, a), cudaGetLastError());
+    cudaError_t e = pdl ? launch_pdl(kern, dim3(grid), dim3(32 * (CG * GW + 1)), smem, s, maps, a)
+                        : (kern<<<grid, 32 * (CG * GW + 1), smem, s>>>(maps, a), cudaGetLastError());
     return cuda_check(e, "gemm launch");
 }
 
