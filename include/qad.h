@@ -217,8 +217,10 @@ void qad_model_destroy(qad_model *model);
  *   agent_row_start, lens  device int32 [n_agents+1], [n_agents]; lens are
  *            the cached lengths before the step (the caller commits accepted
  *            tokens afterwards; rejected slots are overwritten next step)
- *   H_out    device fp32 [M][hidden]: the residual stream after the last layer
- *   ws       device workspace of qad_decode_step_ws_bytes(model, M) bytes
+ *   H_out    device fp32 [M][hidden], 16-byte aligned: the residual stream
+ *            after the last layer
+ *   ws       device workspace of qad_decode_step_ws_bytes(model, M) bytes,
+ *            256-byte aligned
  * 1 <= M <= 16, n_agents <= max_agents. */
 size_t qad_decode_step_ws_bytes(const qad_model *model, int M);
 int qad_decode_step(qad_model *model, const uint16_t *X, int M, const int *agent_row_start,
@@ -254,7 +256,8 @@ int qad_decode_step_launches(const qad_model *model);
  * [M][n_qh hd]), h after the o projection (fp32 [M][hidden]), x2 (bf16),
  * gate|up (fp32 [M][2 inter]), silu(gate)*up (bf16 [M][inter]) and h after
  * the layer (fp32), each at a 256-byte aligned offset in that order, into
- * layer l's slice. Pass dbg = NULL to detach. Graph capture refuses a model
+ * layer l's slice. The buffer must be 256-byte aligned. Pass dbg = NULL to
+ * detach. Graph capture refuses a model
  * with a debug buffer attached. */
 size_t qad_decode_step_debug_bytes(const qad_model *model, int M);
 int qad_model_set_debug(qad_model *model, void *dbg, size_t bytes);
@@ -262,9 +265,10 @@ int qad_model_set_debug(qad_model *model, void *dbg, size_t bytes);
 /* Per-launch event profiler. While enabled, every eager qad_decode_step records
  * a CUDA event before and after each of its launches (which serialises the
  * launch chain) and qad_model_profile_read() accumulates the elapsed times per
- * kernel class into ms[k], count[k] (k: 0 init, 1 prep, 2 qkv GEMM, 3 qkv
- * split/append, 4 attention + combine, 5 o GEMM, 6 gate|up GEMM, 7 down GEMM;
- * n_kinds >= 8) and returns the number of classes. Read after every profiled
+ * kernel class into ms[k], count[k] (k: 0 init, 1 prep (including the
+ * attention split merge), 2 qkv GEMM, 3 attention (including the k/v append),
+ * 4 o GEMM, 5 gate|up GEMM, 6 down GEMM; n_kinds >= 7) and returns the number
+ * of classes. Read after every profiled
  * step (a step not read before the next one is dropped). Enabling resets the
  * totals. Graph capture refuses a model with the profiler on. */
 int qad_model_set_profile(qad_model *model, int enable);

@@ -78,7 +78,7 @@ SIGNATURES = {
     "qad_model_profile_read": (C.c_int, [C.c_void_p, C.POINTER(C.c_double), C.POINTER(C.c_longlong), C.c_int]),
 }
 
-PROFILE_KINDS = ["init", "prep", "gemm_qkv", "qkv_post", "attn", "gemm_o", "gemm_gate_up", "gemm_down"]
+PROFILE_KINDS = ["init", "prep", "gemm_qkv", "attn", "gemm_o", "gemm_gate_up", "gemm_down"]
 
 
 def lib():

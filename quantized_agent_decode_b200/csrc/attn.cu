@@ -23,15 +23,18 @@
 
 namespace qad {
 
-constexpr int QG = 24;          // query vectors per CTA
+constexpr int QG = ATT_QG;      // query vectors per CTA
 constexpr int KT = 16;          // keys per tile (one MMA M tile)
 constexpr int ATT_WARPS = 4;
 constexpr int ATT_STAGES = 3;
 constexpr int TILE_BYTES = KT * 128 * 2;  // 4 KB (K) ; V follows
-constexpr int PART_FLOATS = QG * 128 + 2 * QG;
+constexpr int PART_FLOATS = ATT_PART_FLOATS;
 
 struct AttnArgs {
-    const uint16_t *Q, *Kc, *Vc;
+    const uint16_t *Q, *Kc, *Vc;   // standalone: bf16 Q [M][n_qh][128]
+    const float *qkv;              // fused: fp32 q | k | v rows [M][ldqkv]
+    uint16_t *Kw, *Vw;             // fused: the caches, written at the new positions
+    int ldqkv;
     const int *lens, *ars;
     int n_kvh, kv_cap, n_qh, G, CH, n_rg, max_splits;
     float scale_log2;
@@ -40,6 +43,11 @@ struct AttnArgs {
 
 __device__ __forceinline__ int swz(int key, int chunk) { return key * 256 + ((chunk ^ (key & 7)) << 4); }
 
+// FUSED: Q and the new rows' k, v come from the fp32 projection (rounded to
+// bf16 here, as the unfused path rounds them before the cache write); key
+// positions len .. len+na-1 are taken from there instead of the cache, and the
+// row-group-0 CTA of the split holding a new position writes it to the cache.
+template <bool FUSED>
 __global__ void __launch_bounds__(128, 2) k_decode_attn(AttnArgs p)
 {
     extern __shared__ __align__(128) uint8_t smem[];
@@ -70,11 +78,22 @@ __global__ void __launch_bounds__(128, 2) k_decode_attn(AttnArgs p)
         const int qi = q0 + 8 * nt + gq;
         const bool ok = qi < R;
         const int j = ok ? qi / p.G : 0, hl = ok ? qi - j * p.G : 0;
-        const uint16_t *qrow = p.Q + ((size_t)(r0 + j) * p.n_qh + g * p.G + hl) * 128;
+        if (FUSED) {
+            const float *qrow = p.qkv + (size_t)(r0 + j) * p.ldqkv + (g * p.G + hl) * 128;
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-            qf[nt][ks][0] = ok ? *reinterpret_cast<const uint32_t *>(qrow + 16 * ks + 2 * c) : 0u;
-            qf[nt][ks][1] = ok ? *reinterpret_cast<const uint32_t *>(qrow + 16 * ks + 8 + 2 * c) : 0u;
+            for (int ks = 0; ks < 8; ++ks) {
+                const float2 f0 = ok ? *reinterpret_cast<const float2 *>(qrow + 16 * ks + 2 * c) : make_float2(0.f, 0.f);
+                const float2 f1 = ok ? *reinterpret_cast<const float2 *>(qrow + 16 * ks + 8 + 2 * c) : make_float2(0.f, 0.f);
+                qf[nt][ks][0] = pack_bf162(f0.x, f0.y);
+                qf[nt][ks][1] = pack_bf162(f1.x, f1.y);
+            }
+        } else {
+            const uint16_t *qrow = p.Q + ((size_t)(r0 + j) * p.n_qh + g * p.G + hl) * 128;
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                qf[nt][ks][0] = ok ? *reinterpret_cast<const uint32_t *>(qrow + 16 * ks + 2 * c) : 0u;
+                qf[nt][ks][1] = ok ? *reinterpret_cast<const uint32_t *>(qrow + 16 * ks + 8 + 2 * c) : 0u;
+            }
         }
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
@@ -104,9 +123,41 @@ __global__ void __launch_bounds__(128, 2) k_decode_attn(AttnArgs p)
     const int my = ntiles > w ? (ntiles - w + ATT_WARPS - 1) / ATT_WARPS : 0;
     uint8_t *wbuf = smem + (size_t)w * ATT_STAGES * 2 * TILE_BYTES;
 
+    const int nq = p.n_qh * 128, nkv = p.n_kvh * 128;
     auto issue = [&](int it) {
         const int kb = kbeg + KT * (w + ATT_WARPS * it);
         uint8_t *st = wbuf + (size_t)(it % ATT_STAGES) * 2 * TILE_BYTES;
+        if (FUSED && kb + KT > len) {
+            // tile reaches the new positions: cached keys below len, new rows from the projection
+#pragma unroll 1
+            for (int i = 0; i < 8; ++i) {
+                const int idx = lane + 32 * i, kk = idx >> 4, ch = idx & 15, kp = kb + kk;
+                if (kp < len || kp >= kend) {
+                    const bool ok = kp < kend;
+                    const size_t src = (size_t)(ok ? kp : 0) * 128 + ch * 8;
+                    cp_async16_zfill(st + swz(kk, ch), Kh + src, ok);
+                    cp_async16_zfill(st + TILE_BYTES + swz(kk, ch), Vh + src, ok);
+                } else {
+                    const float *row = p.qkv + (size_t)(r0 + kp - len) * p.ldqkv + nq + g * 128 + ch * 8;
+                    const float4 k0 = *reinterpret_cast<const float4 *>(row);
+                    const float4 k1 = *reinterpret_cast<const float4 *>(row + 4);
+                    const float4 v0 = *reinterpret_cast<const float4 *>(row + nkv);
+                    const float4 v1 = *reinterpret_cast<const float4 *>(row + nkv + 4);
+                    const uint4 kw = make_uint4(pack_bf162(k0.x, k0.y), pack_bf162(k0.z, k0.w),
+                                                pack_bf162(k1.x, k1.y), pack_bf162(k1.z, k1.w));
+                    const uint4 vw = make_uint4(pack_bf162(v0.x, v0.y), pack_bf162(v0.z, v0.w),
+                                                pack_bf162(v1.x, v1.y), pack_bf162(v1.z, v1.w));
+                    *reinterpret_cast<uint4 *>(st + swz(kk, ch)) = kw;
+                    *reinterpret_cast<uint4 *>(st + TILE_BYTES + swz(kk, ch)) = vw;
+                    if (rg == 0) {
+                        const size_t dst = head_off + (size_t)kp * 128 + ch * 8;
+                        *reinterpret_cast<uint4 *>(p.Kw + dst) = kw;
+                        *reinterpret_cast<uint4 *>(p.Vw + dst) = vw;
+                    }
+                }
+            }
+            return;
+        }
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const int idx = lane + 32 * i, kk = idx >> 4, ch = idx & 15;
@@ -330,14 +381,32 @@ size_t attn_smem_bytes()
     return stages > merge ? stages : merge;
 }
 
-int launch_attn(const AttnPlan &pl, const uint16_t *Q, const uint16_t *Kc, const uint16_t *Vc, const int *lens,
-                const int *ars, int n_agents, int kv_cap, int n_qh, int n_kvh, float scale, uint16_t *O, float *part,
-                cudaStream_t s, bool pdl)
+template <bool FUSED>
+static int launch_split_kernel(const AttnPlan &pl, const AttnArgs &p, int n_agents, cudaStream_t s, bool pdl)
 {
-    AttnArgs p;
-    p.Q = Q;
-    p.Kc = Kc;
-    p.Vc = Vc;
+    const size_t smem = attn_smem_bytes();
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+        int rc = cuda_check(
+            cudaFuncSetAttribute(k_decode_attn<FUSED>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem),
+            "cudaFuncSetAttribute(attn)");
+        if (rc)
+            return rc;
+        if (dev >= 0 && dev < 64)
+            attr_set[dev] = true;
+    }
+    dim3 grid(pl.max_splits, pl.n_rg, n_agents * p.n_kvh);
+    cudaError_t e = pdl ? launch_pdl(k_decode_attn<FUSED>, grid, dim3(128), smem, s, p)
+                        : (k_decode_attn<FUSED><<<grid, 128, smem, s>>>(p), cudaGetLastError());
+    return cuda_check(e, "attn launch");
+}
+
+static AttnArgs attn_args(const AttnPlan &pl, const int *lens, const int *ars, int kv_cap, int n_qh, int n_kvh,
+                          float scale, float *part)
+{
+    AttnArgs p = {};
     p.lens = lens;
     p.ars = ars;
     p.n_kvh = n_kvh;
@@ -349,23 +418,52 @@ int launch_attn(const AttnPlan &pl, const uint16_t *Q, const uint16_t *Kc, const
     p.max_splits = pl.max_splits;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.part = part;
-    const size_t smem = attn_smem_bytes();
-    static bool attr_set[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-        int rc = cuda_check(cudaFuncSetAttribute(k_decode_attn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem),
-                            "cudaFuncSetAttribute(attn)");
-        if (rc)
-            return rc;
-        if (dev >= 0 && dev < 64)
-            attr_set[dev] = true;
-    }
-    dim3 grid(pl.max_splits, pl.n_rg, n_agents * n_kvh);
-    cudaError_t e = pdl ? launch_pdl(k_decode_attn, grid, dim3(128), smem, s, p)
-                        : (k_decode_attn<<<grid, 128, smem, s>>>(p), cudaGetLastError());
-    if (e != cudaSuccess)
-        return cuda_check(e, "attn launch");
+    return p;
+}
+
+int launch_attn_fused(const AttnPlan &pl, const float *qkv, int ldqkv, uint16_t *Kc, uint16_t *Vc, const int *lens,
+                      const int *ars, int n_agents, int kv_cap, int n_qh, int n_kvh, float scale, float *part,
+                      cudaStream_t s, bool pdl)
+{
+    AttnArgs p = attn_args(pl, lens, ars, kv_cap, n_qh, n_kvh, scale, part);
+    p.qkv = qkv;
+    p.ldqkv = ldqkv;
+    p.Kc = Kc;
+    p.Vc = Vc;
+    p.Kw = Kc;
+    p.Vw = Vc;
+    return launch_split_kernel<true>(pl, p, n_agents, s, pdl);
+}
+
+AttnPartView attn_part_view(const AttnPlan &pl, const float *part, const int *ars, const int *lens, int kv_cap,
+                            int n_qh, int n_kvh)
+{
+    AttnPartView v;
+    v.part = part;
+    v.ars = ars;
+    v.lens = lens;
+    v.n_kvh = n_kvh;
+    v.G = pl.G;
+    v.n_rg = pl.n_rg;
+    v.max_splits = pl.max_splits;
+    v.CH = pl.CH;
+    v.kv_cap = kv_cap;
+    v.n_qh = n_qh;
+    return v;
+}
+
+int launch_attn(const AttnPlan &pl, const uint16_t *Q, const uint16_t *Kc, const uint16_t *Vc, const int *lens,
+                const int *ars, int n_agents, int kv_cap, int n_qh, int n_kvh, float scale, uint16_t *O, float *part,
+                cudaStream_t s, bool pdl)
+{
+    AttnArgs p = attn_args(pl, lens, ars, kv_cap, n_qh, n_kvh, scale, part);
+    p.Q = Q;
+    p.Kc = Kc;
+    p.Vc = Vc;
+    int rc = launch_split_kernel<false>(pl, p, n_agents, s, pdl);
+    if (rc)
+        return rc;
+    cudaError_t e;
     dim3 g2(QG, pl.n_rg, n_agents * n_kvh);
     e = pdl ? launch_pdl(k_attn_combine, g2, dim3(128), 0, s, p, O)
             : (k_attn_combine<<<g2, 128, 0, s>>>(p, O), cudaGetLastError());

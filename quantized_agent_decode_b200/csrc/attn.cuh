@@ -4,6 +4,20 @@
 
 namespace qad {
 
+// Partial results of one (agent, kv-head, row group of 24 query vectors, key
+// split): unnormalised O [24][128] fp32, then the running max m[24] (log2
+// domain) and the sum l[24]. Record index
+// ((agent * n_kvh + kv_head) * n_rg + rg) * max_splits + split.
+constexpr int ATT_QG = 24;
+constexpr int ATT_PART_FLOATS = ATT_QG * 128 + 2 * ATT_QG;
+
+// What a consumer needs to merge the splits of one query vector.
+struct AttnPartView {
+    const float *part;
+    const int *ars, *lens;
+    int n_kvh, G, n_rg, max_splits, CH, kv_cap, n_qh;
+};
+
 struct AttnPlan {
     int G;           // q-heads per kv-head
     int n_rg;        // groups of 24 query vectors per (agent, kv-head)
@@ -13,8 +27,18 @@ struct AttnPlan {
 };
 
 AttnPlan attn_plan(int n_agents, int n_qh, int n_kvh, int kv_cap, int max_rows_per_agent);
+// Standalone form: Q bf16, caches already holding the new rows, O bf16 (combine included).
 int launch_attn(const AttnPlan &pl, const uint16_t *Q, const uint16_t *Kc, const uint16_t *Vc, const int *lens,
                 const int *ars, int n_agents, int kv_cap, int n_qh, int n_kvh, float scale, uint16_t *O, float *part,
                 cudaStream_t s, bool pdl);
+// Fused form used by the decode step: Q and the new rows' k, v are read from the
+// fp32 q|k|v projection [M][ldqkv]; the split holding each new position also
+// writes that row's k, v (bf16) into the caches. Writes only the partials
+// (the o-projection prep merges them).
+int launch_attn_fused(const AttnPlan &pl, const float *qkv, int ldqkv, uint16_t *Kc, uint16_t *Vc, const int *lens,
+                      const int *ars, int n_agents, int kv_cap, int n_qh, int n_kvh, float scale, float *part,
+                      cudaStream_t s, bool pdl);
+AttnPartView attn_part_view(const AttnPlan &pl, const float *part, const int *ars, const int *lens, int kv_cap,
+                            int n_qh, int n_kvh);
 
 }  // namespace qad

@@ -251,6 +251,11 @@ __device__ __forceinline__ uint2 lds_v2(const void *p)
     asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(smem_u32(p)));
     return v;
 }
+__device__ __forceinline__ float2 lds_v2f(const void *p)
+{
+    const uint2 v = lds_v2(p);
+    return make_float2(__uint_as_float(v.x), __uint_as_float(v.y));
+}
 __device__ __forceinline__ uint32_t lds_u32(const void *p)
 {
     uint32_t v;

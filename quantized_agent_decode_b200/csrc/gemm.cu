@@ -46,49 +46,57 @@ __device__ int g_gemm_status;
 
 // ------------------------------------------------------------- fragment layout
 // Activation rows r = 8*nt + g (nt < NT, g < 8); blocks b < nblk; k-steps
-// s < 16; lane quad c < 4. Block-major, so one block's fragments are one
-// contiguous bulk copy and a warp's 32 lanes read 32 consecutive entries.
-//   XP (uint2 units): [b][s][g][c][nt] = {b0, b1}: the two B registers of the
+// s < 16; lane quad c < 4. One record per block (rec_bytes), so a GEMM unit
+// fetches its block's operand with one bulk copy and a warp's 32 lanes read 32
+// consecutive entries.
+//   X (uint2 units): [s][g][c][nt] = {b0, b1}: the two B registers of the
 //       m16n8k16 fragment: b0 = (x[k0], x[k0+2]), b1 = (x[k0+1], x[k0+3]) with
-//       k0 = 256 b + frag_k0(s, c), as fp16 of x * 2^e_r.
-//   SP (uint2 units): [b][g][c][nt] = {(Shi_2c, Shi_2c+1), (Slo_2c, Slo_2c+1)}
+//       k0 = 256 b + frag_k0(s, c), as fp16 of x * 2^e(r,b).
+//   S (uint2 units): [g][c][nt] = {(Shi_2c, Shi_2c+1), (Slo_2c, Slo_2c+1)}
 //       with S_j the sum of the 32 fp16 activations of Q4_K sub-block j split
 //       into two fp16 parts (Q4_K only).
-//   RS: 16 floats, 2^-e_r (0 for rows >= M).
-static inline size_t xp_words(int nblk, int nt) { return (size_t)8 * nblk * 16 * 4 * nt * 2; }
-static inline size_t sp_words(int nblk, int nt) { return (size_t)8 * nblk * 4 * nt * 2; }
+//   RS: 16 floats, 2^-e(r,b) (0 for rows >= M).
+// e(r,b) puts the block's largest |x| in [512, 1024): fp16 holds every bf16
+// value of the block exactly unless it is 2^24 times smaller than that max.
 static inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-size_t frag_bytes(int K, int nt)
-{
-    int nblk = K / 256;
-    return align256(xp_words(nblk, nt) * 4) + align256(sp_words(nblk, nt) * 4) + 256;
-}
+size_t frag_bytes(int K, int nt) { return align256((size_t)(K / 256) * rec_bytes(4, nt)); }
 
-FragBuf frag_carve(void *ws, int K, int nt)
+FragBuf frag_carve(void *ws, int, int)
 {
-    int nblk = K / 256;
-    char *p = (char *)ws;
     FragBuf f;
-    f.xp = (uint32_t *)p;
-    p += align256(xp_words(nblk, nt) * 4);
-    f.sp = (uint32_t *)p;
-    p += align256(sp_words(nblk, nt) * 4);
-    f.rs = (float *)p;
+    f.rec = (uint8_t *)ws;
     return f;
 }
 
 // Which activation column feeds logical k-slot (s, c). The weight-side decode
 // below produces, for lane quad c and k-step s, the weights at within-block
 // positions k0, k0+2 (first B register) and k0+1, k0+3 (second).
-template <int FMT>
-__device__ __forceinline__ int frag_k0(int s, int c)
+__host__ __device__ constexpr int frag_k0(int fmt, int s, int c)
 {
-    if (FMT == 4)  // quant bytes 32c..32c+31: word s>>1, low (s even) or high (s odd) nibbles
-        return 64 * c + 4 * (s >> 1) + 32 * (s & 1);
-    else           // half c>>1, l-range 16*(c&1); word s>>2; t = s&3 selects the 32-weight quarter
-        return 128 * (c >> 1) + 16 * (c & 1) + 4 * (s >> 2) + 32 * (s & 3);
+    // Q4_K: quant bytes 32c..32c+31: word s>>1, low (s even) or high (s odd) nibbles.
+    // Q6_K: half c>>1, l-range 16*(c&1); word s>>2; s&3 selects the 32-weight quarter.
+    return fmt == 4 ? 64 * c + 4 * (s >> 1) + 32 * (s & 1) : 128 * (c >> 1) + 16 * (c & 1) + 4 * (s >> 2) + 32 * (s & 3);
 }
+
+// The inverse: the slot (s, c) whose k0 is 4t (t < 64), so thread t of a block
+// reads columns 4t..4t+3 and its loads coalesce. For Q4_K, t >> 3 is the
+// sub-block 2c + (s & 1).
+__host__ __device__ constexpr int slot_s(int fmt, int t)
+{
+    return fmt == 4 ? 2 * (t & 7) + ((t >> 3) & 1) : 4 * (t & 3) + ((t & 31) >> 3);
+}
+__host__ __device__ constexpr int slot_c(int fmt, int t) { return fmt == 4 ? t >> 4 : 2 * (t >> 5) + ((t >> 2) & 1); }
+
+constexpr bool slot_maps_consistent()
+{
+    for (int fmt = 4; fmt <= 6; fmt += 2)
+        for (int t = 0; t < 64; ++t)
+            if (frag_k0(fmt, slot_s(fmt, t), slot_c(fmt, t)) != 4 * t || slot_s(fmt, t) > 15 || slot_c(fmt, t) > 3)
+                return false;
+    return true;
+}
+static_assert(slot_maps_consistent(), "fragment slot maps must invert frag_k0");
 
 // ------------------------------------------------------------- prep kernel
 
@@ -112,139 +120,179 @@ __device__ __forceinline__ float warp_max(float v)
         v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
     return v;
 }
-__device__ float block_sum(float v, float *red)
-{
-    v = warp_sum(v);
-    int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-    __syncthreads();
-    if (l == 0)
-        red[w] = v;
-    __syncthreads();
-    v = (l < (int)(blockDim.x >> 5)) ? red[l] : 0.f;
-    return warp_sum(v);
-}
-__device__ float block_max(float v, float *red)
-{
-    v = warp_max(v);
-    int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-    __syncthreads();
-    if (l == 0)
-        red[w] = v;
-    __syncthreads();
-    v = (l < (int)(blockDim.x >> 5)) ? red[l] : 0.f;
-    return warp_max(v);
-}
 __device__ __forceinline__ float round_half(float v) { return __half2float(__float2half_rn(v)); }
 
-// One CTA per activation row r < 8*NT (rows >= M write zero fragments).
-// Phase 1 forms the row exactly as the GEMM must see it (bf16 values: the
-// input itself, RMSNorm of the fp32 residual, or silu(gate)*up), phase 2 picks
-// the power-of-two scale that puts max|x| in [512, 1024) and writes the row's
-// fragments and sub-block sums.
-template <int FMT, int NT>
-__global__ void __launch_bounds__(512) k_prep(PrepArgs a)
+// silu(g) * u in fp32; below g = -80, 1 + e^-g equals e^-g in fp32 and e^-g
+// would overflow past -88, so the product g*u*e^g is formed in the log domain
+// (an exact zero stays zero).
+__device__ __forceinline__ float silu_mul(float g, float u)
 {
-    extern __shared__ uint16_t sxb[];  // the row as bf16 bits
-    __shared__ float red[32];
-    const int r = blockIdx.x, tid = threadIdx.x, nth = blockDim.x;
+    if (g >= -80.f)
+        return g / (1.f + expf(-g)) * u;
+    const float p = g * u;
+    return p == 0.f ? p : copysignf(expf(g + logf(fabsf(p))), p);
+}
+
+// Grid (ceil(nblk / 4), 8*NT): CTA (x, r) forms row r's blocks 4x..4x+3, one
+// 64-thread quarter per block, thread t of a quarter owning columns 4t..4t+3.
+// The values are formed exactly as the GEMM must see them (bf16: the input
+// itself, RMSNorm of the fp32 residual, silu(gate)*up, or the merged
+// attention output), then scaled per (row, block) into fp16 fragments.
+template <int FMT, int NT>
+__global__ void __launch_bounds__(256) k_prep(PrepArgs a)
+{
+    __shared__ float red[8];
+    __shared__ float s_inv;
+    const int r = blockIdx.y, tid = threadIdx.x, q = tid >> 6, t = tid & 63;
     const int K = a.K, nblk = K >> 8;
+    const int b = 4 * blockIdx.x + q;
     const PrepSrc &S = a.src;
     pdl_trigger();
     pdl_wait();
     if (S.zero) {
-        long long per = (S.zero_n + gridDim.x - 1) / gridDim.x;
-        long long z0 = (long long)r * per, z1 = min(S.zero_n, z0 + per);
-        for (long long i = z0 + tid; i < z1; i += nth)
-            S.zero[i] = 0.f;
+        const long long nct = (long long)gridDim.x * gridDim.y, ct = (long long)blockIdx.y * gridDim.x + blockIdx.x;
+        const long long per = ((S.zero_n + nct - 1) / nct + 3) & ~3LL;
+        const long long z0 = ct * per, z1 = min(S.zero_n, z0 + per);
+        if ((S.zero_n & 3) == 0 && ((uintptr_t)S.zero & 15) == 0) {
+            for (long long i = z0 + 4 * tid; i < z1; i += 4 * 256)
+                *reinterpret_cast<float4 *>(S.zero + i) = make_float4(0.f, 0.f, 0.f, 0.f);
+        } else {
+            for (long long i = z0 + tid; i < z1; i += 256)
+                S.zero[i] = 0.f;
+        }
     }
     const bool live = r < a.M;
-    float mx = 0.f;
-    if (live) {
+    if (S.kind == PREP_RMSNORM && live) {
+        // the whole row's mean square, recomputed by every CTA of the row in the same order
+        const float4 *h4 = reinterpret_cast<const float4 *>(S.xf + (size_t)r * S.ldx);
+        float ss = 0.f;
+        for (int i = tid; i < (K >> 2); i += 256) {
+            const float4 v = h4[i];
+            ss = fmaf(v.x, v.x, ss);
+            ss = fmaf(v.y, v.y, ss);
+            ss = fmaf(v.z, v.z, ss);
+            ss = fmaf(v.w, v.w, ss);
+        }
+        ss = warp_sum(ss);
+        if ((tid & 31) == 0)
+            red[tid >> 5] = ss;
+        __syncthreads();
+        if (tid == 0) {
+            float tot = 0.f;
+            for (int w = 0; w < 8; ++w)
+                tot += red[w];
+            s_inv = 1.f / sqrtf(tot / (float)K + S.eps);
+        }
+        __syncthreads();
+    }
+    const bool act = live && b < nblk;
+    const int k = 256 * b + 4 * t;
+    uint16_t v[4] = {0, 0, 0, 0};
+    if (act) {
         if (S.kind == PREP_BF16) {
-            const uint16_t *x = S.xb + (size_t)r * S.ldx;
-            for (int k = tid; k < K; k += nth) {
-                const uint16_t v = x[k];
-                sxb[k] = v;
-                mx = fmaxf(mx, fabsf(bf16_to_f(v)));
-            }
+            const uint2 w = *reinterpret_cast<const uint2 *>(S.xb + (size_t)r * S.ldx + k);
+            v[0] = (uint16_t)(w.x & 0xFFFF);
+            v[1] = (uint16_t)(w.x >> 16);
+            v[2] = (uint16_t)(w.y & 0xFFFF);
+            v[3] = (uint16_t)(w.y >> 16);
         } else if (S.kind == PREP_RMSNORM) {
-            const float *h = S.xf + (size_t)r * S.ldx;
-            float ss = 0.f;
-            for (int k = tid; k < K; k += nth) {
-                float v = h[k];
-                ss = fmaf(v, v, ss);
-            }
-            ss = block_sum(ss, red);
-            const float inv = 1.f / sqrtf(ss / (float)K + S.eps);
-            for (int k = tid; k < K; k += nth) {
-                const uint16_t v = f_to_bf16(h[k] * inv);
-                sxb[k] = v;
-                mx = fmaxf(mx, fabsf(bf16_to_f(v)));
-            }
-        } else {
+            const float4 h = *reinterpret_cast<const float4 *>(S.xf + (size_t)r * S.ldx + k);
+            const float inv = s_inv;
+            v[0] = f_to_bf16(h.x * inv);
+            v[1] = f_to_bf16(h.y * inv);
+            v[2] = f_to_bf16(h.z * inv);
+            v[3] = f_to_bf16(h.w * inv);
+        } else if (S.kind == PREP_SILU) {
             const float *gp = S.xf + (size_t)r * S.ldx;
-            for (int k = tid; k < K; k += nth) {
-                const float gg = gp[k], uu = gp[K + k];
-                float r;
-                if (gg >= -80.f) {
-                    r = gg / (1.f + expf(-gg)) * uu;
-                } else {
-                    // 1 + e^-g == e^-g in fp32 here; e^-g would overflow below -88, so
-                    // form g*u*e^g in the log domain (exact zero stays zero)
-                    const float p = gg * uu;
-                    r = p == 0.f ? p : copysignf(expf(gg + logf(fabsf(p))), p);
+            const float4 g = *reinterpret_cast<const float4 *>(gp + k);
+            const float4 u = *reinterpret_cast<const float4 *>(gp + K + k);
+            v[0] = f_to_bf16(silu_mul(g.x, u.x));
+            v[1] = f_to_bf16(silu_mul(g.y, u.y));
+            v[2] = f_to_bf16(silu_mul(g.z, u.z));
+            v[3] = f_to_bf16(silu_mul(g.w, u.w));
+        } else {
+            // merge the key splits of query vector (row r, head k / 128), dims k%128 .. +3
+            const AttnPartView &P = S.att;
+            int ag = 0;
+            while (ag + 1 < S.n_agents && P.ars[ag + 1] <= r)
+                ++ag;
+            const int na = P.ars[ag + 1] - P.ars[ag], j = r - P.ars[ag];
+            const int head = k >> 7, d = k & 127;
+            const int g = head / P.G, hl = head - g * P.G;
+            const int qi = j * P.G + hl, rg = qi / ATT_QG, qq = qi - rg * ATT_QG;
+            const int L = min(P.lens[ag] + na, P.kv_cap);
+            const int nsp = (L + P.CH - 1) / P.CH;
+            const float *base = P.part + ((((size_t)ag * P.n_kvh + g) * P.n_rg + rg) * P.max_splits) * ATT_PART_FLOATS;
+            float Mx = -INFINITY;
+            for (int sp = 0; sp < nsp; ++sp)
+                Mx = fmaxf(Mx, base[(size_t)sp * ATT_PART_FLOATS + ATT_QG * 128 + qq]);
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            float Ls = 0.f;
+            if (Mx != -INFINITY)
+                for (int sp = 0; sp < nsp; ++sp) {
+                    const float *pp = base + (size_t)sp * ATT_PART_FLOATS;
+                    const float wgt = exp2f(pp[ATT_QG * 128 + qq] - Mx);
+                    const float4 o = *reinterpret_cast<const float4 *>(pp + qq * 128 + d);
+                    acc.x += wgt * o.x;
+                    acc.y += wgt * o.y;
+                    acc.z += wgt * o.z;
+                    acc.w += wgt * o.w;
+                    Ls += wgt * pp[ATT_QG * 128 + ATT_QG + qq];
                 }
-                const uint16_t v = f_to_bf16(r);
-                sxb[k] = v;
-                mx = fmaxf(mx, fabsf(bf16_to_f(v)));
-            }
+            const bool pos = Ls > 0.f;
+            v[0] = f_to_bf16(pos ? acc.x / Ls : 0.f);
+            v[1] = f_to_bf16(pos ? acc.y / Ls : 0.f);
+            v[2] = f_to_bf16(pos ? acc.z / Ls : 0.f);
+            v[3] = f_to_bf16(pos ? acc.w / Ls : 0.f);
         }
         if (S.dbg)
-            for (int k = tid; k < K; k += nth)
-                S.dbg[(size_t)r * S.ld_dbg + k] = sxb[k];
+            *reinterpret_cast<uint2 *>(S.dbg + (size_t)r * S.ld_dbg + k) =
+                make_uint2(v[0] | (uint32_t)v[1] << 16, v[2] | (uint32_t)v[3] << 16);
     }
-    mx = block_max(mx, red);
+    float x[4];
+    float mx = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        x[i] = bf16_to_f(v[i]);
+        mx = fmaxf(mx, fabsf(x[i]));
+    }
+    // max over the block's two warps
+    mx = warp_max(mx);
+    if ((tid & 31) == 0)
+        red[tid >> 5] = mx;
+    __syncthreads();
+    mx = fmaxf(red[2 * q], red[2 * q + 1]);
     int e = 0;
     if (mx > 0.f) {
         int E;
         frexpf(mx, &E);  // mx in [2^(E-1), 2^E)
         e = min(126, max(-126, 10 - E));
     }
+    if (b >= nblk)
+        return;
     const float sc = ldexpf(1.f, e);
-    if (tid == 0)
-        a.fb.rs[r] = live ? ldexpf(1.f, -e) : 0.f;
-    __syncthreads();
+    uint8_t *rec = a.fb.rec + (size_t)b * rec_bytes(FMT, NT);
     const int g = r & 7, nt = r >> 3;
-    uint2 *xp = reinterpret_cast<uint2 *>(a.fb.xp);
-    for (int it = tid; it < nblk * 64; it += nth) {
-        const int b = it >> 6, s = (it >> 2) & 15, c = it & 3;
-        uint2 v = make_uint2(0u, 0u);
-        if (live) {
-            const int k = 256 * b + frag_k0<FMT>(s, c);
-            v.x = pack_half2(bf16_to_f(sxb[k]) * sc, bf16_to_f(sxb[k + 2]) * sc);
-            v.y = pack_half2(bf16_to_f(sxb[k + 1]) * sc, bf16_to_f(sxb[k + 3]) * sc);
-        }
-        xp[((((size_t)b * 16 + s) * 8 + g) * 4 + c) * NT + nt] = v;
-    }
+    const int s = slot_s(FMT, t), c = slot_c(FMT, t);
+    const float h0 = round_half(x[0] * sc), h1 = round_half(x[1] * sc), h2 = round_half(x[2] * sc),
+                h3 = round_half(x[3] * sc);
+    reinterpret_cast<uint2 *>(rec)[((s * 8 + g) * 4 + c) * NT + nt] =
+        make_uint2(pack_half2(h0, h2), pack_half2(h1, h3));
     if (FMT == 4) {
-        uint2 *sp = reinterpret_cast<uint2 *>(a.fb.sp);
-        for (int it = tid; it < nblk * 4; it += nth) {
-            const int b = it >> 2, c = it & 3;
-            uint2 v = make_uint2(0u, 0u);
-            if (live) {
-                const uint16_t *x0 = sxb + 256 * b + 64 * c;
-                float s0 = 0.f, s1 = 0.f;
-                for (int k = 0; k < 32; ++k) {
-                    s0 += round_half(bf16_to_f(x0[k]) * sc);
-                    s1 += round_half(bf16_to_f(x0[32 + k]) * sc);
-                }
-                const float h0 = round_half(s0), h1 = round_half(s1);
-                v.x = pack_half2(h0, h1);
-                v.y = pack_half2(s0 - h0, s1 - h1);
-            }
-            sp[(((size_t)b * 8 + g) * 4 + c) * NT + nt] = v;
+        // sub-block j = t >> 3 is the 8 lanes t & ~7 .. +7 (fp32 sum of its fp16 values)
+        float sj = (h0 + h1) + (h2 + h3);
+        sj += __shfl_xor_sync(0xffffffffu, sj, 1);
+        sj += __shfl_xor_sync(0xffffffffu, sj, 2);
+        sj += __shfl_xor_sync(0xffffffffu, sj, 4);
+        const float sj1 = __shfl_down_sync(0xffffffffu, sj, 8);  // sub-block j + 1
+        if ((t & 15) == 0) {
+            const float hi0 = round_half(sj), hi1 = round_half(sj1);
+            reinterpret_cast<uint2 *>(rec + 4096 * NT)[(g * 4 + c) * NT + nt] =
+                make_uint2(pack_half2(hi0, hi1), pack_half2(sj - hi0, sj1 - hi1));
         }
     }
+    if (t == 0)
+        reinterpret_cast<float *>(rec + rec_bytes(FMT, NT) - 64)[r] = live ? ldexpf(1.f, -e) : 0.f;
 }
 
 // ------------------------------------------------------------- GEMM kernels
@@ -273,9 +321,13 @@ template <int FMT, int NT>
 struct Stage {
     static constexpr int W_BYTES = TILE_ROWS * (FMT == 4 ? 144 : Q6A_BYTES);
     static constexpr int D_BYTES = FMT == 4 ? 0 : TILE_ROWS * 16;   // 8 fp16 d per row (aligned group of 8 blocks)
-    static constexpr int X_BYTES = 4096 * NT;                       // [s 16][g 8][c 4][nt][2 words]
-    static constexpr int S_BYTES = FMT == 4 ? 256 * NT : 0;         // [g 8][c 4][nt][2 words]
-    static constexpr int BYTES = W_BYTES + D_BYTES + X_BYTES + S_BYTES;
+    static constexpr int X_BYTES = 4096 * NT;                       // the block's operand record:
+    static constexpr int S_BYTES = FMT == 4 ? 256 * NT : 0;         //   X, S, then 16 row scales
+    static constexpr int R_BYTES = rec_bytes(FMT, NT);
+    // every stage starts on a 128-byte boundary (tensor-map copy destinations)
+    static constexpr int COPY_BYTES = W_BYTES + D_BYTES + R_BYTES;  // what lands per unit
+    static constexpr int BYTES = (COPY_BYTES + 127) / 128 * 128;
+    static_assert(W_BYTES % 128 == 0 && D_BYTES % 128 == 0 && R_BYTES % 16 == 0, "stage field alignment");
 };
 
 template <int FMT>
@@ -296,8 +348,7 @@ struct WeightMaps {
 
 struct GemmArgs {
     int N, nblk, M, ldy, units;
-    const uint32_t *xp, *sp;
-    const float *rs;
+    const uint8_t *rec;  // operand records, rec_bytes(FMT, NT) apart
     float *Y;
 };
 
@@ -313,7 +364,7 @@ __device__ __forceinline__ void flush_rows(float (&tot)[NT][4], const GemmArgs &
             const int n = n0 + g + 8 * (e >> 1);
             const int r = 8 * nt + 2 * c + (e & 1);
             if (n < a.N && r < a.M)
-                atomicAdd(a.Y + (size_t)r * a.ldy + n, a.rs[r] * tot[nt][e]);
+                atomicAdd(a.Y + (size_t)r * a.ldy + n, tot[nt][e]);
             tot[nt][e] = 0.f;
         }
 }
@@ -341,9 +392,21 @@ __device__ __forceinline__ uint32_t u4w(const uint4 &v, int i)
 
 // One Q4_K block of this warp's 16 rows against all activation rows.
 // W16: the warp's first row in the stage; XS/SS: the block's fragments.
+// Row scales 2^-e(r,b) of the four accumulator rows this lane owns per n-tile.
 template <int NT>
-__device__ __forceinline__ void q4_block(const uint8_t *W16, const uint8_t *XS, const uint8_t *SS, int g, int c,
-                                         uint32_t selT, bool hib, float (&tot)[NT][4])
+__device__ __forceinline__ void lds_rs(const uint8_t *RS, int c, float (&rs)[NT][2])
+{
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        const float2 v = lds_v2f(RS + 4 * (8 * nt + 2 * c));
+        rs[nt][0] = v.x;
+        rs[nt][1] = v.y;
+    }
+}
+
+template <int NT>
+__device__ __forceinline__ void q4_block(const uint8_t *W16, const uint8_t *XS, const uint8_t *SS, const uint8_t *RS,
+                                         int g, int c, uint32_t selT, bool hib, float (&tot)[NT][4])
 {
     uint4 hdr[2], q0[2], q1[2];
 #pragma unroll
@@ -417,6 +480,8 @@ __device__ __forceinline__ void q4_block(const uint8_t *W16, const uint8_t *XS, 
     // mins: sum_j m_j * S_j, S split into two fp16 parts along k
     uint32_t sb[NT][2];
     lds_b<NT>(SS + (g * 4 + c) * 8 * NT, sb);
+    float rs[NT][2];
+    lds_rs<NT>(RS, c, rs);
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
         float accm[4];
@@ -424,8 +489,8 @@ __device__ __forceinline__ void q4_block(const uint8_t *W16, const uint8_t *XS, 
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const int rh = e >> 1;
-            tot[nt][e] = fmaf(dd[rh], acc[nt][e], tot[nt][e]);
-            tot[nt][e] = fmaf(-dm[rh], accm[e], tot[nt][e]);
+            const float y = fmaf(dd[rh], acc[nt][e], -dm[rh] * accm[e]);
+            tot[nt][e] = fmaf(rs[nt][e & 1], y, tot[nt][e]);
         }
     }
 }
@@ -435,8 +500,8 @@ constexpr uint32_t H2_1152 = 0x64806480u;  // 1152.0
 // One Q6_K-like block (packed layout) of this warp's 16 rows. A16: the warp's
 // first row in plane A of the stage; D16: its first row of the d tile.
 template <int NT>
-__device__ __forceinline__ void q6_block(const uint8_t *A16, const uint8_t *D16, int bsub, const uint8_t *XS, int g,
-                                         int c, float (&tot)[NT][4])
+__device__ __forceinline__ void q6_block(const uint8_t *A16, const uint8_t *D16, int bsub, const uint8_t *XS,
+                                         const uint8_t *RS, int g, int c, float (&tot)[NT][4])
 {
     uint4 QL0[2], QL1[2], QH[2];
     uint32_t SC[2][4];
@@ -493,11 +558,13 @@ __device__ __forceinline__ void q6_block(const uint8_t *A16, const uint8_t *D16,
             }
         }
     }
+    float rs[NT][2];
+    lds_rs<NT>(RS, c, rs);
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-            tot[nt][e] = fmaf(dd[e >> 1], acc[nt][e], tot[nt][e]);
+            tot[nt][e] = fmaf(dd[e >> 1] * rs[nt][e & 1], acc[nt][e], tot[nt][e]);
 }
 
 template <int FMT, int NT>
@@ -532,18 +599,13 @@ __global__ void __launch_bounds__(32 * (CG * GW + 1), 1) k_qgemm(const __grid_co
             uint8_t *st = smem + (size_t)(i % S) * St::BYTES;
             uint64_t *bar = &full[i % S];
             if (weights) {
-                mbar_arrive_expect_tx(bar, (uint32_t)St::BYTES);
+                mbar_arrive_expect_tx(bar, (uint32_t)St::COPY_BYTES);
                 tma_load_2d(st, &maps.w, b * (FMT == 4 ? 144 : Q6A_BYTES), t * TILE_ROWS, bar);
                 if (FMT == 6)
                     tma_load_2d(st + St::W_BYTES, &maps.d, b & ~7, t * TILE_ROWS, bar);
             }
-            if (frags) {
-                uint8_t *xs = st + St::W_BYTES + St::D_BYTES;
-                bulk_g2s(xs, reinterpret_cast<const uint8_t *>(a.xp) + (size_t)b * St::X_BYTES, St::X_BYTES, bar);
-                if (FMT == 4)
-                    bulk_g2s(xs + St::X_BYTES, reinterpret_cast<const uint8_t *>(a.sp) + (size_t)b * St::S_BYTES,
-                             St::S_BYTES, bar);
-            }
+            if (frags)
+                bulk_g2s(st + St::W_BYTES + St::D_BYTES, a.rec + (size_t)b * St::R_BYTES, St::R_BYTES, bar);
         };
         const int pre = min(S, n_units);
         int t = n_units > 0 ? u0 / a.nblk : 0, b = u0 - t * a.nblk;
@@ -607,11 +669,12 @@ __global__ void __launch_bounds__(32 * (CG * GW + 1), 1) k_qgemm(const __grid_co
             return;
         }
         const uint8_t *XS = st + St::W_BYTES + St::D_BYTES;
+        const uint8_t *RS = XS + St::R_BYTES - 64;
         if (FMT == 4)
-            q4_block<NT>(st + (size_t)(16 * wi) * 144, XS, XS + St::X_BYTES, g, c, selT, hib, tot);
+            q4_block<NT>(st + (size_t)(16 * wi) * 144, XS, XS + St::X_BYTES, RS, g, c, selT, hib, tot);
         else
-            q6_block<NT>(st + (size_t)(16 * wi) * Q6A_BYTES, st + St::W_BYTES + (size_t)(16 * wi) * 16, b & 7, XS, g,
-                         c, tot);
+            q6_block<NT>(st + (size_t)(16 * wi) * Q6A_BYTES, st + St::W_BYTES + (size_t)(16 * wi) * 16, b & 7, XS, RS,
+                         g, c, tot);
         __syncwarp();
         if (lane == 0)
             mbar_arrive(&empty[i % S]);
@@ -673,28 +736,14 @@ int launch_prep(int fmt, int K, int M, const PrepSrc &src, const FragBuf &fb, cu
 {
     const int nt = frag_nt(M);
     PrepArgs a{src, K, M, fb};
-    const size_t smem = (size_t)K * sizeof(uint16_t);
     void (*kern)(PrepArgs);
     if (fmt == 4)
         kern = nt == 1 ? k_prep<4, 1> : k_prep<4, 2>;
     else
         kern = nt == 1 ? k_prep<6, 1> : k_prep<6, 2>;
-    if (smem > 48 * 1024) {
-        // once per (device, kernel variant): room for the longest row (K <= 65536)
-        static bool done[64][4] = {};
-        int dev = 0;
-        cudaGetDevice(&dev);
-        const int v = (fmt == 4 ? 0 : 2) + (nt - 1);
-        if (dev < 0 || dev >= 64 || !done[dev][v]) {
-            int rc = set_smem(kern, (size_t)65536 * sizeof(uint16_t));
-            if (rc)
-                return rc;
-            if (dev >= 0 && dev < 64)
-                done[dev][v] = true;
-        }
-    }
-    cudaError_t e = pdl ? launch_pdl(kern, dim3(8 * nt), dim3(512), smem, s, a)
-                        : (kern<<<8 * nt, 512, smem, s>>>(a), cudaGetLastError());
+    const dim3 grid((K / 256 + 3) / 4, 8 * nt);
+    cudaError_t e = pdl ? launch_pdl(kern, grid, dim3(256), 0, s, a)
+                        : (kern<<<grid, 256, 0, s>>>(a), cudaGetLastError());
     return cuda_check(e, "prep launch");
 }
 
@@ -725,9 +774,7 @@ int launch_gemm(int fmt, const WeightMapsBlob &maps_blob, int N, int K, int M, c
     a.M = M;
     a.ldy = ldy;
     a.units = ((N + TILE_ROWS - 1) / TILE_ROWS) * a.nblk;
-    a.xp = fb.xp;
-    a.sp = fb.sp;
-    a.rs = fb.rs;
+    a.rec = fb.rec;
     a.Y = Y;
     void (*kern)(const WeightMaps, GemmArgs);
     size_t smem;
@@ -822,6 +869,8 @@ static int gemm_entry(int fmt, const void *W, int N, int K, const uint16_t *X, i
         return qad::fail(QAD_ERR_INVALID, "%s: workspace must be 256-byte aligned", name);
     if ((uintptr_t)W & 15)
         return qad::fail(QAD_ERR_INVALID, "%s: weights must be 16-byte aligned", name);
+    if ((uintptr_t)X & 7)
+        return qad::fail(QAD_ERR_INVALID, "%s: activations must be 8-byte aligned", name);
     if (ws_bytes < qad_gemm_ws_bytes(K, M))
         return qad::fail(QAD_ERR_WORKSPACE, "%s: workspace %zu < %zu bytes", name, ws_bytes, qad_gemm_ws_bytes(K, M));
     qad::WeightMapsBlob maps;

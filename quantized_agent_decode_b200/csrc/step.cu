@@ -11,12 +11,12 @@
 // programmatic dependent launch (each GEMM starts streaming its weights while
 // its producer drains) and replayed as one CUDA graph.
 //
-// Per layer (rounding points as in the layer definition of qad.h):
+// Per layer, nine launches (rounding points as in the layer definition of qad.h):
 //   prep(rmsnorm h)          -> fp16 fragments; zeroes the qkv buffer
 //   q4k_gemm(Wqkv)           -> qkv fp32 (atomic partial sums)
-//   qkv_post                 -> Q bf16; k, v bf16 appended at each row's position
-//   decode_attn + combine    -> O bf16
-//   prep(O)                  -> fragments
+//   decode_attn (fused)      -> per-split partials; Q, k, v rounded to bf16 from
+//                               qkv, k and v appended at each row's position
+//   prep(merge splits -> O)  -> O bf16 -> fragments
 //   q4k_gemm(Wo)             -> h += ...
 //   prep(rmsnorm h)          -> fragments; zeroes the gate|up buffer
 //   q4k_gemm(Wgu)            -> gate|up fp32
@@ -33,9 +33,7 @@ struct qad_step_graph {
 };
 
 // Kernel classes timed by the optional per-launch event profiler.
-enum ProfKind {
-    PK_INIT = 0, PK_PREP, PK_GEMM_QKV, PK_QKV_POST, PK_ATTN, PK_GEMM_O, PK_GEMM_GU, PK_GEMM_DOWN, PK_COUNT
-};
+enum ProfKind { PK_INIT = 0, PK_PREP, PK_GEMM_QKV, PK_ATTN, PK_GEMM_O, PK_GEMM_GU, PK_GEMM_DOWN, PK_COUNT };
 
 struct qad_model {
     qad_model_desc d;
@@ -64,7 +62,7 @@ namespace qad {
 static inline size_t a256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct StepLayout {
-    size_t qkv, qb, ob, gu, frag, part, x_in, ars_in, lens_in, h_out, total;
+    size_t qkv, gu, frag, part, x_in, ars_in, lens_in, h_out, total;
     AttnPlan plan;
 };
 
@@ -90,10 +88,6 @@ static StepLayout step_layout(const qad_model_desc &d, int M)
     size_t off = 0;
     L.qkv = off;
     off += a256((size_t)M * nqkv * 4);
-    L.qb = off;
-    off += a256((size_t)M * nq * 2);
-    L.ob = off;
-    off += a256((size_t)M * nq * 2);
     L.gu = off;
     off += a256((size_t)M * 2 * d.inter * 4);
     L.frag = off;
@@ -155,34 +149,6 @@ __global__ void k_init_h(const uint16_t *__restrict__ X, float *__restrict__ h, 
         h[i] = bf16_to_f(X[i]);
 }
 
-// Split the fused q|k|v projection of row r: Q as bf16 for attention, and the
-// row's k and v as bf16 appended to its agent's cache at position len + j.
-__global__ void k_qkv_post(const float *__restrict__ qkv, uint16_t *__restrict__ Qb, uint16_t *__restrict__ Kc,
-                           uint16_t *__restrict__ Vc, const int *__restrict__ ars, const int *__restrict__ lens,
-                           int n_agents, int nq, int nkv, int n_kvh, int hd, int kv_cap)
-{
-    const int r = blockIdx.x;
-    pdl_trigger();
-    pdl_wait();
-    int a = 0;
-    while (a < n_agents && !(ars[a] <= r && r < ars[a + 1]))
-        ++a;
-    if (a == n_agents)
-        return;
-    const int pos = lens[a] + (r - ars[a]);
-    const float *src = qkv + (size_t)r * (nq + 2 * nkv);
-    for (int i = threadIdx.x; i < nq; i += blockDim.x)
-        Qb[(size_t)r * nq + i] = f_to_bf16(src[i]);
-    if (pos < 0 || pos >= kv_cap)
-        return;
-    for (int i = threadIdx.x; i < nkv; i += blockDim.x) {
-        const int g = i / hd, dd = i - g * hd;
-        const size_t dst = (((size_t)a * n_kvh + g) * kv_cap + pos) * hd + dd;
-        Kc[dst] = f_to_bf16(src[nq + i]);
-        Vc[dst] = f_to_bf16(src[nq + nkv + i]);
-    }
-}
-
 // Profiler: events around each launch (serialises the chain; eager steps only).
 struct Prof {
     qad_model *m;
@@ -228,7 +194,6 @@ static int run_step(qad_model *m, const uint16_t *X, int M, const int *ars, int 
     const StepLayout L = step_layout(d, M);
     const int nt = frag_nt(M);
     float *qkv = (float *)(ws + L.qkv), *gu = (float *)(ws + L.gu);
-    uint16_t *Qb = (uint16_t *)(ws + L.qb), *Ob = (uint16_t *)(ws + L.ob);
     float *part = (float *)(ws + L.part);
     const AttnPlan plan = attn_plan(n_agents, d.n_qh, d.n_kvh, d.kv_cap, max_rows);
     const float scale = 1.0f / sqrtf((float)hd);
@@ -267,22 +232,17 @@ static int run_step(qad_model *m, const uint16_t *X, int M, const int *ars, int 
         QAD_PROF(PK_GEMM_QKV, launch_gemm(4, m->mqkv[l], nqkv, H, M, fb, qkv, nqkv, s, true));
         if (dbg && (rc = copy_d2d(dbg + DL.qkv, qkv, (size_t)M * nqkv * 4, s)))
             return rc;
-        // Q, and k/v appended to the caches
-        QAD_PROF(PK_QKV_POST, cuda_check(launch_pdl(k_qkv_post, dim3(M), dim3(256), 0, s, (const float *)qkv, Qb,
-                                                     m->kc[l], m->vc[l], ars, lens, n_agents, nq, nkv, d.n_kvh, hd,
-                                                     d.kv_cap),
-                                          "qkv_post launch"));
-        // attention over each agent's cache
-        QAD_PROF(PK_ATTN, launch_attn(plan, Qb, m->kc[l], m->vc[l], lens, ars, n_agents, d.kv_cap, d.n_qh, d.n_kvh,
-                                      scale, Ob, part, s, true));
-        if (dbg && (rc = copy_d2d(dbg + DL.attn, Ob, (size_t)M * nq * 2, s)))
-            return rc;
-        // h += O Wo^T
+        // attention over each agent's cache; k, v of the new rows appended
+        QAD_PROF(PK_ATTN, launch_attn_fused(plan, qkv, nqkv, m->kc[l], m->vc[l], lens, ars, n_agents, d.kv_cap,
+                                            d.n_qh, d.n_kvh, scale, part, s, true));
+        // O = merged splits (bf16); h += O Wo^T
         fb = frag_carve(ws + L.frag, nq, nt);
         src = PrepSrc{};
-        src.kind = PREP_BF16;
-        src.xb = Ob;
-        src.ldx = nq;
+        src.kind = PREP_ATTN;
+        src.att = attn_part_view(plan, part, ars, lens, d.kv_cap, d.n_qh, d.n_kvh);
+        src.n_agents = n_agents;
+        src.dbg = dbg ? (uint16_t *)(dbg + DL.attn) : nullptr;
+        src.ld_dbg = nq;
         QAD_PROF(PK_PREP, launch_prep(4, nq, M, src, fb, s, true));
         QAD_PROF(PK_GEMM_O, launch_gemm(4, m->mo[l], H, nq, M, fb, h, H, s, true));
         if (dbg && (rc = copy_d2d(dbg + DL.hmid, h, (size_t)M * H * 4, s)))
@@ -335,6 +295,8 @@ static int check_step_args(const qad_model *m, const void *X, int M, const void 
         return fail(QAD_ERR_UNSUPPORTED, "decode_step: rows per agent x group exceeds 96");
     if ((uintptr_t)ws & 255)
         return fail(QAD_ERR_INVALID, "decode_step: workspace must be 256-byte aligned");
+    if ((uintptr_t)H_out & 15)
+        return fail(QAD_ERR_INVALID, "decode_step: H_out must be 16-byte aligned");
     if (ws_bytes < step_layout(m->d, M).total)
         return fail(QAD_ERR_WORKSPACE, "decode_step: workspace %zu < %zu bytes", ws_bytes, step_layout(m->d, M).total);
     return QAD_OK;
@@ -427,6 +389,8 @@ extern "C" int qad_model_set_debug(qad_model *m, void *dbg, size_t bytes)
 {
     if (!m)
         return qad::fail(QAD_ERR_INVALID, "qad_model_set_debug: null model");
+    if ((uintptr_t)dbg & 255)
+        return qad::fail(QAD_ERR_INVALID, "qad_model_set_debug: buffer must be 256-byte aligned");
     m->dbg = dbg;
     m->dbg_bytes = bytes;
     return QAD_OK;
@@ -449,7 +413,7 @@ extern "C" int qad_decode_step_launches(const qad_model *m)
 {
     if (!m)
         return 0;
-    return 1 + 11 * m->d.n_layers;
+    return 1 + 9 * m->d.n_layers;
 }
 
 extern "C" int qad_step_graph_create(qad_model *m, const uint16_t *X, int M, const int *agent_row_start, int n_agents,
