@@ -304,6 +304,36 @@ def run_reference(args, ws, rank):
 
 # ------------------------------------------------------------------ GPU arm
 
+def time_gate_up(w, stream, reps=5):
+    """Device time per gate|up call (prep + Q4_K GEMM) over the stack's 64 matrices:
+    the calls are captured once as a graph and replayed; returns (us per call,
+    algorithmic bytes per call: weights + bf16 input rows + fp32 output rows)."""
+    import quantized_agent_decode_b200 as q
+    sh = w.shape
+    N, K, M = 2 * sh.inter, sh.hidden, w.M
+    X = synth.bf16_normal_torch(synth.torch_gen(w.seed, "cuda", 4242), (M, K), "cuda")
+    Y = torch.zeros(M, N, device="cuda")
+    ws = q.alloc_ws(q.gemm_ws_bytes(K, M))
+    with torch.cuda.stream(stream):
+        for W in w.w_gu:
+            q.q4k_gemm(W, N, K, X, M, Y, ws=ws, stream=stream)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            for W in w.w_gu:
+                q.q4k_gemm(W, N, K, X, M, Y, ws=ws, stream=stream)
+        graph.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            graph.replay()
+        e1.record(stream)
+    stream.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / (reps * len(w.w_gu))
+    nbytes = w.w_gu[0].numel() + M * K * 2 + M * N * 4
+    del graph
+    return us, nbytes
+
+
 def run_gpu(args, ws, rank, local):
     import quantized_agent_decode_b200 as q
     from quantized_agent_decode_b200 import build
@@ -313,20 +343,6 @@ def run_gpu(args, ws, rank, local):
     w = Workload(args.workload)
     stream = torch.cuda.Stream()
     torch.cuda.synchronize()
-
-    # per-kernel durations (eager, event-bracketed launches) for the roofline
-    w.model.set_profile(True)
-    with torch.cuda.stream(stream):
-        for _ in range(2):
-            w.step(stream)
-            stream.synchronize()
-            w.model.profile_read()
-        w.model.set_profile(True)  # reset totals after warm-up
-        for _ in range(3):
-            w.step(stream)
-            stream.synchronize()
-            prof = w.model.profile_read()
-    w.model.set_profile(False)
 
     # graph-replayed timed region
     g = w.graph(stream)
@@ -367,19 +383,14 @@ def run_gpu(args, ws, rank, local):
     d2h = Hh.numel() * 4
     g.close()
 
+    # dominant kernel: the gate|up Q4_K GEMM (largest matrix of the layer), timed
+    # over all 64 layers' matrices (6.4 GB, far above L2) as one replayed graph
+    gu_us, gu_bytes = time_gate_up(w, stream)
     if rank != 0:
         return 0
     peak, peak_kind = measured_peaks()
     L = w.shape.n_layers
-    # dominant kernel: the gate|up Q4_K GEMM (largest weight matrix of the layer)
-    gu_ms, gu_n = prof["gemm_gate_up"]
-    gu_bytes = (w.w_gu[0].numel() + w.M * w.shape.hidden * 2 + w.M * 2 * w.shape.inter * 4)
-    gu_avg_s = gu_ms / max(gu_n, 1) / 1e3
-    achieved = gu_bytes / gu_avg_s / 1e9
-    prof_total = sum(v[0] for v in prof.values())
-    shares = {k: round(v[0] / prof_total, 4) for k, v in prof.items()}
-    per_kernel = {k: {"avg_us": round(v[0] / max(v[1], 1) * 1e3, 2), "launches_per_step": v[1] // 3}
-                  for k, v in prof.items()}
+    achieved = gu_bytes / (gu_us * 1e-6) / 1e9
     value = weight_stream_gbs(w.weight_bytes, ws, ms_step)
     cpu = {}
     if ws == 1 and not args.no_cpu_baseline:
@@ -401,14 +412,15 @@ def run_gpu(args, ws, rank, local):
                    "cached_tokens": w.ctx, "weight_bytes_per_step": w.weight_bytes,
                    "kv_bytes_per_step": w.kv_bytes, "parallelism": f"replicas{ws}",
                    "l2": "inputs larger than L2 (13.7 GB of weights per step), no flush"},
-        "roofline": {"bound": "hbm", "kernel": "q4k gate|up GEMM (N=34816, K=5120)",
+        "roofline": {"bound": "hbm", "kernel": "q4k gate|up GEMM (N=34816, K=5120, M=12)",
                      "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_kind": peak_kind,
                      "traffic": kernel_traffic("gemm.cu", "q4k_gemm_gate_up_traffic.json"),
-                     "duration_us": gu_avg_s * 1e6, "bytes_per_launch": gu_bytes,
-                     "timing": "CUDA events around each launch, eager profiled steps"},
+                     "duration_us": gu_us, "bytes_per_launch": gu_bytes,
+                     "timing": "CUDA events on the replaying stream around a graph of the 64 layers' gate|up "
+                               "calls (prep + GEMM each; the time includes the prep)"},
         "step_stream_gbs": (w.weight_bytes + w.kv_bytes) / (ms_step / 1e3) / 1e9,
-        "kernel_shares": shares, "kernels": per_kernel,
+        "kernel_shares": "profiles/step_launches_stack12_ctx1k.md (ncu launch list)",
         "e2e": {"value": weight_stream_gbs(w.weight_bytes, ws, e2e_ms), "unit": "GB/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": w.model.launches() * args.steps,
@@ -428,7 +440,8 @@ KERNELS = {  # single-kernel cases for profiler captures: (format, N, K)
 
 def run_kernel(args):
     """Time one matrix of the stack through the public GEMM entry point (prep +
-    GEMM per call), rotating 8 weight copies so every call streams from HBM."""
+    GEMM per call), rotating 8 weight copies so every call streams from HBM; the
+    8 calls are replayed as one CUDA graph, so the time is device time."""
     import quantized_agent_decode_b200 as q
     from quantized_agent_decode_b200 import build
     build.build()
@@ -443,7 +456,8 @@ def run_kernel(args):
         ars = torch.arange(0, 13, 3, dtype=torch.int32, device="cuda")
         O = torch.zeros(12, n_qh, 128, dtype=torch.bfloat16, device="cuda")
         ws = q.alloc_ws(q.decode_attn_ws_bytes(A, n_qh, n_kvh, cap, 3))
-        fn = lambda i: q.decode_attn(Qd, Kd, Vd, lens, ars, A, 3, cap, n_qh, n_kvh, 128, O, ws=ws)  # noqa: E731
+        fn = lambda i, st: q.decode_attn(Qd, Kd, Vd, lens, ars, A, 3, cap, n_qh, n_kvh, 128, O, ws=ws,  # noqa: E731
+                                         stream=st)
         nbytes = 2 * A * n_kvh * cap * 128 * 2
     else:
         fmt, N, K = KERNELS[args.kernel]
@@ -456,18 +470,29 @@ def run_kernel(args):
         Y = torch.zeros(M, N, device="cuda")
         ws = q.alloc_ws(q.gemm_ws_bytes(K, M))
         gemm = q.q4k_gemm if fmt == 4 else q.q6k_gemm
-        fn = lambda i: gemm(Ws[i % 8], N, K, X, M, Y, ws=ws)  # noqa: E731
+        fn = lambda i, st: gemm(Ws[i % 8], N, K, X, M, Y, ws=ws, stream=st)  # noqa: E731
         nbytes = Ws[0].numel()
-    for i in range(args.warmup):
-        fn(i)
+    # 8 calls (8 weight copies) captured once and replayed: device time only, no host launch cost
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        for i in range(8):
+            fn(i, stream)
+    stream.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(8):
+            fn(i, stream)
+    for _ in range(args.warmup):
+        graph.replay()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for i in range(args.steps):
-        fn(i)
+    reps = max(1, args.steps // 8)
+    e0.record()  # graph.replay() launches on the current stream
+    for _ in range(reps):
+        graph.replay()
     e1.record()
     torch.cuda.synchronize()
-    us = e0.elapsed_time(e1) / args.steps * 1e3
+    us = e0.elapsed_time(e1) / (reps * 8) * 1e3
     print(json.dumps({"kernel": args.kernel, "rows": args.rows, "us_per_call": us,
                       "gbs": nbytes / us / 1e3, "bytes": nbytes, "device_status": q.device_status()}), flush=True)
     return 0

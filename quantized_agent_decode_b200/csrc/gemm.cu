@@ -10,26 +10,29 @@
 // multiply-accumulate hidden under it.
 //
 // Design (sm_100a):
-//  * Each quantized byte is loaded exactly once, by one thread, with 16-byte
-//    streaming loads (Q4_K blocks are 16-byte aligned; the 210-byte Q6_K-like
-//    blocks are read as 4-byte words and realigned with funnel shifts).
+//  * A producer warp streams each unit (a tile of weight rows x one 256-wide
+//    block) into a ring of shared-memory stages with one 2-D tensor-map load
+//    (TMA), plus one bulk copy of that block's activation record; each stage
+//    completes on an mbarrier. Every quantized byte leaves HBM exactly once.
 //  * The block is decoded in registers into fp16 tensor-core operands that are
 //    EXACT: for Q4_K, A = sc_j * q (<= 945) and the mins enter through a second
 //    small MMA against per-sub-block activation sums; for Q6_K, A = sc * (q-32)
-//    (|.| <= 2048 for |sc| <= 64). The fp16 values come from the "1024 + q"
-//    exponent trick (OR of the nibble into the mantissa of 1024.0) followed by
-//    one fused multiply-add that applies the scale.
+//    (|.| <= 4096). The fp16 values come from the "1024 + q" exponent trick (OR
+//    of the nibble into the mantissa of 1024.0) followed by one fused
+//    multiply-add that applies the scale.
 //  * M = 12 rows need ~16 multiply-adds per weight, four times what the FP32
 //    pipes deliver at the HBM rate, so the product runs on the tensor cores as
-//    m16n8k16 warp MMAs (weights = A, the 16 padded activation rows = B).
+//    m16n8k16 warp MMAs (weights = A, the 16 padded activation rows = B). Each
+//    consumer warp owns 32 weight rows (two m16 tiles), so every activation
+//    fragment read from shared memory feeds four MMAs.
 //  * The activations are prepared once per GEMM (k_prep) into fp16 B
 //    fragments in exactly the register order each lane consumes, with a
-//    per-row power-of-two scale so fp16's range always holds them.
-//  * Work is split stream-K style over all warps of a persistent grid (one CTA
-//    per SM): unit = (tile of 16*MT weight rows, one 256-wide block); each warp
-//    takes a contiguous run of units, accumulates in registers, and adds its
-//    partial tile sums into Y with fp32 atomics when its run leaves a tile.
-//  * Programmatic dependent launch: the first unit's weights are requested
+//    power-of-two scale per (row, block) so fp16's range always holds them.
+//  * Work is split stream-K style over a persistent grid (one CTA per SM):
+//    each CTA takes a contiguous run of units, its consumer groups take them
+//    round-robin and accumulate in registers, adding partial tile sums into Y
+//    with fp32 atomics when a group's run leaves a tile.
+//  * Programmatic dependent launch: the first units' weights are requested
 //    before griddepcontrol.wait, so the weight stream starts while the
 //    producer of the activations is still finishing.
 #include <cuda.h>
@@ -37,6 +40,7 @@
 #include <mutex>
 
 #include "gemm.cuh"
+
 
 namespace qad {
 
@@ -312,33 +316,42 @@ __global__ void __launch_bounds__(256) k_prep(PrepArgs a)
 // so every field is 16-byte aligned) followed by plane D [N][ceil8(nblk)] fp16
 // d. 210-byte GGUF blocks cannot be addressed by TMA (16-byte start rule).
 
-constexpr int GW = 8;                // consumer warps per group (16 rows each)
-constexpr int CG = 2;                // consumer groups, taking alternate units
-constexpr int TILE_ROWS = 16 * GW;   // weight rows per CTA unit
+constexpr int RW = 32;               // weight rows per consumer warp (two m16 tiles)
 constexpr int Q6A_BYTES = 208;       // plane A bytes per Q6_K block
+
+// CG consumer groups of GW warps take units round-robin; each warp owns RW
+// weight rows of the unit. Stages are reused every S units and S is a multiple
+// of CG, so unit i and unit i + S (the next use of a stage) belong to the same
+// group: a group never waits on a stage phase whose predecessor it has not
+// itself seen complete (parity waits cannot tell phase u from phase u - 2).
+template <int FMT>
+struct Cfg {
+    static constexpr int GW = 4;                       // warps per consumer group
+    static constexpr int CG = FMT == 4 ? 3 : 2;        // consumer groups
+    static constexpr int TILE = RW * GW;               // weight rows per unit
+    static constexpr int S = 6;                        // pipeline stages
+    static constexpr int THREADS = 32 * (CG * GW + 1);
+    static constexpr int ROW_BYTES = FMT == 4 ? 144 : Q6A_BYTES;
+    static_assert(S % CG == 0, "stage reuse must stay within one consumer group");
+};
 
 template <int FMT, int NT>
 struct Stage {
-    static constexpr int W_BYTES = TILE_ROWS * (FMT == 4 ? 144 : Q6A_BYTES);
-    static constexpr int D_BYTES = FMT == 4 ? 0 : TILE_ROWS * 16;   // 8 fp16 d per row (aligned group of 8 blocks)
-    static constexpr int X_BYTES = 4096 * NT;                       // the block's operand record:
-    static constexpr int S_BYTES = FMT == 4 ? 256 * NT : 0;         //   X, S, then 16 row scales
+    static constexpr int W_BYTES = Cfg<FMT>::TILE * Cfg<FMT>::ROW_BYTES;
+    static constexpr int D_BYTES = FMT == 4 ? 0 : Cfg<FMT>::TILE * 16;  // 8 fp16 d per row (aligned group of 8 blocks)
+    static constexpr int X_BYTES = 4096 * NT;                          // the block's operand record:
+    static constexpr int S_BYTES = FMT == 4 ? 256 * NT : 0;            //   X, S, then 16 row scales
     static constexpr int R_BYTES = rec_bytes(FMT, NT);
+    static constexpr int COPY_BYTES = W_BYTES + D_BYTES + R_BYTES;     // what lands per unit
     // every stage starts on a 128-byte boundary (tensor-map copy destinations)
-    static constexpr int COPY_BYTES = W_BYTES + D_BYTES + R_BYTES;  // what lands per unit
     static constexpr int BYTES = (COPY_BYTES + 127) / 128 * 128;
     static_assert(W_BYTES % 128 == 0 && D_BYTES % 128 == 0 && R_BYTES % 16 == 0, "stage field alignment");
-};
-
-template <int FMT>
-struct Stages {
-    static constexpr int N = FMT == 4 ? 6 : 5;
 };
 
 template <int FMT, int NT>
 constexpr size_t gemm_smem_bytes()
 {
-    return (size_t)Stages<FMT>::N * Stage<FMT, NT>::BYTES + 2 * Stages<FMT>::N * sizeof(uint64_t);
+    return (size_t)Cfg<FMT>::S * Stage<FMT, NT>::BYTES + 2 * Cfg<FMT>::S * sizeof(uint64_t);
 }
 
 struct WeightMaps {
@@ -354,6 +367,7 @@ struct GemmArgs {
 
 enum { ERR_FULL_TIMEOUT = 1, ERR_EMPTY_TIMEOUT = 2 };
 
+// Add a warp's partial sums of 16 weight rows (n0 + g, n0 + g + 8) to Y.
 template <int NT>
 __device__ __forceinline__ void flush_rows(float (&tot)[NT][4], const GemmArgs &a, int n0, int g, int c)
 {
@@ -390,9 +404,7 @@ __device__ __forceinline__ uint32_t u4w(const uint4 &v, int i)
     return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
 }
 
-// One Q4_K block of this warp's 16 rows against all activation rows.
-// W16: the warp's first row in the stage; XS/SS: the block's fragments.
-// Row scales 2^-e(r,b) of the four accumulator rows this lane owns per n-tile.
+// Row scales 2^-e(r,b) of the activation rows this lane's accumulators hold.
 template <int NT>
 __device__ __forceinline__ void lds_rs(const uint8_t *RS, int c, float (&rs)[NT][2])
 {
@@ -404,23 +416,19 @@ __device__ __forceinline__ void lds_rs(const uint8_t *RS, int c, float (&rs)[NT]
     }
 }
 
+// One Q4_K block of this warp's 32 weight rows (tiles mt = 0, 1; this lane
+// decodes rows 16 mt + g and 16 mt + g + 8, indexed q = 2 mt + rh) against
+// all activation rows. W: the warp's first row in the stage; XS/SS/RS: the
+// block's operand record.
 template <int NT>
-__device__ __forceinline__ void q4_block(const uint8_t *W16, const uint8_t *XS, const uint8_t *SS, const uint8_t *RS,
-                                         int g, int c, uint32_t selT, bool hib, float (&tot)[NT][4])
+__device__ __forceinline__ void q4_block(const uint8_t *W, const uint8_t *XS, const uint8_t *SS, const uint8_t *RS,
+                                         int g, int c, uint32_t selT, bool hib, float (&tot)[2][NT][4])
 {
-    uint4 hdr[2], q0[2], q1[2];
+    uint32_t SCl[4], NGl[4], SCh[4], NGh[4], AM[4];
+    float dd[4], dm[4];
 #pragma unroll
-    for (int rh = 0; rh < 2; ++rh) {
-        const uint8_t *row = W16 + (g + 8 * rh) * 144;
-        hdr[rh] = lds_v4(row);
-        q0[rh] = lds_v4(row + 16 + 32 * c);
-        q1[rh] = lds_v4(row + 32 + 32 * c);
-    }
-    uint32_t SCl[2], NGl[2], SCh[2], NGh[2], AM[2];
-    float dd[2], dm[2];
-#pragma unroll
-    for (int rh = 0; rh < 2; ++rh) {
-        const uint4 h = hdr[rh];
+    for (int q = 0; q < 4; ++q) {
+        const uint4 h = lds_v4(W + (16 * (q >> 1) + g + 8 * (q & 1)) * 144);
         // scales/mins of sub-blocks 2c and 2c+1 (bytes (2c)&3, +1 of the packed words)
         const uint32_t scA = h.y & 0x3F3F3F3Fu, mA = h.z & 0x3F3F3F3Fu;
         const uint32_t scB = (h.w & 0x0F0F0F0Fu) | ((h.y >> 2) & 0x30303030u);
@@ -429,150 +437,169 @@ __device__ __forceinline__ void q4_block(const uint8_t *W16, const uint8_t *XS, 
         const uint32_t Tl = prmt(T, 0x64u, 0x4040u);                     // 1024 + sc_lo (x2)
         const uint32_t Th = prmt(T, 0x64u, 0x4141u);                     // 1024 + sc_hi (x2)
         const uint32_t Tm = prmt(T, 0x64u, 0x4342u);                     // 1024 + (m_lo, m_hi)
-        SCl[rh] = hsub2(Tl, H2_1024);                                    // sc_lo
-        NGl[rh] = hmul2(SCl[rh], H2_NEG1024);                            // -1024 sc_lo
-        SCh[rh] = hfma2(Th, H2_SIXTEENTH, H2_NEG64);                     // sc_hi / 16
-        NGh[rh] = hmul2(SCh[rh], H2_NEG1024);                            // -64 sc_hi
-        AM[rh] = hsub2(Tm, H2_1024);                                     // (m_lo, m_hi)
-        dd[rh] = half_lo(h.x);
-        dm[rh] = half_hi(h.x);
+        SCl[q] = hsub2(Tl, H2_1024);                                     // sc_lo
+        NGl[q] = hmul2(SCl[q], H2_NEG1024);                              // -1024 sc_lo
+        SCh[q] = hfma2(Th, H2_SIXTEENTH, H2_NEG64);                      // sc_hi / 16
+        NGh[q] = hmul2(SCh[q], H2_NEG1024);                              // -64 sc_hi
+        AM[q] = hsub2(Tm, H2_1024);                                      // (m_lo, m_hi)
+        dd[q] = half_lo(h.x);
+        dm[q] = half_hi(h.x);
     }
-    float acc[NT][4], acc2[NT][4];  // two independent chains: low and high nibbles
+    float acc[2][NT][4];
     const uint8_t *xl = XS + (g * 4 + c) * 8 * NT;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        uint32_t blo[NT][2], bhi[NT][2];
-        lds_b<NT>(xl + (2 * i) * 256 * NT, blo);
-        lds_b<NT>(xl + (2 * i + 1) * 256 * NT, bhi);
-        const uint32_t w0 = i < 4 ? u4w(q0[0], i) : u4w(q1[0], i - 4);
-        const uint32_t w1 = i < 4 ? u4w(q0[1], i) : u4w(q1[1], i - 4);
-        const uint32_t w0s = w0 >> 8, w1s = w1 >> 8;
-        // low nibbles: sub-block 2c, k-step 2i
-        const uint32_t a0 = hfma2(and_or(w0, 0x000F000Fu, H2_1024), SCl[0], NGl[0]);
-        const uint32_t a1 = hfma2(and_or(w1, 0x000F000Fu, H2_1024), SCl[1], NGl[1]);
-        const uint32_t a2 = hfma2(and_or(w0s, 0x000F000Fu, H2_1024), SCl[0], NGl[0]);
-        const uint32_t a3 = hfma2(and_or(w1s, 0x000F000Fu, H2_1024), SCl[1], NGl[1]);
+    for (int half = 0; half < 2; ++half) {
+        uint4 qw[4];  // quant words 4 half .. 4 half + 3 of this lane's 32 bytes, per row
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            if (i == 0)
-                mma_f16_zero(acc[nt], a0, a1, a2, a3, blo[nt][0], blo[nt][1]);
-            else
-                mma_f16(acc[nt], a0, a1, a2, a3, blo[nt][0], blo[nt][1]);
-        }
-        // high nibbles: sub-block 2c+1, k-step 2i+1
-        const uint32_t c0 = hfma2(and_or(w0, 0x00F000F0u, H2_1024), SCh[0], NGh[0]);
-        const uint32_t c1 = hfma2(and_or(w1, 0x00F000F0u, H2_1024), SCh[1], NGh[1]);
-        const uint32_t c2 = hfma2(and_or(w0s, 0x00F000F0u, H2_1024), SCh[0], NGh[0]);
-        const uint32_t c3 = hfma2(and_or(w1s, 0x00F000F0u, H2_1024), SCh[1], NGh[1]);
+        for (int q = 0; q < 4; ++q)
+            qw[q] = lds_v4(W + (16 * (q >> 1) + g + 8 * (q & 1)) * 144 + 16 + 32 * c + 16 * half);
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            if (i == 0)
-                mma_f16_zero(acc2[nt], c0, c1, c2, c3, bhi[nt][0], bhi[nt][1]);
-            else
-                mma_f16(acc2[nt], c0, c1, c2, c3, bhi[nt][0], bhi[nt][1]);
+        for (int ii = 0; ii < 4; ++ii) {
+            const int i = 4 * half + ii;
+            uint32_t blo[NT][2], bhi[NT][2];
+            lds_b<NT>(xl + (2 * i) * 256 * NT, blo);
+            lds_b<NT>(xl + (2 * i + 1) * 256 * NT, bhi);
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt) {
+                const int q0 = 2 * mt, q1 = 2 * mt + 1;
+                const uint32_t w0 = u4w(qw[q0], ii), w1 = u4w(qw[q1], ii);
+                const uint32_t w0s = w0 >> 8, w1s = w1 >> 8;
+                // low nibbles: sub-block 2c, k-step 2i
+                const uint32_t a0 = hfma2(and_or(w0, 0x000F000Fu, H2_1024), SCl[q0], NGl[q0]);
+                const uint32_t a1 = hfma2(and_or(w1, 0x000F000Fu, H2_1024), SCl[q1], NGl[q1]);
+                const uint32_t a2 = hfma2(and_or(w0s, 0x000F000Fu, H2_1024), SCl[q0], NGl[q0]);
+                const uint32_t a3 = hfma2(and_or(w1s, 0x000F000Fu, H2_1024), SCl[q1], NGl[q1]);
+                // high nibbles: sub-block 2c+1, k-step 2i+1
+                const uint32_t c0 = hfma2(and_or(w0, 0x00F000F0u, H2_1024), SCh[q0], NGh[q0]);
+                const uint32_t c1 = hfma2(and_or(w1, 0x00F000F0u, H2_1024), SCh[q1], NGh[q1]);
+                const uint32_t c2 = hfma2(and_or(w0s, 0x00F000F0u, H2_1024), SCh[q0], NGh[q0]);
+                const uint32_t c3 = hfma2(and_or(w1s, 0x00F000F0u, H2_1024), SCh[q1], NGh[q1]);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    if (i == 0)
+                        mma_f16_zero(acc[mt][nt], a0, a1, a2, a3, blo[nt][0], blo[nt][1]);
+                    else
+                        mma_f16(acc[mt][nt], a0, a1, a2, a3, blo[nt][0], blo[nt][1]);
+                    mma_f16(acc[mt][nt], c0, c1, c2, c3, bhi[nt][0], bhi[nt][1]);
+                }
+            }
         }
     }
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-            acc[nt][e] += acc2[nt][e];
     // mins: sum_j m_j * S_j, S split into two fp16 parts along k
     uint32_t sb[NT][2];
     lds_b<NT>(SS + (g * 4 + c) * 8 * NT, sb);
     float rs[NT][2];
     lds_rs<NT>(RS, c, rs);
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-        float accm[4];
-        mma_f16_zero(accm, AM[0], AM[1], AM[0], AM[1], sb[nt][0], sb[nt][1]);
+    for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int rh = e >> 1;
-            const float y = fmaf(dd[rh], acc[nt][e], -dm[rh] * accm[e]);
-            tot[nt][e] = fmaf(rs[nt][e & 1], y, tot[nt][e]);
+        for (int nt = 0; nt < NT; ++nt) {
+            float accm[4];
+            mma_f16_zero(accm, AM[2 * mt], AM[2 * mt + 1], AM[2 * mt], AM[2 * mt + 1], sb[nt][0], sb[nt][1]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int q = 2 * mt + (e >> 1);
+                const float y = fmaf(dd[q], acc[mt][nt][e], -dm[q] * accm[e]);
+                tot[mt][nt][e] = fmaf(rs[nt][e & 1], y, tot[mt][nt][e]);
+            }
         }
-    }
 }
 
 constexpr uint32_t H2_1152 = 0x64806480u;  // 1152.0
 
-// One Q6_K-like block (packed layout) of this warp's 16 rows. A16: the warp's
-// first row in plane A of the stage; D16: its first row of the d tile.
+// One Q6_K-like block (packed layout) of this warp's 32 weight rows. A: the
+// warp's first row in plane A of the stage; D: its first row of the d tile.
 template <int NT>
-__device__ __forceinline__ void q6_block(const uint8_t *A16, const uint8_t *D16, int bsub, const uint8_t *XS,
-                                         const uint8_t *RS, int g, int c, float (&tot)[NT][4])
+__device__ __forceinline__ void q6_block(const uint8_t *A, const uint8_t *D, int bsub, const uint8_t *XS,
+                                         const uint8_t *RS, int g, int c, float (&tot)[2][NT][4])
 {
-    uint4 QL0[2], QL1[2], QH[2];
-    uint32_t SC[2][4];
-    float dd[2];
+    uint32_t SC[4][4];
+    float dd[4];
     const int h = c >> 1, lq = 16 * (c & 1);
+    const uint32_t j = (uint32_t)(c & 1);
+    const uint32_t sel0 = j | 0x40u | (j << 8) | 0x4000u, sel1 = (j + 2) | 0x40u | ((j + 2) << 8) | 0x4000u;
 #pragma unroll
-    for (int rh = 0; rh < 2; ++rh) {
-        const uint8_t *blk = A16 + (g + 8 * rh) * Q6A_BYTES;
-        QL0[rh] = lds_v4(blk + 64 * h + lq);
-        QL1[rh] = lds_v4(blk + 64 * h + 32 + lq);
-        QH[rh] = lds_v4(blk + 128 + 32 * h + lq);
+    for (int q = 0; q < 4; ++q) {
+        const int row = 16 * (q >> 1) + g + 8 * (q & 1);
+        const uint8_t *blk = A + row * Q6A_BYTES;
         // int8 scales of sub-blocks 8h + 2t + (c&1): bytes (c&1) + 2t of the 8 scale bytes
         const uint2 sw = lds_v2(blk + 192 + 8 * h);
         const uint32_t s0 = sw.x ^ 0x80808080u, s1 = sw.y ^ 0x80808080u;
-        const uint32_t j = (uint32_t)(c & 1);
-        const uint32_t sel0 = j | 0x40u | (j << 8) | 0x4000u, sel1 = (j + 2) | 0x40u | ((j + 2) << 8) | 0x4000u;
         // (sc + 128) + 1024 - 1152 = sc, exact in fp16
-        SC[rh][0] = hsub2(prmt(s0, 0x64u, sel0), H2_1152);
-        SC[rh][1] = hsub2(prmt(s0, 0x64u, sel1), H2_1152);
-        SC[rh][2] = hsub2(prmt(s1, 0x64u, sel0), H2_1152);
-        SC[rh][3] = hsub2(prmt(s1, 0x64u, sel1), H2_1152);
-        const uint32_t dw = lds_u32(D16 + (g + 8 * rh) * 16 + (bsub & 6) * 2);
-        dd[rh] = __half2float(__ushort_as_half((unsigned short)(dw >> ((bsub & 1) * 16))));
+        SC[q][0] = hsub2(prmt(s0, 0x64u, sel0), H2_1152);
+        SC[q][1] = hsub2(prmt(s0, 0x64u, sel1), H2_1152);
+        SC[q][2] = hsub2(prmt(s1, 0x64u, sel0), H2_1152);
+        SC[q][3] = hsub2(prmt(s1, 0x64u, sel1), H2_1152);
+        const uint32_t dw = lds_u32(D + row * 16 + (bsub & 6) * 2);
+        dd[q] = __half2float(__ushort_as_half((unsigned short)(dw >> ((bsub & 1) * 16))));
     }
-    float acc[NT][4];
+    float acc[2][NT][4];
     const uint8_t *xl = XS + (g * 4 + c) * 8 * NT;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        uint32_t qt[2][4];
+    for (int half = 0; half < 2; ++half) {
+        uint2 L0[4], L1[4], HH[4];  // words 2 half, 2 half + 1 of ql (two quarters) and qh, per row
 #pragma unroll
-        for (int rh = 0; rh < 2; ++rh) {
-            const uint32_t l0 = u4w(QL0[rh], i), l1 = u4w(QL1[rh], i), hh = u4w(QH[rh], i);
-            qt[rh][0] = (l0 & 0x0F0F0F0Fu) | ((hh << 4) & 0x30303030u);
-            qt[rh][1] = (l1 & 0x0F0F0F0Fu) | ((hh << 2) & 0x30303030u);
-            qt[rh][2] = ((l0 >> 4) & 0x0F0F0F0Fu) | (hh & 0x30303030u);
-            qt[rh][3] = ((l1 >> 4) & 0x0F0F0F0Fu) | ((hh >> 2) & 0x30303030u);
+        for (int q = 0; q < 4; ++q) {
+            const uint8_t *blk = A + (16 * (q >> 1) + g + 8 * (q & 1)) * Q6A_BYTES;
+            L0[q] = lds_v2(blk + 64 * h + lq + 8 * half);
+            L1[q] = lds_v2(blk + 64 * h + 32 + lq + 8 * half);
+            HH[q] = lds_v2(blk + 128 + 32 * h + lq + 8 * half);
         }
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
-            const int s = 4 * i + t;
-            uint32_t bf[NT][2];
-            lds_b<NT>(xl + s * 256 * NT, bf);
-            // pairs (bytes 0,2) and (bytes 1,3) -> 1024 + q -> q - 32 -> sc*(q-32)
-            const uint32_t a0 = hmul2(hsub2(prmt(qt[0][t], 0x64u, 0x4240u), H2_1056), SC[0][t]);
-            const uint32_t a1 = hmul2(hsub2(prmt(qt[1][t], 0x64u, 0x4240u), H2_1056), SC[1][t]);
-            const uint32_t a2 = hmul2(hsub2(prmt(qt[0][t], 0x64u, 0x4341u), H2_1056), SC[0][t]);
-            const uint32_t a3 = hmul2(hsub2(prmt(qt[1][t], 0x64u, 0x4341u), H2_1056), SC[1][t]);
+        for (int ii = 0; ii < 2; ++ii) {
+            const int i = 2 * half + ii;
+            uint32_t qt[4][4];
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                if (s == 0)
-                    mma_f16_zero(acc[nt], a0, a1, a2, a3, bf[nt][0], bf[nt][1]);
-                else
-                    mma_f16(acc[nt], a0, a1, a2, a3, bf[nt][0], bf[nt][1]);
+            for (int q = 0; q < 4; ++q) {
+                const uint32_t l0 = ii ? L0[q].y : L0[q].x, l1 = ii ? L1[q].y : L1[q].x;
+                const uint32_t hh = ii ? HH[q].y : HH[q].x;
+                qt[q][0] = (l0 & 0x0F0F0F0Fu) | ((hh << 4) & 0x30303030u);
+                qt[q][1] = (l1 & 0x0F0F0F0Fu) | ((hh << 2) & 0x30303030u);
+                qt[q][2] = ((l0 >> 4) & 0x0F0F0F0Fu) | (hh & 0x30303030u);
+                qt[q][3] = ((l1 >> 4) & 0x0F0F0F0Fu) | ((hh >> 2) & 0x30303030u);
+            }
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                const int s = 4 * i + t;
+                uint32_t bf[NT][2];
+                lds_b<NT>(xl + s * 256 * NT, bf);
+#pragma unroll
+                for (int mt = 0; mt < 2; ++mt) {
+                    const int q0 = 2 * mt, q1 = 2 * mt + 1;
+                    // pairs (bytes 0,2) and (bytes 1,3) -> 1024 + q -> q - 32 -> sc*(q-32)
+                    const uint32_t a0 = hmul2(hsub2(prmt(qt[q0][t], 0x64u, 0x4240u), H2_1056), SC[q0][t]);
+                    const uint32_t a1 = hmul2(hsub2(prmt(qt[q1][t], 0x64u, 0x4240u), H2_1056), SC[q1][t]);
+                    const uint32_t a2 = hmul2(hsub2(prmt(qt[q0][t], 0x64u, 0x4341u), H2_1056), SC[q0][t]);
+                    const uint32_t a3 = hmul2(hsub2(prmt(qt[q1][t], 0x64u, 0x4341u), H2_1056), SC[q1][t]);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        if (s == 0)
+                            mma_f16_zero(acc[mt][nt], a0, a1, a2, a3, bf[nt][0], bf[nt][1]);
+                        else
+                            mma_f16(acc[mt][nt], a0, a1, a2, a3, bf[nt][0], bf[nt][1]);
+                    }
+                }
             }
         }
     }
     float rs[NT][2];
     lds_rs<NT>(RS, c, rs);
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+    for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-            tot[nt][e] = fmaf(dd[e >> 1] * rs[nt][e & 1], acc[nt][e], tot[nt][e]);
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                tot[mt][nt][e] = fmaf(dd[2 * mt + (e >> 1)] * rs[nt][e & 1], acc[mt][nt][e], tot[mt][nt][e]);
 }
 
 template <int FMT, int NT>
-__global__ void __launch_bounds__(32 * (CG * GW + 1), 1) k_qgemm(const __grid_constant__ WeightMaps maps, GemmArgs a)
+__global__ void __launch_bounds__(Cfg<FMT>::THREADS, 1) k_qgemm(const __grid_constant__ WeightMaps maps, GemmArgs a)
 {
     extern __shared__ __align__(128) uint8_t smem[];
     using St = Stage<FMT, NT>;
-    constexpr int S = Stages<FMT>::N;
+    using Cf = Cfg<FMT>;
+    constexpr int S = Cf::S, GW = Cf::GW, CG = Cf::CG, TILE = Cf::TILE;
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + (size_t)S * St::BYTES);
     uint64_t *empty = full + S;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -582,7 +609,7 @@ __global__ void __launch_bounds__(32 * (CG * GW + 1), 1) k_qgemm(const __grid_co
     if (threadIdx.x == 0) {
         for (int i = 0; i < S; ++i) {
             mbar_init(&full[i], 1);
-            mbar_init(&empty[i], GW);  // the 8 warps of the consumer group that used the stage
+            mbar_init(&empty[i], GW);  // the warps of the consumer group that used the stage
         }
         mbar_fence_init();
     }
@@ -600,9 +627,9 @@ __global__ void __launch_bounds__(32 * (CG * GW + 1), 1) k_qgemm(const __grid_co
             uint64_t *bar = &full[i % S];
             if (weights) {
                 mbar_arrive_expect_tx(bar, (uint32_t)St::COPY_BYTES);
-                tma_load_2d(st, &maps.w, b * (FMT == 4 ? 144 : Q6A_BYTES), t * TILE_ROWS, bar);
+                tma_load_2d(st, &maps.w, b * Cf::ROW_BYTES, t * TILE, bar);
                 if (FMT == 6)
-                    tma_load_2d(st + St::W_BYTES, &maps.d, b & ~7, t * TILE_ROWS, bar);
+                    tma_load_2d(st + St::W_BYTES, &maps.d, b & ~7, t * TILE, bar);
             }
             if (frags)
                 bulk_g2s(st + St::W_BYTES + St::D_BYTES, a.rec + (size_t)b * St::R_BYTES, St::R_BYTES, bar);
@@ -643,19 +670,21 @@ __global__ void __launch_bounds__(32 * (CG * GW + 1), 1) k_qgemm(const __grid_co
         return;
     }
 
-    // ---------------------------------------------------- consumer groups (alternate units)
+    // ---------------------------------------------------- consumer groups (round-robin units)
     const int grp = warp / GW, wi = warp % GW;
     const int g = lane >> 2, c = lane & 3;
     const int jj = 2 * (c & 1);
     const uint32_t selT = (uint32_t)(jj | ((jj + 1) << 4) | ((jj + 4) << 8) | ((jj + 5) << 12));
     const bool hib = c >= 2;
     pdl_wait();
-    float tot[NT][4];
+    float tot[2][NT][4];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+    for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-            tot[nt][e] = 0.f;
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                tot[mt][nt][e] = 0.f;
     int t = 0, b = 0;
     if (grp < n_units) {
         t = (u0 + grp) / a.nblk;
@@ -671,9 +700,9 @@ __global__ void __launch_bounds__(32 * (CG * GW + 1), 1) k_qgemm(const __grid_co
         const uint8_t *XS = st + St::W_BYTES + St::D_BYTES;
         const uint8_t *RS = XS + St::R_BYTES - 64;
         if (FMT == 4)
-            q4_block<NT>(st + (size_t)(16 * wi) * 144, XS, XS + St::X_BYTES, RS, g, c, selT, hib, tot);
+            q4_block<NT>(st + (size_t)(RW * wi) * 144, XS, XS + St::X_BYTES, RS, g, c, selT, hib, tot);
         else
-            q6_block<NT>(st + (size_t)(16 * wi) * Q6A_BYTES, st + St::W_BYTES + (size_t)(16 * wi) * 16, b & 7, XS, RS,
+            q6_block<NT>(st + (size_t)(RW * wi) * Q6A_BYTES, st + St::W_BYTES + (size_t)(RW * wi) * 16, b & 7, XS, RS,
                          g, c, tot);
         __syncwarp();
         if (lane == 0)
@@ -684,8 +713,10 @@ __global__ void __launch_bounds__(32 * (CG * GW + 1), 1) k_qgemm(const __grid_co
             bn -= a.nblk;
             ++tn;
         }
-        if (tn != t || i + CG >= n_units)
-            flush_rows<NT>(tot, a, t * TILE_ROWS + 16 * wi, g, c);
+        if (tn != t || i + CG >= n_units) {
+            flush_rows<NT>(tot[0], a, t * TILE + RW * wi, g, c);
+            flush_rows<NT>(tot[1], a, t * TILE + RW * wi + 16, g, c);
+        }
         t = tn;
         b = bn;
     }
@@ -753,14 +784,15 @@ int make_weight_maps(int fmt, const void *W, int N, int K, WeightMapsBlob *out)
     WeightMaps *m = reinterpret_cast<WeightMaps *>(out);
     const int nblk = K / 256;
     if (fmt == 4)
-        return encode_tmap_2d(&m->w, W, 1, (uint64_t)nblk * 144, (uint64_t)N, (uint64_t)nblk * 144, 144, TILE_ROWS);
+        return encode_tmap_2d(&m->w, W, 1, (uint64_t)nblk * 144, (uint64_t)N, (uint64_t)nblk * 144, 144,
+                              Cfg<4>::TILE);
     int rc = encode_tmap_2d(&m->w, W, 1, (uint64_t)nblk * Q6A_BYTES, (uint64_t)N, (uint64_t)nblk * Q6A_BYTES,
-                            Q6A_BYTES, TILE_ROWS);
+                            Q6A_BYTES, Cfg<6>::TILE);
     if (rc)
         return rc;
     const int nblk8 = (nblk + 7) & ~7;
     const uint8_t *D = (const uint8_t *)W + (size_t)N * nblk * Q6A_BYTES;
-    return encode_tmap_2d(&m->d, D, 2, (uint64_t)nblk8, (uint64_t)N, (uint64_t)nblk8 * 2, 8, TILE_ROWS);
+    return encode_tmap_2d(&m->d, D, 2, (uint64_t)nblk8, (uint64_t)N, (uint64_t)nblk8 * 2, 8, Cfg<6>::TILE);
 }
 
 int launch_gemm(int fmt, const WeightMapsBlob &maps_blob, int N, int K, int M, const FragBuf &fb, float *Y, int ldy,
@@ -773,7 +805,8 @@ int launch_gemm(int fmt, const WeightMapsBlob &maps_blob, int N, int K, int M, c
     a.nblk = K / 256;
     a.M = M;
     a.ldy = ldy;
-    a.units = ((N + TILE_ROWS - 1) / TILE_ROWS) * a.nblk;
+    const int tile = fmt == 4 ? Cfg<4>::TILE : Cfg<6>::TILE;
+    a.units = ((N + tile - 1) / tile) * a.nblk;
     a.rec = fb.rec;
     a.Y = Y;
     void (*kern)(const WeightMaps, GemmArgs);
@@ -797,8 +830,9 @@ int launch_gemm(int fmt, const WeightMapsBlob &maps_blob, int N, int K, int M, c
             done[dev][v] = true;
     }
     const int grid = num_sms();
-    cudaError_t e = pdl ? launch_pdl(kern, dim3(grid), dim3(32 * (CG * GW + 1)), smem, s, maps, a)
-                        : (kern<<<grid, 32 * (CG * GW + 1), smem, s>>>(maps, a), cudaGetLastError());
+    const int threads = fmt == 4 ? Cfg<4>::THREADS : Cfg<6>::THREADS;
+    cudaError_t e = pdl ? launch_pdl(kern, dim3(grid), dim3(threads), smem, s, maps, a)
+                        : (kern<<<grid, threads, smem, s>>>(maps, a), cudaGetLastError());
     return cuda_check(e, "gemm launch");
 }
 
