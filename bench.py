@@ -170,6 +170,18 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ helpers
 
+def measured_bf16_tflops(sustained=False):
+    """Dense bf16 tensor throughput from MEASURED_PEAKS.json (fp16 runs at the same rate)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        v = d.get("bf16_tflops_sustained" if sustained else "bf16_tflops")
+        if v:
+            return float(v)
+    return 1590.0
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -433,6 +445,10 @@ def run_gpu(args, ws, rank, local):
     return 0
 
 
+DENSE_KERNELS = {  # prefill chunk (2048 prompt rows + 12 decode rows) through one matrix: (format, N, K, M)
+    "pf_gate_up": (4, 34816, 5120, 2060), "pf_down": (6, 5120, 17408, 2060), "pf_qkv": (4, 8192, 5120, 2060),
+}
+
 KERNELS = {  # single-kernel cases for profiler captures: (format, N, K)
     "qkv": (4, 8192, 5120), "o": (4, 5120, 6144), "gate_up": (4, 34816, 5120), "down": (6, 5120, 17408),
 }
@@ -446,7 +462,20 @@ def run_kernel(args):
     from quantized_agent_decode_b200 import build
     build.build()
     g = synth.torch_gen(SEED, "cuda", 77)
-    if args.kernel == "attn23k":
+    if args.kernel in DENSE_KERNELS:
+        fmt, N, K, M = DENSE_KERNELS[args.kernel]
+        mk = synth.q4k_matrix_torch if fmt == 4 else synth.q6k_matrix_torch
+        Ws = [mk(g, N, K, "cuda") for _ in range(2)]
+        if fmt == 6:
+            Ws = [q.q6k_pack(w, N, K) for w in Ws]
+        X = synth.bf16_normal_torch(g, (M, K), "cuda")
+        Y = torch.empty(M, N, device="cuda")
+        ws = q.alloc_ws(q.dense_gemm_ws_bytes(K, M))
+        gemm = q.q4k_gemm_dense if fmt == 4 else q.q6k_gemm_dense
+        fn = lambda i, st: gemm(Ws[i % 2], N, K, X, M, Y, ws=ws, stream=st)  # noqa: E731
+        nbytes = Ws[0].numel()
+        flops = 2.0 * M * N * K
+    elif args.kernel == "attn23k":
         A, L, n_qh, n_kvh = 4, 23000, 48, 8
         cap = L + 3
         Kd = synth.bf16_normal_torch(g, (A, n_kvh, cap, 128), "cuda")
@@ -472,6 +501,8 @@ def run_kernel(args):
         gemm = q.q4k_gemm if fmt == 4 else q.q6k_gemm
         fn = lambda i, st: gemm(Ws[i % 8], N, K, X, M, Y, ws=ws, stream=st)  # noqa: E731
         nbytes = Ws[0].numel()
+    if args.kernel not in DENSE_KERNELS:
+        flops = None
     # 8 calls (8 weight copies) captured once and replayed: device time only, no host launch cost
     stream = torch.cuda.Stream()
     with torch.cuda.stream(stream):
@@ -493,8 +524,14 @@ def run_kernel(args):
     e1.record()
     torch.cuda.synchronize()
     us = e0.elapsed_time(e1) / (reps * 8) * 1e3
-    print(json.dumps({"kernel": args.kernel, "rows": args.rows, "us_per_call": us,
-                      "gbs": nbytes / us / 1e3, "bytes": nbytes, "device_status": q.device_status()}), flush=True)
+    out = {"kernel": args.kernel, "rows": args.rows, "us_per_call": us, "gbs": nbytes / us / 1e3, "bytes": nbytes,
+           "device_status": q.device_status()}
+    if flops:
+        peak = measured_bf16_tflops()
+        out.update({"rows": DENSE_KERNELS[args.kernel][3], "tflops": flops / us / 1e6, "flop_per_call": flops,
+                    "peak_tflops": peak, "frac": flops / us / 1e6 / peak if peak else None,
+                    "dense_status": q.dense_status()})
+    print(json.dumps(out), flush=True)
     return 0
 
 
@@ -506,7 +543,7 @@ def main():
     ap.add_argument("--workload", default="stack12_ctx1k", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel", choices=sorted(list(KERNELS) + ["attn23k"]),
+    ap.add_argument("--kernel", choices=sorted(list(KERNELS) + list(DENSE_KERNELS) + ["attn23k"]),
                     help="time one kernel of the step instead (profiler captures)")
     ap.add_argument("--rows", type=int, default=12)
     args = ap.parse_args()

@@ -115,7 +115,7 @@ int qad_q6k_pack(const void *W, int N, int K, void *W_packed, void *stream);
  * streams are decoding, and plain C integrations that only hold pointers to
  * buffers owned elsewhere. Arguments and result are those of qad_q4k_gemm
  * without the workspace: the scratch is a fixed array of
- * qad_q4k_gemm_noalloc_scratch_bytes() bytes (1 MiB; enough for K <= 30720 at
+ * qad_q4k_gemm_noalloc_scratch_bytes() bytes (1 MiB; enough for K <= 30464 at
  * 16 rows) in device memory that every GPU loading this library holds until
  * the process exits. Calls that need more scratch fail with
  * QAD_ERR_UNSUPPORTED before any launch. The first call on each device looks
@@ -139,6 +139,34 @@ int qad_q4k_gemm(const void *W, int N, int K, const uint16_t *X, int M, float *Y
                  void *ws, size_t ws_bytes, void *stream);
 int qad_q6k_gemm(const void *W, int N, int K, const uint16_t *X, int M, float *Y, int accumulate,
                  void *ws, size_t ws_bytes, void *stream);
+
+/* ---------------------------------------------------------------- prefill-chunk GEMM
+ * OpenJet page, section 真正重要的是少互相堵车: a long prompt is processed in
+ * chunks (2048 prompt rows of one agent, plus the 12 decode rows) through the
+ * same quantized weights; at that M the product is compute-bound.
+ *
+ * Y[m][n] = sum_k w[n][k] * x[m][k] for M >= 1 rows on the 5th-generation
+ * tensor cores (tcgen05, fp16 operands, fp32 accumulate in TMEM). The weights
+ * are dequantized in shared memory to fp16: w = fp16(d*sc)*q - fp16(dmin*m)
+ * (Q4_K) or fp16(d*sc)*(q - 32) (Q6_K-like), so each weight carries a
+ * relative rounding error <= 2^-11 on top of the exact definition; x enters as
+ * fp16 of x * 2^e_m with a per-row power of two (exact for bf16 rows whose
+ * dynamic range is below 2^38).
+ *   W   device: Q4_K [N][K/256][144] (qad_q4k_gemm_dense) or the packed
+ *       Q6_K-like layout of qad_q6k_pack (qad_q6k_gemm_dense); 16-byte aligned
+ *   X   device bf16 [M][K], 16-byte aligned;  Y  device fp32 [M][N], overwritten
+ *   ws  device workspace of qad_dense_gemm_ws_bytes(K, M) bytes, 256-byte aligned
+ * K % 256 == 0, K <= 65536. Returns 0 or a negative QAD_ERR_* code. Launches
+ * two kernels on `stream`. */
+size_t qad_dense_gemm_ws_bytes(int K, int M);
+int qad_q4k_gemm_dense(const void *W, int N, int K, const uint16_t *X, int M, float *Y, void *ws,
+                       size_t ws_bytes, void *stream);
+int qad_q6k_gemm_dense(const void *W, int N, int K, const uint16_t *X, int M, float *Y, void *ws,
+                       size_t ws_bytes, void *stream);
+/* 0 if every pipeline wait of the dense GEMM completed since the last reset
+ * (else 1 raw blocks, 2 activation tiles, 3 weight tiles, 4 accumulator,
+ * 5 teardown); reset != 0 clears it. Negative QAD_ERR_* on a CUDA error. */
+int qad_dense_status(int reset);
 
 /* ---------------------------------------------------------------- attention
  * Grouped-query decode attention of each agent's rows over that agent's own

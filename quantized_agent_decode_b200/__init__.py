@@ -54,6 +54,12 @@ SIGNATURES = {
                                C.c_void_p, C.c_size_t, C.c_void_p]),
     "qad_q6k_gemm": (C.c_int, [C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_int, C.c_void_p, C.c_int,
                                C.c_void_p, C.c_size_t, C.c_void_p]),
+    "qad_dense_gemm_ws_bytes": (C.c_size_t, [C.c_int, C.c_int]),
+    "qad_q4k_gemm_dense": (C.c_int, [C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p,
+                                     C.c_size_t, C.c_void_p]),
+    "qad_q6k_gemm_dense": (C.c_int, [C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p,
+                                     C.c_size_t, C.c_void_p]),
+    "qad_dense_status": (C.c_int, [C.c_int]),
     "qad_decode_attn_ws_bytes": (C.c_size_t, [C.c_int] * 5),
     "qad_decode_attn": (C.c_int, [C.c_void_p] * 5 + [C.c_int] * 6 + [C.c_float, C.c_void_p, C.c_void_p,
                                                                      C.c_size_t, C.c_void_p]),
@@ -189,6 +195,34 @@ def q4k_gemm_noalloc(W, N, K, X, M, Y, accumulate=False, stream=None):
     _check(lib().qad_q4k_gemm_noalloc(_dev(W, "W"), N, K, _dev(X, "X"), M, _dev(Y, "Y"), int(bool(accumulate)),
                                       _stream(stream)), "qad_q4k_gemm_noalloc")
     return Y
+
+
+def dense_gemm_ws_bytes(K: int, M: int) -> int:
+    return int(lib().qad_dense_gemm_ws_bytes(K, M))
+
+
+def dense_status(reset: bool = True) -> int:
+    """0 if every pipeline wait of the dense (prefill) GEMM completed since the last reset."""
+    return _check(lib().qad_dense_status(int(reset)), "qad_dense_status")
+
+
+def _dense(fn, W, N, K, X, M, Y, ws, stream):
+    _require_gpu()
+    if ws is None:
+        ws = alloc_ws(dense_gemm_ws_bytes(K, M), X.device)
+    _check(getattr(lib(), fn)(_dev(W, "W"), N, K, _dev(X, "X"), M, _dev(Y, "Y"), _dev(ws, "ws"),
+                              ws.numel() * ws.element_size(), _stream(stream)), fn)
+    return Y
+
+
+def q4k_gemm_dense(W, N, K, X, M, Y, ws=None, stream=None):
+    """Prefill-chunk GEMM on tcgen05: Y[M,N] (fp32, overwritten) = X[M,K] (bf16) @ W^T, W Q4_K."""
+    return _dense("qad_q4k_gemm_dense", W, N, K, X, M, Y, ws, stream)
+
+
+def q6k_gemm_dense(W, N, K, X, M, Y, ws=None, stream=None):
+    """Prefill-chunk GEMM on tcgen05 with W in the packed Q6_K-like layout (q6k_pack)."""
+    return _dense("qad_q6k_gemm_dense", W, N, K, X, M, Y, ws, stream)
 
 
 def q6k_packed_bytes(N: int, K: int) -> int:

@@ -1,0 +1,565 @@
+// dense.cu -- the prefill-chunk GEMM: Y[m][n] = sum_k w[n][k] x[m][k] for a
+// chunk of M ~ 2060 activation rows (2048 prompt tokens of one agent plus the
+// 12 decode rows) against the same Q4_K / Q6_K-like weights as the decode step.
+//
+// [OpenJet page] = rebasdaily.com 2026-10-29, "OpenJet ... multi-agent
+// serving", section 真正重要的是少互相堵车: a 20K-token prompt arrives while
+// other agents decode; its chunks run through the same weights. At M = 2060
+// the product is compute-bound (~2 FLOP per weight per row), so it belongs
+// on the 5th-generation tensor cores.
+//
+// Design (sm_100a, one CTA per SM, persistent over output tiles):
+//  * Output tile = 128 weight rows x 256 activation rows. The accumulator
+//    D[128][256] fp32 lives in TMEM (256 columns); one elected thread issues
+//    tcgen05.mma kind::f16 (M=128, N=256, K=16) with both operands in shared
+//    memory (K-major, no swizzle: 8-row x 16-byte core matrices).
+//  * A producer warp streams the raw quantized blocks of the tile's 128 rows
+//    by TMA (one block of 256 k per stage) and the activation tiles (256 rows
+//    x 64 k fp16, already in core-matrix order) by one bulk copy per k-step.
+//  * Four dequant warps turn each 64-wide k-step of the raw blocks into fp16
+//    weights in core-matrix order: w = fp16(d*sc) * q - fp16(dmin*m) for Q4_K
+//    (q exact in fp16, one fused multiply-add per pair), w = fp16(d*sc) *
+//    (q - 32) for Q6_K. The same warps then read the accumulator out of TMEM,
+//    apply the activation row scale and store Y.
+//  * Activations enter as fp16 of x * 2^e_m (per-row power of two putting the
+//    row's max |x| in [2^14, 2^15)); a prep kernel writes them straight into
+//    the tile order the bulk copies want, zero-padding M to whole tiles.
+//  * Every mbarrier wait is bounded; on a timeout the CTA records a status,
+//    skips the rest of its work, waits for its own copies and MMAs, frees its
+//    TMEM and exits.
+#include <cuda.h>
+
+#include "dense.cuh"
+#include "gemm.cuh"
+
+namespace qad {
+
+__device__ int g_dense_status;
+
+namespace dn {
+constexpr int TN = 128;            // weight rows per tile (MMA M)
+constexpr int TM = 256;            // activation rows per tile (MMA N)
+constexpr int KS = 64;             // k per pipeline step
+constexpr int SR = 2;              // raw-block stages
+constexpr int SB = 3;              // activation-tile stages
+constexpr int SA = 3;              // dequantized-weight stages
+constexpr int B_BYTES = TM * KS * 2;   // 32 KB
+constexpr int A_BYTES = TN * KS * 2;   // 16 KB
+constexpr int THREADS = 192;       // producer, MMA, 4 dequant/epilogue warps
+constexpr int Q6A = 208;
+template <int FMT>
+struct Raw {
+    static constexpr int W = TN * (FMT == 4 ? 144 : Q6A);
+    static constexpr int D = FMT == 4 ? 0 : TN * 16;
+    static constexpr int COPY = W + D;
+    static constexpr int BYTES = (COPY + 1023) / 1024 * 1024;
+};
+template <int FMT>
+constexpr size_t smem_bytes()
+{
+    return 1024 /* alignment slack */ + (size_t)SR * Raw<FMT>::BYTES + (size_t)SB * B_BYTES + (size_t)SA * A_BYTES +
+           256 /* barriers + tmem slot */;
+}
+enum { ST_RAW = 1, ST_B = 2, ST_A = 3, ST_ACC = 4, ST_DONE = 5 };
+}  // namespace dn
+
+struct DenseArgs {
+    int N, K, M, mt, nt, nblk;
+    const uint16_t *x16;  // activation tiles (dense_x16 layout)
+    const float *rs;      // per activation row 2^-e (0 past M)
+    float *Y;
+    int ldy;
+};
+
+// Activation tile layout: [m_tile][k-step][k-chunk 8][256 rows][8 fp16]; one
+// (m_tile, k-step) is 32 KB contiguous, i.e. exactly the B operand of one
+// k-step in core-matrix order (chunk stride 4096 B, 8-row stride 128 B).
+__global__ void __launch_bounds__(256) k_prep_dense(const uint16_t *__restrict__ X, int ldx, int M, int K,
+                                                    uint16_t *__restrict__ x16, float *__restrict__ rs)
+{
+    __shared__ float red[8];
+    const int r = blockIdx.x, tid = threadIdx.x;
+    const int mt = r / dn::TM, rr = r % dn::TM, ksteps = K / dn::KS;
+    const bool live = r < M;
+    float mx = 0.f;
+    if (live)
+        for (int q = tid; q < K / 8; q += 256) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(X + (size_t)r * ldx + 8 * q);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                mx = fmaxf(mx, fabsf(bf16_to_f((uint16_t)(w[i] & 0xFFFF))));
+                mx = fmaxf(mx, fabsf(bf16_to_f((uint16_t)(w[i] >> 16))));
+            }
+        }
+#pragma unroll
+    for (int o = 16; o; o >>= 1)
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if ((tid & 31) == 0)
+        red[tid >> 5] = mx;
+    __syncthreads();
+    mx = 0.f;
+    for (int i = 0; i < 8; ++i)
+        mx = fmaxf(mx, red[i]);
+    int e = 0;
+    if (mx > 0.f) {
+        int E;
+        frexpf(mx, &E);  // mx in [2^(E-1), 2^E)
+        e = min(126, max(-126, 15 - E));
+    }
+    const float sc = ldexpf(1.f, e);
+    if (tid == 0)
+        rs[r] = live ? ldexpf(1.f, -e) : 0.f;
+    for (int q = tid; q < K / 8; q += 256) {
+        uint4 o = make_uint4(0u, 0u, 0u, 0u);
+        if (live) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(X + (size_t)r * ldx + 8 * q);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            uint32_t h[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                h[i] = pack_half2(bf16_to_f((uint16_t)(w[i] & 0xFFFF)) * sc, bf16_to_f((uint16_t)(w[i] >> 16)) * sc);
+            o = make_uint4(h[0], h[1], h[2], h[3]);
+        }
+        const int ks = q / 8, ch = q % 8;
+        const size_t off = ((((size_t)mt * ksteps + ks) * 8 + ch) * dn::TM + rr) * 8;
+        *reinterpret_cast<uint4 *>(x16 + off) = o;
+    }
+}
+
+// fp16 pair (v, v)
+__device__ __forceinline__ uint32_t h2dup(float v)
+{
+    const uint32_t h = __half_as_ushort(__float2half_rn(v));
+    return h | (h << 16);
+}
+
+// 64 fp16 weights of row n for k-step kk (0..3) of a Q4_K block -> 8 chunks of
+// the A stage (chunk c at c * 2048 + n * 16).
+__device__ __forceinline__ void dequant_q4(const uint8_t *blk, int kk, uint8_t *A, int n)
+{
+    const uint4 h = lds_v4(blk);
+    const float d = half_lo(h.x), dmin = half_hi(h.x);
+    const uint32_t s[3] = {h.y, h.z, h.w};  // the 12 packed scale/min bytes
+    auto byte = [&](int i) { return (s[i >> 2] >> (8 * (i & 3))) & 0xFFu; };
+    float sc[2], mn[2];
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+        const int j = 2 * kk + t;  // sub-block
+        if (j < 4) {
+            sc[t] = (float)(byte(j) & 63);
+            mn[t] = (float)(byte(j + 4) & 63);
+        } else {
+            sc[t] = (float)((byte(j + 4) & 0xF) | ((byte(j - 4) >> 6) << 4));
+            mn[t] = (float)((byte(j + 4) >> 4) | ((byte(j) >> 6) << 4));
+        }
+    }
+    // low nibbles: sub-block 2kk, k 0..31 of the step; high: 2kk+1, k 32..63
+    const uint32_t aL = h2dup(d * sc[0]), bL = h2dup(-dmin * mn[0]);
+    const uint32_t aH = h2dup(d * sc[1] * 0.0625f), bH = h2dup(-dmin * mn[1]);
+    const uint4 q0 = lds_v4(blk + 16 + 32 * kk), q1 = lds_v4(blk + 32 + 32 * kk);
+    const uint32_t qw[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        uint32_t lo[4], hi[4];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const uint32_t w = qw[2 * c + u];
+            const uint32_t t01 = prmt(w, w, 0x1100u), t23 = prmt(w, w, 0x3322u);
+            // (1024 + q) -> q exact -> a*q + b
+            lo[2 * u] = hfma2(hsub2(and_or(t01, 0x000F000Fu, H2_1024), H2_1024), aL, bL);
+            lo[2 * u + 1] = hfma2(hsub2(and_or(t23, 0x000F000Fu, H2_1024), H2_1024), aL, bL);
+            hi[2 * u] = hfma2(hsub2(and_or(t01, 0x00F000F0u, H2_1024), H2_1024), aH, bH);
+            hi[2 * u + 1] = hfma2(hsub2(and_or(t23, 0x00F000F0u, H2_1024), H2_1024), aH, bH);
+        }
+        *reinterpret_cast<uint4 *>(A + c * 2048 + n * 16) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        *reinterpret_cast<uint4 *>(A + (4 + c) * 2048 + n * 16) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    }
+}
+
+constexpr uint32_t H2_1056D = 0x64206420u;  // 1056.0
+
+// Q6_K-like (packed plane A, d from the D tile): k-step kk = half h, group sel.
+__device__ __forceinline__ void dequant_q6(const uint8_t *blk, float d, int kk, uint8_t *A, int n)
+{
+    const int h = kk >> 1, sel = kk & 1;
+    const uint2 sw = lds_v2(blk + 192 + 8 * h);
+    const int8_t *scb = reinterpret_cast<const int8_t *>(&sw);
+    uint32_t a[4];
+#pragma unroll
+    for (int g = 0; g < 4; ++g)  // 16-weight groups of the step: scales 4 sel + g
+        a[g] = h2dup(d * (float)scb[4 * sel + g]);
+#pragma unroll
+    for (int part = 0; part < 2; ++part) {  // k 0..31 (ql[l], qh bits 4sel), k 32..63 (ql[l+32], bits 4sel+2)
+        const uint8_t *ql = blk + 64 * h + 32 * part;
+        const uint8_t *qh = blk + 128 + 32 * h;
+        const int sh = 4 * sel + 2 * part;
+#pragma unroll
+        for (int c2 = 0; c2 < 4; ++c2) {  // chunk = 4 part + c2: k 8 c2 .. 8 c2 + 7 of the part
+            const uint2 L = lds_v2(ql + 8 * c2), Hh = lds_v2(qh + 8 * c2);
+            const uint32_t lw[2] = {L.x, L.y}, hw[2] = {Hh.x, Hh.y};
+            uint32_t o[4];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const uint32_t q = ((lw[u] >> (4 * sel)) & 0x0F0F0F0Fu) | (((hw[u] >> sh) & 0x03030303u) << 4);
+                const uint32_t t01 = prmt(q, q, 0x1100u), t23 = prmt(q, q, 0x3322u);
+                const uint32_t sc = a[2 * part + (c2 >> 1)];
+                o[2 * u] = hmul2(hsub2(and_or(t01, 0x003F003Fu, H2_1024), H2_1056D), sc);
+                o[2 * u + 1] = hmul2(hsub2(and_or(t23, 0x003F003Fu, H2_1024), H2_1056D), sc);
+            }
+            *reinterpret_cast<uint4 *>(A + (4 * part + c2) * 2048 + n * 16) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+    }
+}
+
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ __forceinline__ void umma_f16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate)
+{
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+                 ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+                 : "memory");
+}
+
+template <int FMT>
+__global__ void __launch_bounds__(dn::THREADS, 1) k_dense_gemm(const __grid_constant__ WeightMapsBlob mapsb, DenseArgs a)
+{
+    using namespace dn;
+    using R = Raw<FMT>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    uint8_t *RAW = smem;
+    uint8_t *BS = RAW + SR * R::BYTES;
+    uint8_t *AS = BS + SB * B_BYTES;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(AS + SA * A_BYTES);
+    uint64_t *raw_full = bar, *raw_empty = bar + SR, *b_full = bar + 2 * SR, *b_empty = b_full + SB;
+    uint64_t *a_full = b_empty + SB, *a_empty = a_full + SA, *acc_full = a_empty + SA, *acc_empty = acc_full + 1;
+    uint64_t *done = acc_empty + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 1);
+    __shared__ int s_bad;
+    const CUtensorMap *mw = reinterpret_cast<const CUtensorMap *>(mapsb.bytes);
+    const CUtensorMap *md = mw + 1;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tiles = a.mt * a.nt;
+    const int ksteps = a.K / KS;
+
+    if (threadIdx.x == 0) {
+        s_bad = 0;
+        for (int i = 0; i < SR; ++i) {
+            mbar_init(&raw_full[i], 1);
+            mbar_init(&raw_empty[i], 4);
+        }
+        for (int i = 0; i < SB; ++i) {
+            mbar_init(&b_full[i], 1);
+            mbar_init(&b_empty[i], 1);
+        }
+        for (int i = 0; i < SA; ++i) {
+            mbar_init(&a_full[i], 4);
+            mbar_init(&a_empty[i], 1);
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(acc_empty, 4);
+        mbar_init(done, 1);
+        mbar_fence_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    auto fail = [&](int code) {
+        atomicExch(&g_dense_status, code);
+        atomicExch(&s_bad, 1);
+    };
+    auto bad = [&]() { return *(volatile int *)&s_bad != 0; };
+
+    if (warp == 0) {
+        // ------------------------------------------------ producer
+        if (lane == 0) {
+            int bk = 0, ks = 0;
+            for (int t = blockIdx.x; t < tiles && !bad(); t += gridDim.x) {
+                const int nt = t / a.mt, mt = t % a.mt;
+                for (int blk = 0; blk < a.nblk && !bad(); ++blk) {
+                    const int s = bk % SR;
+                    if (bk >= SR && !mbar_wait(&raw_empty[s], ((bk / SR) - 1) & 1)) {
+                        fail(ST_RAW);
+                        break;
+                    }
+                    uint8_t *st = RAW + s * R::BYTES;
+                    mbar_arrive_expect_tx(&raw_full[s], (uint32_t)R::COPY);
+                    tma_load_2d(st, mw, blk * (FMT == 4 ? 144 : Q6A), nt * TN, &raw_full[s]);
+                    if (FMT == 6)
+                        tma_load_2d(st + R::W, md, blk & ~7, nt * TN, &raw_full[s]);
+                    ++bk;
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const int sb = ks % SB;
+                        if (ks >= SB && !mbar_wait(&b_empty[sb], ((ks / SB) - 1) & 1)) {
+                            fail(ST_B);
+                            break;
+                        }
+                        mbar_arrive_expect_tx(&b_full[sb], (uint32_t)B_BYTES);
+                        bulk_g2s(BS + sb * B_BYTES, a.x16 + ((size_t)mt * ksteps + 4 * blk + kk) * (B_BYTES / 2),
+                                 B_BYTES, &b_full[sb]);
+                        ++ks;
+                    }
+                }
+            }
+            // every issued copy lands before teardown
+            for (int k = max(0, bk - SR); k < bk; ++k)
+                if (!mbar_wait(&raw_full[k % SR], (k / SR) & 1, 20000))
+                    fail(ST_RAW);
+            for (int k = max(0, ks - SB); k < ks; ++k)
+                if (!mbar_wait(&b_full[k % SB], (k / SB) & 1, 20000))
+                    fail(ST_B);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = umma_idesc_f16(TN, TM);
+            int ks = 0, tc = 0;
+            bool issued = false;
+            for (int t = blockIdx.x; t < tiles && !bad(); t += gridDim.x, ++tc) {
+                if (tc > 0) {
+                    if (!mbar_wait(acc_empty, (tc - 1) & 1)) {
+                        fail(ST_ACC);
+                        break;
+                    }
+                    tc_fence_after();
+                }
+                for (int k = 0; k < ksteps; ++k, ++ks) {
+                    const int sa = ks % SA, sb = ks % SB;
+                    if (!mbar_wait(&a_full[sa], (ks / SA) & 1) || !mbar_wait(&b_full[sb], (ks / SB) & 1)) {
+                        fail(ST_A);
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t abase = smem_u32(AS + sa * A_BYTES), bbase = smem_u32(BS + sb * B_BYTES);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const uint64_t ad = umma_desc_k_noswz(abase + j * 2 * (TN * 16), TN * 16, 128);
+                        const uint64_t bd = umma_desc_k_noswz(bbase + j * 2 * (TM * 16), TM * 16, 128);
+                        umma_f16_ss(tmem, ad, bd, idesc, (k | j) != 0);
+                    }
+                    issued = true;
+                    umma_commit(&a_empty[sa]);
+                    umma_commit(&b_empty[sb]);
+                }
+                if (bad())
+                    break;
+                umma_commit(acc_full);
+            }
+            // every MMA this thread issued has completed before TMEM is freed
+            if (issued) {
+                umma_commit(done);
+                if (!mbar_wait(done, 0, 20000))
+                    fail(ST_DONE);
+            }
+        }
+    } else {
+        // ------------------------------------------------ dequant + epilogue (weight row n)
+        const int quarter = warp & 3;
+        const int n = 32 * quarter + lane;
+        int bk = 0, ks = 0, tc = 0;
+        for (int t = blockIdx.x; t < tiles && !bad(); t += gridDim.x, ++tc) {
+            const int nt = t / a.mt, mt = t % a.mt;
+            for (int blk = 0; blk < a.nblk && !bad(); ++blk, ++bk) {
+                const int s = bk % SR;
+                if (!__all_sync(0xffffffffu, mbar_wait(&raw_full[s], (bk / SR) & 1))) {
+                    fail(ST_RAW);
+                    break;
+                }
+                const uint8_t *st = RAW + s * R::BYTES;
+                float d6 = 0.f;
+                if (FMT == 6) {
+                    const uint32_t dw = lds_u32(st + R::W + n * 16 + (blk & 6) * 2);
+                    d6 = __half2float(__ushort_as_half((unsigned short)(dw >> ((blk & 1) * 16))));
+                }
+                for (int kk = 0; kk < 4; ++kk, ++ks) {
+                    const int sa = ks % SA;
+                    if (ks >= SA && !__all_sync(0xffffffffu, mbar_wait(&a_empty[sa], ((ks / SA) - 1) & 1))) {
+                        fail(ST_A);
+                        break;
+                    }
+                    uint8_t *A = AS + sa * A_BYTES;
+                    if (FMT == 4)
+                        dequant_q4(st + n * 144, kk, A, n);
+                    else
+                        dequant_q6(st + n * Q6A, d6, kk, A, n);
+                    fence_proxy_async();
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(&a_full[sa]);
+                }
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&raw_empty[s]);
+            }
+            if (bad())
+                break;
+            // epilogue: D[n][m] * 2^-e_m -> Y[m][n]
+            if (!__all_sync(0xffffffffu, mbar_wait(acc_full, tc & 1))) {
+                fail(ST_ACC);
+                break;
+            }
+            tc_fence_after();
+            const int ng = nt * TN + n;
+#pragma unroll 1
+            for (int j = 0; j < TM / 16; ++j) {
+                uint32_t v[16];
+                tmem_ld_x16(tmem + ((uint32_t)(32 * quarter) << 16) + 16 * j, v);
+                tmem_wait_ld();
+                const int m0 = mt * TM + 16 * j;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int m = m0 + i;
+                    if (m < a.M && ng < a.N)
+                        a.Y[(size_t)m * a.ldy + ng] = __uint_as_float(v[i]) * a.rs[m];
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(acc_empty);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
+// ------------------------------------------------------------- host side
+
+// Tensor maps of the weights with 128-row boxes: [0] the Q4_K matrix or the
+// Q6_K plane A, [1] the Q6_K plane D.
+int make_dense_maps(int fmt, const void *W, int N, int K, WeightMapsBlob *out)
+{
+    static_assert(sizeof(WeightMapsBlob) >= 2 * sizeof(CUtensorMap), "blob too small");
+    CUtensorMap *m = reinterpret_cast<CUtensorMap *>(out->bytes);
+    const int nblk = K / 256;
+    if (fmt == 4)
+        return encode_tmap_2d(&m[0], W, 1, (uint64_t)nblk * 144, (uint64_t)N, (uint64_t)nblk * 144, 144, dn::TN);
+    int rc = encode_tmap_2d(&m[0], W, 1, (uint64_t)nblk * dn::Q6A, (uint64_t)N, (uint64_t)nblk * dn::Q6A, dn::Q6A,
+                            dn::TN);
+    if (rc)
+        return rc;
+    const int nblk8 = (nblk + 7) & ~7;
+    const uint8_t *D = (const uint8_t *)W + (size_t)N * nblk * dn::Q6A;
+    return encode_tmap_2d(&m[1], D, 2, (uint64_t)nblk8, (uint64_t)N, (uint64_t)nblk8 * 2, 8, dn::TN);
+}
+
+size_t dense_ws_bytes(int K, int M)
+{
+    const size_t mpad = (size_t)(M + dn::TM - 1) / dn::TM * dn::TM;
+    return mpad * (size_t)K * 2 + ((mpad * 4 + 255) & ~(size_t)255);
+}
+
+template <int FMT>
+static int launch_dense_t(const WeightMapsBlob &maps, const DenseArgs &a, cudaStream_t s)
+{
+    const size_t smem = dn::smem_bytes<FMT>();
+    static bool done[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || !done[dev]) {
+        int rc = cuda_check(
+            cudaFuncSetAttribute(k_dense_gemm<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem),
+            "cudaFuncSetAttribute(dense)");
+        if (rc)
+            return rc;
+        if (dev >= 0 && dev < 64)
+            done[dev] = true;
+    }
+    const int tiles = a.mt * a.nt;
+    const int grid = tiles < num_sms() ? tiles : num_sms();
+    k_dense_gemm<FMT><<<grid, dn::THREADS, smem, s>>>(maps, a);
+    return cuda_check(cudaGetLastError(), "dense gemm launch");
+}
+
+int launch_dense(int fmt, const void *W, int N, int K, const uint16_t *X, int M, float *Y, void *ws,
+                 cudaStream_t s)
+{
+    WeightMapsBlob maps;
+    int rc = make_dense_maps(fmt, W, N, K, &maps);
+    if (rc)
+        return rc;
+    const int mt = (M + dn::TM - 1) / dn::TM;
+    uint16_t *x16 = (uint16_t *)ws;
+    float *rs = (float *)((char *)ws + (size_t)mt * dn::TM * K * 2);
+    k_prep_dense<<<mt * dn::TM, 256, 0, s>>>(X, K, M, K, x16, rs);
+    rc = cuda_check(cudaGetLastError(), "dense prep launch");
+    if (rc)
+        return rc;
+    DenseArgs a;
+    a.N = N;
+    a.K = K;
+    a.M = M;
+    a.mt = mt;
+    a.nt = (N + dn::TN - 1) / dn::TN;
+    a.nblk = K / 256;
+    a.x16 = x16;
+    a.rs = rs;
+    a.Y = Y;
+    a.ldy = N;
+    return fmt == 4 ? launch_dense_t<4>(maps, a, s) : launch_dense_t<6>(maps, a, s);
+}
+
+}  // namespace qad
+
+// ------------------------------------------------------------- C ABI
+
+extern "C" size_t qad_dense_gemm_ws_bytes(int K, int M)
+{
+    if (K <= 0 || K % 256 || M <= 0)
+        return 0;
+    return qad::dense_ws_bytes(K, M);
+}
+
+extern "C" int qad_dense_status(int reset)
+{
+    int v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, qad::g_dense_status, sizeof(int));
+    if (e != cudaSuccess)
+        return qad::cuda_check(e, "qad_dense_status");
+    if (reset && v) {
+        const int z = 0;
+        e = cudaMemcpyToSymbol(qad::g_dense_status, &z, sizeof(int));
+        if (e != cudaSuccess)
+            return qad::cuda_check(e, "qad_dense_status reset");
+    }
+    return v;
+}
+
+static int dense_entry(int fmt, const void *W, int N, int K, const uint16_t *X, int M, float *Y, void *ws,
+                       size_t ws_bytes, void *stream)
+{
+    const char *name = fmt == 4 ? "qad_q4k_gemm_dense" : "qad_q6k_gemm_dense";
+    if (!W || !X || !Y || !ws || N <= 0 || K <= 0 || M <= 0)
+        return qad::fail(QAD_ERR_INVALID, "%s: null pointer or non-positive size (N=%d K=%d M=%d)", name, N, K, M);
+    if (K % 256 || K > 65536 || N > (1 << 24))
+        return qad::fail(QAD_ERR_UNSUPPORTED, "%s: need K %% 256 == 0, K <= 65536 (K=%d N=%d)", name, K, N);
+    if (((uintptr_t)W | (uintptr_t)X) & 15 || (uintptr_t)ws & 255)
+        return qad::fail(QAD_ERR_INVALID, "%s: W and X must be 16-byte aligned, ws 256-byte aligned", name);
+    if (ws_bytes < qad::dense_ws_bytes(K, M))
+        return qad::fail(QAD_ERR_WORKSPACE, "%s: workspace %zu < %zu bytes", name, ws_bytes, qad::dense_ws_bytes(K, M));
+    return qad::launch_dense(fmt, W, N, K, X, M, Y, ws, (cudaStream_t)stream);
+}
+
+extern "C" int qad_q4k_gemm_dense(const void *W, int N, int K, const uint16_t *X, int M, float *Y, void *ws,
+                                  size_t ws_bytes, void *stream)
+{
+    return dense_entry(4, W, N, K, X, M, Y, ws, ws_bytes, stream);
+}
+
+extern "C" int qad_q6k_gemm_dense(const void *W, int N, int K, const uint16_t *X, int M, float *Y, void *ws,
+                                  size_t ws_bytes, void *stream)
+{
+    return dense_entry(6, W, N, K, X, M, Y, ws, ws_bytes, stream);
+}

@@ -63,6 +63,20 @@ def test_version_and_error_text(qlib):
     assert L.qad_gemm_ws_bytes(5120, 12) > 0
 
 
+def test_dense_gemm_argument_checks(qlib):
+    """The prefill-chunk GEMM validates its arguments on the host before any launch."""
+    L = qlib.lib()
+    fake = C.c_void_p(0x10000)  # aligned, never dereferenced: every call below fails its checks first
+    assert L.qad_q4k_gemm_dense(None, 128, 256, fake, 4, fake, fake, 1 << 20, None) == -1
+    assert L.qad_q4k_gemm_dense(fake, 128, 300, fake, 4, fake, fake, 1 << 20, None) == -2
+    assert b"K % 256" in L.qad_last_error()
+    assert L.qad_q6k_gemm_dense(fake, 128, 256, C.c_void_p(0x10008), 4, fake, fake, 1 << 20, None) == -1
+    need = L.qad_dense_gemm_ws_bytes(512, 300)
+    assert need == 512 * 512 * 2 + 512 * 4  # M padded to two 256-row tiles, plus the row scales
+    assert L.qad_q4k_gemm_dense(fake, 128, 512, fake, 300, fake, fake, need - 1, None) == -3
+    assert L.qad_dense_gemm_ws_bytes(100, 4) == 0 and L.qad_dense_gemm_ws_bytes(256, 0) == 0
+
+
 def test_pack_rows_matches_oracle(qlib, orc):
     gd = golden("pack_rows.json")
     H = 64
