@@ -16,11 +16,14 @@
 //  * A producer warp streams the raw quantized blocks of the tile's 128 rows
 //    by TMA (one block of 256 k per stage) and the activation tiles (256 rows
 //    x 64 k fp16, already in core-matrix order) by one bulk copy per k-step.
-//  * Four dequant warps turn each 64-wide k-step of the raw blocks into fp16
-//    weights in core-matrix order: w = fp16(d*sc) * q - fp16(dmin*m) for Q4_K
-//    (q exact in fp16, one fused multiply-add per pair), w = fp16(d*sc) *
-//    (q - 32) for Q6_K. The same warps then read the accumulator out of TMEM,
-//    apply the activation row scale and store Y.
+//  * Eight dequant warps turn each 64-wide k-step of the raw blocks into fp16
+//    weights in core-matrix order (one weight row per thread, one 32-wide half
+//    of the k-step per warp): w = fp16(d*sc) * q - fp16(dmin*m) for Q4_K (q
+//    exact in fp16, one fused multiply-add per pair), w = fp16(d*sc) * (q - 32)
+//    for Q6_K.
+//  * Two accumulators (512 TMEM columns): four epilogue warps read tile t out
+//    of TMEM, apply the activation row scales and store Y while the MMAs of
+//    tile t + 1 run.
 //  * Activations enter as fp16 of x * 2^e_m (per-row power of two putting the
 //    row's max |x| in [2^14, 2^15)); a prep kernel writes them straight into
 //    the tile order the bulk copies want, zero-padding M to whole tiles.
@@ -45,7 +48,9 @@ constexpr int SB = 3;              // activation-tile stages
 constexpr int SA = 3;              // dequantized-weight stages
 constexpr int B_BYTES = TM * KS * 2;   // 32 KB
 constexpr int A_BYTES = TN * KS * 2;   // 16 KB
-constexpr int THREADS = 192;       // producer, MMA, 4 dequant/epilogue warps
+constexpr int DQW = 8;             // dequant warps: two per weight-row quarter (k halves)
+constexpr int EPW = 4;             // epilogue warps (one per TMEM lane quarter)
+constexpr int THREADS = 32 * (2 + DQW + EPW);  // + producer, MMA issuer
 constexpr int Q6A = 208;
 template <int FMT>
 struct Raw {
@@ -134,63 +139,58 @@ __device__ __forceinline__ uint32_t h2dup(float v)
     return h | (h << 16);
 }
 
-// 64 fp16 weights of row n for k-step kk (0..3) of a Q4_K block -> 8 chunks of
-// the A stage (chunk c at c * 2048 + n * 16).
-__device__ __forceinline__ void dequant_q4(const uint8_t *blk, int kk, uint8_t *A, int n)
+// 32 fp16 weights of row n for k-step kk (0..3) of a Q4_K block: half 0 = the
+// low nibbles (k 0..31 of the step, chunks 0..3), half 1 = the high nibbles
+// (k 32..63, chunks 4..7); chunk c of the A stage sits at c * 2048 + n * 16.
+__device__ __forceinline__ void dequant_q4(const uint8_t *blk, int kk, int half, uint8_t *A, int n)
 {
     const uint4 h = lds_v4(blk);
     const float d = half_lo(h.x), dmin = half_hi(h.x);
-    const uint32_t s[3] = {h.y, h.z, h.w};  // the 12 packed scale/min bytes
-    auto byte = [&](int i) { return (s[i >> 2] >> (8 * (i & 3))) & 0xFFu; };
-    float sc[2], mn[2];
-#pragma unroll
-    for (int t = 0; t < 2; ++t) {
-        const int j = 2 * kk + t;  // sub-block
-        if (j < 4) {
-            sc[t] = (float)(byte(j) & 63);
-            mn[t] = (float)(byte(j + 4) & 63);
-        } else {
-            sc[t] = (float)((byte(j + 4) & 0xF) | ((byte(j - 4) >> 6) << 4));
-            mn[t] = (float)((byte(j + 4) >> 4) | ((byte(j) >> 6) << 4));
-        }
+    // byte i of the 12 packed scale/min bytes (h.y, h.z, h.w)
+    auto byte = [&](int i) { return ((i < 4 ? h.y : i < 8 ? h.z : h.w) >> (8 * (i & 3))) & 0xFFu; };
+    const int j = 2 * kk + half;  // sub-block
+    float sc, mn;
+    if (j < 4) {
+        sc = (float)(byte(j) & 63);
+        mn = (float)(byte(j + 4) & 63);
+    } else {
+        sc = (float)((byte(j + 4) & 0xF) | ((byte(j - 4) >> 6) << 4));
+        mn = (float)((byte(j + 4) >> 4) | ((byte(j) >> 6) << 4));
     }
-    // low nibbles: sub-block 2kk, k 0..31 of the step; high: 2kk+1, k 32..63
-    const uint32_t aL = h2dup(d * sc[0]), bL = h2dup(-dmin * mn[0]);
-    const uint32_t aH = h2dup(d * sc[1] * 0.0625f), bH = h2dup(-dmin * mn[1]);
+    // the high nibble enters as 16 q, so its scale is d*sc/16
+    const uint32_t av = h2dup(half ? d * sc * 0.0625f : d * sc), bv = h2dup(-dmin * mn);
+    const uint32_t mask = half ? 0x00F000F0u : 0x000F000Fu;
     const uint4 q0 = lds_v4(blk + 16 + 32 * kk), q1 = lds_v4(blk + 32 + 32 * kk);
     const uint32_t qw[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-        uint32_t lo[4], hi[4];
+        uint32_t o[4];
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
             const uint32_t w = qw[2 * c + u];
             const uint32_t t01 = prmt(w, w, 0x1100u), t23 = prmt(w, w, 0x3322u);
             // (1024 + q) -> q exact -> a*q + b
-            lo[2 * u] = hfma2(hsub2(and_or(t01, 0x000F000Fu, H2_1024), H2_1024), aL, bL);
-            lo[2 * u + 1] = hfma2(hsub2(and_or(t23, 0x000F000Fu, H2_1024), H2_1024), aL, bL);
-            hi[2 * u] = hfma2(hsub2(and_or(t01, 0x00F000F0u, H2_1024), H2_1024), aH, bH);
-            hi[2 * u + 1] = hfma2(hsub2(and_or(t23, 0x00F000F0u, H2_1024), H2_1024), aH, bH);
+            o[2 * u] = hfma2(hsub2(and_or(t01, mask, H2_1024), H2_1024), av, bv);
+            o[2 * u + 1] = hfma2(hsub2(and_or(t23, mask, H2_1024), H2_1024), av, bv);
         }
-        *reinterpret_cast<uint4 *>(A + c * 2048 + n * 16) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-        *reinterpret_cast<uint4 *>(A + (4 + c) * 2048 + n * 16) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4 *>(A + (4 * half + c) * 2048 + n * 16) = make_uint4(o[0], o[1], o[2], o[3]);
     }
 }
 
 constexpr uint32_t H2_1056D = 0x64206420u;  // 1056.0
 
-// Q6_K-like (packed plane A, d from the D tile): k-step kk = half h, group sel.
-__device__ __forceinline__ void dequant_q6(const uint8_t *blk, float d, int kk, uint8_t *A, int n)
+// Q6_K-like (packed plane A, d from the D tile): k-step kk = half h, group sel;
+// `part` 0 writes k 0..31 of the step (chunks 0..3), part 1 k 32..63.
+__device__ __forceinline__ void dequant_q6(const uint8_t *blk, float d, int kk, int part, uint8_t *A, int n)
 {
     const int h = kk >> 1, sel = kk & 1;
     const uint2 sw = lds_v2(blk + 192 + 8 * h);
     const int8_t *scb = reinterpret_cast<const int8_t *>(&sw);
-    uint32_t a[4];
+    uint32_t a[2];
 #pragma unroll
-    for (int g = 0; g < 4; ++g)  // 16-weight groups of the step: scales 4 sel + g
-        a[g] = h2dup(d * (float)scb[4 * sel + g]);
-#pragma unroll
-    for (int part = 0; part < 2; ++part) {  // k 0..31 (ql[l], qh bits 4sel), k 32..63 (ql[l+32], bits 4sel+2)
+    for (int g = 0; g < 2; ++g)  // 16-weight groups of the part: scales 4 sel + 2 part + g
+        a[g] = h2dup(d * (float)scb[4 * sel + 2 * part + g]);
+    {  // part 0: k 0..31 (ql[l], qh bits 4sel); part 1: k 32..63 (ql[l+32], qh bits 4sel+2)
         const uint8_t *ql = blk + 64 * h + 32 * part;
         const uint8_t *qh = blk + 128 + 32 * h;
         const int sh = 4 * sel + 2 * part;
@@ -203,7 +203,7 @@ __device__ __forceinline__ void dequant_q6(const uint8_t *blk, float d, int kk, 
             for (int u = 0; u < 2; ++u) {
                 const uint32_t q = ((lw[u] >> (4 * sel)) & 0x0F0F0F0Fu) | (((hw[u] >> sh) & 0x03030303u) << 4);
                 const uint32_t t01 = prmt(q, q, 0x1100u), t23 = prmt(q, q, 0x3322u);
-                const uint32_t sc = a[2 * part + (c2 >> 1)];
+                const uint32_t sc = a[c2 >> 1];
                 o[2 * u] = hmul2(hsub2(and_or(t01, 0x003F003Fu, H2_1024), H2_1056D), sc);
                 o[2 * u + 1] = hmul2(hsub2(and_or(t23, 0x003F003Fu, H2_1024), H2_1056D), sc);
             }
@@ -235,8 +235,8 @@ __global__ void __launch_bounds__(dn::THREADS, 1) k_dense_gemm(const __grid_cons
     uint8_t *AS = BS + SB * B_BYTES;
     uint64_t *bar = reinterpret_cast<uint64_t *>(AS + SA * A_BYTES);
     uint64_t *raw_full = bar, *raw_empty = bar + SR, *b_full = bar + 2 * SR, *b_empty = b_full + SB;
-    uint64_t *a_full = b_empty + SB, *a_empty = a_full + SA, *acc_full = a_empty + SA, *acc_empty = acc_full + 1;
-    uint64_t *done = acc_empty + 1;
+    uint64_t *a_full = b_empty + SB, *a_empty = a_full + SA, *acc_full = a_empty + SA, *acc_empty = acc_full + 2;
+    uint64_t *done = acc_empty + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 1);
     __shared__ int s_bad;
     const CUtensorMap *mw = reinterpret_cast<const CUtensorMap *>(mapsb.bytes);
@@ -249,23 +249,25 @@ __global__ void __launch_bounds__(dn::THREADS, 1) k_dense_gemm(const __grid_cons
         s_bad = 0;
         for (int i = 0; i < SR; ++i) {
             mbar_init(&raw_full[i], 1);
-            mbar_init(&raw_empty[i], 4);
+            mbar_init(&raw_empty[i], DQW);
         }
         for (int i = 0; i < SB; ++i) {
             mbar_init(&b_full[i], 1);
             mbar_init(&b_empty[i], 1);
         }
         for (int i = 0; i < SA; ++i) {
-            mbar_init(&a_full[i], 4);
+            mbar_init(&a_full[i], DQW);
             mbar_init(&a_empty[i], 1);
         }
-        mbar_init(acc_full, 1);
-        mbar_init(acc_empty, 4);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&acc_full[i], 1);
+            mbar_init(&acc_empty[i], EPW);
+        }
         mbar_init(done, 1);
         mbar_fence_init();
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, 256);
+        tmem_alloc(tmem_slot, 512);  // two 256-column accumulators
         tmem_relinquish();
     }
     tc_fence_before();
@@ -324,8 +326,9 @@ __global__ void __launch_bounds__(dn::THREADS, 1) k_dense_gemm(const __grid_cons
             int ks = 0, tc = 0;
             bool issued = false;
             for (int t = blockIdx.x; t < tiles && !bad(); t += gridDim.x, ++tc) {
-                if (tc > 0) {
-                    if (!mbar_wait(acc_empty, (tc - 1) & 1)) {
+                const int acc = tc & 1;
+                if (tc >= 2) {  // the epilogue has drained this accumulator's previous tile
+                    if (!mbar_wait(&acc_empty[acc], ((tc >> 1) - 1) & 1)) {
                         fail(ST_ACC);
                         break;
                     }
@@ -343,7 +346,7 @@ __global__ void __launch_bounds__(dn::THREADS, 1) k_dense_gemm(const __grid_cons
                     for (int j = 0; j < 4; ++j) {
                         const uint64_t ad = umma_desc_k_noswz(abase + j * 2 * (TN * 16), TN * 16, 128);
                         const uint64_t bd = umma_desc_k_noswz(bbase + j * 2 * (TM * 16), TM * 16, 128);
-                        umma_f16_ss(tmem, ad, bd, idesc, (k | j) != 0);
+                        umma_f16_ss(tmem + 256 * acc, ad, bd, idesc, (k | j) != 0);
                     }
                     issued = true;
                     umma_commit(&a_empty[sa]);
@@ -351,7 +354,7 @@ __global__ void __launch_bounds__(dn::THREADS, 1) k_dense_gemm(const __grid_cons
                 }
                 if (bad())
                     break;
-                umma_commit(acc_full);
+                umma_commit(&acc_full[acc]);
             }
             // every MMA this thread issued has completed before TMEM is freed
             if (issued) {
@@ -360,13 +363,12 @@ __global__ void __launch_bounds__(dn::THREADS, 1) k_dense_gemm(const __grid_cons
                     fail(ST_DONE);
             }
         }
-    } else {
-        // ------------------------------------------------ dequant + epilogue (weight row n)
-        const int quarter = warp & 3;
+    } else if (warp < 2 + DQW) {
+        // ------------------------------------------------ dequant (weight row n, one k half)
+        const int dw = warp - 2, quarter = dw & 3, half = dw >> 2;
         const int n = 32 * quarter + lane;
-        int bk = 0, ks = 0, tc = 0;
-        for (int t = blockIdx.x; t < tiles && !bad(); t += gridDim.x, ++tc) {
-            const int nt = t / a.mt, mt = t % a.mt;
+        int bk = 0, ks = 0;
+        for (int t = blockIdx.x; t < tiles && !bad(); t += gridDim.x) {
             for (int blk = 0; blk < a.nblk && !bad(); ++blk, ++bk) {
                 const int s = bk % SR;
                 if (!__all_sync(0xffffffffu, mbar_wait(&raw_full[s], (bk / SR) & 1))) {
@@ -376,8 +378,8 @@ __global__ void __launch_bounds__(dn::THREADS, 1) k_dense_gemm(const __grid_cons
                 const uint8_t *st = RAW + s * R::BYTES;
                 float d6 = 0.f;
                 if (FMT == 6) {
-                    const uint32_t dw = lds_u32(st + R::W + n * 16 + (blk & 6) * 2);
-                    d6 = __half2float(__ushort_as_half((unsigned short)(dw >> ((blk & 1) * 16))));
+                    const uint32_t dwd = lds_u32(st + R::W + n * 16 + (blk & 6) * 2);
+                    d6 = __half2float(__ushort_as_half((unsigned short)(dwd >> ((blk & 1) * 16))));
                 }
                 for (int kk = 0; kk < 4; ++kk, ++ks) {
                     const int sa = ks % SA;
@@ -387,9 +389,9 @@ __global__ void __launch_bounds__(dn::THREADS, 1) k_dense_gemm(const __grid_cons
                     }
                     uint8_t *A = AS + sa * A_BYTES;
                     if (FMT == 4)
-                        dequant_q4(st + n * 144, kk, A, n);
+                        dequant_q4(st + n * 144, kk, half, A, n);
                     else
-                        dequant_q6(st + n * Q6A, d6, kk, A, n);
+                        dequant_q6(st + n * Q6A, d6, kk, half, A, n);
                     fence_proxy_async();
                     __syncwarp();
                     if (lane == 0)
@@ -399,39 +401,49 @@ __global__ void __launch_bounds__(dn::THREADS, 1) k_dense_gemm(const __grid_cons
                 if (lane == 0)
                     mbar_arrive(&raw_empty[s]);
             }
-            if (bad())
-                break;
-            // epilogue: D[n][m] * 2^-e_m -> Y[m][n]
-            if (!__all_sync(0xffffffffu, mbar_wait(acc_full, tc & 1))) {
+        }
+    } else {
+        // ------------------------------------------------ epilogue: D[n][m] * 2^-e_m -> Y[m][n]
+        const int quarter = warp & 3;  // TMEM lanes 32 quarter .. + 31 (this warp's access window)
+        const int n = 32 * quarter + lane;
+        int tc = 0;
+        for (int t = blockIdx.x; t < tiles && !bad(); t += gridDim.x, ++tc) {
+            const int nt = t / a.mt, mt = t % a.mt, acc = tc & 1;
+            float rsv[TM / 32];  // row scales of this tile's 256 activation rows, 8 per lane
+#pragma unroll
+            for (int i = 0; i < TM / 32; ++i)
+                rsv[i] = a.rs[mt * TM + 32 * i + lane];
+            if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[acc], (tc >> 1) & 1))) {
                 fail(ST_ACC);
                 break;
             }
             tc_fence_after();
             const int ng = nt * TN + n;
-#pragma unroll 1
+            const bool col_ok = ng < a.N;
+#pragma unroll
             for (int j = 0; j < TM / 16; ++j) {
                 uint32_t v[16];
-                tmem_ld_x16(tmem + ((uint32_t)(32 * quarter) << 16) + 16 * j, v);
+                tmem_ld_x16(tmem + 256 * acc + ((uint32_t)(32 * quarter) << 16) + 16 * j, v);
                 tmem_wait_ld();
-                const int m0 = mt * TM + 16 * j;
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    const int m = m0 + i;
-                    if (m < a.M && ng < a.N)
-                        a.Y[(size_t)m * a.ldy + ng] = __uint_as_float(v[i]) * a.rs[m];
+                    const int mm = 16 * j + i, m = mt * TM + mm;
+                    const float r = __shfl_sync(0xffffffffu, rsv[mm / 32], mm % 32);
+                    if (m < a.M && col_ok)
+                        a.Y[(size_t)m * a.ldy + ng] = __uint_as_float(v[i]) * r;
                 }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
-                mbar_arrive(acc_empty);
+                mbar_arrive(&acc_empty[acc]);
         }
     }
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, 256);
+        tmem_dealloc(tmem, 512);
     }
 }
 
