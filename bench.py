@@ -475,6 +475,17 @@ def run_kernel(args):
         fn = lambda i, st: gemm(Ws[i % 2], N, K, X, M, Y, ws=ws, stream=st)  # noqa: E731
         nbytes = Ws[0].numel()
         flops = 2.0 * M * N * K
+    elif args.kernel == "pfattn23k":
+        len_, C, n_qh, n_kvh = 23000, 2048, 48, 8
+        cap = len_ + C
+        Kd = synth.bf16_normal_torch(g, (n_kvh, cap, 128), "cuda")
+        Vd = synth.bf16_normal_torch(g, (n_kvh, cap, 128), "cuda")
+        Qd = synth.bf16_normal_torch(g, (C, n_qh, 128), "cuda")
+        O = torch.zeros(C, n_qh, 128, dtype=torch.bfloat16, device="cuda")
+        fn = lambda i, st: q.prefill_attn(Qd, Kd, Vd, len_, C, cap, n_qh, n_kvh, 128, O, stream=st)  # noqa: E731
+        nbytes = 2 * n_kvh * cap * 128 * 2
+        # QK^T and PV over the visible keys: row j sees len + j + 1 keys
+        flops = 4.0 * 128 * n_qh * (C * (len_ + 1) + C * (C - 1) / 2)
     elif args.kernel == "attn23k":
         A, L, n_qh, n_kvh = 4, 23000, 48, 8
         cap = L + 3
@@ -501,7 +512,7 @@ def run_kernel(args):
         gemm = q.q4k_gemm if fmt == 4 else q.q6k_gemm
         fn = lambda i, st: gemm(Ws[i % 8], N, K, X, M, Y, ws=ws, stream=st)  # noqa: E731
         nbytes = Ws[0].numel()
-    if args.kernel not in DENSE_KERNELS:
+    if args.kernel not in DENSE_KERNELS and args.kernel != "pfattn23k":
         flops = None
     # 8 calls (8 weight copies) captured once and replayed: device time only, no host launch cost
     stream = torch.cuda.Stream()
@@ -528,9 +539,10 @@ def run_kernel(args):
            "device_status": q.device_status()}
     if flops:
         peak = measured_bf16_tflops()
-        out.update({"rows": DENSE_KERNELS[args.kernel][3], "tflops": flops / us / 1e6, "flop_per_call": flops,
+        out.update({"rows": DENSE_KERNELS[args.kernel][3] if args.kernel in DENSE_KERNELS else 2048,
+                    "tflops": flops / us / 1e6, "flop_per_call": flops,
                     "peak_tflops": peak, "frac": flops / us / 1e6 / peak if peak else None,
-                    "dense_status": q.dense_status()})
+                    "dense_status": q.dense_status() if args.kernel in DENSE_KERNELS else None})
     print(json.dumps(out), flush=True)
     return 0
 
@@ -543,7 +555,7 @@ def main():
     ap.add_argument("--workload", default="stack12_ctx1k", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel", choices=sorted(list(KERNELS) + list(DENSE_KERNELS) + ["attn23k"]),
+    ap.add_argument("--kernel", choices=sorted(list(KERNELS) + list(DENSE_KERNELS) + ["attn23k", "pfattn23k"]),
                     help="time one kernel of the step instead (profiler captures)")
     ap.add_argument("--rows", type=int, default=12)
     args = ap.parse_args()

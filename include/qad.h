@@ -192,6 +192,22 @@ int qad_decode_attn(const uint16_t *Q, const uint16_t *Kc, const uint16_t *Vc, c
                     int n_qh, int n_kvh, int hd, float scale, uint16_t *O, void *ws, size_t ws_bytes,
                     void *stream);
 
+/* ---------------------------------------------------------------- prefill-chunk attention
+ * OpenJet page, section 真正重要的是少互相堵车: a prompt chunk of one agent
+ * (C rows at positions len .. len+C-1) attends causally over the agent's own
+ * cache: row j, q-head h (kv-head h / (n_qh/n_kvh)) sees keys 0 .. len+j,
+ *   o = softmax(q . K[0..len+j]^T * scale) V[0..len+j]
+ * (the decode attention's definition with C rows). The chunk's k, v must
+ * already be in the cache at positions len .. len+C-1.
+ *   Q       device bf16 [C][n_qh][128]
+ *   Kc, Vc  device bf16 [n_kvh][kv_cap][128] (this agent's cache); len + C <= kv_cap
+ *   O       device bf16 [C][n_qh][128], written
+ * Tensor-core products with fp32 softmax; the probabilities enter the PV
+ * product rounded to bf16 (relative error <= 2^-9). hd must be 128. Q, caches
+ * and O 16-byte aligned. Returns 0 or a negative QAD_ERR_* code. */
+int qad_prefill_attn(const uint16_t *Q, const uint16_t *Kc, const uint16_t *Vc, int len, int C, int kv_cap,
+                     int n_qh, int n_kvh, int hd, float scale, uint16_t *O, void *stream);
+
 /* ---------------------------------------------------------------- row packer
  * Host-only. Stacks every agent's rows (next token + drafts) agent-major into
  * one batch ([OpenJet page], section 只搬一次权重). An agent paused for a tool

@@ -60,6 +60,7 @@ SIGNATURES = {
     "qad_q6k_gemm_dense": (C.c_int, [C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p,
                                      C.c_size_t, C.c_void_p]),
     "qad_dense_status": (C.c_int, [C.c_int]),
+    "qad_prefill_attn": (C.c_int, [C.c_void_p] * 3 + [C.c_int] * 6 + [C.c_float, C.c_void_p, C.c_void_p]),
     "qad_decode_attn_ws_bytes": (C.c_size_t, [C.c_int] * 5),
     "qad_decode_attn": (C.c_int, [C.c_void_p] * 5 + [C.c_int] * 6 + [C.c_float, C.c_void_p, C.c_void_p,
                                                                      C.c_size_t, C.c_void_p]),
@@ -259,6 +260,17 @@ def decode_attn(Q, Kc, Vc, lens, agent_row_start, n_agents, max_rows_per_agent, 
 
 
 # ------------------------------------------------------------------ row packer (host)
+
+def prefill_attn(Q, Kc, Vc, len_, C, kv_cap, n_qh, n_kvh, hd, O, scale=None, stream=None):
+    """Causal attention of a C-row prompt chunk at positions len_.. over one agent's cache
+    (Kc, Vc bf16 [n_kvh][kv_cap][hd] holding the chunk's k, v); O bf16 [C][n_qh][hd]."""
+    _require_gpu()
+    if scale is None:
+        scale = hd ** -0.5
+    _check(lib().qad_prefill_attn(_dev(Q, "Q"), _dev(Kc, "Kc"), _dev(Vc, "Vc"), int(len_), int(C), int(kv_cap),
+                                  n_qh, n_kvh, hd, float(scale), _dev(O, "O"), _stream(stream)), "qad_prefill_attn")
+    return O
+
 
 def pack_rows(agent_rows, lens, hidden: int, max_rows: int = QAD_MAX_ROWS):
     """agent_rows: list of CPU bf16 tensors [n_a, hidden] (n_a may be 0).
