@@ -315,6 +315,15 @@ int qad_model_set_debug(qad_model *model, void *dbg, size_t bytes);
  * of classes. Read after every profiled
  * step (a step not read before the next one is dropped). Enabling resets the
  * totals. Graph capture refuses a model with the profiler on. */
+/* Per-launch device trace (works in eager steps and in graphs captured while
+ * it is attached). With a device buffer of 3 * n_records u64 attached, launch
+ * k of each following step (k < n_records; launch order: init, then per layer
+ * prep, qkv GEMM, attention, prep, o GEMM, prep, gate|up GEMM, prep, down
+ * GEMM) records %globaltimer nanoseconds into words 3k..3k+2 with atomicMin:
+ * the first CTA's start, the first CTA past its wait on the previous kernel,
+ * and the bitwise NOT of the last warp's exit. Fill the buffer with 0xFF bytes
+ * before a step. Pass buf = NULL to detach. Returns 0 or QAD_ERR_INVALID. */
+int qad_model_set_trace(qad_model *model, unsigned long long *buf, int n_records);
 int qad_model_set_profile(qad_model *model, int enable);
 int qad_model_profile_read(qad_model *model, double *ms, long long *count, int n_kinds);
 

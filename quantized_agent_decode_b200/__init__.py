@@ -81,6 +81,7 @@ SIGNATURES = {
     "qad_decode_step_launches": (C.c_int, [C.c_void_p]),
     "qad_decode_step_debug_bytes": (C.c_size_t, [C.c_void_p, C.c_int]),
     "qad_model_set_debug": (C.c_int, [C.c_void_p, C.c_void_p, C.c_size_t]),
+    "qad_model_set_trace": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int]),
     "qad_model_set_profile": (C.c_int, [C.c_void_p, C.c_int]),
     "qad_model_profile_read": (C.c_int, [C.c_void_p, C.POINTER(C.c_double), C.POINTER(C.c_longlong), C.c_int]),
 }
@@ -342,6 +343,27 @@ class Model:
         self._dbg = alloc_ws(n)
         _check(lib().qad_model_set_debug(self.handle, _dev(self._dbg, "dbg"), n), "qad_model_set_debug")
         return self._dbg
+
+    def set_trace(self, enable: bool):
+        """Attach (or detach) a per-launch device trace buffer; returns it (int64 [launches][3])."""
+        if not enable:
+            _check(lib().qad_model_set_trace(self.handle, None, 0), "qad_model_set_trace")
+            self._trace = None
+            return None
+        n = self.launches()
+        self._trace = torch.full((n, 3), -1, dtype=torch.int64, device="cuda")
+        _check(lib().qad_model_set_trace(self.handle, C.c_void_p(self._trace.data_ptr()), n), "qad_model_set_trace")
+        return self._trace
+
+    def trace_reset(self, stream=None):
+        self._trace.fill_(-1)
+
+    def trace_read(self):
+        """Per launch (start_ns, ready_ns, end_ns) relative to the first start, as a CPU int64 tensor."""
+        t = self._trace.cpu()
+        end = ~t[:, 2]
+        out = torch.stack([t[:, 0], t[:, 1], end], 1)
+        return out - out[:, 0].min()
 
     def set_profile(self, enable: bool):
         _check(lib().qad_model_set_profile(self.handle, int(bool(enable))), "qad_model_set_profile")

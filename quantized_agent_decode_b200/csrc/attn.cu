@@ -39,6 +39,7 @@ struct AttnArgs {
     int n_kvh, kv_cap, n_qh, G, CH, n_rg, max_splits;
     float scale_log2;
     float *part;
+    unsigned long long *trace;
 };
 
 __device__ __forceinline__ int swz(int key, int chunk) { return key * 256 + ((chunk ^ (key & 7)) << 4); }
@@ -54,53 +55,28 @@ __global__ void __launch_bounds__(128, 2) k_decode_attn(AttnArgs p)
     const int sp = blockIdx.x, rg = blockIdx.y, ag = blockIdx.z;
     const int a = ag / p.n_kvh, g = ag - a * p.n_kvh;
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31, gq = lane >> 2, c = lane & 3;
+    trace_start(p.trace);
     pdl_trigger();
-    pdl_wait();
+    // Agent offsets, lengths and the cached keys below len are constant for the
+    // whole step, so they are read before waiting on the previous kernel; Q and
+    // the new rows' k, v (fused form) only after it.
     const int r0 = p.ars[a], na = p.ars[a + 1] - r0;
     const int len = p.lens[a];
     const int R = na * p.G;
     const int q0 = rg * QG;
-    if (q0 >= R)
+    if (q0 >= R) {
+        trace_end(p.trace);
         return;
+    }
     const int L = min(len + na, p.kv_cap);
     const int kbeg = sp * p.CH;
-    if (kbeg >= L)
+    if (kbeg >= L) {
+        trace_end(p.trace);
         return;
+    }
     const int kend = min(L, kbeg + p.CH);
     const size_t head_off = ((size_t)a * p.n_kvh + g) * (size_t)p.kv_cap * 128;
     const uint16_t *Kh = p.Kc + head_off, *Vh = p.Vc + head_off;
-
-    // Q^T fragments: b0 = Q[q][16ks+2c..], b1 = Q[q][16ks+8+2c..] for q = q0 + 8nt + gq
-    uint32_t qf[3][8][2];
-    int qpos[3][2];  // last visible key of the two query columns this lane owns (per nt)
-#pragma unroll
-    for (int nt = 0; nt < 3; ++nt) {
-        const int qi = q0 + 8 * nt + gq;
-        const bool ok = qi < R;
-        const int j = ok ? qi / p.G : 0, hl = ok ? qi - j * p.G : 0;
-        if (FUSED) {
-            const float *qrow = p.qkv + (size_t)(r0 + j) * p.ldqkv + (g * p.G + hl) * 128;
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const float2 f0 = ok ? *reinterpret_cast<const float2 *>(qrow + 16 * ks + 2 * c) : make_float2(0.f, 0.f);
-                const float2 f1 = ok ? *reinterpret_cast<const float2 *>(qrow + 16 * ks + 8 + 2 * c) : make_float2(0.f, 0.f);
-                qf[nt][ks][0] = pack_bf162(f0.x, f0.y);
-                qf[nt][ks][1] = pack_bf162(f1.x, f1.y);
-            }
-        } else {
-            const uint16_t *qrow = p.Q + ((size_t)(r0 + j) * p.n_qh + g * p.G + hl) * 128;
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                qf[nt][ks][0] = ok ? *reinterpret_cast<const uint32_t *>(qrow + 16 * ks + 2 * c) : 0u;
-                qf[nt][ks][1] = ok ? *reinterpret_cast<const uint32_t *>(qrow + 16 * ks + 8 + 2 * c) : 0u;
-            }
-        }
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const int qc = q0 + 8 * nt + 2 * c + e;
-            qpos[nt][e] = qc < R ? len + qc / p.G : -1;
-        }
-    }
 
     float o[8][3][4];
 #pragma unroll
@@ -167,12 +143,54 @@ __global__ void __launch_bounds__(128, 2) k_decode_attn(AttnArgs p)
             cp_async16_zfill(st + TILE_BYTES + swz(kk, ch), Vh + src, ok);
         }
     };
-    if (my > 0)
-        issue(0);
-    cp_async_commit();
-    if (my > 1)
-        issue(1);
-    cp_async_commit();
+    // tiles of cached keys only (always the earlier ones) stream before the wait
+    auto cached_tile = [&](int it) { return !FUSED || kbeg + KT * (w + ATT_WARPS * it) + KT <= len; };
+    int pre = 0;
+    while (pre < 2 && pre < my && cached_tile(pre)) {
+        issue(pre);
+        cp_async_commit();
+        ++pre;
+    }
+    pdl_wait();
+    trace_ready(p.trace);
+    for (int it = pre; it < 2; ++it) {
+        if (it < my)
+            issue(it);
+        cp_async_commit();
+    }
+
+    // Q^T fragments: b0 = Q[q][16ks+2c..], b1 = Q[q][16ks+8+2c..] for q = q0 + 8nt + gq
+    uint32_t qf[3][8][2];
+    int qpos[3][2];  // last visible key of the two query columns this lane owns (per nt)
+#pragma unroll
+    for (int nt = 0; nt < 3; ++nt) {
+        const int qi = q0 + 8 * nt + gq;
+        const bool ok = qi < R;
+        const int j = ok ? qi / p.G : 0, hl = ok ? qi - j * p.G : 0;
+        if (FUSED) {
+            const float *qrow = p.qkv + (size_t)(r0 + j) * p.ldqkv + (g * p.G + hl) * 128;
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const float2 f0 = ok ? *reinterpret_cast<const float2 *>(qrow + 16 * ks + 2 * c) : make_float2(0.f, 0.f);
+                const float2 f1 = ok ? *reinterpret_cast<const float2 *>(qrow + 16 * ks + 8 + 2 * c) : make_float2(0.f, 0.f);
+                qf[nt][ks][0] = pack_bf162(f0.x, f0.y);
+                qf[nt][ks][1] = pack_bf162(f1.x, f1.y);
+            }
+        } else {
+            const uint16_t *qrow = p.Q + ((size_t)(r0 + j) * p.n_qh + g * p.G + hl) * 128;
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                qf[nt][ks][0] = ok ? *reinterpret_cast<const uint32_t *>(qrow + 16 * ks + 2 * c) : 0u;
+                qf[nt][ks][1] = ok ? *reinterpret_cast<const uint32_t *>(qrow + 16 * ks + 8 + 2 * c) : 0u;
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int qc = q0 + 8 * nt + 2 * c + e;
+            qpos[nt][e] = qc < R ? len + qc / p.G : -1;
+        }
+    }
+
 
     for (int it = 0; it < my; ++it) {
         if (it + 2 < my)
@@ -318,6 +336,7 @@ __global__ void __launch_bounds__(128, 2) k_decode_attn(AttnArgs p)
         out[QG * 128 + tid] = M;
         out[QG * 128 + QG + tid] = Lsum;
     }
+    trace_end(p.trace);
 }
 
 // One CTA per (query vector, row group, agent*kv-head); thread = dimension.
@@ -423,9 +442,10 @@ static AttnArgs attn_args(const AttnPlan &pl, const int *lens, const int *ars, i
 
 int launch_attn_fused(const AttnPlan &pl, const float *qkv, int ldqkv, uint16_t *Kc, uint16_t *Vc, const int *lens,
                       const int *ars, int n_agents, int kv_cap, int n_qh, int n_kvh, float scale, float *part,
-                      cudaStream_t s, bool pdl)
+                      cudaStream_t s, bool pdl, unsigned long long *trace)
 {
     AttnArgs p = attn_args(pl, lens, ars, kv_cap, n_qh, n_kvh, scale, part);
+    p.trace = trace;
     p.qkv = qkv;
     p.ldqkv = ldqkv;
     p.Kc = Kc;

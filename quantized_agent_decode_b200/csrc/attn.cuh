@@ -37,7 +37,7 @@ int launch_attn(const AttnPlan &pl, const uint16_t *Q, const uint16_t *Kc, const
 // (the o-projection prep merges them).
 int launch_attn_fused(const AttnPlan &pl, const float *qkv, int ldqkv, uint16_t *Kc, uint16_t *Vc, const int *lens,
                       const int *ars, int n_agents, int kv_cap, int n_qh, int n_kvh, float scale, float *part,
-                      cudaStream_t s, bool pdl);
+                      cudaStream_t s, bool pdl, unsigned long long *trace = nullptr);
 AttnPartView attn_part_view(const AttnPlan &pl, const float *part, const int *ars, const int *lens, int kv_cap,
                             int n_qh, int n_kvh);
 

@@ -47,6 +47,32 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 // ----------------------------------------------------------------- PDL controls
 
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Optional per-launch trace record: 3 x u64 of %globaltimer ns, all reduced with
+// atomicMin so one 0xFF fill resets them: [0] first CTA start, [1] first CTA
+// past its dependency wait, [2] ~(last warp exit).
+__device__ __forceinline__ unsigned long long gtimer()
+{
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ void trace_start(unsigned long long *rec)
+{
+    if (rec && threadIdx.x == 0)
+        atomicMin(rec, gtimer());
+}
+__device__ __forceinline__ void trace_ready(unsigned long long *rec)
+{
+    if (rec && threadIdx.x == 0)
+        atomicMin(rec + 1, gtimer());
+}
+// called by one lane of every warp as it finishes
+__device__ __forceinline__ void trace_end(unsigned long long *rec)
+{
+    if (rec && (threadIdx.x & 31) == 0)
+        atomicMin(rec + 2, ~gtimer());
+}
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // ----------------------------------------------------------------- loads

@@ -108,6 +108,7 @@ struct PrepArgs {
     PrepSrc src;
     int K, M;
     FragBuf fb;
+    unsigned long long *trace;
 };
 
 __device__ __forceinline__ float warp_sum(float v)
@@ -151,8 +152,31 @@ __global__ void __launch_bounds__(256) k_prep(PrepArgs a)
     const int K = a.K, nblk = K >> 8;
     const int b = 4 * blockIdx.x + q;
     const PrepSrc &S = a.src;
+    trace_start(a.trace);
     pdl_trigger();
+    const bool live = r < a.M;
+    const bool act = live && b < nblk;
+    const int k = 256 * b + 4 * t;
+    // PREP_ATTN: which agent / query vector / partial records this thread merges.
+    // Agent offsets and lengths are constant for the whole step, so they are read
+    // before waiting on the previous kernel.
+    const float *att_base = nullptr;
+    int att_nsp = 0, att_qq = 0, att_d = 0;
+    if (S.kind == PREP_ATTN && act) {
+        const AttnPartView &P = S.att;
+        int ag = 0;
+        while (ag + 1 < S.n_agents && P.ars[ag + 1] <= r)
+            ++ag;
+        const int na = P.ars[ag + 1] - P.ars[ag], j = r - P.ars[ag];
+        const int head = k >> 7, g = head / P.G, hl = head - g * P.G;
+        const int qi = j * P.G + hl, rg = qi / ATT_QG;
+        att_qq = qi - rg * ATT_QG;
+        att_d = k & 127;
+        att_nsp = (min(P.lens[ag] + na, P.kv_cap) + P.CH - 1) / P.CH;
+        att_base = P.part + ((((size_t)ag * P.n_kvh + g) * P.n_rg + rg) * P.max_splits) * ATT_PART_FLOATS;
+    }
     pdl_wait();
+    trace_ready(a.trace);
     if (S.zero) {
         const long long nct = (long long)gridDim.x * gridDim.y, ct = (long long)blockIdx.y * gridDim.x + blockIdx.x;
         const long long per = ((S.zero_n + nct - 1) / nct + 3) & ~3LL;
@@ -165,13 +189,17 @@ __global__ void __launch_bounds__(256) k_prep(PrepArgs a)
                 S.zero[i] = 0.f;
         }
     }
-    const bool live = r < a.M;
+    float4 own = make_float4(0.f, 0.f, 0.f, 0.f);  // RMSNorm: this thread's 4 values, kept from the sum pass
     if (S.kind == PREP_RMSNORM && live) {
-        // the whole row's mean square, recomputed by every CTA of the row in the same order
+        // the whole row's mean square, recomputed by every CTA of the row in the same
+        // order; float4 index 256 * blockIdx.x + tid is this thread's own k .. k+3
         const float4 *h4 = reinterpret_cast<const float4 *>(S.xf + (size_t)r * S.ldx);
+        const int mine = 256 * blockIdx.x + tid;
         float ss = 0.f;
         for (int i = tid; i < (K >> 2); i += 256) {
             const float4 v = h4[i];
+            if (i == mine)
+                own = v;
             ss = fmaf(v.x, v.x, ss);
             ss = fmaf(v.y, v.y, ss);
             ss = fmaf(v.z, v.z, ss);
@@ -189,8 +217,6 @@ __global__ void __launch_bounds__(256) k_prep(PrepArgs a)
         }
         __syncthreads();
     }
-    const bool act = live && b < nblk;
-    const int k = 256 * b + 4 * t;
     uint16_t v[4] = {0, 0, 0, 0};
     if (act) {
         if (S.kind == PREP_BF16) {
@@ -200,12 +226,11 @@ __global__ void __launch_bounds__(256) k_prep(PrepArgs a)
             v[2] = (uint16_t)(w.y & 0xFFFF);
             v[3] = (uint16_t)(w.y >> 16);
         } else if (S.kind == PREP_RMSNORM) {
-            const float4 h = *reinterpret_cast<const float4 *>(S.xf + (size_t)r * S.ldx + k);
             const float inv = s_inv;
-            v[0] = f_to_bf16(h.x * inv);
-            v[1] = f_to_bf16(h.y * inv);
-            v[2] = f_to_bf16(h.z * inv);
-            v[3] = f_to_bf16(h.w * inv);
+            v[0] = f_to_bf16(own.x * inv);
+            v[1] = f_to_bf16(own.y * inv);
+            v[2] = f_to_bf16(own.z * inv);
+            v[3] = f_to_bf16(own.w * inv);
         } else if (S.kind == PREP_SILU) {
             const float *gp = S.xf + (size_t)r * S.ldx;
             const float4 g = *reinterpret_cast<const float4 *>(gp + k);
@@ -215,33 +240,24 @@ __global__ void __launch_bounds__(256) k_prep(PrepArgs a)
             v[2] = f_to_bf16(silu_mul(g.z, u.z));
             v[3] = f_to_bf16(silu_mul(g.w, u.w));
         } else {
-            // merge the key splits of query vector (row r, head k / 128), dims k%128 .. +3
-            const AttnPartView &P = S.att;
-            int ag = 0;
-            while (ag + 1 < S.n_agents && P.ars[ag + 1] <= r)
-                ++ag;
-            const int na = P.ars[ag + 1] - P.ars[ag], j = r - P.ars[ag];
-            const int head = k >> 7, d = k & 127;
-            const int g = head / P.G, hl = head - g * P.G;
-            const int qi = j * P.G + hl, rg = qi / ATT_QG, qq = qi - rg * ATT_QG;
-            const int L = min(P.lens[ag] + na, P.kv_cap);
-            const int nsp = (L + P.CH - 1) / P.CH;
-            const float *base = P.part + ((((size_t)ag * P.n_kvh + g) * P.n_rg + rg) * P.max_splits) * ATT_PART_FLOATS;
+            // merge the key splits of query vector (row r, head k / 128), dims k%128 .. +3:
+            // the global max first, then the weighted sums (the loads of each pass are
+            // independent of one another, so they overlap)
             float Mx = -INFINITY;
-            for (int sp = 0; sp < nsp; ++sp)
-                Mx = fmaxf(Mx, base[(size_t)sp * ATT_PART_FLOATS + ATT_QG * 128 + qq]);
+            for (int sp = 0; sp < att_nsp; ++sp)
+                Mx = fmaxf(Mx, att_base[(size_t)sp * ATT_PART_FLOATS + ATT_QG * 128 + att_qq]);
             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
             float Ls = 0.f;
             if (Mx != -INFINITY)
-                for (int sp = 0; sp < nsp; ++sp) {
-                    const float *pp = base + (size_t)sp * ATT_PART_FLOATS;
-                    const float wgt = exp2f(pp[ATT_QG * 128 + qq] - Mx);
-                    const float4 o = *reinterpret_cast<const float4 *>(pp + qq * 128 + d);
+                for (int sp = 0; sp < att_nsp; ++sp) {
+                    const float *pp = att_base + (size_t)sp * ATT_PART_FLOATS;
+                    const float wgt = exp2f(pp[ATT_QG * 128 + att_qq] - Mx);
+                    const float4 o = *reinterpret_cast<const float4 *>(pp + att_qq * 128 + att_d);
                     acc.x += wgt * o.x;
                     acc.y += wgt * o.y;
                     acc.z += wgt * o.z;
                     acc.w += wgt * o.w;
-                    Ls += wgt * pp[ATT_QG * 128 + ATT_QG + qq];
+                    Ls += wgt * pp[ATT_QG * 128 + ATT_QG + att_qq];
                 }
             const bool pos = Ls > 0.f;
             v[0] = f_to_bf16(pos ? acc.x / Ls : 0.f);
@@ -272,8 +288,10 @@ __global__ void __launch_bounds__(256) k_prep(PrepArgs a)
         frexpf(mx, &E);  // mx in [2^(E-1), 2^E)
         e = min(126, max(-126, 10 - E));
     }
-    if (b >= nblk)
+    if (b >= nblk) {
+        trace_end(a.trace);
         return;
+    }
     const float sc = ldexpf(1.f, e);
     uint8_t *rec = a.fb.rec + (size_t)b * rec_bytes(FMT, NT);
     const int g = r & 7, nt = r >> 3;
@@ -297,6 +315,7 @@ __global__ void __launch_bounds__(256) k_prep(PrepArgs a)
     }
     if (t == 0)
         reinterpret_cast<float *>(rec + rec_bytes(FMT, NT) - 64)[r] = live ? ldexpf(1.f, -e) : 0.f;
+    trace_end(a.trace);
 }
 
 // ------------------------------------------------------------- GEMM kernels
@@ -324,10 +343,17 @@ constexpr int Q6A_BYTES = 208;       // plane A bytes per Q6_K block
 // of CG, so unit i and unit i + S (the next use of a stage) belong to the same
 // group: a group never waits on a stage phase whose predecessor it has not
 // itself seen complete (parity waits cannot tell phase u from phase u - 2).
+// Consumer groups per CTA (build-time tunables).
+#ifndef QAD_Q4_GROUPS
+#define QAD_Q4_GROUPS 3
+#endif
+#ifndef QAD_Q6_GROUPS
+#define QAD_Q6_GROUPS 2
+#endif
 template <int FMT>
 struct Cfg {
     static constexpr int GW = 4;                       // warps per consumer group
-    static constexpr int CG = FMT == 4 ? 3 : 2;        // consumer groups
+    static constexpr int CG = FMT == 4 ? QAD_Q4_GROUPS : QAD_Q6_GROUPS;  // consumer groups
     static constexpr int TILE = RW * GW;               // weight rows per unit
     static constexpr int S = 6;                        // pipeline stages
     static constexpr int THREADS = 32 * (CG * GW + 1);
@@ -363,6 +389,7 @@ struct GemmArgs {
     int N, nblk, M, ldy, units;
     const uint8_t *rec;  // operand records, rec_bytes(FMT, NT) apart
     float *Y;
+    unsigned long long *trace;
 };
 
 enum { ERR_FULL_TIMEOUT = 1, ERR_EMPTY_TIMEOUT = 2 };
@@ -614,6 +641,7 @@ __global__ void __launch_bounds__(Cfg<FMT>::THREADS, 1) k_qgemm(const __grid_con
         mbar_fence_init();
     }
     __syncthreads();
+    trace_start(a.trace);
     pdl_trigger();
 
     if (warp == CG * GW) {
@@ -667,6 +695,7 @@ __global__ void __launch_bounds__(Cfg<FMT>::THREADS, 1) k_qgemm(const __grid_con
         for (int k = max(0, i - S); k < i; ++k)
             if (!mbar_wait(&full[k % S], (k / S) & 1, 20000))
                 atomicExch(&g_gemm_status, ERR_FULL_TIMEOUT);
+        trace_end(a.trace);
         return;
     }
 
@@ -677,6 +706,7 @@ __global__ void __launch_bounds__(Cfg<FMT>::THREADS, 1) k_qgemm(const __grid_con
     const uint32_t selT = (uint32_t)(jj | ((jj + 1) << 4) | ((jj + 4) << 8) | ((jj + 5) << 12));
     const bool hib = c >= 2;
     pdl_wait();
+    trace_ready(a.trace);
     float tot[2][NT][4];
 #pragma unroll
     for (int mt = 0; mt < 2; ++mt)
@@ -720,6 +750,7 @@ __global__ void __launch_bounds__(Cfg<FMT>::THREADS, 1) k_qgemm(const __grid_con
         t = tn;
         b = bn;
     }
+    trace_end(a.trace);
 }
 
 // Q6_K-like GGUF blocks -> packed device layout (plane A: first 208 bytes of
@@ -763,10 +794,11 @@ static int set_smem(K kernel, size_t bytes)
 
 int frag_nt(int M) { return M <= 8 ? 1 : 2; }
 
-int launch_prep(int fmt, int K, int M, const PrepSrc &src, const FragBuf &fb, cudaStream_t s, bool pdl)
+int launch_prep(int fmt, int K, int M, const PrepSrc &src, const FragBuf &fb, cudaStream_t s, bool pdl,
+                unsigned long long *trace)
 {
     const int nt = frag_nt(M);
-    PrepArgs a{src, K, M, fb};
+    PrepArgs a{src, K, M, fb, trace};
     void (*kern)(PrepArgs);
     if (fmt == 4)
         kern = nt == 1 ? k_prep<4, 1> : k_prep<4, 2>;
@@ -796,7 +828,7 @@ int make_weight_maps(int fmt, const void *W, int N, int K, WeightMapsBlob *out)
 }
 
 int launch_gemm(int fmt, const WeightMapsBlob &maps_blob, int N, int K, int M, const FragBuf &fb, float *Y, int ldy,
-                cudaStream_t s, bool pdl)
+                cudaStream_t s, bool pdl, unsigned long long *trace)
 {
     const int nt = frag_nt(M);
     const WeightMaps &maps = reinterpret_cast<const WeightMaps &>(maps_blob);
@@ -809,6 +841,7 @@ int launch_gemm(int fmt, const WeightMapsBlob &maps_blob, int N, int K, int M, c
     a.units = ((N + tile - 1) / tile) * a.nblk;
     a.rec = fb.rec;
     a.Y = Y;
+    a.trace = trace;
     void (*kern)(const WeightMaps, GemmArgs);
     size_t smem;
     if (fmt == 4) {

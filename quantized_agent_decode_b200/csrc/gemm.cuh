@@ -44,9 +44,11 @@ struct alignas(64) WeightMapsBlob {
 int make_weight_maps(int fmt, const void *W, int N, int K, WeightMapsBlob *out);
 // The prep runs one 256-thread CTA per (row < 8*nt, group of 4 blocks); the
 // GEMM runs one CTA per SM.
-int launch_prep(int fmt, int K, int M, const PrepSrc &src, const FragBuf &fb, cudaStream_t s, bool pdl);
+// trace: optional 3-word launch record (see trace_start in common.cuh), or nullptr.
+int launch_prep(int fmt, int K, int M, const PrepSrc &src, const FragBuf &fb, cudaStream_t s, bool pdl,
+                unsigned long long *trace = nullptr);
 int launch_gemm(int fmt, const WeightMapsBlob &maps, int N, int K, int M, const FragBuf &fb, float *Y, int ldy,
-                cudaStream_t s, bool pdl);
+                cudaStream_t s, bool pdl, unsigned long long *trace = nullptr);
 size_t q6k_packed_bytes(long long N, int K);
 int launch_q6k_pack(const void *W, int N, int K, void *P, cudaStream_t s);
 

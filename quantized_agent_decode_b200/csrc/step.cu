@@ -50,6 +50,8 @@ struct qad_model {
     std::vector<uint16_t *> kc, vc;
     void *dbg = nullptr;
     size_t dbg_bytes = 0;
+    unsigned long long *trace = nullptr;  // 3 words per launch (see trace_start)
+    int trace_n = 0;
     // graph cache of the host-buffer entry point
     qad_step_graph *hg = nullptr;
     int hg_M = -1, hg_agents = -1, hg_rows = -1;
@@ -141,12 +143,15 @@ static DbgLayout dbg_layout(const qad_model_desc &d, int M)
 }
 
 // h[r][k] = X[r][k] (bf16 -> fp32): the residual stream starts at the input rows.
-__global__ void k_init_h(const uint16_t *__restrict__ X, float *__restrict__ h, int n)
+__global__ void k_init_h(const uint16_t *__restrict__ X, float *__restrict__ h, int n, unsigned long long *trace)
 {
+    trace_start(trace);
     pdl_trigger();
     pdl_wait();
+    trace_ready(trace);
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x)
         h[i] = bf16_to_f(X[i]);
+    trace_end(trace);
 }
 
 // Profiler: events around each launch (serialises the chain; eager steps only).
@@ -213,7 +218,12 @@ static int run_step(qad_model *m, const uint16_t *X, int M, const int *ars, int 
         if ((rc = P.end()))                             \
             return rc;                                  \
     } while (0)
-    QAD_PROF(PK_INIT, (k_init_h<<<(M * H + 255) / 256, 256, 0, s>>>(X, h, M * H),
+    int slot = 0;
+    auto tr = [&]() -> unsigned long long * {  // this launch's trace record, if tracing
+        const int k = slot++;
+        return m->trace && k < m->trace_n ? m->trace + 3 * (size_t)k : nullptr;
+    };
+    QAD_PROF(PK_INIT, (k_init_h<<<(M * H + 255) / 256, 256, 0, s>>>(X, h, M * H, tr()),
                        cuda_check(cudaGetLastError(), "init launch")));
     for (int l = 0; l < d.n_layers; ++l) {
         char *dbg = m->dbg ? (char *)m->dbg + (size_t)l * DL.per_layer : nullptr;
@@ -228,13 +238,13 @@ static int run_step(qad_model *m, const uint16_t *X, int M, const int *ars, int 
         src.zero_n = (long long)M * nqkv;
         src.dbg = dbg ? (uint16_t *)(dbg + DL.x1) : nullptr;
         src.ld_dbg = H;
-        QAD_PROF(PK_PREP, launch_prep(4, H, M, src, fb, s, true));
-        QAD_PROF(PK_GEMM_QKV, launch_gemm(4, m->mqkv[l], nqkv, H, M, fb, qkv, nqkv, s, true));
+        QAD_PROF(PK_PREP, launch_prep(4, H, M, src, fb, s, true, tr()));
+        QAD_PROF(PK_GEMM_QKV, launch_gemm(4, m->mqkv[l], nqkv, H, M, fb, qkv, nqkv, s, true, tr()));
         if (dbg && (rc = copy_d2d(dbg + DL.qkv, qkv, (size_t)M * nqkv * 4, s)))
             return rc;
         // attention over each agent's cache; k, v of the new rows appended
         QAD_PROF(PK_ATTN, launch_attn_fused(plan, qkv, nqkv, m->kc[l], m->vc[l], lens, ars, n_agents, d.kv_cap,
-                                            d.n_qh, d.n_kvh, scale, part, s, true));
+                                            d.n_qh, d.n_kvh, scale, part, s, true, tr()));
         // O = merged splits (bf16); h += O Wo^T
         fb = frag_carve(ws + L.frag, nq, nt);
         src = PrepSrc{};
@@ -243,8 +253,8 @@ static int run_step(qad_model *m, const uint16_t *X, int M, const int *ars, int 
         src.n_agents = n_agents;
         src.dbg = dbg ? (uint16_t *)(dbg + DL.attn) : nullptr;
         src.ld_dbg = nq;
-        QAD_PROF(PK_PREP, launch_prep(4, nq, M, src, fb, s, true));
-        QAD_PROF(PK_GEMM_O, launch_gemm(4, m->mo[l], H, nq, M, fb, h, H, s, true));
+        QAD_PROF(PK_PREP, launch_prep(4, nq, M, src, fb, s, true, tr()));
+        QAD_PROF(PK_GEMM_O, launch_gemm(4, m->mo[l], H, nq, M, fb, h, H, s, true, tr()));
         if (dbg && (rc = copy_d2d(dbg + DL.hmid, h, (size_t)M * H * 4, s)))
             return rc;
         // x2 = bf16(rmsnorm(h)) -> gate | up
@@ -258,8 +268,8 @@ static int run_step(qad_model *m, const uint16_t *X, int M, const int *ars, int 
         src.zero_n = (long long)M * 2 * I;
         src.dbg = dbg ? (uint16_t *)(dbg + DL.x2) : nullptr;
         src.ld_dbg = H;
-        QAD_PROF(PK_PREP, launch_prep(4, H, M, src, fb, s, true));
-        QAD_PROF(PK_GEMM_GU, launch_gemm(4, m->mgu[l], 2 * I, H, M, fb, gu, 2 * I, s, true));
+        QAD_PROF(PK_PREP, launch_prep(4, H, M, src, fb, s, true, tr()));
+        QAD_PROF(PK_GEMM_GU, launch_gemm(4, m->mgu[l], 2 * I, H, M, fb, gu, 2 * I, s, true, tr()));
         if (dbg && (rc = copy_d2d(dbg + DL.gu, gu, (size_t)M * 2 * I * 4, s)))
             return rc;
         // h += bf16(silu(gate) * up) Wdown^T
@@ -270,8 +280,8 @@ static int run_step(qad_model *m, const uint16_t *X, int M, const int *ars, int 
         src.ldx = 2 * I;
         src.dbg = dbg ? (uint16_t *)(dbg + DL.act) : nullptr;
         src.ld_dbg = I;
-        QAD_PROF(PK_PREP, launch_prep(6, I, M, src, fb, s, true));
-        QAD_PROF(PK_GEMM_DOWN, launch_gemm(6, m->mdown[l], H, I, M, fb, h, H, s, true));
+        QAD_PROF(PK_PREP, launch_prep(6, I, M, src, fb, s, true, tr()));
+        QAD_PROF(PK_GEMM_DOWN, launch_gemm(6, m->mdown[l], H, I, M, fb, h, H, s, true, tr()));
         if (dbg && (rc = copy_d2d(dbg + DL.hout, h, (size_t)M * H * 4, s)))
             return rc;
     }
@@ -393,6 +403,17 @@ extern "C" int qad_model_set_debug(qad_model *m, void *dbg, size_t bytes)
         return qad::fail(QAD_ERR_INVALID, "qad_model_set_debug: buffer must be 256-byte aligned");
     m->dbg = dbg;
     m->dbg_bytes = bytes;
+    return QAD_OK;
+}
+
+extern "C" int qad_model_set_trace(qad_model *m, unsigned long long *buf, int n_records)
+{
+    if (!m || n_records < 0 || (buf && n_records == 0))
+        return qad::fail(QAD_ERR_INVALID, "qad_model_set_trace: null model or bad record count");
+    if ((uintptr_t)buf & 7)
+        return qad::fail(QAD_ERR_INVALID, "qad_model_set_trace: buffer must be 8-byte aligned");
+    m->trace = buf;
+    m->trace_n = buf ? n_records : 0;
     return QAD_OK;
 }
 
