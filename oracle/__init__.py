@@ -61,6 +61,9 @@ def lib():
         L.orc_pack_rows.restype = C.c_int
         L.orc_pack_rows.argtypes = [C.POINTER(C.c_void_p), i32p, i32p, C.c_int, C.c_int,
                                     u16p, i32p, i32p, i32p]
+        L.orc_argmax.restype = C.c_long
+        L.orc_argmax.argtypes = [f64p, C.c_long]
+        L.orc_accept_greedy.argtypes = [i32p, i32p, i32p, C.c_int, i32p, i32p, i32p]
         L.orc_decode_layer.argtypes = [u8p, u8p, u8p, u8p, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
                                        C.c_double, f64p, C.c_int, i32p, C.c_int, i32p, u16p, u16p,
                                        C.c_int, C.c_int] + [C.c_void_p] * 7
@@ -211,6 +214,26 @@ def pack_rows(agent_rows, lens, H: int):
     m = lib().orc_pack_rows(ptrs, n_rows, np.ascontiguousarray(lens, np.int32), n, H, X, ra, rp, ars)
     assert m == M
     return X[:M], ra[:M], rp[:M], ars
+
+
+def argmax(v: np.ndarray) -> int:
+    """First index of the maximum of a 1-D float64 array."""
+    v = np.ascontiguousarray(v, np.float64)
+    return int(lib().orc_argmax(v, v.size))
+
+
+def accept_greedy(row_argmax, row_tokens, ars, lens):
+    """Greedy draft acceptance: returns (new lens, out_tokens, n_accept)."""
+    ars = np.ascontiguousarray(ars, np.int32)
+    n = len(ars) - 1
+    M = int(ars[-1])
+    lens2 = np.array(lens, np.int32, copy=True)
+    out = np.zeros(max(M, 1), np.int32)
+    acc = np.zeros(max(n, 1), np.int32)
+    lib().orc_accept_greedy(np.ascontiguousarray(row_argmax, np.int32).reshape(-1) if M else np.zeros(1, np.int32),
+                            np.ascontiguousarray(row_tokens, np.int32).reshape(-1) if M else np.zeros(1, np.int32),
+                            ars, n, lens2, out, acc)
+    return lens2, out[:M], acc[:n]
 
 
 def decode_layer(Wqkv, Wo, Wgu, Wdown, H, I, n_qh, n_kvh, hd, h, ars, lens, Kc, Vc, cap,

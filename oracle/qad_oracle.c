@@ -419,6 +419,45 @@ int orc_pack_rows(const uint16_t *const *rows, const int *n_rows, const int *len
     return r;
 }
 
+/* First index of the largest value (ties resolve to the lowest index). */
+long orc_argmax(const double *v, long n)
+{
+    long best = 0;
+    for (long i = 1; i < n; ++i)
+        if (v[i] > v[best])
+            best = i;
+    return best;
+}
+
+/* Greedy verification of the drafts and commit of the KV lengths
+ * ([OpenJet page], section 只搬一次权重: the two draft tokens of every agent
+ * are checked in the same forward pass as its next token). The pages do not
+ * state the acceptance rule; the reading taken is greedy: row j of an agent
+ * (position lens[a] + j, input token row_tokens[r0 + j]) predicts
+ * row_argmax[r0 + j]; draft j + 1 (the input of row j + 1) is accepted iff
+ * every earlier draft was and row_argmax[r0 + j] == row_tokens[r0 + j + 1].
+ * With k drafts accepted the agent emits row_argmax[r0 .. r0 + k] (k + 1
+ * tokens: the accepted drafts and the next token after them), its cache holds
+ * valid keys up to position lens[a] + k, so lens[a] += k + 1; the rows after
+ * r0 + k are rejected (their cache slots are overwritten by the next step).
+ *   out_tokens[r]: the emitted token of row r, or -1 for rejected rows
+ *   n_accept[a]:   k (agents with no rows: 0, lens unchanged) */
+void orc_accept_greedy(const int *row_argmax, const int *row_tokens, const int *ars, int n_agents, int *lens,
+                       int *out_tokens, int *n_accept)
+{
+    for (int a = 0; a < n_agents; ++a) {
+        const int r0 = ars[a], n = ars[a + 1] - ars[a];
+        int k = 0;
+        while (k + 1 < n && row_argmax[r0 + k] == row_tokens[r0 + k + 1])
+            ++k;
+        for (int j = 0; j < n; ++j)
+            out_tokens[r0 + j] = j <= k ? row_argmax[r0 + j] : -1;
+        n_accept[a] = n > 0 ? k : 0;
+        if (n > 0)
+            lens[a] += k + 1;
+    }
+}
+
 /* One decoder layer of the synthetic stack for the packed batch, with the
  * rounding points of the design notes:
  *   x1  = bf16(rmsnorm(h))

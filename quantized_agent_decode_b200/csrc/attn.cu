@@ -21,6 +21,11 @@
 // hi + lo pair of bf16 values, so its rounding error is ~2^-17 relative.
 #include "attn.cuh"
 
+// Fewest keys one split of the decode attention covers (build-time tunable, multiple of 64).
+#ifndef QAD_ATTN_MIN_SPLIT_KEYS
+#define QAD_ATTN_MIN_SPLIT_KEYS 256
+#endif
+
 namespace qad {
 
 constexpr int QG = ATT_QG;      // query vectors per CTA
@@ -385,8 +390,8 @@ AttnPlan attn_plan(int n_agents, int n_qh, int n_kvh, int kv_cap, int max_rows_p
         splits = 1;
     int ch = (kv_cap + splits - 1) / splits;
     ch = ((ch + 63) / 64) * 64;
-    if (ch < 64)
-        ch = 64;
+    if (ch < QAD_ATTN_MIN_SPLIT_KEYS)  // short caches: fewer, longer splits (less partial traffic)
+        ch = QAD_ATTN_MIN_SPLIT_KEYS;
     pl.CH = ch;
     pl.max_splits = (kv_cap + ch - 1) / ch;
     pl.part_bytes = (size_t)n_agents * n_kvh * pl.n_rg * pl.max_splits * PART_FLOATS * sizeof(float);
