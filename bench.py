@@ -475,6 +475,19 @@ def run_kernel(args):
         fn = lambda i, st: gemm(Ws[i % 2], N, K, X, M, Y, ws=ws, stream=st)  # noqa: E731
         nbytes = Ws[0].numel()
         flops = 2.0 * M * N * K
+    elif args.kernel == "verify":
+        hidden, vocab, M = 5120, 151936, 12
+        Wh = synth.q4k_matrix_torch(g, vocab, hidden, "cuda")
+        Hd = synth.bf16_normal_torch(g, (M, hidden), "cuda").float()
+        ars = torch.arange(0, 13, 3, dtype=torch.int32, device="cuda")
+        toks = torch.randint(0, vocab, (M,), generator=g, dtype=torch.int32, device="cuda")
+        lens = torch.full((4,), 1024, dtype=torch.int32, device="cuda")
+        out = torch.empty(M, dtype=torch.int32, device="cuda")
+        acc = torch.empty(4, dtype=torch.int32, device="cuda")
+        ws = q.alloc_ws(q.verify_ws_bytes(hidden, vocab, M))
+        fn = lambda i, st: q.verify_step(Hd, M, hidden, Wh, vocab, ars, 4, toks, lens, out, acc, ws=ws,  # noqa: E731
+                                         stream=st)
+        nbytes = Wh.numel()
     elif args.kernel == "pfattn23k":
         len_, C, n_qh, n_kvh = 23000, 2048, 48, 8
         cap = len_ + C
@@ -555,7 +568,7 @@ def main():
     ap.add_argument("--workload", default="stack12_ctx1k", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel", choices=sorted(list(KERNELS) + list(DENSE_KERNELS) + ["attn23k", "pfattn23k"]),
+    ap.add_argument("--kernel", choices=sorted(list(KERNELS) + list(DENSE_KERNELS) + ["attn23k", "pfattn23k", "verify"]),
                     help="time one kernel of the step instead (profiler captures)")
     ap.add_argument("--rows", type=int, default=12)
     args = ap.parse_args()

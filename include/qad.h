@@ -192,6 +192,32 @@ int qad_decode_attn(const uint16_t *Q, const uint16_t *Kc, const uint16_t *Vc, c
                     int n_qh, int n_kvh, int hd, float scale, uint16_t *O, void *ws, size_t ws_bytes,
                     void *stream);
 
+/* ---------------------------------------------------------------- verify tail
+ * OpenJet page, section 只搬一次权重: every agent's drafts are checked in the
+ * same pass as its next token. The acceptance rule is not on the page; the
+ * rule implemented is greedy. For the step's final hidden states H:
+ *   logits = bf16(rmsnorm(H)) . W_head^T          (Q4_K head, fp32 [M][vocab])
+ *   row_argmax[r] = first index of the row's maximum logit (fp32 decision)
+ *   per agent a (rows r0 .. r0+n-1, inputs row_tokens[]): draft j+1 (the input
+ *   of row j+1) is accepted iff all earlier drafts were and
+ *   row_argmax[r0+j] == row_tokens[r0+j+1]; with k accepted,
+ *   out_tokens[r0+j] = row_argmax[r0+j] for j <= k and -1 after,
+ *   n_accept[a] = k, lens[a] += k + 1 (agents with no rows: unchanged).
+ *   H          device fp32 [M][hidden], 16-byte aligned
+ *   W_head     device Q4_K [vocab][hidden/256][144], 16-byte aligned
+ *   agent_row_start device int32 [n_agents+1]; row_tokens device int32 [M]
+ *   lens       device int32 [n_agents], updated in place (the KV-length commit)
+ *   out_tokens device int32 [M]; n_accept device int32 [n_agents]
+ *   row_argmax optional device int32 [M]; logits_out optional device fp32
+ *              [M][vocab] (else the logits live in ws)
+ *   ws         device workspace of qad_verify_ws_bytes(hidden, vocab, M) bytes
+ * 1 <= M <= 16, hidden % 256 == 0. Four launches on `stream`. Returns 0 or a
+ * negative QAD_ERR_* code. */
+size_t qad_verify_ws_bytes(int hidden, int vocab, int M);
+int qad_verify_step(const float *H, int M, int hidden, float rms_eps, const void *W_head, int vocab,
+                    const int *agent_row_start, int n_agents, const int *row_tokens, int *lens, int *out_tokens,
+                    int *n_accept, int *row_argmax, float *logits_out, void *ws, size_t ws_bytes, void *stream);
+
 /* ---------------------------------------------------------------- prefill-chunk attention
  * OpenJet page, section 真正重要的是少互相堵车: a prompt chunk of one agent
  * (C rows at positions len .. len+C-1) attends causally over the agent's own

@@ -60,6 +60,9 @@ SIGNATURES = {
     "qad_q6k_gemm_dense": (C.c_int, [C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p,
                                      C.c_size_t, C.c_void_p]),
     "qad_dense_status": (C.c_int, [C.c_int]),
+    "qad_verify_ws_bytes": (C.c_size_t, [C.c_int, C.c_int, C.c_int]),
+    "qad_verify_step": (C.c_int, [C.c_void_p, C.c_int, C.c_int, C.c_float, C.c_void_p, C.c_int, C.c_void_p, C.c_int]
+                        + [C.c_void_p] * 7 + [C.c_size_t, C.c_void_p]),
     "qad_prefill_attn": (C.c_int, [C.c_void_p] * 3 + [C.c_int] * 6 + [C.c_float, C.c_void_p, C.c_void_p]),
     "qad_decode_attn_ws_bytes": (C.c_size_t, [C.c_int] * 5),
     "qad_decode_attn": (C.c_int, [C.c_void_p] * 5 + [C.c_int] * 6 + [C.c_float, C.c_void_p, C.c_void_p,
@@ -261,6 +264,26 @@ def decode_attn(Q, Kc, Vc, lens, agent_row_start, n_agents, max_rows_per_agent, 
 
 
 # ------------------------------------------------------------------ row packer (host)
+
+def verify_ws_bytes(hidden: int, vocab: int, M: int) -> int:
+    return int(lib().qad_verify_ws_bytes(hidden, vocab, M))
+
+
+def verify_step(H, M, hidden, W_head, vocab, agent_row_start, n_agents, row_tokens, lens, out_tokens, n_accept,
+                row_argmax=None, logits=None, rms_eps=1e-6, ws=None, stream=None):
+    """Logits through the Q4_K head, per-row argmax, greedy draft acceptance and the
+    in-place KV-length commit (see qad_verify_step in include/qad.h)."""
+    _require_gpu()
+    if ws is None:
+        ws = alloc_ws(verify_ws_bytes(hidden, vocab, M), H.device)
+    opt = lambda t, n: None if t is None else _dev(t, n)  # noqa: E731
+    _check(lib().qad_verify_step(_dev(H, "H"), M, hidden, float(rms_eps), _dev(W_head, "W_head"), vocab,
+                                 _dev(agent_row_start, "agent_row_start"), n_agents, _dev(row_tokens, "row_tokens"),
+                                 _dev(lens, "lens"), _dev(out_tokens, "out_tokens"), _dev(n_accept, "n_accept"),
+                                 opt(row_argmax, "row_argmax"), opt(logits, "logits"), _dev(ws, "ws"),
+                                 ws.numel() * ws.element_size(), _stream(stream)), "qad_verify_step")
+    return out_tokens
+
 
 def prefill_attn(Q, Kc, Vc, len_, C, kv_cap, n_qh, n_kvh, hd, O, scale=None, stream=None):
     """Causal attention of a C-row prompt chunk at positions len_.. over one agent's cache

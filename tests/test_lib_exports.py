@@ -53,6 +53,28 @@ def test_build_targets_sm100a_only():
     assert build.ARCH == ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
+def _prototype_arg_counts():
+    """Number of parameters of every qad_* prototype in include/*.h."""
+    counts = {}
+    inc = os.path.join(ROOT, "include")
+    for fn in os.listdir(inc):
+        if not fn.endswith(".h"):
+            continue
+        text = re.sub(r"/\*.*?\*/", "", open(os.path.join(inc, fn)).read(), flags=re.S)
+        for m in re.finditer(r"\b(qad_[a-z0-9_]+)\s*\(([^;{]*?)\)\s*;", text):
+            args = m.group(2).strip()
+            counts[m.group(1)] = 0 if args in ("", "void") else args.count(",") + 1
+    return counts
+
+
+def test_binding_signatures_match_header(qlib):
+    """Every ctypes signature in the binding has as many parameters as its C prototype."""
+    counts = _prototype_arg_counts()
+    for name, (_, argtypes) in qlib.SIGNATURES.items():
+        assert name in counts, name
+        assert len(argtypes) == counts[name], (name, len(argtypes), counts[name])
+
+
 def test_version_and_error_text(qlib):
     L = qlib.lib()
     assert L.qad_version() >= 100
