@@ -449,6 +449,46 @@ DENSE_KERNELS = {  # prefill chunk (2048 prompt rows + 12 decode rows) through o
     "pf_gate_up": (4, 34816, 5120, 2060), "pf_down": (6, 5120, 17408, 2060), "pf_qkv": (4, 8192, 5120, 2060),
 }
 
+STEP_LAUNCHES = ["prep_rms_attn", "gemm_qkv", "attn", "prep_merge", "gemm_o", "prep_rms_mlp", "gemm_gate_up",
+                 "prep_silu", "gemm_down"]
+
+
+def run_trace(args):
+    """Per-launch device timeline of one replayed step (qad_model_set_trace): for each
+    launch kind the mean wait (start -> dependency met), run (-> last warp exit) and
+    critical-path share (previous launch's end -> this launch's end), in microseconds."""
+    from quantized_agent_decode_b200 import build
+    build.build()
+    w = Workload(args.workload)
+    stream = torch.cuda.Stream()
+    w.model.set_trace(True)
+    g = w.graph(stream)
+    for _ in range(max(args.warmup, 1)):
+        g.launch(stream)
+    stream.synchronize()
+    w.model.trace_reset()
+    torch.cuda.synchronize()
+    g.launch(stream)
+    stream.synchronize()
+    t = w.model.trace_read().numpy() / 1000.0
+    names = ["init"] + STEP_LAUNCHES * w.shape.n_layers
+    kinds, prev = {}, 0.0
+    for i, nm in enumerate(names):
+        st, rd, en = t[i]
+        d = kinds.setdefault(nm, [0, 0.0, 0.0, 0.0])
+        d[0] += 1
+        d[1] += rd - st
+        d[2] += en - rd
+        d[3] += en - prev
+        prev = en
+    out = {"workload": w.desc, "step_us": round(float(t[:, 2].max()), 1),
+           "per_launch_kind_us": {k: {"wait": round(v[1] / v[0], 2), "run": round(v[2] / v[0], 2),
+                                      "critical": round(v[3] / v[0], 2), "per_step": v[0]} for k, v in kinds.items()}}
+    print(json.dumps(out), flush=True)
+    g.close()
+    return 0
+
+
 KERNELS = {  # single-kernel cases for profiler captures: (format, N, K)
     "qkv": (4, 8192, 5120), "o": (4, 5120, 6144), "gate_up": (4, 34816, 5120), "down": (6, 5120, 17408),
 }
@@ -571,9 +611,12 @@ def main():
     ap.add_argument("--kernel", choices=sorted(list(KERNELS) + list(DENSE_KERNELS) + ["attn23k", "pfattn23k", "verify"]),
                     help="time one kernel of the step instead (profiler captures)")
     ap.add_argument("--rows", type=int, default=12)
+    ap.add_argument("--trace", action="store_true", help="print the per-launch device timeline of one step")
     args = ap.parse_args()
     if args.kernel:
         return run_kernel(args)
+    if args.trace:
+        return run_trace(args)
     ws, rank, local = (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
                        int(os.environ.get("LOCAL_RANK", "0")))
     if args.impl == "reference":
