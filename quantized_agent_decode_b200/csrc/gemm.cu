@@ -138,6 +138,23 @@ __device__ __forceinline__ float silu_mul(float g, float u)
     return p == 0.f ? p : copysignf(expf(g + logf(fabsf(p))), p);
 }
 
+// Zero the next GEMM's output (its atomics accumulate into it); this CTA's share.
+__device__ __forceinline__ void zero_next_output(const PrepSrc &S)
+{
+    if (S.zero) {
+        const long long nct = (long long)gridDim.x * gridDim.y, ct = (long long)blockIdx.y * gridDim.x + blockIdx.x;
+        const long long per = ((S.zero_n + nct - 1) / nct + 3) & ~3LL;
+        const long long z0 = ct * per, z1 = min(S.zero_n, z0 + per);
+        if ((S.zero_n & 3) == 0 && ((uintptr_t)S.zero & 15) == 0) {
+            for (long long i = z0 + 4 * (long long)threadIdx.x; i < z1; i += 4 * 256)
+                *reinterpret_cast<float4 *>(S.zero + i) = make_float4(0.f, 0.f, 0.f, 0.f);
+        } else {
+            for (long long i = z0 + threadIdx.x; i < z1; i += 256)
+                S.zero[i] = 0.f;
+        }
+    }
+}
+
 // Grid (ceil(nblk / 4), 8*NT): CTA (x, r) forms row r's blocks 4x..4x+3, one
 // 64-thread quarter per block, thread t of a quarter owning columns 4t..4t+3.
 // The values are formed exactly as the GEMM must see them (bf16: the input
@@ -177,18 +194,6 @@ __global__ void __launch_bounds__(256) k_prep(PrepArgs a)
     }
     pdl_wait();
     trace_ready(a.trace);
-    if (S.zero) {
-        const long long nct = (long long)gridDim.x * gridDim.y, ct = (long long)blockIdx.y * gridDim.x + blockIdx.x;
-        const long long per = ((S.zero_n + nct - 1) / nct + 3) & ~3LL;
-        const long long z0 = ct * per, z1 = min(S.zero_n, z0 + per);
-        if ((S.zero_n & 3) == 0 && ((uintptr_t)S.zero & 15) == 0) {
-            for (long long i = z0 + 4 * tid; i < z1; i += 4 * 256)
-                *reinterpret_cast<float4 *>(S.zero + i) = make_float4(0.f, 0.f, 0.f, 0.f);
-        } else {
-            for (long long i = z0 + tid; i < z1; i += 256)
-                S.zero[i] = 0.f;
-        }
-    }
     float4 own = make_float4(0.f, 0.f, 0.f, 0.f);  // RMSNorm: this thread's 4 values, kept from the sum pass
     if (S.kind == PREP_RMSNORM && live) {
         // the whole row's mean square, recomputed by every CTA of the row in the same
@@ -289,6 +294,7 @@ __global__ void __launch_bounds__(256) k_prep(PrepArgs a)
         e = min(126, max(-126, 10 - E));
     }
     if (b >= nblk) {
+        zero_next_output(S);
         trace_end(a.trace);
         return;
     }
@@ -315,6 +321,7 @@ __global__ void __launch_bounds__(256) k_prep(PrepArgs a)
     }
     if (t == 0)
         reinterpret_cast<float *>(rec + rec_bytes(FMT, NT) - 64)[r] = live ? ldexpf(1.f, -e) : 0.f;
+    zero_next_output(S);  // last: the next GEMM's output is not read by this kernel
     trace_end(a.trace);
 }
 
