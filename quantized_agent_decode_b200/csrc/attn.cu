@@ -31,7 +31,8 @@ namespace qad {
 constexpr int QG = ATT_QG;      // query vectors per CTA
 constexpr int KT = 16;          // keys per tile (one MMA M tile)
 constexpr int ATT_WARPS = 4;
-constexpr int ATT_STAGES = 3;
+constexpr int ATT_STAGES_LONG = 3;   // per-warp ring for long caches (two CTAs per SM)
+constexpr int ATT_STAGES_SHORT = 6;  // short caches: a split's cached tiles all in flight at once
 constexpr int TILE_BYTES = KT * 128 * 2;  // 4 KB (K) ; V follows
 constexpr int PART_FLOATS = ATT_PART_FLOATS;
 
@@ -53,7 +54,7 @@ __device__ __forceinline__ int swz(int key, int chunk) { return key * 256 + ((ch
 // bf16 here, as the unfused path rounds them before the cache write); key
 // positions len .. len+na-1 are taken from there instead of the cache, and the
 // row-group-0 CTA of the split holding a new position writes it to the cache.
-template <bool FUSED>
+template <bool FUSED, int STAGES>
 __global__ void __launch_bounds__(128, 2) k_decode_attn(AttnArgs p)
 {
     extern __shared__ __align__(128) uint8_t smem[];
@@ -102,12 +103,12 @@ __global__ void __launch_bounds__(128, 2) k_decode_attn(AttnArgs p)
 
     const int ntiles = (kend - kbeg + KT - 1) / KT;
     const int my = ntiles > w ? (ntiles - w + ATT_WARPS - 1) / ATT_WARPS : 0;
-    uint8_t *wbuf = smem + (size_t)w * ATT_STAGES * 2 * TILE_BYTES;
+    uint8_t *wbuf = smem + (size_t)w * STAGES * 2 * TILE_BYTES;
 
     const int nq = p.n_qh * 128, nkv = p.n_kvh * 128;
     auto issue = [&](int it) {
         const int kb = kbeg + KT * (w + ATT_WARPS * it);
-        uint8_t *st = wbuf + (size_t)(it % ATT_STAGES) * 2 * TILE_BYTES;
+        uint8_t *st = wbuf + (size_t)(it % STAGES) * 2 * TILE_BYTES;
         if (FUSED && kb + KT > len) {
             // tile reaches the new positions: cached keys below len, new rows from the projection
 #pragma unroll 1
@@ -151,14 +152,14 @@ __global__ void __launch_bounds__(128, 2) k_decode_attn(AttnArgs p)
     // tiles of cached keys only (always the earlier ones) stream before the wait
     auto cached_tile = [&](int it) { return !FUSED || kbeg + KT * (w + ATT_WARPS * it) + KT <= len; };
     int pre = 0;
-    while (pre < 2 && pre < my && cached_tile(pre)) {
+    while (pre < STAGES - 1 && pre < my && cached_tile(pre)) {
         issue(pre);
         cp_async_commit();
         ++pre;
     }
     pdl_wait();
     trace_ready(p.trace);
-    for (int it = pre; it < 2; ++it) {
+    for (int it = pre; it < STAGES - 1; ++it) {
         if (it < my)
             issue(it);
         cp_async_commit();
@@ -198,12 +199,12 @@ __global__ void __launch_bounds__(128, 2) k_decode_attn(AttnArgs p)
 
 
     for (int it = 0; it < my; ++it) {
-        if (it + 2 < my)
-            issue(it + 2);
+        if (it + STAGES - 1 < my)
+            issue(it + STAGES - 1);
         cp_async_commit();
-        cp_async_wait<2>();
+        cp_async_wait<STAGES - 1>();
         __syncwarp();
-        const uint8_t *Ks = wbuf + (size_t)(it % ATT_STAGES) * 2 * TILE_BYTES;
+        const uint8_t *Ks = wbuf + (size_t)(it % STAGES) * 2 * TILE_BYTES;
         const uint8_t *Vs = Ks + TILE_BYTES;
         const int kb = kbeg + KT * (w + ATT_WARPS * it);
 
@@ -318,7 +319,8 @@ __global__ void __launch_bounds__(128, 2) k_decode_attn(AttnArgs p)
     __syncthreads();
     const size_t pidx = (((size_t)a * p.n_kvh + g) * p.n_rg + rg) * p.max_splits + sp;
     float *out = p.part + pidx * PART_FLOATS;
-    for (int idx = tid; idx < QG * 128; idx += blockDim.x) {
+    const int nqv = min(QG, R - q0);  // real query vectors of this group (the rest is padding)
+    for (int idx = tid; idx < nqv * 128; idx += blockDim.x) {
         const int q = idx >> 7;
         float M = -INFINITY;
 #pragma unroll
@@ -331,7 +333,7 @@ __global__ void __launch_bounds__(128, 2) k_decode_attn(AttnArgs p)
                 acc += exp2f(sM[ww * QG + q] - M) * sO[((size_t)ww * QG + q) * 128 + (idx & 127)];
         out[idx] = acc;
     }
-    if (tid < QG) {
+    if (tid < nqv) {
         float M = -INFINITY, Lsum = 0.f;
         for (int ww = 0; ww < ATT_WARPS; ++ww)
             M = fmaxf(M, sM[ww * QG + tid]);
@@ -384,6 +386,24 @@ AttnPlan attn_plan(int n_agents, int n_qh, int n_kvh, int kv_cap, int max_rows_p
     pl.n_rg = (max_rows_per_agent * pl.G + QG - 1) / QG;
     // one wave: two resident CTAs per SM (registers and shared memory allow two)
     const int pairs = n_agents * n_kvh * pl.n_rg;
+    // Short caches: at most one CTA per SM, and the split small enough that each
+    // warp's tiles (16 keys each, 4 warps) all fit its 6-stage ring, so every
+    // cached key is in flight before the kernel waits for its queries.
+    {
+        int sp = num_sms() / pairs;
+        if (sp < 1)
+            sp = 1;
+        int ch = (kv_cap + sp - 1) / sp;
+        ch = ((ch + 63) / 64) * 64;
+        if ((ch / KT + ATT_WARPS - 1) / ATT_WARPS <= ATT_STAGES_SHORT - 1) {
+            pl.CH = ch;
+            pl.stages = ATT_STAGES_SHORT;
+            pl.max_splits = (kv_cap + ch - 1) / ch;
+            pl.part_bytes = (size_t)n_agents * n_kvh * pl.n_rg * pl.max_splits * PART_FLOATS * sizeof(float);
+            return pl;
+        }
+    }
+    pl.stages = ATT_STAGES_LONG;
     const int target = 2 * num_sms();
     int splits = target / pairs;
     if (splits < 1)
@@ -398,23 +418,23 @@ AttnPlan attn_plan(int n_agents, int n_qh, int n_kvh, int kv_cap, int max_rows_p
     return pl;
 }
 
-size_t attn_smem_bytes()
+size_t attn_smem_bytes(int nstages)
 {
-    const size_t stages = (size_t)ATT_WARPS * ATT_STAGES * 2 * TILE_BYTES;
+    const size_t stages = (size_t)ATT_WARPS * nstages * 2 * TILE_BYTES;
     const size_t merge = ((size_t)ATT_WARPS * QG * 128 + 2 * ATT_WARPS * QG) * sizeof(float);
     return stages > merge ? stages : merge;
 }
 
-template <bool FUSED>
-static int launch_split_kernel(const AttnPlan &pl, const AttnArgs &p, int n_agents, cudaStream_t s, bool pdl)
+template <bool FUSED, int STAGES>
+static int launch_split_kernel_t(const AttnPlan &pl, const AttnArgs &p, int n_agents, cudaStream_t s, bool pdl)
 {
-    const size_t smem = attn_smem_bytes();
+    const size_t smem = attn_smem_bytes(STAGES);
     static bool attr_set[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64 || !attr_set[dev]) {
         int rc = cuda_check(
-            cudaFuncSetAttribute(k_decode_attn<FUSED>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem),
+            cudaFuncSetAttribute(k_decode_attn<FUSED, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem),
             "cudaFuncSetAttribute(attn)");
         if (rc)
             return rc;
@@ -422,9 +442,16 @@ static int launch_split_kernel(const AttnPlan &pl, const AttnArgs &p, int n_agen
             attr_set[dev] = true;
     }
     dim3 grid(pl.max_splits, pl.n_rg, n_agents * p.n_kvh);
-    cudaError_t e = pdl ? launch_pdl(k_decode_attn<FUSED>, grid, dim3(128), smem, s, p)
-                        : (k_decode_attn<FUSED><<<grid, 128, smem, s>>>(p), cudaGetLastError());
+    cudaError_t e = pdl ? launch_pdl(k_decode_attn<FUSED, STAGES>, grid, dim3(128), smem, s, p)
+                        : (k_decode_attn<FUSED, STAGES><<<grid, 128, smem, s>>>(p), cudaGetLastError());
     return cuda_check(e, "attn launch");
+}
+
+template <bool FUSED>
+static int launch_split_kernel(const AttnPlan &pl, const AttnArgs &p, int n_agents, cudaStream_t s, bool pdl)
+{
+    return pl.stages == ATT_STAGES_SHORT ? launch_split_kernel_t<FUSED, ATT_STAGES_SHORT>(pl, p, n_agents, s, pdl)
+                                         : launch_split_kernel_t<FUSED, ATT_STAGES_LONG>(pl, p, n_agents, s, pdl);
 }
 
 static AttnArgs attn_args(const AttnPlan &pl, const int *lens, const int *ars, int kv_cap, int n_qh, int n_kvh,

@@ -23,6 +23,7 @@ struct AttnPlan {
     int n_rg;        // groups of 24 query vectors per (agent, kv-head)
     int CH;          // keys per split (multiple of 64)
     int max_splits;  // splits covering kv_cap keys
+    int stages;      // per-warp cp.async ring depth of the kernel variant
     size_t part_bytes;
 };
 
