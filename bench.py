@@ -491,6 +491,7 @@ def run_trace(args):
 
 KERNELS = {  # single-kernel cases for profiler captures: (format, N, K)
     "qkv": (4, 8192, 5120), "o": (4, 5120, 6144), "gate_up": (4, 34816, 5120), "down": (6, 5120, 17408),
+    "gate": (4, 17408, 5120),  # one MLP gate (or up) projection alone
 }
 
 
