@@ -61,6 +61,12 @@ def lib():
         L.orc_pack_rows.restype = C.c_int
         L.orc_pack_rows.argtypes = [C.POINTER(C.c_void_p), i32p, i32p, C.c_int, C.c_int,
                                     u16p, i32p, i32p, i32p]
+        L.orc_double_to_half.restype = C.c_uint16
+        L.orc_double_to_half.argtypes = [C.c_double]
+        L.orc_q8_0_quantize.argtypes = [np.ctypeslib.ndpointer(np.float32, flags="C_CONTIGUOUS"), C.c_long, i8p,
+                                        u16p]
+        L.orc_decode_attn_q8.argtypes = [u16p, i8p, u16p, i8p, u16p, i32p, i32p, C.c_int, C.c_int, C.c_int,
+                                         C.c_int, C.c_int, C.c_double, f64p, C.c_void_p, C.c_int]
         L.orc_argmax.restype = C.c_long
         L.orc_argmax.argtypes = [f64p, C.c_long]
         L.orc_accept_greedy.argtypes = [i32p, i32p, i32p, C.c_int, i32p, i32p, i32p]
@@ -214,6 +220,34 @@ def pack_rows(agent_rows, lens, H: int):
     m = lib().orc_pack_rows(ptrs, n_rows, np.ascontiguousarray(lens, np.int32), n, H, X, ra, rp, ars)
     assert m == M
     return X[:M], ra[:M], rp[:M], ars
+
+
+def double_to_half(x: float) -> int:
+    return int(lib().orc_double_to_half(float(x)))
+
+
+def q8_0_quantize(x: np.ndarray):
+    """float32 [..., n] (n % 32 == 0) -> (int8 codes [..., n], fp16 scale bits [..., n / 32])."""
+    x = np.ascontiguousarray(x, np.float32)
+    q = np.zeros(x.shape, np.int8)
+    d = np.zeros(x.shape[:-1] + (x.shape[-1] // 32,), np.uint16)
+    lib().orc_q8_0_quantize(x.reshape(-1), x.size, q.reshape(-1), d.reshape(-1))
+    return q, d
+
+
+def decode_attn_q8(Q, Kq, Kd, Vq, Vd, lens, ars, n_qh, n_kvh, hd, cap, scale=None, nthreads: int = 0):
+    """Attention over a q8_0 cache: O, B float64 [M, n_qh, hd]."""
+    lens = np.ascontiguousarray(lens, np.int32)
+    ars = np.ascontiguousarray(ars, np.int32)
+    M = int(ars[-1])
+    O = np.zeros((M, n_qh, hd), np.float64)
+    B = np.zeros((M, n_qh, hd), np.float64)
+    lib().orc_decode_attn_q8(np.ascontiguousarray(Q, np.uint16).reshape(-1),
+                             np.ascontiguousarray(Kq, np.int8).reshape(-1), np.ascontiguousarray(Kd, np.uint16).reshape(-1),
+                             np.ascontiguousarray(Vq, np.int8).reshape(-1), np.ascontiguousarray(Vd, np.uint16).reshape(-1),
+                             lens, ars, len(lens), cap, n_qh, n_kvh, hd, 1.0 / np.sqrt(hd) if scale is None else float(scale),
+                             O.reshape(-1), _ptr(B.reshape(-1)), nthreads or max_threads())
+    return O, B
 
 
 def argmax(v: np.ndarray) -> int:

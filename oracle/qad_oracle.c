@@ -372,6 +372,119 @@ void orc_decode_attn(const uint16_t *Q, const uint16_t *Kc, const uint16_t *Vc,
     }
 }
 
+/* fp16 bits of x, rounded to nearest with ties to even (subnormals kept). */
+uint16_t orc_double_to_half(double x)
+{
+    if (isnan(x))
+        return 0x7E00;
+    uint16_t sign = signbit(x) ? 0x8000 : 0;
+    double a = fabs(x);
+    if (a == 0.0)
+        return sign;
+    int e;
+    frexp(a, &e);                 /* a = f * 2^e, f in [0.5, 1) */
+    int q = e - 11;               /* 11 significant bits: a = M * 2^q, M in [1024, 2048) */
+    if (q < -24)
+        q = -24;                  /* subnormal spacing of fp16 is 2^-24 */
+    double R = nearbyint(ldexp(a, -q));
+    double r = ldexp(R, q);
+    if (r >= 65520.0)             /* rounds past the largest finite value 65504 */
+        return sign | 0x7C00;
+    /* encode r exactly */
+    if (r < ldexp(1.0, -14))
+        return sign | (uint16_t)(r * ldexp(1.0, 24));             /* subnormal: r / 2^-24 */
+    int ex;
+    double f = frexp(r, &ex);     /* r = f * 2^ex, f in [0.5, 1) */
+    uint16_t mant = (uint16_t)(ldexp(f, 11) - 1024.0);             /* 10 fraction bits */
+    return sign | (uint16_t)((ex - 1 + 15) << 10) | mant;
+}
+
+/* q8_0 quantisation of n values (n % 32 == 0), the GGUF q8_0 rule: per block of
+ * 32 values d = amax / 127, q = round(x / d) (half away from zero) with the
+ * reciprocal taken once, d stored as fp16. The code is decided in fp32 (the
+ * kernel's precision): x, amax, d, 1/d and x * (1/d) are all fp32 operations.
+ * Used for the q8_0 KV-cache variant (dual-4090 page, section 真正昂贵的是
+ * "同时记住": llama.cpp's q8_0 KV cache per agent). */
+void orc_q8_0_quantize(const float *x, long n, int8_t *q, uint16_t *d)
+{
+    for (long b = 0; b < n / 32; ++b) {
+        float amax = 0.0f;
+        for (int i = 0; i < 32; ++i) {
+            float v = fabsf(x[32 * b + i]);
+            if (v > amax)
+                amax = v;
+        }
+        float dF = amax / 127.0f;
+        float id = dF != 0.0f ? 1.0f / dF : 0.0f;
+        for (int i = 0; i < 32; ++i)
+            q[32 * b + i] = (int8_t)roundf(x[32 * b + i] * id);
+        d[b] = orc_double_to_half((double)dF);
+    }
+}
+
+/* Grouped-query attention of orc_decode_attn over a q8_0 cache: key/value
+ * element (agent a, kv-head g, position t, dim k) = half(Kd[.., t, k / 32]) *
+ * Kq[.., t, k] (exact in double). Kq, Vq int8 [A][n_kvh][cap][hd]; Kd, Vd fp16
+ * [A][n_kvh][cap][hd / 32]. */
+void orc_decode_attn_q8(const uint16_t *Q, const int8_t *Kq, const uint16_t *Kd, const int8_t *Vq,
+                        const uint16_t *Vd, const int *lens, const int *ars, int n_agents, int cap, int n_qh,
+                        int n_kvh, int hd, double scale, double *O, double *B, int nthreads)
+{
+    int M = ars[n_agents];
+    const int nb = hd / 32;
+#pragma omp parallel num_threads(nthreads > 0 ? nthreads : 1)
+    {
+        double *s = NULL;
+        int s_cap = 0;
+#pragma omp for schedule(dynamic) collapse(2)
+        for (int r = 0; r < M; ++r)
+            for (int h = 0; h < n_qh; ++h) {
+                int a = 0;
+                while (!(ars[a] <= r && r < ars[a + 1]))
+                    ++a;
+                int j = r - ars[a];
+                int nk = lens[a] + j + 1;
+                int g = h * n_kvh / n_qh;
+                if (nk > s_cap) {
+                    free(s);
+                    s_cap = nk;
+                    s = malloc(sizeof(double) * (size_t)s_cap);
+                }
+                const uint16_t *q = Q + ((size_t)r * n_qh + h) * hd;
+                const size_t hb = ((size_t)a * n_kvh + g) * (size_t)cap;
+                double mx = -INFINITY;
+                for (int t = 0; t < nk; ++t) {
+                    double dot = 0.0;
+                    for (int k = 0; k < hd; ++k)
+                        dot += orc_bf16_to_double(q[k]) * orc_half_to_double(Kd[(hb + t) * nb + k / 32]) *
+                               (double)Kq[(hb + t) * hd + k];
+                    s[t] = scale * dot;
+                    if (s[t] > mx)
+                        mx = s[t];
+                }
+                double z = 0.0;
+                for (int t = 0; t < nk; ++t) {
+                    s[t] = exp(s[t] - mx);
+                    z += s[t];
+                }
+                double *o = O + ((size_t)r * n_qh + h) * hd;
+                double *bb = B ? B + ((size_t)r * n_qh + h) * hd : NULL;
+                for (int k = 0; k < hd; ++k) {
+                    double acc = 0.0, aabs = 0.0;
+                    for (int t = 0; t < nk; ++t) {
+                        double v = orc_half_to_double(Vd[(hb + t) * nb + k / 32]) * (double)Vq[(hb + t) * hd + k];
+                        acc += s[t] * v;
+                        aabs += s[t] * fabs(v);
+                    }
+                    o[k] = acc / z;
+                    if (bb)
+                        bb[k] = aabs / z;
+                }
+            }
+        free(s);
+    }
+}
+
 /* ------------------------------------------------------------------ glue */
 
 /* RMSNorm with unit gain, then bf16: out = bf16(h / sqrt(mean(h^2) + eps)). */
