@@ -73,6 +73,9 @@ def lib():
         L.orc_decode_layer.argtypes = [u8p, u8p, u8p, u8p, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
                                        C.c_double, f64p, C.c_int, i32p, C.c_int, i32p, u16p, u16p,
                                        C.c_int, C.c_int] + [C.c_void_p] * 7
+        L.orc_decode_layer_q8.argtypes = [u8p, u8p, u8p, u8p, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
+                                          C.c_double, f64p, C.c_int, i32p, C.c_int, i32p, i8p, u16p, i8p, u16p,
+                                          C.c_int, C.c_int] + [C.c_void_p] * 7
         L.orc_max_threads.restype = C.c_int
         _lib = L
     return _lib
@@ -273,6 +276,7 @@ def accept_greedy(row_argmax, row_tokens, ars, lens):
 def decode_layer(Wqkv, Wo, Wgu, Wdown, H, I, n_qh, n_kvh, hd, h, ars, lens, Kc, Vc, cap,
                  eps=1e-6, nthreads: int = 0, want=False):
     """One layer on the fp64 residual ``h`` [M, H] (in place); caches updated in place.
+    Kc, Vc are bf16 arrays, or (codes int8, scales fp16 bits) pairs for a q8_0 cache.
     With want=True also returns the intermediates dict."""
     M = h.shape[0]
     nq, nkv = n_qh * hd, n_kvh * hd
@@ -284,11 +288,15 @@ def decode_layer(Wqkv, Wo, Wgu, Wdown, H, I, n_qh, n_kvh, hd, h, ars, lens, Kc, 
                      act=np.zeros((M, I), np.uint16))
     names = ["x1", "qkv", "attn", "hmid", "x2", "gu", "act"]
     ptrs = [_ptr(inter.get(k)) for k in names]
-    lib().orc_decode_layer(np.ascontiguousarray(Wqkv, np.uint8).reshape(-1),
-                           np.ascontiguousarray(Wo, np.uint8).reshape(-1),
-                           np.ascontiguousarray(Wgu, np.uint8).reshape(-1),
-                           np.ascontiguousarray(Wdown, np.uint8).reshape(-1),
-                           H, I, n_qh, n_kvh, hd, eps, h, M, np.ascontiguousarray(ars, np.int32),
-                           len(lens), np.ascontiguousarray(lens, np.int32), Kc.reshape(-1), Vc.reshape(-1),
-                           cap, nthreads or max_threads(), *ptrs)
+    W = [np.ascontiguousarray(w, np.uint8).reshape(-1) for w in (Wqkv, Wo, Wgu, Wdown)]
+    common = (H, I, n_qh, n_kvh, hd, eps, h, M, np.ascontiguousarray(ars, np.int32), len(lens),
+              np.ascontiguousarray(lens, np.int32))
+    if isinstance(Kc, tuple):
+        for a in (*Kc, *Vc):
+            assert a.flags["C_CONTIGUOUS"]  # updated in place
+        lib().orc_decode_layer_q8(*W, *common, Kc[0].reshape(-1), Kc[1].reshape(-1), Vc[0].reshape(-1),
+                                  Vc[1].reshape(-1), cap, nthreads or max_threads(), *ptrs)
+    else:
+        lib().orc_decode_layer(*W, *common, Kc.reshape(-1), Vc.reshape(-1), cap, nthreads or max_threads(),
+                               *ptrs)
     return inter

@@ -585,12 +585,20 @@ void orc_accept_greedy(const int *row_argmax, const int *row_tokens, const int *
  * h is the fp64 residual stream [M][H], updated in place. The caches are
  * updated in place. Intermediates are returned when the pointers are non-null
  * (used by teacher-forced checks). */
-void orc_decode_layer(const uint8_t *Wqkv, const uint8_t *Wo, const uint8_t *Wgu,
-                      const uint8_t *Wdown, int H, int I, int n_qh, int n_kvh, int hd,
-                      double eps, double *h, int M, const int *ars, int n_agents,
-                      const int *lens, uint16_t *Kc, uint16_t *Vc, int cap, int nthreads,
-                      uint16_t *x1_out, double *qkv_out, uint16_t *attn_out,
-                      double *hmid_out, uint16_t *x2_out, double *gu_out, uint16_t *act_out)
+/* KV cache of one layer: bf16 planes, or q8_0 codes plus fp16 scales. */
+typedef struct {
+    int q8;
+    uint16_t *Kc, *Vc;             /* bf16 [A][n_kvh][cap][hd] */
+    int8_t *Kq, *Vq;               /* q8_0 codes [A][n_kvh][cap][hd] */
+    uint16_t *Kd, *Vd;             /* q8_0 scales [A][n_kvh][cap][hd/32] */
+} orc_kv;
+
+static void decode_layer_impl(const uint8_t *Wqkv, const uint8_t *Wo, const uint8_t *Wgu,
+                              const uint8_t *Wdown, int H, int I, int n_qh, int n_kvh, int hd,
+                              double eps, double *h, int M, const int *ars, int n_agents,
+                              const int *lens, orc_kv kv, int cap, int nthreads,
+                              uint16_t *x1_out, double *qkv_out, uint16_t *attn_out,
+                              double *hmid_out, uint16_t *x2_out, double *gu_out, uint16_t *act_out)
 {
     int nq = n_qh * hd, nkv = n_kvh * hd, nqkv = nq + 2 * nkv;
     uint16_t *x1 = malloc(sizeof(uint16_t) * (size_t)M * H);
@@ -611,15 +619,32 @@ void orc_decode_layer(const uint8_t *Wqkv, const uint8_t *Wo, const uint8_t *Wgu
         int pos = lens[a] + (r - ars[a]);
         for (int i = 0; i < nq; ++i)
             Qb[(size_t)r * nq + i] = orc_double_to_bf16(qkv[(size_t)r * nqkv + i]);
-        for (int g = 0; g < n_kvh; ++g)
-            for (int d = 0; d < hd; ++d) {
-                size_t dst = (((size_t)a * n_kvh + g) * cap + pos) * hd + d;
-                Kc[dst] = orc_double_to_bf16(qkv[(size_t)r * nqkv + nq + g * hd + d]);
-                Vc[dst] = orc_double_to_bf16(qkv[(size_t)r * nqkv + nq + nkv + g * hd + d]);
+        for (int g = 0; g < n_kvh; ++g) {
+            size_t row = ((size_t)a * n_kvh + g) * cap + pos;
+            if (!kv.q8) {
+                for (int d = 0; d < hd; ++d) {
+                    kv.Kc[row * hd + d] = orc_double_to_bf16(qkv[(size_t)r * nqkv + nq + g * hd + d]);
+                    kv.Vc[row * hd + d] = orc_double_to_bf16(qkv[(size_t)r * nqkv + nq + nkv + g * hd + d]);
+                }
+            } else {
+                /* q8_0 append: the fp32 projection row, 32-value blocks */
+                float *kf = malloc(sizeof(float) * 2 * (size_t)hd), *vf = kf + hd;
+                for (int d = 0; d < hd; ++d) {
+                    kf[d] = (float)qkv[(size_t)r * nqkv + nq + g * hd + d];
+                    vf[d] = (float)qkv[(size_t)r * nqkv + nq + nkv + g * hd + d];
+                }
+                orc_q8_0_quantize(kf, hd, kv.Kq + row * hd, kv.Kd + row * (hd / 32));
+                orc_q8_0_quantize(vf, hd, kv.Vq + row * hd, kv.Vd + row * (hd / 32));
+                free(kf);
             }
+        }
     }
-    orc_decode_attn(Qb, Kc, Vc, lens, ars, n_agents, cap, n_qh, n_kvh, hd,
-                    1.0 / sqrt((double)hd), o, NULL, nthreads);
+    if (!kv.q8)
+        orc_decode_attn(Qb, kv.Kc, kv.Vc, lens, ars, n_agents, cap, n_qh, n_kvh, hd,
+                        1.0 / sqrt((double)hd), o, NULL, nthreads);
+    else
+        orc_decode_attn_q8(Qb, kv.Kq, kv.Kd, kv.Vq, kv.Vd, lens, ars, n_agents, cap, n_qh, n_kvh, hd,
+                           1.0 / sqrt((double)hd), o, NULL, nthreads);
     for (size_t i = 0; i < (size_t)M * nq; ++i)
         ob[i] = orc_double_to_bf16(o[i]);
     orc_gemm(4, Wo, H, nq, ob, M, y, NULL, nthreads);
@@ -655,6 +680,33 @@ void orc_decode_layer(const uint8_t *Wqkv, const uint8_t *Wo, const uint8_t *Wgu
     free(y);
     free(x2);
     free(act);
+}
+
+/* One decoder layer over bf16 caches (the rounding points listed at the top). */
+void orc_decode_layer(const uint8_t *Wqkv, const uint8_t *Wo, const uint8_t *Wgu,
+                      const uint8_t *Wdown, int H, int I, int n_qh, int n_kvh, int hd,
+                      double eps, double *h, int M, const int *ars, int n_agents,
+                      const int *lens, uint16_t *Kc, uint16_t *Vc, int cap, int nthreads,
+                      uint16_t *x1_out, double *qkv_out, uint16_t *attn_out,
+                      double *hmid_out, uint16_t *x2_out, double *gu_out, uint16_t *act_out)
+{
+    orc_kv kv = {0, Kc, Vc, NULL, NULL, NULL, NULL};
+    decode_layer_impl(Wqkv, Wo, Wgu, Wdown, H, I, n_qh, n_kvh, hd, eps, h, M, ars, n_agents, lens, kv,
+                      cap, nthreads, x1_out, qkv_out, attn_out, hmid_out, x2_out, gu_out, act_out);
+}
+
+/* The same layer over a q8_0 cache: the new rows' k, v are the fp32 values of
+ * the projection, quantised by orc_q8_0_quantize; attention dequantises. */
+void orc_decode_layer_q8(const uint8_t *Wqkv, const uint8_t *Wo, const uint8_t *Wgu,
+                         const uint8_t *Wdown, int H, int I, int n_qh, int n_kvh, int hd,
+                         double eps, double *h, int M, const int *ars, int n_agents,
+                         const int *lens, int8_t *Kq, uint16_t *Kd, int8_t *Vq, uint16_t *Vd, int cap,
+                         int nthreads, uint16_t *x1_out, double *qkv_out, uint16_t *attn_out,
+                         double *hmid_out, uint16_t *x2_out, double *gu_out, uint16_t *act_out)
+{
+    orc_kv kv = {1, NULL, NULL, Kq, Vq, Kd, Vd};
+    decode_layer_impl(Wqkv, Wo, Wgu, Wdown, H, I, n_qh, n_kvh, hd, eps, h, M, ars, n_agents, lens, kv,
+                      cap, nthreads, x1_out, qkv_out, attn_out, hmid_out, x2_out, gu_out, act_out);
 }
 
 int orc_max_threads(void)

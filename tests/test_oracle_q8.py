@@ -1,5 +1,6 @@
 """Pins of the oracle's fp16 rounding, q8_0 quantiser and q8_0-cache attention."""
 import numpy as np
+import pytest
 
 import synth
 from conftest import SEED
@@ -63,3 +64,80 @@ def test_q8_attention_equals_bf16_attention_on_exact_values(orc):
     O8, B8 = orc.decode_attn_q8(Q, Kq, Kd, Vq, Vd, lens, ars, n_qh, n_kvh, hd, cap)
     O, B = orc.decode_attn(Q, Kb, Vb, lens, ars, n_qh, n_kvh, hd, cap)
     assert np.array_equal(O8, O) and np.array_equal(B8, B)
+
+
+def test_q8_0_matches_gguf_quantiser(orc):
+    """The gguf package's Q8_0 quantiser (numpy, float32) is an independent
+    implementation of the same block format."""
+    gguf = pytest.importorskip("gguf")
+    rng = np.random.default_rng(14)
+    x = (rng.standard_normal((300, 32)) * 10.0 ** rng.integers(-4, 4, (300, 1))).astype(np.float32)
+    x[0] = 0.0
+    x[1, :] = np.arange(32) - 15.5          # halves: ties at every value once scaled
+    x[2, :] = np.round(rng.standard_normal(32) * 50).astype(np.float32)
+    x[2, 5] = 127.0                          # d = 1 exactly
+    x[3, :] = 1e-6 * (np.arange(32) - 16)    # scale in the fp16 subnormal range
+    q, d = orc.q8_0_quantize(x)
+    ref = gguf.quants.quantize(x.reshape(-1), gguf.GGMLQuantizationType.Q8_0).reshape(300, 34)
+    assert np.array_equal(d[:, 0], ref[:, :2].copy().view(np.uint16)[:, 0])
+    assert np.array_equal(q, ref[:, 2:].view(np.int8))
+
+
+def test_q8_decode_layer_appends_and_attends(orc):
+    """The q8_0 layer: everything before the append equals the bf16 layer; the
+    appended codes are the gguf Q8_0 blocks of the fp32 projection; the
+    attention output matches torch SDPA over the dequantised cache."""
+    gguf = pytest.importorskip("gguf")
+    import torch
+    import torch.nn.functional as F
+    H, I, n_qh, n_kvh, hd = 256, 512, 4, 2, 128
+    nq, nkv = n_qh * hd, n_kvh * hd
+    lens = np.array([6, 0, 11], np.int32)
+    ars = np.array([0, 3, 5, 6], np.int32)
+    M, A, cap = 6, 3, 20
+    Wqkv = synth.q4k_matrix_np(SEED, 50, nq + 2 * nkv, H)
+    Wo = synth.q4k_matrix_np(SEED, 51, H, nq)
+    Wgu = synth.q4k_matrix_np(SEED, 52, 2 * I, H)
+    Wd = synth.q6k_matrix_np(SEED, 53, H, I)
+    rng = np.random.default_rng(15)
+    Kq = rng.integers(-127, 128, (A, n_kvh, cap, hd)).astype(np.int8)
+    Vq = rng.integers(-127, 128, (A, n_kvh, cap, hd)).astype(np.int8)
+    Kd = (np.abs(rng.standard_normal((A, n_kvh, cap, hd // 32))) * 0.02 + 1e-3).astype(np.float16).view(np.uint16)
+    Vd = (np.abs(rng.standard_normal((A, n_kvh, cap, hd // 32))) * 0.02 + 1e-3).astype(np.float16).view(np.uint16)
+    h0 = orc.bf16_array_to_f64(synth.bf16_normal_np(SEED, 56, (M, H)))
+    h8, hb = h0.copy(), h0.copy()
+    K8, V8 = (Kq.copy(), Kd.copy()), (Vq.copy(), Vd.copy())
+    i8 = orc.decode_layer(Wqkv, Wo, Wgu, Wd, H, I, n_qh, n_kvh, hd, h8, ars, lens, K8, V8, cap, want=True)
+    Kb = synth.bf16_normal_np(SEED, 54, (A, n_kvh, cap, hd))
+    Vb = synth.bf16_normal_np(SEED, 55, (A, n_kvh, cap, hd))
+    ib = orc.decode_layer(Wqkv, Wo, Wgu, Wd, H, I, n_qh, n_kvh, hd, hb, ars, lens, Kb, Vb, cap, want=True)
+    assert np.array_equal(i8["x1"], ib["x1"]) and np.array_equal(i8["qkv"], ib["qkv"])
+
+    def gq8(v):
+        blk = gguf.quants.quantize(v.astype(np.float32).reshape(-1), gguf.GGMLQuantizationType.Q8_0).reshape(-1, 34)
+        return blk[:, 2:].view(np.int8).reshape(-1), blk[:, :2].copy().view(np.uint16).reshape(-1)
+    for r in range(M):
+        a = int(np.searchsorted(ars, r, side="right") - 1)
+        pos = lens[a] + r - ars[a]
+        for g in range(n_kvh):
+            for plane, off in ((K8, nq), (V8, nq + nkv)):
+                q, d = gq8(i8["qkv"][r, off + g * hd: off + (g + 1) * hd])
+                assert np.array_equal(plane[0][a, g, pos], q) and np.array_equal(plane[1][a, g, pos], d)
+    # attention over the dequantised cache, restated with torch SDPA
+    deq = lambda P: np.repeat(P[1].view(np.float16).astype(np.float64), 32, axis=3) * P[0]  # noqa: E731
+    Kf, Vf = torch.from_numpy(deq(K8)), torch.from_numpy(deq(V8))
+    Q = torch.from_numpy(orc.bf16_array_to_f64(orc.f64_array_to_bf16(i8["qkv"][:, :nq]))).reshape(M, n_qh, hd)
+    G = n_qh // n_kvh
+    o = torch.zeros(M, n_qh, hd, dtype=torch.float64)
+    for a in range(A):
+        r0, r1 = int(ars[a]), int(ars[a + 1])
+        if r1 == r0:
+            continue
+        nk = int(lens[a]) + r1 - r0
+        mask = torch.arange(nk)[None, :] <= (torch.arange(r1 - r0) + int(lens[a]))[:, None]
+        o[r0:r1] = F.scaled_dot_product_attention(Q[r0:r1].permute(1, 0, 2), Kf[a, :, :nk].repeat_interleave(G, 0),
+                                                  Vf[a, :, :nk].repeat_interleave(G, 0),
+                                                  attn_mask=mask).permute(1, 0, 2)
+    o = o.reshape(M, nq).numpy()
+    got = orc.bf16_array_to_f64(i8["attn"])
+    assert np.abs(got - o).max() <= 2.0 ** -8 * np.abs(o).max()
