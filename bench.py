@@ -49,7 +49,10 @@ WORKLOADS = {
                       "1024 cached tokens per agent", 64, 3, 4, 1024),
     "stack12_ctx23k": ("64-layer Q4_K stack, 12 rows = 4 agents x 3, 23000 cached tokens per agent "
                        "(GQA 48/8 heads, bf16 KV)", 64, 3, 4, 23000),
+    "stack12_ctx23k_q8": ("64-layer Q4_K stack, 12 rows = 4 agents x 3, 23000 cached tokens per agent "
+                          "(GQA 48/8 heads, q8_0 KV)", 64, 3, 4, 23000),
 }
+KV_Q8_WORKLOADS = {"stack12_ctx23k_q8"}
 for _m in (1, 2, 3, 4, 6, 8, 12, 16):
     WORKLOADS[f"stack_m{_m}"] = (f"64-layer Q4_K stack, {_m} rows (row-count sweep), 1024 cached tokens",
                                  64, _m, 1, 1024)
@@ -73,6 +76,7 @@ class Workload:
         self.shape, self.rows_per_agent, self.n_agents, self.ctx = sh, rpa, na, cl
         self.M = rpa * na
         self.kv_cap = cl + rpa
+        self.kv_q8 = name in KV_Q8_WORKLOADS
         g = synth.torch_gen(seed, device, 0)
         H, I, hd = sh.hidden, sh.inter, sh.head_dim
         nq, nkv = sh.n_qh * hd, sh.n_kvh * hd
@@ -86,11 +90,22 @@ class Workload:
             self.w_gu.append(torch.cat([synth.q4k_matrix_torch(gl, I, H, device),
                                         synth.q4k_matrix_torch(gl, I, H, device)]))
             self.w_down.append(q.q6k_pack(synth.q6k_matrix_torch(gl, H, I, device), H, I))
-            self.kc.append(synth.bf16_normal_torch(gl, (na, sh.n_kvh, self.kv_cap, hd), device))
-            self.vc.append(synth.bf16_normal_torch(gl, (na, sh.n_kvh, self.kv_cap, hd), device))
+            if self.kv_q8:
+                for caches in (self.kc, self.vc):
+                    buf = torch.empty(q.kv_cache_bytes(q.KV_Q8_0, na, sh.n_kvh, self.kv_cap, hd),
+                                      dtype=torch.uint8, device=device)
+                    codes, scales = q.q8_cache_planes(buf, na, sh.n_kvh, self.kv_cap, hd)
+                    c8, s16 = synth.q8_planes_torch(gl, na * sh.n_kvh * self.kv_cap, hd, device)
+                    codes.view(-1, hd).copy_(c8)
+                    scales.view(-1, hd // 32).copy_(s16.view(torch.int16))
+                    caches.append(buf)
+            else:
+                self.kc.append(synth.bf16_normal_torch(gl, (na, sh.n_kvh, self.kv_cap, hd), device))
+                self.vc.append(synth.bf16_normal_torch(gl, (na, sh.n_kvh, self.kv_cap, hd), device))
         self.model = q.Model(hidden=H, inter=I, n_qh=sh.n_qh, n_kvh=sh.n_kvh, head_dim=hd, max_agents=na,
                              kv_cap=self.kv_cap, w_qkv=self.w_qkv, w_o=self.w_o, w_gu=self.w_gu,
-                             w_down=self.w_down, k_cache=self.kc, v_cache=self.vc)
+                             w_down=self.w_down, k_cache=self.kc, v_cache=self.vc,
+                             kv_format=q.KV_Q8_0 if self.kv_q8 else q.KV_BF16)
         self.X = synth.bf16_normal_torch(g, (self.M, H), device)
         self.ars = torch.arange(0, self.M + 1, rpa, dtype=torch.int32, device=device)
         self.lens = torch.full((na,), cl, dtype=torch.int32, device=device)
@@ -98,7 +113,8 @@ class Workload:
         self.ws = q.alloc_ws(self.model.ws_bytes(self.M), device)
         self.weight_bytes = sum(t.numel() for ts in (self.w_qkv, self.w_o, self.w_gu, self.w_down) for t in ts)
         # (the packed down projection carries each block's 210 bytes plus up to 14 bytes of row padding)
-        self.kv_bytes = 2 * L * na * sh.n_kvh * (cl + rpa) * hd * 2  # keys read per step (incl. new rows)
+        # keys and values read per step (incl. new rows): bf16, or q8_0 codes + one fp16 scale per 32
+        self.kv_bytes = 2 * L * na * sh.n_kvh * (cl + rpa) * (hd + hd // 16 if self.kv_q8 else hd * 2)
         self.act_bytes = L * self.M * (2 * H * 4 + 2 * I * 4 + (nq + 2 * nkv) * 4)  # fp32 outputs/residual
 
     def down_gguf(self, layer):
@@ -247,16 +263,17 @@ def barrier(ws):
 _SAMPLE_CACHE = {}
 
 
-def oracle_layer_sample(seed=SEED, ctx=1024, rows_per_agent=3, n_agents=4, threads=0):
+def oracle_layer_sample(seed=SEED, ctx=1024, rows_per_agent=3, n_agents=4, threads=0, kv_q8=False):
     """One decoder layer of the same stack through the fp64 CPU oracle (inputs
     drawn once and reused). Returns (seconds, weight bytes of the layer, threads used)."""
     import oracle
-    key = (seed, ctx, rows_per_agent, n_agents)
+    key = (seed, ctx, rows_per_agent, n_agents, kv_q8)
     if key not in _SAMPLE_CACHE:
-        _SAMPLE_CACHE[key] = _oracle_layer_inputs(seed, ctx, rows_per_agent, n_agents)
+        _SAMPLE_CACHE[key] = _oracle_layer_inputs(seed, ctx, rows_per_agent, n_agents, kv_q8)
     Wqkv, Wo, Wgu, Wd, Kc0, Vc0, h0, ars, lens, cap = _SAMPLE_CACHE[key]
     sh = synth.StackShape(n_layers=1)
-    Kc, Vc, h = Kc0.copy(), Vc0.copy(), h0.copy()
+    cp = lambda c: tuple(a.copy() for a in c) if isinstance(c, tuple) else c.copy()  # noqa: E731
+    Kc, Vc, h = cp(Kc0), cp(Vc0), h0.copy()
     nth = threads or oracle.max_threads()
     t0 = time.perf_counter()
     oracle.decode_layer(Wqkv, Wo, Wgu, Wd, sh.hidden, sh.inter, sh.n_qh, sh.n_kvh, sh.head_dim, h, ars, lens,
@@ -266,7 +283,7 @@ def oracle_layer_sample(seed=SEED, ctx=1024, rows_per_agent=3, n_agents=4, threa
     return dt, wbytes, nth
 
 
-def _oracle_layer_inputs(seed, ctx, rows_per_agent, n_agents):
+def _oracle_layer_inputs(seed, ctx, rows_per_agent, n_agents, kv_q8=False):
     import oracle
     sh = synth.StackShape(n_layers=1)
     H, I, hd = sh.hidden, sh.inter, sh.head_dim
@@ -277,8 +294,17 @@ def _oracle_layer_inputs(seed, ctx, rows_per_agent, n_agents):
     Wgu = np.concatenate([synth.q4k_matrix_np(seed, 5, I, H), synth.q4k_matrix_np(seed, 6, I, H)])
     Wd = synth.q6k_matrix_np(seed, 7, H, I)
     cap = ctx + rows_per_agent
-    Kc = synth.bf16_normal_np(seed, 8, (n_agents, sh.n_kvh, cap, hd))
-    Vc = synth.bf16_normal_np(seed, 9, (n_agents, sh.n_kvh, cap, hd))
+    if kv_q8:
+        g = synth.torch_gen(seed, "cpu", 8)
+        planes = []
+        for _ in range(2):
+            c8, s16 = synth.q8_planes_torch(g, n_agents * sh.n_kvh * cap, hd, "cpu")
+            planes.append((c8.numpy().reshape(n_agents, sh.n_kvh, cap, hd),
+                           s16.numpy().view(np.uint16).reshape(n_agents, sh.n_kvh, cap, hd // 32)))
+        Kc, Vc = planes
+    else:
+        Kc = synth.bf16_normal_np(seed, 8, (n_agents, sh.n_kvh, cap, hd))
+        Vc = synth.bf16_normal_np(seed, 9, (n_agents, sh.n_kvh, cap, hd))
     M = rows_per_agent * n_agents
     h = oracle.bf16_array_to_f64(synth.bf16_normal_np(seed, 10, (M, H)))
     ars = np.arange(0, M + 1, rows_per_agent, dtype=np.int32)
@@ -293,10 +319,11 @@ def run_reference(args, ws, rank):
         return 0
     desc, L, rpa, na, cl = WORKLOADS[args.workload]
     for _ in range(args.warmup):
-        oracle_layer_sample(ctx=cl, rows_per_agent=rpa, n_agents=na)
+        oracle_layer_sample(ctx=cl, rows_per_agent=rpa, n_agents=na, kv_q8=args.workload in KV_Q8_WORKLOADS)
     times = []
     for _ in range(args.steps):
-        dt, wb, nth = oracle_layer_sample(ctx=cl, rows_per_agent=rpa, n_agents=na)
+        dt, wb, nth = oracle_layer_sample(ctx=cl, rows_per_agent=rpa, n_agents=na,
+                                          kv_q8=args.workload in KV_Q8_WORKLOADS)
         times.append(dt)
     t = statistics.median(times)
     step_s = t * L
@@ -409,7 +436,8 @@ def run_gpu(args, ws, rank, local):
         # repeat one decoder layer of the same stack (fresh caches each time) for >= 10 s of CPU work
         tot, n = 0.0, 0
         while tot < 10.0 and n < L:
-            dt, wb, nth = oracle_layer_sample(ctx=w.ctx, rows_per_agent=w.rows_per_agent, n_agents=w.n_agents)
+            dt, wb, nth = oracle_layer_sample(ctx=w.ctx, rows_per_agent=w.rows_per_agent, n_agents=w.n_agents,
+                                              kv_q8=w.kv_q8)
             tot += dt
             n += 1
         cpu = {"value": wb * n / tot / 1e9, "unit": "GB/s", "cores": nth, "kind": "oracle",
@@ -553,6 +581,20 @@ def run_kernel(args):
         fn = lambda i, st: q.decode_attn(Qd, Kd, Vd, lens, ars, A, 3, cap, n_qh, n_kvh, 128, O, ws=ws,  # noqa: E731
                                          stream=st)
         nbytes = 2 * A * n_kvh * cap * 128 * 2
+    elif args.kernel == "attn23k_q8":
+        A, L, n_qh, n_kvh = 4, 23000, 48, 8
+        cap = L + 3
+        Kq, Kd = synth.q8_planes_torch(g, A * n_kvh * cap, 128, "cuda")
+        Vq, Vd = synth.q8_planes_torch(g, A * n_kvh * cap, 128, "cuda")
+        Kd, Vd = Kd.view(torch.int16), Vd.view(torch.int16)
+        Qd = synth.bf16_normal_torch(g, (12, n_qh, 128), "cuda")
+        lens = torch.full((A,), L, dtype=torch.int32, device="cuda")
+        ars = torch.arange(0, 13, 3, dtype=torch.int32, device="cuda")
+        O = torch.zeros(12, n_qh, 128, dtype=torch.bfloat16, device="cuda")
+        ws = q.alloc_ws(q.decode_attn_ws_bytes(A, n_qh, n_kvh, cap, 3))
+        fn = lambda i, st: q.decode_attn_q8(Qd, Kq, Kd, Vq, Vd, lens, ars, A, 3, cap, n_qh, n_kvh, 128,  # noqa: E731
+                                            O, ws=ws, stream=st)
+        nbytes = 2 * A * n_kvh * cap * (128 + 8)
     else:
         fmt, N, K = KERNELS[args.kernel]
         mk = synth.q4k_matrix_torch if fmt == 4 else synth.q6k_matrix_torch
@@ -609,7 +651,7 @@ def main():
     ap.add_argument("--workload", default="stack12_ctx1k", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel", choices=sorted(list(KERNELS) + list(DENSE_KERNELS) + ["attn23k", "pfattn23k", "verify"]),
+    ap.add_argument("--kernel", choices=sorted(list(KERNELS) + list(DENSE_KERNELS) + ["attn23k", "attn23k_q8", "pfattn23k", "verify"]),
                     help="time one kernel of the step instead (profiler captures)")
     ap.add_argument("--rows", type=int, default=12)
     ap.add_argument("--trace", action="store_true", help="print the per-launch device timeline of one step")

@@ -192,6 +192,38 @@ int qad_decode_attn(const uint16_t *Q, const uint16_t *Kc, const uint16_t *Vc, c
                     int n_qh, int n_kvh, int hd, float scale, uint16_t *O, void *ws, size_t ws_bytes,
                     void *stream);
 
+/* ---------------------------------------------------------------- q8_0 KV cache
+ * dual-4090 page (rebasdaily.com 2026-09-10, llama.cpp agent concurrency on two
+ * RTX 4090s): its tests keep the KV cache in q8_0. Block format (llama.cpp's
+ * q8_0): 32 consecutive values share one fp16 scale and hold int8 codes,
+ *   d = amax / 127 (fp32 division), id = d != 0 ? 1 / d : 0 (fp32),
+ *   q_i = roundf(x_i * id) (fp32 product, ties away from zero), scale = fp16_RNE(d),
+ * value = fp16(d) * q. A q8_0 cache tensor is ONE allocation of
+ * qad_kv_cache_bytes(QAD_KV_Q8_0, ...) bytes: the codes [agents][n_kvh][kv_cap][hd]
+ * int8 first, then, at the next 256-byte boundary, the scales
+ * [agents][n_kvh][kv_cap][hd/32] fp16. Values must be finite and within the
+ * fp16 range. */
+#define QAD_KV_BF16 0
+#define QAD_KV_Q8_0 8
+/* Bytes of one K (or V) cache tensor of the given format; 0 for invalid
+ * arguments (hd must be 128). */
+size_t qad_kv_cache_bytes(int kv_format, int n_agents, int n_kvh, int kv_cap, int hd);
+/* q8_0 of n values (n % 32 == 0): x device fp32 (x_is_bf16 == 0) or bf16
+ * [n], 16-byte aligned; q device int8 [n], 16-byte aligned; d device fp16
+ * [n/32]. One launch on `stream`. Bit-exact with the definition above. */
+int qad_q8_0_quantize(const void *x, int x_is_bf16, long long n, int8_t *q, uint16_t *d, void *stream);
+/* Decode attention (the definition of qad_decode_attn) over a q8_0 cache:
+ *   Kq, Vq  device int8 codes [n_agents][n_kvh][kv_cap][hd], 16-byte aligned
+ *   Kd, Vd  device fp16 scales [n_agents][n_kvh][kv_cap][hd/32], 8-byte aligned
+ * Other arguments, limits and the workspace are those of qad_decode_attn
+ * (qad_decode_attn_ws_bytes). Keys enter the product exactly (int8 codes,
+ * per-block scales applied in fp32); V is dequantised to fp16 (one rounding)
+ * and the probabilities are fp16. Q 8-byte aligned. */
+int qad_decode_attn_q8(const uint16_t *Q, const int8_t *Kq, const uint16_t *Kd, const int8_t *Vq,
+                       const uint16_t *Vd, const int *lens, const int *agent_row_start, int n_agents,
+                       int max_rows_per_agent, int kv_cap, int n_qh, int n_kvh, int hd, float scale,
+                       uint16_t *O, void *ws, size_t ws_bytes, void *stream);
+
 /* ---------------------------------------------------------------- verify tail
  * OpenJet page, section 只搬一次权重: every agent's drafts are checked in the
  * same pass as its next token. The acceptance rule is not on the page; the
@@ -259,9 +291,13 @@ int qad_pack_rows(const qad_agent_rows *agents, int n_agents, int hidden, int ma
  *   w_o    Q4_K [hidden][n_qh hd]
  *   w_gu   Q4_K [2 inter][hidden]               rows: gate, then up
  *   w_down Q6_K-like [hidden][inter], packed by qad_q6k_pack
- *   k_cache, v_cache bf16 [max_agents][n_kvh][kv_cap][hd]
+ *   k_cache, v_cache bf16 [max_agents][n_kvh][kv_cap][hd] (kv_format
+ *          QAD_KV_BF16), or q8_0 cache allocations of qad_kv_cache_bytes(
+ *          QAD_KV_Q8_0, max_agents, n_kvh, kv_cap, hd) bytes (kv_format
+ *          QAD_KV_Q8_0; the new rows' k, v are quantised from the fp32
+ *          projection)
  * The descriptor's pointer arrays are host arrays of n_layers entries and are
- * copied by qad_model_create. */
+ * copied by qad_model_create. A zero-initialised kv_format is bf16. */
 typedef struct {
     int n_layers, hidden, inter, n_qh, n_kvh, head_dim;
     int max_agents, kv_cap;
@@ -272,6 +308,7 @@ typedef struct {
     const void *const *w_down;
     uint16_t *const *k_cache;
     uint16_t *const *v_cache;
+    int kv_format;
 } qad_model_desc;
 
 typedef struct qad_model qad_model;

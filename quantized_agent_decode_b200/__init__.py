@@ -30,7 +30,10 @@ class ModelDesc(C.Structure):
                 ("n_kvh", C.c_int), ("head_dim", C.c_int), ("max_agents", C.c_int), ("kv_cap", C.c_int),
                 ("rms_eps", C.c_float), ("w_qkv", C.POINTER(C.c_void_p)), ("w_o", C.POINTER(C.c_void_p)),
                 ("w_gu", C.POINTER(C.c_void_p)), ("w_down", C.POINTER(C.c_void_p)),
-                ("k_cache", C.POINTER(C.c_void_p)), ("v_cache", C.POINTER(C.c_void_p))]
+                ("k_cache", C.POINTER(C.c_void_p)), ("v_cache", C.POINTER(C.c_void_p)), ("kv_format", C.c_int)]
+
+
+KV_BF16, KV_Q8_0 = 0, 8
 
 
 class AgentRows(C.Structure):
@@ -65,6 +68,10 @@ SIGNATURES = {
                         + [C.c_void_p] * 7 + [C.c_size_t, C.c_void_p]),
     "qad_prefill_attn": (C.c_int, [C.c_void_p] * 3 + [C.c_int] * 6 + [C.c_float, C.c_void_p, C.c_void_p]),
     "qad_decode_attn_ws_bytes": (C.c_size_t, [C.c_int] * 5),
+    "qad_kv_cache_bytes": (C.c_size_t, [C.c_int] * 5),
+    "qad_q8_0_quantize": (C.c_int, [C.c_void_p, C.c_int, C.c_longlong, C.c_void_p, C.c_void_p, C.c_void_p]),
+    "qad_decode_attn_q8": (C.c_int, [C.c_void_p] * 7 + [C.c_int] * 6 + [C.c_float, C.c_void_p, C.c_void_p,
+                                                                        C.c_size_t, C.c_void_p]),
     "qad_decode_attn": (C.c_int, [C.c_void_p] * 5 + [C.c_int] * 6 + [C.c_float, C.c_void_p, C.c_void_p,
                                                                      C.c_size_t, C.c_void_p]),
     "qad_pack_rows": (C.c_int, [C.POINTER(AgentRows), C.c_int, C.c_int, C.c_int, C.c_void_p, C.c_void_p,
@@ -316,13 +323,58 @@ def pack_rows(agent_rows, lens, hidden: int, max_rows: int = QAD_MAX_ROWS):
     return X[:M], ra[:M], rp[:M], ars
 
 
+def kv_cache_bytes(kv_format, n_agents, n_kvh, kv_cap, hd=128) -> int:
+    """Bytes of one K (or V) cache tensor: bf16, or q8_0 codes + (256-aligned) fp16 scales."""
+    return int(lib().qad_kv_cache_bytes(kv_format, n_agents, n_kvh, kv_cap, hd))
+
+
+def q8_cache_planes(buf, n_agents, n_kvh, kv_cap, hd=128):
+    """Views (codes int8 [A][n_kvh][cap][hd], scales fp16 bits int16 [A][n_kvh][cap][hd/32]) of a
+    uint8 q8_0 cache allocation of kv_cache_bytes(KV_Q8_0, ...) bytes."""
+    n = n_agents * n_kvh * kv_cap * hd
+    off = (n + 255) // 256 * 256
+    codes = buf[:n].view(torch.int8).view(n_agents, n_kvh, kv_cap, hd)
+    scales = buf[off:off + n // 16].view(torch.int16).view(n_agents, n_kvh, kv_cap, hd // 32)
+    return codes, scales
+
+
+def q8_0_quantize(x, q=None, d=None, stream=None):
+    """q8_0 of a fp32 or bf16 device tensor (numel % 32 == 0): (codes int8, scales fp16 bits int16)."""
+    _require_gpu()
+    n = x.numel()
+    if q is None:
+        q = torch.empty(n, dtype=torch.int8, device=x.device)
+    if d is None:
+        d = torch.empty(n // 32, dtype=torch.int16, device=x.device)
+    if x.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("q8_0_quantize: x must be float32 or bfloat16")
+    _check(lib().qad_q8_0_quantize(_dev(x, "x"), int(x.dtype == torch.bfloat16), n, _dev(q, "q"), _dev(d, "d"),
+                                   _stream(stream)), "qad_q8_0_quantize")
+    return q, d
+
+
+def decode_attn_q8(Q, Kq, Kd, Vq, Vd, lens, agent_row_start, n_agents, max_rows_per_agent, kv_cap, n_qh, n_kvh, hd,
+                   O, scale=None, ws=None, stream=None):
+    _require_gpu()
+    if scale is None:
+        scale = hd ** -0.5
+    if ws is None:
+        ws = alloc_ws(decode_attn_ws_bytes(n_agents, n_qh, n_kvh, kv_cap, max_rows_per_agent), Q.device)
+    _check(lib().qad_decode_attn_q8(_dev(Q, "Q"), _dev(Kq, "Kq"), _dev(Kd, "Kd"), _dev(Vq, "Vq"), _dev(Vd, "Vd"),
+                                    _dev(lens, "lens"), _dev(agent_row_start, "agent_row_start"), n_agents,
+                                    max_rows_per_agent, kv_cap, n_qh, n_kvh, hd, float(scale), _dev(O, "O"),
+                                    _dev(ws, "ws"), ws.numel() * ws.element_size(), _stream(stream)),
+           "qad_decode_attn_q8")
+    return O
+
+
 # ------------------------------------------------------------------ model / decode step
 
 class Model:
     """A decoder stack whose weights and KV caches live in caller-owned device tensors."""
 
     def __init__(self, *, hidden, inter, n_qh, n_kvh, head_dim, max_agents, kv_cap, w_qkv, w_o, w_gu, w_down,
-                 k_cache, v_cache, rms_eps=1e-6):
+                 k_cache, v_cache, rms_eps=1e-6, kv_format=KV_BF16):
         _require_gpu()
         L = len(w_qkv)
         self._keep = (w_qkv, w_o, w_gu, w_down, k_cache, v_cache)
@@ -331,12 +383,13 @@ class Model:
             assert len(ts) == L, name
             arrs.append((C.c_void_p * L)(*[_dev(t, name).value for t in ts]))
         self._arrs = arrs
-        d = ModelDesc(L, hidden, inter, n_qh, n_kvh, head_dim, max_agents, kv_cap, rms_eps, *arrs)
+        d = ModelDesc(L, hidden, inter, n_qh, n_kvh, head_dim, max_agents, kv_cap, rms_eps, *arrs, kv_format)
         h = C.c_void_p()
         _check(lib().qad_model_create(C.byref(d), C.byref(h)), "qad_model_create")
         self.handle = h
         self.n_layers, self.hidden, self.inter = L, hidden, inter
         self.n_qh, self.n_kvh, self.head_dim, self.max_agents, self.kv_cap = n_qh, n_kvh, head_dim, max_agents, kv_cap
+        self.kv_format = kv_format
         self._dbg = None
 
     def close(self):

@@ -515,10 +515,16 @@ int launch_attn(const AttnPlan &pl, const uint16_t *Q, const uint16_t *Kc, const
     int rc = launch_split_kernel<false>(pl, p, n_agents, s, pdl);
     if (rc)
         return rc;
-    cudaError_t e;
+    return launch_attn_combine(pl, part, lens, ars, n_agents, kv_cap, n_qh, n_kvh, O, s, pdl);
+}
+
+int launch_attn_combine(const AttnPlan &pl, const float *part, const int *lens, const int *ars, int n_agents,
+                        int kv_cap, int n_qh, int n_kvh, uint16_t *O, cudaStream_t s, bool pdl)
+{
+    AttnArgs p = attn_args(pl, lens, ars, kv_cap, n_qh, n_kvh, 1.f, const_cast<float *>(part));
     dim3 g2(QG, pl.n_rg, n_agents * n_kvh);
-    e = pdl ? launch_pdl(k_attn_combine, g2, dim3(128), 0, s, p, O)
-            : (k_attn_combine<<<g2, 128, 0, s>>>(p, O), cudaGetLastError());
+    cudaError_t e = pdl ? launch_pdl(k_attn_combine, g2, dim3(128), 0, s, p, O)
+                        : (k_attn_combine<<<g2, 128, 0, s>>>(p, O), cudaGetLastError());
     return cuda_check(e, "attn combine launch");
 }
 

@@ -39,6 +39,19 @@ int launch_attn(const AttnPlan &pl, const uint16_t *Q, const uint16_t *Kc, const
 int launch_attn_fused(const AttnPlan &pl, const float *qkv, int ldqkv, uint16_t *Kc, uint16_t *Vc, const int *lens,
                       const int *ars, int n_agents, int kv_cap, int n_qh, int n_kvh, float scale, float *part,
                       cudaStream_t s, bool pdl, unsigned long long *trace = nullptr);
+// Combine the splits of a standalone launch into bf16 O [M][n_qh][128].
+int launch_attn_combine(const AttnPlan &pl, const float *part, const int *lens, const int *ars, int n_agents,
+                        int kv_cap, int n_qh, int n_kvh, uint16_t *O, cudaStream_t s, bool pdl);
+// q8_0 cache: int8 codes [A][n_kvh][kv_cap][128] and fp16 scales [A][n_kvh][kv_cap][4]
+// (one per 32 values) for K and for V. Same plan and partial records as the bf16 form.
+int launch_attn_q8_fused(const AttnPlan &pl, const float *qkv, int ldqkv, int8_t *Kq, uint16_t *Kd, int8_t *Vq,
+                         uint16_t *Vd, const int *lens, const int *ars, int n_agents, int kv_cap, int n_qh, int n_kvh,
+                         float scale, float *part, cudaStream_t s, bool pdl, unsigned long long *trace = nullptr);
+int launch_attn_q8(const AttnPlan &pl, const uint16_t *Q, const int8_t *Kq, const uint16_t *Kd, const int8_t *Vq,
+                   const uint16_t *Vd, const int *lens, const int *ars, int n_agents, int kv_cap, int n_qh, int n_kvh,
+                   float scale, uint16_t *O, float *part, cudaStream_t s, bool pdl);
+// Byte offset of the scale plane inside one q8_0 cache allocation.
+size_t kv_q8_scale_offset(int n_agents, int n_kvh, int kv_cap);
 AttnPartView attn_part_view(const AttnPlan &pl, const float *part, const int *ars, const int *lens, int kv_cap,
                             int n_qh, int n_kvh);
 

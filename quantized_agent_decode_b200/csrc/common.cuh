@@ -165,6 +165,7 @@ constexpr uint32_t H2_1056 = 0x64206420u;   // 1056.0
 constexpr uint32_t H2_ONE = 0x3C003C00u;    // 1.0
 constexpr uint32_t H2_SIXTEENTH = 0x2C002C00u; // 0.0625
 constexpr uint32_t H2_NEG64 = 0xD400D400u;  // -64.0
+constexpr uint32_t H2_1152 = 0x64806480u;   // 1152.0 = 1024 + 128
 
 // ----------------------------------------------------------------- tensor core (legacy warp MMA)
 
@@ -394,6 +395,13 @@ __device__ __forceinline__ void cp_async16_zfill(void *smem, const void *gmem, b
     uint32_t a = (uint32_t)__cvta_generic_to_shared(smem);
     int n = valid ? 16 : 0;
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(a), "l"(gmem), "r"(n));
+}
+// 8-byte copy through L1 (the .cg form moves 16 bytes only); zero fill when !valid.
+__device__ __forceinline__ void cp_async8_zfill(void *smem, const void *gmem, bool valid)
+{
+    uint32_t a = (uint32_t)__cvta_generic_to_shared(smem);
+    int n = valid ? 8 : 0;
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(a), "l"(gmem), "r"(n));
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;"); }
 template <int N>

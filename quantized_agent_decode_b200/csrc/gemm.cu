@@ -539,7 +539,6 @@ __device__ __forceinline__ void q4_block(const uint8_t *W, const uint8_t *XS, co
         }
 }
 
-constexpr uint32_t H2_1152 = 0x64806480u;  // 1152.0
 
 // One Q6_K-like block (packed layout) of this warp's 32 weight rows. A: the
 // warp's first row in plane A of the stage; D: its first row of the d tile.

@@ -243,8 +243,16 @@ static int run_step(qad_model *m, const uint16_t *X, int M, const int *ars, int 
         if (dbg && (rc = copy_d2d(dbg + DL.qkv, qkv, (size_t)M * nqkv * 4, s)))
             return rc;
         // attention over each agent's cache; k, v of the new rows appended
-        QAD_PROF(PK_ATTN, launch_attn_fused(plan, qkv, nqkv, m->kc[l], m->vc[l], lens, ars, n_agents, d.kv_cap,
-                                            d.n_qh, d.n_kvh, scale, part, s, true, tr()));
+        if (d.kv_format == QAD_KV_Q8_0) {
+            const size_t so = kv_q8_scale_offset(d.max_agents, d.n_kvh, d.kv_cap);
+            int8_t *Kq = (int8_t *)m->kc[l], *Vq = (int8_t *)m->vc[l];
+            uint16_t *Kd = (uint16_t *)((char *)m->kc[l] + so), *Vd = (uint16_t *)((char *)m->vc[l] + so);
+            QAD_PROF(PK_ATTN, launch_attn_q8_fused(plan, qkv, nqkv, Kq, Kd, Vq, Vd, lens, ars, n_agents, d.kv_cap,
+                                                   d.n_qh, d.n_kvh, scale, part, s, true, tr()));
+        } else {
+            QAD_PROF(PK_ATTN, launch_attn_fused(plan, qkv, nqkv, m->kc[l], m->vc[l], lens, ars, n_agents, d.kv_cap,
+                                                d.n_qh, d.n_kvh, scale, part, s, true, tr()));
+        }
         // O = merged splits (bf16); h += O Wo^T
         fb = frag_carve(ws + L.frag, nq, nt);
         src = PrepSrc{};
@@ -323,6 +331,9 @@ extern "C" int qad_model_create(const qad_model_desc *desc, qad_model **out)
         d.kv_cap <= 0 || !(d.rms_eps >= 0.f) || !d.w_qkv || !d.w_o || !d.w_gu || !d.w_down || !d.k_cache ||
         !d.v_cache)
         return qad::fail(QAD_ERR_INVALID, "qad_model_create: invalid descriptor");
+    if (d.kv_format != QAD_KV_BF16 && d.kv_format != QAD_KV_Q8_0)
+        return qad::fail(QAD_ERR_UNSUPPORTED, "qad_model_create: kv_format %d (need QAD_KV_BF16 or QAD_KV_Q8_0)",
+                         d.kv_format);
     if (d.head_dim != 128 || d.n_qh % d.n_kvh || d.hidden % 256 || d.inter % 256 || (d.n_qh * d.head_dim) % 256 ||
         d.hidden > 65536 || d.inter > 65536)
         return qad::fail(QAD_ERR_UNSUPPORTED,

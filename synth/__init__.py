@@ -126,6 +126,15 @@ def bf16_normal_torch(gen: torch.Generator, shape, device, scale: float = 1.0) -
     return t.to(torch.bfloat16)
 
 
+def q8_planes_torch(gen: torch.Generator, n_rows: int, hd: int, device):
+    """A q8_0-shaped cache of n_rows rows drawn in ``device`` memory: int8 codes
+    [n_rows, hd] (normal, sd 42, clipped to +-127) and fp16 scales [n_rows, hd/32]
+    uniform in [0.01, 0.03) (values of roughly N(0,1) size)."""
+    codes = torch.randn((n_rows, hd), device=device, generator=gen).mul_(42.0).round_().clamp_(-127, 127)
+    scales = torch.rand((n_rows, hd // 32), device=device, generator=gen).mul_(0.02).add_(0.01)
+    return codes.to(torch.int8), scales.to(torch.float16)
+
+
 # ---------------------------------------------------------------- model shapes
 
 class StackShape:

@@ -68,8 +68,9 @@ def bf16_close(gpu_bits, ref_bits, orc, frac=1e-3):
 class Stack:
     """A small synthetic stack with ragged agents, built on the GPU from host arrays."""
 
-    def __init__(self, q, n_layers, H, I, n_qh, n_kvh, n_rows, lens, seed, extra_cap=4):
+    def __init__(self, q, n_layers, H, I, n_qh, n_kvh, n_rows, lens, seed, extra_cap=4, kv="bf16", orc=None):
         self.q = q
+        self.kv = kv
         self.L, self.H, self.I, self.n_qh, self.n_kvh = n_layers, H, I, n_qh, n_kvh
         hd = 128
         self.nq, self.nkv = n_qh * hd, n_kvh * hd
@@ -92,24 +93,51 @@ class Stack:
                 down=synth.q6k_matrix_np(SEED, t + 7, H, I),
                 kc=synth.bf16_normal_np(SEED, t + 8, (self.A, n_kvh, self.cap, hd)),
                 vc=synth.bf16_normal_np(SEED, t + 9, (self.A, n_kvh, self.cap, hd))))
+            if kv == "q8_0":  # the cached rows: q8_0 of N(0,1) values (the oracle's quantiser)
+                w = self.W[-1]
+                for name in ("kc", "vc"):
+                    w[name + "8"] = orc.q8_0_quantize(orc.bf16_array_to_f64(w[name]).astype(np.float32))
         self.X = synth.bf16_normal_np(SEED, seed + 7777, (self.M, H))
         dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()  # noqa: E731
         bdev = lambda a: dev(a.view(np.int16)).view(torch.bfloat16)  # noqa: E731
         self.d = dict(qkv=[dev(w["qkv"]) for w in self.W], o=[dev(w["o"]) for w in self.W],
                       gu=[dev(w["gu"]) for w in self.W],
-                      down=[q.q6k_pack(dev(w["down"]), H, I) for w in self.W],
-                      kc=[bdev(w["kc"]) for w in self.W], vc=[bdev(w["vc"]) for w in self.W])
+                      down=[q.q6k_pack(dev(w["down"]), H, I) for w in self.W])
+        if kv == "q8_0":
+            nbytes = q.kv_cache_bytes(q.KV_Q8_0, self.A, n_kvh, self.cap)
+            self.d["kc"] = [torch.zeros(nbytes, dtype=torch.uint8, device="cuda") for _ in self.W]
+            self.d["vc"] = [torch.zeros(nbytes, dtype=torch.uint8, device="cuda") for _ in self.W]
+            self.reset_caches()
+        else:
+            self.d["kc"] = [bdev(w["kc"]) for w in self.W]
+            self.d["vc"] = [bdev(w["vc"]) for w in self.W]
         self.model = q.Model(hidden=H, inter=I, n_qh=n_qh, n_kvh=n_kvh, head_dim=hd, max_agents=self.A,
                              kv_cap=self.cap, w_qkv=self.d["qkv"], w_o=self.d["o"], w_gu=self.d["gu"],
-                             w_down=self.d["down"], k_cache=self.d["kc"], v_cache=self.d["vc"])
+                             w_down=self.d["down"], k_cache=self.d["kc"], v_cache=self.d["vc"],
+                             kv_format=q.KV_Q8_0 if kv == "q8_0" else q.KV_BF16)
         self.Xd = bdev(self.X)
         self.arsd = dev(self.ars)
         self.lensd = dev(self.lens)
         self.Hd = torch.empty(self.M, H, dtype=torch.float32, device="cuda")
         self.ws = q.alloc_ws(self.model.ws_bytes(self.M))
 
+    def planes(self, l):
+        """Host copies (Kq, Kd, Vq, Vd) of layer l's q8_0 caches."""
+        out = []
+        for buf in (self.d["kc"][l], self.d["vc"][l]):
+            codes, scales = self.q.q8_cache_planes(buf, self.A, self.n_kvh, self.cap)
+            out += [codes.cpu().numpy(), scales.cpu().numpy().view(np.uint16)]
+        return out
+
     def reset_caches(self):
         for l in range(self.L):
+            if self.kv == "q8_0":
+                for name in ("kc", "vc"):
+                    codes, scales = self.q.q8_cache_planes(self.d[name][l], self.A, self.n_kvh, self.cap)
+                    qn, dn = self.W[l][name + "8"]
+                    codes.copy_(torch.from_numpy(qn))
+                    scales.copy_(torch.from_numpy(dn.view(np.int16)))
+                continue
             self.d["kc"][l].copy_(torch.from_numpy(self.W[l]["kc"].view(np.int16)).view(torch.bfloat16))
             self.d["vc"][l].copy_(torch.from_numpy(self.W[l]["vc"].view(np.int16)).view(torch.bfloat16))
 
@@ -120,9 +148,10 @@ class Stack:
         return dbg
 
 
-def check_layer(st, orc, dbg, l, h_in, kc_after, vc_after, rows=None):
+def check_layer(st, orc, dbg, l, h_in, kc_after, vc_after, rows=None, q8=None):
     """Teacher-forced checks of layer l. h_in: the layer's fp32 input (GPU values).
-    rows: optional subset of output rows for the GEMM checks (full size)."""
+    rows: optional subset of output rows for the GEMM checks (full size).
+    q8: (Kq, Kd, Vq, Vd) host copies of a q8_0 cache after the step (kc/vc unused)."""
     v = dbg_views(dbg, l, st.M, st.H, st.I, st.nq, st.nqkv)
     W = st.W[l] if isinstance(st.W[l], dict) else st.W[l]()
     # x1 = bf16(rmsnorm(h))
@@ -138,6 +167,22 @@ def check_layer(st, orc, dbg, l, h_in, kc_after, vc_after, rows=None):
         assert ratio.max() <= 1.0, ratio.max()
 
     gemm_check(4, W["qkv"], st.nqkv, st.H, v["x1"], v["qkv"])
+    if q8 is not None:
+        # k, v appended as q8_0 of the fp32 projection, bit-exact (same fp32 decisions)
+        Kq, Kd, Vq, Vd = q8
+        for r in range(st.M):
+            a = int(np.searchsorted(st.ars, r, side="right") - 1)
+            pos = st.lens[a] + r - st.ars[a]
+            kq, kd = orc.q8_0_quantize(v["qkv"][r, st.nq:st.nq + st.nkv].reshape(st.n_kvh, 128))
+            vq, vd = orc.q8_0_quantize(v["qkv"][r, st.nq + st.nkv:].reshape(st.n_kvh, 128))
+            assert np.array_equal(Kq[a, :, pos], kq) and np.array_equal(Kd[a, :, pos], kd)
+            assert np.array_equal(Vq[a, :, pos], vq) and np.array_equal(Vd[a, :, pos], vd)
+        Qb = orc.f64_array_to_bf16(v["qkv"][:, :st.nq].astype(np.float64)).reshape(st.M, st.n_qh, 128)
+        O_ref, B = orc.decode_attn_q8(Qb, Kq, Kd, Vq, Vd, st.lens, st.ars, st.n_qh, st.n_kvh, 128, st.cap)
+        o = orc.bf16_array_to_f64(v["attn"]).reshape(O_ref.shape)
+        # fp16 V and P leave the fp32 result within 2e-3 * B; bf16 output: half an ulp (2^-8 relative) more
+        assert (np.abs(o - O_ref) <= 2e-3 * B + np.abs(O_ref) * 2.0 ** -8 + 1e-30).all()
+        return _check_after_attn(st, orc, v, W, h_in, gemm_check)
     # k, v appended as bf16 of the fp32 projection, exactly
     kvb = orc.f64_array_to_bf16(v["qkv"][:, st.nq:].astype(np.float64)) if rows is None else None
     for r in range(st.M):
@@ -155,6 +200,10 @@ def check_layer(st, orc, dbg, l, h_in, kc_after, vc_after, rows=None):
     O_ref, B = orc.decode_attn(Qb, kc_after, vc_after, st.lens, st.ars, st.n_qh, st.n_kvh, 128, st.cap)
     o = orc.bf16_array_to_f64(v["attn"]).reshape(O_ref.shape)
     assert (np.abs(o - O_ref) <= 2e-3 * B + np.abs(O_ref) * 2.0 ** -9 + 1e-30).all()
+    return _check_after_attn(st, orc, v, W, h_in, gemm_check)
+
+
+def _check_after_attn(st, orc, v, W, h_in, gemm_check):
     # h += O Wo^T
     gemm_check(4, W["o"], st.H, st.nq, v["attn"], v["hmid"], base=h_in.astype(np.float64))
     # x2, gate|up
@@ -178,6 +227,20 @@ def test_step_teacher_forced_small_stack(q, orc, n_rows, lens):
     h = orc.bf16_array_to_f64(st.X).astype(np.float32)
     for l in range(st.L):
         h = check_layer(st, orc, dbg, l, h, kc[l], vc[l])
+    assert np.array_equal(h, st.Hd.cpu().numpy())
+    assert q.device_status() == 0
+
+
+@pytest.mark.parametrize("n_rows,lens", [([3, 1, 2], [40, 0, 7]), ([3, 3, 3, 3], [5, 17, 33, 2]),
+                                         ([0, 2, 3], [9, 0, 130])])
+def test_step_q8_0_cache_teacher_forced(q, orc, n_rows, lens):
+    """The same step over q8_0 caches: appended codes bit-exact, attention within
+    the attention tolerance of the oracle over the GPU's caches."""
+    st = Stack(q, 2, 512, 1024, 8, 2, n_rows, lens, seed=20 + len(n_rows), kv="q8_0", orc=orc)
+    dbg = st.run()
+    h = orc.bf16_array_to_f64(st.X).astype(np.float32)
+    for l in range(st.L):
+        h = check_layer(st, orc, dbg, l, h, None, None, q8=st.planes(l))
     assert np.array_equal(h, st.Hd.cpu().numpy())
     assert q.device_status() == 0
 
