@@ -34,6 +34,7 @@ constexpr int ATT_WARPS = 4;
 constexpr int ATT_STAGES_LONG = 3;   // per-warp ring for long caches (two CTAs per SM)
 constexpr int ATT_STAGES_SHORT = 6;  // short caches: a split's cached tiles all in flight at once
 constexpr int TILE_BYTES = KT * 128 * 2;  // 4 KB (K) ; V follows
+constexpr float M_SLACK = 8.f;            // scores may pass the reference maximum by 2^8
 constexpr int PART_FLOATS = ATT_PART_FLOATS;
 
 struct AttnArgs {
@@ -106,9 +107,24 @@ __global__ void __launch_bounds__(128, 2) k_decode_attn(AttnArgs p)
     uint8_t *wbuf = smem + (size_t)w * STAGES * 2 * TILE_BYTES;
 
     const int nq = p.n_qh * 128, nkv = p.n_kvh * 128;
-    auto issue = [&](int it) {
+    // per-lane constants of a full tile's copies: chunk (lane & 15) of keys lane/16 + 2i
+    // (i = 0..7); keys 8 apart share the swizzle, so 4 offsets cover the 8 rows
+    int cp_dst[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        cp_dst[i] = swz((lane >> 4) + 2 * i, lane & 15);
+    const int cp_src = (lane >> 4) * 128 + (lane & 15) * 8;  // elements
+    auto issue = [&](int it, uint8_t *st) {
         const int kb = kbeg + KT * (w + ATT_WARPS * it);
-        uint8_t *st = wbuf + (size_t)(it % STAGES) * 2 * TILE_BYTES;
+        if (!(FUSED && kb + KT > len) && kb + KT <= kend) {  // a full tile of cached keys
+            const uint16_t *ks = Kh + (size_t)kb * 128 + cp_src, *vs = Vh + (size_t)kb * 128 + cp_src;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                cp_async16(st + cp_dst[i & 3] + (i >> 2) * 2048, ks + 256 * i);
+                cp_async16(st + TILE_BYTES + cp_dst[i & 3] + (i >> 2) * 2048, vs + 256 * i);
+            }
+            return;
+        }
         if (FUSED && kb + KT > len) {
             // tile reaches the new positions: cached keys below len, new rows from the projection
 #pragma unroll 1
@@ -151,9 +167,10 @@ __global__ void __launch_bounds__(128, 2) k_decode_attn(AttnArgs p)
     };
     // tiles of cached keys only (always the earlier ones) stream before the wait
     auto cached_tile = [&](int it) { return !FUSED || kbeg + KT * (w + ATT_WARPS * it) + KT <= len; };
+    auto stage = [&](int i) { return wbuf + (size_t)i * 2 * TILE_BYTES; };
     int pre = 0;
     while (pre < STAGES - 1 && pre < my && cached_tile(pre)) {
-        issue(pre);
+        issue(pre, stage(pre));
         cp_async_commit();
         ++pre;
     }
@@ -161,7 +178,7 @@ __global__ void __launch_bounds__(128, 2) k_decode_attn(AttnArgs p)
     trace_ready(p.trace);
     for (int it = pre; it < STAGES - 1; ++it) {
         if (it < my)
-            issue(it);
+            issue(it, stage(it));
         cp_async_commit();
     }
 
@@ -198,13 +215,16 @@ __global__ void __launch_bounds__(128, 2) k_decode_attn(AttnArgs p)
     }
 
 
+    int cur = 0, nxt = STAGES - 1;  // ring slots of tile it and of tile it + STAGES - 1
     for (int it = 0; it < my; ++it) {
         if (it + STAGES - 1 < my)
-            issue(it + STAGES - 1);
+            issue(it + STAGES - 1, stage(nxt));
+        nxt = nxt + 1 == STAGES ? 0 : nxt + 1;
         cp_async_commit();
         cp_async_wait<STAGES - 1>();
         __syncwarp();
-        const uint8_t *Ks = wbuf + (size_t)(it % STAGES) * 2 * TILE_BYTES;
+        const uint8_t *Ks = stage(cur);
+        cur = cur + 1 == STAGES ? 0 : cur + 1;
         const uint8_t *Vs = Ks + TILE_BYTES;
         const int kb = kbeg + KT * (w + ATT_WARPS * it);
 
@@ -223,39 +243,57 @@ __global__ void __launch_bounds__(128, 2) k_decode_attn(AttnArgs p)
             for (int nt = 0; nt < 3; ++nt)
                 mma_bf16(s[nt], a0, a1, a2, a3, qf[nt][ks][0], qf[nt][ks][1]);
         }
-        // online softmax per query column (keys gq and gq+8 of this lane)
+        // Online softmax against a reference maximum m per query column that moves only
+        // when a score passes it by more than M_SLACK (log2 units), so most tiles need no
+        // cross-lane reduction and no rescale (P <= 2^8, far inside bf16's range; the
+        // reference cancels in every merge). Masks only on tiles past the cached keys.
+        const bool interior = kb + KT <= kend && kb + KT <= len;
+        float v[3][4];
+        bool over = false;
+#pragma unroll
+        for (int nt = 0; nt < 3; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                float v0 = s[nt][e] * p.scale_log2, v1 = s[nt][e + 2] * p.scale_log2;
+                if (!interior) {
+                    const int k0 = kb + gq, k1 = kb + gq + 8;
+                    v0 = (k0 < kend && k0 <= qpos[nt][e]) ? v0 : -INFINITY;
+                    v1 = (k1 < kend && k1 <= qpos[nt][e]) ? v1 : -INFINITY;
+                }
+                over |= fmaxf(v0, v1) > m[nt][e] + M_SLACK;
+                v[nt][e] = v0;
+                v[nt][e + 2] = v1;
+            }
+        if (__any_sync(0xffffffffu, over)) {
+#pragma unroll
+            for (int nt = 0; nt < 3; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    float mx = fmaxf(v[nt][e], v[nt][e + 2]);
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+                    const float mn = fmaxf(m[nt][e], mx);
+                    const float corr = mn == -INFINITY ? 1.f : ex2_approx(m[nt][e] - mn);
+                    m[nt][e] = mn;
+                    l[nt][e] *= corr;
+#pragma unroll
+                    for (int dt = 0; dt < 8; ++dt) {
+                        o[dt][nt][e] *= corr;
+                        o[dt][nt][e + 2] *= corr;
+                    }
+                }
+        }
         uint32_t bh[3][2], bl[3][2];
 #pragma unroll
         for (int nt = 0; nt < 3; ++nt) {
             float pv[4];
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-                const int k0 = kb + gq, k1 = kb + gq + 8;
-                const float v0 = (k0 < kend && k0 <= qpos[nt][e]) ? s[nt][e] * p.scale_log2 : -INFINITY;
-                const float v1 = (k1 < kend && k1 <= qpos[nt][e]) ? s[nt][e + 2] * p.scale_log2 : -INFINITY;
-                float mx = fmaxf(v0, v1);
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-                const float mn = fmaxf(m[nt][e], mx);
-                float corr, p0, p1;
-                if (mn == -INFINITY) {
-                    corr = 1.f;
-                    p0 = p1 = 0.f;
-                } else {
-                    corr = exp2f(m[nt][e] - mn);
-                    p0 = exp2f(v0 - mn);
-                    p1 = exp2f(v1 - mn);
-                }
-                m[nt][e] = mn;
-                l[nt][e] = l[nt][e] * corr + p0 + p1;
-                pv[e] = p0;
-                pv[e + 2] = p1;
-#pragma unroll
-                for (int dt = 0; dt < 8; ++dt) {
-                    o[dt][nt][e] *= corr;
-                    o[dt][nt][e + 2] *= corr;
-                }
+                const bool none = m[nt][e] == -INFINITY;
+                pv[e] = none ? 0.f : ex2_approx(v[nt][e] - m[nt][e]);
+                pv[e + 2] = none ? 0.f : ex2_approx(v[nt][e + 2] - m[nt][e]);
+                l[nt][e] += pv[e] + pv[e + 2];
             }
             // P^T fragment (keys x queries) via an in-register transpose, as bf16 hi + lo
             const uint32_t h0 = pack_bf162(pv[0], pv[1]), h1 = pack_bf162(pv[2], pv[3]);

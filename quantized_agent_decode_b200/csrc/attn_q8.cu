@@ -23,9 +23,9 @@
 // permuted so that each lane reads its codes with 8- and 16-byte shared-memory
 // loads (the sum over k and the choice of MMA rows are order-free); the
 // partial records use the natural order.
-// The rescale of the running output by the softmax correction is skipped when
-// no query column's maximum grew (the correction is then exactly 1), and the
-// causal/tail masks run only on tiles that reach past the cached length.
+// The cross-lane reduction of a tile's maximum and the rescale of the running
+// output run only when some score passes the running maximum, and the
+// causal/tail masks only on tiles that reach past the cached length.
 #include "attn.cuh"
 
 namespace qad {
@@ -40,7 +40,7 @@ constexpr int SCB = KT * 8;                  // fp16 scales of one tile (128 B)
 constexpr int STAGE = 2 * TILE + 2 * SCB;    // K codes | V codes | K scales | V scales
 constexpr int STAGES_SHORT = 6;
 constexpr int STAGES_LONG = 5;
-constexpr float P_LOG2_SCALE = 15.f;         // probabilities enter the PV product as fp16 P * 2^15
+constexpr float P_LOG2_SCALE = 15.f;         // P enters the PV product as fp16 2^(v - m + 15) <= 2^15
 
 struct Q8Args {
     const uint16_t *Q;          // standalone: bf16 Q [M][n_qh][128]
@@ -142,10 +142,27 @@ __global__ void __launch_bounds__(128, 2) k_decode_attn_q8(Q8Args p)
     uint8_t *wbuf = smem + (size_t)w * STAGES * STAGE;
     const int nq = p.n_qh * 128, nkv = p.n_kvh * 128;
 
-    auto issue = [&](int it) {
+    // per-lane constants of the copies: chunk (lane & 7) of keys lane/8 + 4i (i = 0..3)
+    const int cp_src = (lane >> 3) * 128 + (lane & 7) * 16;
+    const int cp_dst0 = q8sw(lane >> 3, lane & 7), cp_dst1 = q8sw((lane >> 3) + 4, lane & 7);
+    const int sc_dst = 2 * TILE + (lane >> 4) * SCB + (lane & 15) * 8;
+    const uint16_t *sc_src = (lane < 16 ? Kdh : Vdh) + (lane & 15) * 4;
+    auto issue = [&](int it, uint8_t *st) {
         const int kb = kbeg + KT * (w + NW * it);
-        uint8_t *st = wbuf + (size_t)(it % STAGES) * STAGE;
         const bool mixed = FUSED && kb + KT > len;  // the tile holds new positions (taken from the projection)
+        if (!mixed && kb + KT <= kend) {            // a full tile of cached keys
+            const int8_t *ks = Kh + (size_t)kb * 128 + cp_src, *vs = Vh + (size_t)kb * 128 + cp_src;
+            cp_async16(st + cp_dst0, ks);
+            cp_async16(st + cp_dst1, ks + 512);
+            cp_async16(st + cp_dst0 + 1024, ks + 1024);
+            cp_async16(st + cp_dst1 + 1024, ks + 1536);
+            cp_async16(st + TILE + cp_dst0, vs);
+            cp_async16(st + TILE + cp_dst1, vs + 512);
+            cp_async16(st + TILE + cp_dst0 + 1024, vs + 1024);
+            cp_async16(st + TILE + cp_dst1 + 1024, vs + 1536);
+            cp_async8_zfill(st + sc_dst, sc_src + (size_t)kb * 4, true);
+            return;
+        }
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int idx = lane + 32 * i, kk = idx >> 3, j = idx & 7, kp = kb + kk;
@@ -167,8 +184,7 @@ __global__ void __launch_bounds__(128, 2) k_decode_attn_q8(Q8Args p)
                     cp_async8_zfill(st + 2 * TILE + SCB + kk * 8, Vdh + src, ok);
             }
         }
-        if constexpr (!FUSED)
-            return;
+        if constexpr (FUSED) {
         if (!mixed)
             return;
         // new positions: quantise the fp32 k, v rows; the row-group-0 CTA also
@@ -216,11 +232,13 @@ __global__ void __launch_bounds__(128, 2) k_decode_attn_q8(Q8Args p)
                 }
             }
         }
+        }
     };
     auto cached_tile = [&](int it) { return !FUSED || kbeg + KT * (w + NW * it) + KT <= len; };
+    auto stage = [&](int i) { return wbuf + (size_t)i * STAGE; };
     int pre = 0;
     while (pre < STAGES - 1 && pre < my && cached_tile(pre)) {
-        issue(pre);
+        issue(pre, stage(pre));
         cp_async_commit();
         ++pre;
     }
@@ -228,7 +246,7 @@ __global__ void __launch_bounds__(128, 2) k_decode_attn_q8(Q8Args p)
     trace_ready(p.trace);
     for (int it = pre; it < STAGES - 1; ++it) {
         if (it < my)
-            issue(it);
+            issue(it, stage(it));
         cp_async_commit();
     }
 
@@ -275,13 +293,23 @@ __global__ void __launch_bounds__(128, 2) k_decode_attn_q8(Q8Args p)
         }
     }
 
+    // per-lane shared-memory offsets of the fragment loads (see q8sw)
+    int offK[4];
+#pragma unroll
+    for (int b = 0; b < 4; ++b)
+        offK[b] = q8sw(gq, 2 * b + (c >> 1)) + (c & 1) * 8;
+    const int offV0 = TILE + q8sw(2 * c, gq), offV1 = TILE + q8sw(2 * c + 1, gq);
+    const int offVd = 2 * TILE + SCB + 2 * c * 8 + (gq >> 1) * 2;
+    int cur = 0, nxt = STAGES - 1;  // ring slots of tile it and of tile it + STAGES - 1
     for (int it = 0; it < my; ++it) {
         if (it + STAGES - 1 < my)
-            issue(it + STAGES - 1);
+            issue(it + STAGES - 1, stage(nxt));
+        nxt = nxt + 1 == STAGES ? 0 : nxt + 1;
         cp_async_commit();
         cp_async_wait<STAGES - 1>();
         __syncwarp();
-        const uint8_t *st = wbuf + (size_t)(it % STAGES) * STAGE;
+        const uint8_t *st = stage(cur);
+        cur = cur + 1 == STAGES ? 0 : cur + 1;
         const int kb = kbeg + KT * (w + NW * it);
 
         // S^T = K Q^T, one MMA pair per 32-value block, scaled per key and block
@@ -291,8 +319,7 @@ __global__ void __launch_bounds__(128, 2) k_decode_attn_q8(Q8Args p)
         float s[3][4];
 #pragma unroll
         for (int b = 0; b < 4; ++b) {
-            const int off = q8sw(gq, 2 * b + (c >> 1)) + (c & 1) * 8;
-            const uint2 x0 = lds_v2(st + off), x1 = lds_v2(st + off + 8 * 128);
+            const uint2 x0 = lds_v2(st + offK[b]), x1 = lds_v2(st + offK[b] + 8 * 128);
             const uint32_t u00 = x0.x ^ 0x80808080u, u01 = x0.y ^ 0x80808080u;
             const uint32_t u10 = x1.x ^ 0x80808080u, u11 = x1.y ^ 0x80808080u;
             const uint32_t A0[4] = {hsub2(prmt(u00, 0x64646464u, 0x4140u), H2_1152), hsub2(prmt(u10, 0x64646464u, 0x4140u), H2_1152),
@@ -318,10 +345,14 @@ __global__ void __launch_bounds__(128, 2) k_decode_attn_q8(Q8Args p)
             }
         }
 
-        // online softmax; masks only where the tile reaches past the cached keys
+        // Online softmax: the cross-lane reduction of the tile maximum and the rescale
+        // run only when some score passes the running maximum m (once m is established,
+        // most tiles skip both). P enters the MMA as fp16 2^(v - m + 15) <= 2^15; fp16
+        // keeps 11 bits down to 2^-29 of the maximum, and the common factor cancels in
+        // every merge. Masks run only on tiles that reach past the cached keys.
         const bool interior = kb + KT <= kend && kb + KT <= len;
-        float v[3][4], mn[3][2];
-        bool grow = false;
+        float v[3][4];
+        bool over = false;
 #pragma unroll
         for (int nt = 0; nt < 3; ++nt)
 #pragma unroll
@@ -332,22 +363,22 @@ __global__ void __launch_bounds__(128, 2) k_decode_attn_q8(Q8Args p)
                     v0 = (k0 < kend && k0 <= qpos[nt][e]) ? v0 : -INFINITY;
                     v1 = (k1 < kend && k1 <= qpos[nt][e]) ? v1 : -INFINITY;
                 }
-                float mx = fmaxf(v0, v1);
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-                mn[nt][e] = fmaxf(m[nt][e], mx);
-                grow |= mn[nt][e] > m[nt][e];
+                over |= fmaxf(v0, v1) > m[nt][e];
                 v[nt][e] = v0;
                 v[nt][e + 2] = v1;
             }
-        if (__any_sync(0xffffffffu, grow)) {
+        if (__any_sync(0xffffffffu, over)) {
 #pragma unroll
             for (int nt = 0; nt < 3; ++nt)
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
-                    const float corr = mn[nt][e] == -INFINITY ? 1.f : exp2f(m[nt][e] - mn[nt][e]);
-                    m[nt][e] = mn[nt][e];
+                    float mx = fmaxf(v[nt][e], v[nt][e + 2]);
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+                    const float mn = fmaxf(m[nt][e], mx);
+                    const float corr = mn == -INFINITY ? 1.f : ex2_approx(m[nt][e] - mn);
+                    m[nt][e] = mn;
                     l[nt][e] *= corr;
 #pragma unroll
                     for (int dt = 0; dt < 8; ++dt) {
@@ -362,12 +393,10 @@ __global__ void __launch_bounds__(128, 2) k_decode_attn_q8(Q8Args p)
             float pv[4];
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-                // P * 2^15: the largest is 32768, and fp16 keeps 11 bits down to 2^-29 before
-                // the scale (the factor is common to o and l and cancels in every merge)
                 const bool none = m[nt][e] == -INFINITY;
                 const float mb = m[nt][e] - P_LOG2_SCALE;
-                pv[e] = none ? 0.f : exp2f(v[nt][e] - mb);
-                pv[e + 2] = none ? 0.f : exp2f(v[nt][e + 2] - mb);
+                pv[e] = none ? 0.f : ex2_approx(v[nt][e] - mb);
+                pv[e + 2] = none ? 0.f : ex2_approx(v[nt][e + 2] - mb);
                 l[nt][e] += pv[e] + pv[e + 2];
             }
             // P^T fragment (keys x queries) via an in-register transpose, fp16
@@ -377,14 +406,14 @@ __global__ void __launch_bounds__(128, 2) k_decode_attn_q8(Q8Args p)
 
         // O^T += V^T P^T. M-tile dt, row gq is output dimension 16 gq + 2 dt,
         // row gq + 8 is 16 gq + 2 dt + 1; K = keys 2c, 2c+1, 2c+8, 2c+9 (natural).
-        const uint8_t *Vs = st + TILE, *Vsc = st + 2 * TILE + SCB;
-        const uint4 R0 = lds_v4(Vs + q8sw(2 * c, gq)), R1 = lds_v4(Vs + q8sw(2 * c + 1, gq));
-        const uint4 R2 = lds_v4(Vs + q8sw(2 * c + 8, gq)), R3 = lds_v4(Vs + q8sw(2 * c + 9, gq));
-        const int sb = (gq >> 1) * 2;  // this lane's 16 dimensions lie in block gq / 2
-        const uint32_t d01 = (uint32_t)*reinterpret_cast<const uint16_t *>(Vsc + (2 * c) * 8 + sb) |
-                             (uint32_t)*reinterpret_cast<const uint16_t *>(Vsc + (2 * c + 1) * 8 + sb) << 16;
-        const uint32_t d89 = (uint32_t)*reinterpret_cast<const uint16_t *>(Vsc + (2 * c + 8) * 8 + sb) |
-                             (uint32_t)*reinterpret_cast<const uint16_t *>(Vsc + (2 * c + 9) * 8 + sb) << 16;
+        // keys 2c+8, 2c+9 sit 1024 bytes after keys 2c, 2c+1 (same swizzle); this lane's 16
+        // dimensions lie in block gq / 2, whose scales are 2 bytes at offVd in each key's 8
+        const uint4 R0 = lds_v4(st + offV0), R1 = lds_v4(st + offV1);
+        const uint4 R2 = lds_v4(st + offV0 + 1024), R3 = lds_v4(st + offV1 + 1024);
+        const uint32_t d01 = (uint32_t)*reinterpret_cast<const uint16_t *>(st + offVd) |
+                             (uint32_t)*reinterpret_cast<const uint16_t *>(st + offVd + 8) << 16;
+        const uint32_t d89 = (uint32_t)*reinterpret_cast<const uint16_t *>(st + offVd + 64) |
+                             (uint32_t)*reinterpret_cast<const uint16_t *>(st + offVd + 72) << 16;
         const uint32_t W0[4] = {R0.x, R0.y, R0.z, R0.w}, W1[4] = {R1.x, R1.y, R1.z, R1.w};
         const uint32_t W2[4] = {R2.x, R2.y, R2.z, R2.w}, W3[4] = {R3.x, R3.y, R3.z, R3.w};
 #pragma unroll

@@ -158,6 +158,15 @@ __device__ __forceinline__ float half_hi(uint32_t v) { return __half2float(__ush
 __device__ __forceinline__ float bf16_to_f(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
 __device__ __forceinline__ uint16_t f_to_bf16(float f) { return __bfloat16_as_ushort(__float2bfloat16_rn(f)); }
 
+// 2^x by the SFU instruction (ex2.approx.ftz: relative error ~2^-22, results
+// below 2^-126 flush to zero, 2^-inf = 0).
+__device__ __forceinline__ float ex2_approx(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // fp16x2 constants (both halves equal)
 constexpr uint32_t H2_1024 = 0x64006400u;   // 1024.0
 constexpr uint32_t H2_NEG1024 = 0xE400E400u;// -1024.0
