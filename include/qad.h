@@ -353,6 +353,33 @@ int qad_step_graph_create(qad_model *model, const uint16_t *X, int M, const int 
 int qad_step_graph_launch(qad_step_graph *g, void *stream);
 void qad_step_graph_destroy(qad_step_graph *g);
 
+/* ---------------------------------------------------------------- mixed step (chunked prefill)
+ * OpenJet page, section 真正重要的是少互相堵车: a long prompt is fed in chunks
+ * so the other agents keep decoding. One mixed step runs the decode batch (M
+ * rows, exactly as qad_decode_step) together with C prompt rows of one more
+ * agent (chunk_agent, positions chunk_len .. chunk_len + C - 1 of its cache),
+ * all R = M + C rows through the dense tensor-core GEMMs of the layer
+ * definition above. The decode rows attend as in qad_decode_step; chunk row j
+ * attends causally to keys 0 .. chunk_len + j of its agent (its own k, v are
+ * appended first), i.e. the same definition with C rows.
+ *   X       device bf16 [R][hidden]: the M decode rows (agent-major) then the C
+ *           chunk rows, 16-byte aligned
+ *   agent_row_start, lens  as qad_decode_step (ignored when M == 0); the chunk
+ *           agent must have no decode rows in this step
+ *   H_out   device fp32 [R][hidden], 16-byte aligned
+ *   ws      qad_mixed_step_ws_bytes(model, M, C) bytes, 256-byte aligned
+ * 0 <= M <= 16, C >= 0, M + C >= 1; bf16 KV caches only (the prompt-chunk
+ * attention reads bf16). Precision: the dense GEMM's (fp16 weight tiles) and
+ * the prefill attention's (bf16 probabilities) for every row. Synchronous
+ * with respect to nothing: all launches go to `stream`. With
+ * qad_model_set_debug, a buffer of qad_mixed_step_debug_bytes(model, M, C)
+ * receives the per-layer intermediates in the qad_decode_step layout for R rows. */
+size_t qad_mixed_step_ws_bytes(const qad_model *model, int M, int C);
+size_t qad_mixed_step_debug_bytes(const qad_model *model, int M, int C);
+int qad_mixed_step(qad_model *model, const uint16_t *X, int M, const int *agent_row_start, int n_agents,
+                   int max_rows_per_agent, const int *lens, int chunk_agent, int chunk_len, int C, float *H_out,
+                   void *ws, size_t ws_bytes, void *stream);
+
 /* Number of kernel launches one qad_decode_step issues (for accounting). */
 int qad_decode_step_launches(const qad_model *model);
 

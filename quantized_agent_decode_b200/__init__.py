@@ -77,6 +77,10 @@ SIGNATURES = {
     "qad_pack_rows": (C.c_int, [C.POINTER(AgentRows), C.c_int, C.c_int, C.c_int, C.c_void_p, C.c_void_p,
                                 C.c_void_p, C.c_void_p]),
     "qad_model_create": (C.c_int, [C.POINTER(ModelDesc), C.POINTER(C.c_void_p)]),
+    "qad_mixed_step_ws_bytes": (C.c_size_t, [C.c_void_p, C.c_int, C.c_int]),
+    "qad_mixed_step_debug_bytes": (C.c_size_t, [C.c_void_p, C.c_int, C.c_int]),
+    "qad_mixed_step": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int, C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_int,
+                                 C.c_int, C.c_int, C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p]),
     "qad_model_destroy": (None, [C.c_void_p]),
     "qad_decode_step_ws_bytes": (C.c_size_t, [C.c_void_p, C.c_int]),
     "qad_decode_step": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int, C.c_void_p, C.c_int, C.c_int, C.c_void_p,
@@ -451,6 +455,26 @@ class Model:
         cnt = (C.c_longlong * n)()
         _check(lib().qad_model_profile_read(self.handle, ms, cnt, n), "qad_model_profile_read")
         return {k: (ms[i], cnt[i]) for i, k in enumerate(PROFILE_KINDS)}
+
+    def mixed_ws_bytes(self, M: int, C: int) -> int:
+        return int(lib().qad_mixed_step_ws_bytes(self.handle, M, C))
+
+    def set_debug_mixed(self, M: int, C: int):
+        """Attach a per-layer intermediates buffer sized for a mixed step of M + C rows."""
+        n = int(lib().qad_mixed_step_debug_bytes(self.handle, M, C))
+        self._dbg = alloc_ws(n)
+        _check(lib().qad_model_set_debug(self.handle, _dev(self._dbg, "dbg"), n), "qad_model_set_debug")
+        return self._dbg
+
+    def mixed_step(self, X, M, agent_row_start, n_agents, max_rows_per_agent, lens, chunk_agent, chunk_len, C, H_out,
+                   ws, stream=None):
+        """Decode rows (M) plus a C-row prompt chunk of chunk_agent at positions chunk_len.. (X: decode rows first)."""
+        ptr = lambda t, n: _dev(t, n) if t is not None else None  # noqa: E731
+        _check(lib().qad_mixed_step(self.handle, _dev(X, "X"), M, ptr(agent_row_start, "agent_row_start"), n_agents,
+                                    max_rows_per_agent, ptr(lens, "lens"), chunk_agent, chunk_len, C,
+                                    _dev(H_out, "H_out"), _dev(ws, "ws"), ws.numel() * ws.element_size(),
+                                    _stream(stream)), "qad_mixed_step")
+        return H_out
 
     def decode_step(self, X, M, agent_row_start, n_agents, max_rows_per_agent, lens, H_out, ws, stream=None):
         _check(lib().qad_decode_step(self.handle, _dev(X, "X"), M, _dev(agent_row_start, "agent_row_start"),

@@ -167,6 +167,17 @@ __device__ __forceinline__ float ex2_approx(float x)
     return y;
 }
 
+// silu(g) * u in fp32; below g = -80, 1 + e^-g equals e^-g in fp32 and e^-g
+// would overflow past -88, so the product g*u*e^g is formed in the log domain
+// (an exact zero stays zero).
+__device__ __forceinline__ float silu_mul(float g, float u)
+{
+    if (g >= -80.f)
+        return g / (1.f + expf(-g)) * u;
+    const float p = g * u;
+    return p == 0.f ? p : copysignf(expf(g + logf(fabsf(p))), p);
+}
+
 // fp16x2 constants (both halves equal)
 constexpr uint32_t H2_1024 = 0x64006400u;   // 1024.0
 constexpr uint32_t H2_NEG1024 = 0xE400E400u;// -1024.0

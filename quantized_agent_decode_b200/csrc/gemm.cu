@@ -127,16 +127,6 @@ __device__ __forceinline__ float warp_max(float v)
 }
 __device__ __forceinline__ float round_half(float v) { return __half2float(__float2half_rn(v)); }
 
-// silu(g) * u in fp32; below g = -80, 1 + e^-g equals e^-g in fp32 and e^-g
-// would overflow past -88, so the product g*u*e^g is formed in the log domain
-// (an exact zero stays zero).
-__device__ __forceinline__ float silu_mul(float g, float u)
-{
-    if (g >= -80.f)
-        return g / (1.f + expf(-g)) * u;
-    const float p = g * u;
-    return p == 0.f ? p : copysignf(expf(g + logf(fabsf(p))), p);
-}
 
 // Zero the next GEMM's output (its atomics accumulate into it); this CTA's share.
 __device__ __forceinline__ void zero_next_output(const PrepSrc &S)

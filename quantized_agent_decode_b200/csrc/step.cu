@@ -25,6 +25,7 @@
 #include <vector>
 
 #include "attn.cuh"
+#include "dense.cuh"
 #include "gemm.cuh"
 
 struct qad_step_graph {
@@ -301,6 +302,200 @@ static int run_step(qad_model *m, const uint16_t *X, int M, const int *ars, int 
     return QAD_OK;
 }
 
+// ------------------------------------------------------------- mixed step: decode rows + one prompt chunk
+//
+// [OpenJet page], section 真正重要的是少互相堵车: a long prompt must not stall the
+// other agents. A mixed step carries the decode batch (M rows, as above) and C
+// prompt rows of one more agent, all R = M + C rows through the dense (tcgen05)
+// GEMMs; the decode rows attend with the split-KV kernel, the chunk with the
+// causal prefill kernel. Per layer: rmsnorm -> qkv -> attention (decode rows
+// append their k, v; the chunk's k, v are appended first) -> o -> residual +
+// rmsnorm -> gate|up -> silu*up -> down -> residual.
+
+// h += Y (when Y is given), then X = bf16(h / sqrt(mean(h^2) + eps)); one CTA per row.
+__global__ void __launch_bounds__(256) k_rows_rmsnorm(float *__restrict__ h, const float *__restrict__ Y,
+                                                      uint16_t *__restrict__ X, int H, float eps)
+{
+    __shared__ float red[8];
+    const int r = blockIdx.x, tid = threadIdx.x;
+    float *hr = h + (size_t)r * H;
+    float ss = 0.f;
+    for (int i = 4 * tid; i < H; i += 1024) {
+        float4 v = *reinterpret_cast<float4 *>(hr + i);
+        if (Y) {
+            const float4 y = *reinterpret_cast<const float4 *>(Y + (size_t)r * H + i);
+            v.x += y.x, v.y += y.y, v.z += y.z, v.w += y.w;
+            *reinterpret_cast<float4 *>(hr + i) = v;
+        }
+        ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1)
+        ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if ((tid & 31) == 0)
+        red[tid >> 5] = ss;
+    __syncthreads();
+    ss = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w)
+        ss += red[w];
+    const float inv = 1.f / sqrtf(ss / (float)H + eps);
+    for (int i = 4 * tid; i < H; i += 1024) {
+        const float4 v = *reinterpret_cast<const float4 *>(hr + i);
+        *reinterpret_cast<uint2 *>(X + (size_t)r * H + i) =
+            make_uint2(pack_bf162(v.x * inv, v.y * inv), pack_bf162(v.z * inv, v.w * inv));
+    }
+}
+
+// act = bf16(silu(gate) * up) from gate|up fp32 [R][2I]; one CTA per row.
+__global__ void __launch_bounds__(256) k_rows_silu(const float *__restrict__ gu, uint16_t *__restrict__ act, int I)
+{
+    const int r = blockIdx.x;
+    const float *g = gu + (size_t)r * 2 * I, *u = g + I;
+    for (int i = 2 * threadIdx.x; i < I; i += 512) {
+        const float2 gv = *reinterpret_cast<const float2 *>(g + i), uv = *reinterpret_cast<const float2 *>(u + i);
+        *reinterpret_cast<uint32_t *>(act + (size_t)r * I + i) = pack_bf162(silu_mul(gv.x, uv.x), silu_mul(gv.y, uv.y));
+    }
+}
+
+// h += Y over n floats.
+__global__ void k_rows_add(float *__restrict__ h, const float *__restrict__ Y, long long n)
+{
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n / 4; i += (long long)gridDim.x * blockDim.x) {
+        float4 v = reinterpret_cast<float4 *>(h)[i];
+        const float4 y = reinterpret_cast<const float4 *>(Y)[i];
+        v.x += y.x, v.y += y.y, v.z += y.z, v.w += y.w;
+        reinterpret_cast<float4 *>(h)[i] = v;
+    }
+}
+
+// Chunk row j (projection row M + j): Q = bf16(q) into Qc [C][nq]; k, v as bf16
+// into the agent's caches (Kc, Vc point at its [n_kvh][cap][128] slice) at pos0 + j.
+__global__ void __launch_bounds__(256) k_chunk_qkv(const float *__restrict__ qkv, int ldqkv, int M, int nq, int n_kvh,
+                                                   uint16_t *__restrict__ Qc, uint16_t *__restrict__ Kc,
+                                                   uint16_t *__restrict__ Vc, int cap, int pos0)
+{
+    const int j = blockIdx.x, nkv = n_kvh * 128;
+    const float *row = qkv + (size_t)(M + j) * ldqkv;
+    for (int i = 2 * threadIdx.x; i < nq; i += 512)
+        *reinterpret_cast<uint32_t *>(Qc + (size_t)j * nq + i) = pack_bf162(row[i], row[i + 1]);
+    for (int i = 2 * threadIdx.x; i < nkv; i += 512) {
+        const int g = i >> 7, dd = i & 127;
+        const size_t dst = ((size_t)g * cap + pos0 + j) * 128 + dd;
+        *reinterpret_cast<uint32_t *>(Kc + dst) = pack_bf162(row[nq + i], row[nq + i + 1]);
+        *reinterpret_cast<uint32_t *>(Vc + dst) = pack_bf162(row[nq + nkv + i], row[nq + nkv + i + 1]);
+    }
+}
+
+struct MixedLayout {
+    size_t x, qkv, y, qc, part, dense, total;
+};
+
+static MixedLayout mixed_layout(const qad_model_desc &d, int M, int C)
+{
+    MixedLayout L;
+    const int R = M + C, nq = d.n_qh * d.head_dim, nqkv = (d.n_qh + 2 * d.n_kvh) * d.head_dim;
+    const int xw = d.hidden > nq ? (d.hidden > d.inter ? d.hidden : d.inter) : (nq > d.inter ? nq : d.inter);
+    const int yw = d.hidden > 2 * d.inter ? d.hidden : 2 * d.inter;
+    size_t off = 0;
+    L.x = off;  // bf16 activations: x1, attention output, x2, act (each dead after its GEMM's prep)
+    off += a256((size_t)R * xw * 2);
+    L.qkv = off;
+    off += a256((size_t)R * nqkv * 4);
+    L.y = off;  // fp32 GEMM outputs: o, gate|up, down
+    off += a256((size_t)R * yw * 4);
+    L.qc = off;
+    off += a256((size_t)(C > 0 ? C : 1) * nq * 2);
+    L.part = off;
+    off += a256(M > 0 ? max_part_bytes(d, M) : 0);
+    L.dense = off;
+    size_t db = dense_ws_bytes(d.hidden, R);
+    if (dense_ws_bytes(nq, R) > db)
+        db = dense_ws_bytes(nq, R);
+    if (dense_ws_bytes(d.inter, R) > db)
+        db = dense_ws_bytes(d.inter, R);
+    off += a256(db);
+    L.total = off;
+    return L;
+}
+
+static int run_mixed(qad_model *m, const uint16_t *X, int M, const int *ars, int n_agents, int max_rows,
+                     const int *lens, int ca, int clen, int C, float *h, char *ws, cudaStream_t s)
+{
+    const qad_model_desc &d = m->d;
+    const int H = d.hidden, I = d.inter, hd = d.head_dim, R = M + C;
+    const int nq = d.n_qh * hd, nkv = d.n_kvh * hd, nqkv = nq + 2 * nkv;
+    const MixedLayout L = mixed_layout(d, M, C);
+    uint16_t *xb = (uint16_t *)(ws + L.x), *Qc = (uint16_t *)(ws + L.qc);
+    float *qkv = (float *)(ws + L.qkv), *y = (float *)(ws + L.y), *part = (float *)(ws + L.part);
+    void *dws = ws + L.dense;
+    const float scale = 1.0f / sqrtf((float)hd);
+    const DbgLayout DL = dbg_layout(d, R);
+    int rc;
+    auto ok = [](const char *what) { return cuda_check(cudaGetLastError(), what); };
+    k_init_h<<<(R * H + 255) / 256, 256, 0, s>>>(X, h, R * H, nullptr);
+    if ((rc = ok("init launch")))
+        return rc;
+    for (int l = 0; l < d.n_layers; ++l) {
+        char *dbg = m->dbg ? (char *)m->dbg + (size_t)l * DL.per_layer : nullptr;
+        k_rows_rmsnorm<<<R, 256, 0, s>>>(h, nullptr, xb, H, d.rms_eps);
+        if ((rc = ok("rmsnorm launch")))
+            return rc;
+        if (dbg && (rc = copy_d2d(dbg + DL.x1, xb, (size_t)R * H * 2, s)))
+            return rc;
+        if ((rc = launch_dense(4, m->wqkv[l], nqkv, H, xb, R, qkv, dws, s)))
+            return rc;
+        if (dbg && (rc = copy_d2d(dbg + DL.qkv, qkv, (size_t)R * nqkv * 4, s)))
+            return rc;
+        if (M > 0) {  // decode rows: split-KV attention (appends their k, v), splits merged into O rows 0..M-1
+            const AttnPlan plan = attn_plan(n_agents, d.n_qh, d.n_kvh, d.kv_cap, max_rows);
+            if ((rc = launch_attn_fused(plan, qkv, nqkv, m->kc[l], m->vc[l], lens, ars, n_agents, d.kv_cap, d.n_qh,
+                                        d.n_kvh, scale, part, s, false)))
+                return rc;
+            if ((rc = launch_attn_combine(plan, part, lens, ars, n_agents, d.kv_cap, d.n_qh, d.n_kvh, xb, s, false)))
+                return rc;
+        }
+        if (C > 0) {  // the chunk: append its k, v, then causal attention into O rows M..R-1
+            const size_t slice = (size_t)ca * d.n_kvh * d.kv_cap * hd;
+            k_chunk_qkv<<<C, 256, 0, s>>>(qkv, nqkv, M, nq, d.n_kvh, Qc, m->kc[l] + slice, m->vc[l] + slice, d.kv_cap,
+                                          clen);
+            if ((rc = ok("chunk qkv launch")))
+                return rc;
+            if ((rc = launch_prefill_attn(Qc, m->kc[l] + slice, m->vc[l] + slice, clen, C, d.kv_cap, d.n_qh, d.n_kvh,
+                                          scale, xb + (size_t)M * nq, s)))
+                return rc;
+        }
+        if (dbg && (rc = copy_d2d(dbg + DL.attn, xb, (size_t)R * nq * 2, s)))
+            return rc;
+        if ((rc = launch_dense(4, m->wo[l], H, nq, xb, R, y, dws, s)))
+            return rc;
+        k_rows_rmsnorm<<<R, 256, 0, s>>>(h, y, xb, H, d.rms_eps);  // h += o; x2
+        if ((rc = ok("rmsnorm launch")))
+            return rc;
+        if (dbg && (rc = copy_d2d(dbg + DL.hmid, h, (size_t)R * H * 4, s)))
+            return rc;
+        if (dbg && (rc = copy_d2d(dbg + DL.x2, xb, (size_t)R * H * 2, s)))
+            return rc;
+        if ((rc = launch_dense(4, m->wgu[l], 2 * I, H, xb, R, y, dws, s)))
+            return rc;
+        if (dbg && (rc = copy_d2d(dbg + DL.gu, y, (size_t)R * 2 * I * 4, s)))
+            return rc;
+        k_rows_silu<<<R, 256, 0, s>>>(y, xb, I);
+        if ((rc = ok("silu launch")))
+            return rc;
+        if (dbg && (rc = copy_d2d(dbg + DL.act, xb, (size_t)R * I * 2, s)))
+            return rc;
+        if ((rc = launch_dense(6, m->wdown[l], H, I, xb, R, y, dws, s)))
+            return rc;
+        k_rows_add<<<(R * H / 4 + 255) / 256, 256, 0, s>>>(h, y, (long long)R * H);
+        if ((rc = ok("residual launch")))
+            return rc;
+        if (dbg && (rc = copy_d2d(dbg + DL.hout, h, (size_t)R * H * 4, s)))
+            return rc;
+    }
+    return QAD_OK;
+}
+
 static int check_step_args(const qad_model *m, const void *X, int M, const void *ars, int n_agents, int max_rows,
                            const void *lens, const void *H_out, const void *ws, size_t ws_bytes)
 {
@@ -439,6 +634,49 @@ extern "C" int qad_decode_step(qad_model *m, const uint16_t *X, int M, const int
         return qad::fail(QAD_ERR_WORKSPACE, "decode_step: debug buffer too small");
     return qad::run_step(m, X, M, agent_row_start, n_agents, max_rows_per_agent, lens, H_out, (char *)ws,
                          (cudaStream_t)stream);
+}
+
+extern "C" size_t qad_mixed_step_ws_bytes(const qad_model *m, int M, int C)
+{
+    if (!m || M < 0 || C < 0 || M + C <= 0 || M > QAD_MAX_ROWS)
+        return 0;
+    return qad::mixed_layout(m->d, M, C).total;
+}
+
+extern "C" size_t qad_mixed_step_debug_bytes(const qad_model *m, int M, int C)
+{
+    if (!m || M < 0 || C < 0 || M + C <= 0 || M > QAD_MAX_ROWS)
+        return 0;
+    return qad::dbg_layout(m->d, M + C).per_layer * m->d.n_layers;
+}
+
+extern "C" int qad_mixed_step(qad_model *m, const uint16_t *X, int M, const int *agent_row_start, int n_agents,
+                              int max_rows_per_agent, const int *lens, int chunk_agent, int chunk_len, int C,
+                              float *H_out, void *ws, size_t ws_bytes, void *stream)
+{
+    if (!m || !X || !H_out || !ws || M < 0 || C < 0 || M + C <= 0)
+        return qad::fail(QAD_ERR_INVALID, "qad_mixed_step: null pointer or empty step");
+    if (M > 0) {
+        int rc = qad::check_step_args(m, X, M, agent_row_start, n_agents, max_rows_per_agent, lens, H_out, ws,
+                                      ws_bytes);
+        if (rc)
+            return rc;
+    }
+    if (m->d.kv_format != QAD_KV_BF16)
+        return qad::fail(QAD_ERR_UNSUPPORTED, "qad_mixed_step: the prompt chunk needs bf16 KV caches");
+    if (C > 0 && (chunk_agent < 0 || chunk_agent >= m->d.max_agents || chunk_len < 0 ||
+                  (long long)chunk_len + C > m->d.kv_cap))
+        return qad::fail(QAD_ERR_INVALID, "qad_mixed_step: chunk agent %d or positions %d..%lld outside the cache",
+                         chunk_agent, chunk_len, (long long)chunk_len + C - 1);
+    if ((uintptr_t)ws & 255 || (uintptr_t)H_out & 15 || (uintptr_t)X & 15)
+        return qad::fail(QAD_ERR_INVALID, "qad_mixed_step: ws 256-byte, X and H_out 16-byte aligned");
+    if (ws_bytes < qad::mixed_layout(m->d, M, C).total)
+        return qad::fail(QAD_ERR_WORKSPACE, "qad_mixed_step: workspace %zu < %zu bytes", ws_bytes,
+                         qad::mixed_layout(m->d, M, C).total);
+    if (m->dbg && m->dbg_bytes < qad_mixed_step_debug_bytes(m, M, C))
+        return qad::fail(QAD_ERR_WORKSPACE, "qad_mixed_step: debug buffer too small");
+    return qad::run_mixed(m, X, M, agent_row_start, n_agents, max_rows_per_agent, lens, chunk_agent, chunk_len, C,
+                          H_out, (char *)ws, (cudaStream_t)stream);
 }
 
 extern "C" int qad_decode_step_launches(const qad_model *m)

@@ -1,0 +1,101 @@
+"""GPU parity of the mixed step (decode rows + one agent's prompt chunk through
+the dense tensor-core GEMMs) against the fp64 oracle, teacher-forced per layer.
+
+The oracle's layer is the same definition with the chunk agent holding C rows
+at positions chunk_len .. chunk_len + C - 1 (causal, like draft rows).
+Tolerances: dense GEMM 2^-10 * B + 1e-3 * A (fp16 weight tiles, see the dense
+GEMM tests); decode-row attention 2e-3 * sum p|v|, chunk-row attention
+2^-8 * sum p|v| (bf16 probabilities), both plus half a bf16 ulp (2^-8
+relative) of the output; bf16 rounding points equal except for rare one-ulp
+flips at rounding ties.
+"""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from conftest import SEED
+from test_gpu_dense import _bound
+from test_gpu_step import Stack, _bits, bf16_close, dbg_views
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def q():
+    import quantized_agent_decode_b200 as q
+    from quantized_agent_decode_b200 import build
+    build.build()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return q
+
+
+def _dense_check(orc, fmt, W, N, K, Xb, Y_gpu, base=None):
+    Yr, A = orc.gemm(fmt, W, N, K, Xb)
+    B = _bound(orc, fmt, W, N, K, Xb)
+    ref = Yr if base is None else base + Yr
+    slack = 0 if base is None else 8 * 2.0 ** -24 * (np.abs(base) + np.abs(Yr))
+    ratio = np.abs(Y_gpu.astype(np.float64) - ref) / (2.0 ** -10 * B + 1e-3 * A + slack + 1e-30)
+    assert ratio.max() <= 1.0, ratio.max()
+
+
+@pytest.mark.parametrize("n_rows,lens,C", [([3, 2, 0], [40, 7, 17], 70), ([3, 3, 0], [5, 300, 0], 130),
+                                           ([0], [9], 64)])
+def test_mixed_step_teacher_forced(q, orc, n_rows, lens, C):
+    """The chunk agent is the last one (no decode rows), so the GPU's row order
+    (decode rows, then the chunk) is the oracle's agent-major order."""
+    st = Stack(q, 2, 512, 1024, 8, 2, n_rows, lens, seed=40 + C, extra_cap=C + 4)
+    M = st.M
+    ca, clen = st.A - 1, int(lens[-1])
+    R = M + C
+    Xc = synth.bf16_normal_np(SEED, 9000 + C, (C, st.H))
+    Xall = np.concatenate([st.X, Xc]) if M else Xc
+    Xd = torch.from_numpy(Xall.view(np.int16)).view(torch.bfloat16).cuda()
+    Hd = torch.empty(R, st.H, dtype=torch.float32, device="cuda")
+    ws = q.alloc_ws(st.model.mixed_ws_bytes(M, C))
+    dbg = st.model.set_debug_mixed(M, C)
+    st.model.mixed_step(Xd, M, st.arsd if M else None, st.A, max(st.max_rows, 1), st.lensd if M else None, ca, clen,
+                        C, Hd, ws)
+    torch.cuda.synchronize()
+    ars_o = np.concatenate([st.ars[:-1], [R]]).astype(np.int32)  # the chunk agent's rows are the last C
+    h = orc.bf16_array_to_f64(Xall).astype(np.float32)
+    for l in range(st.L):
+        v = dbg_views(dbg, l, R, st.H, st.I, st.nq, st.nqkv)
+        W = st.W[l]
+        kc = _bits(st.d["kc"][l]).reshape(W["kc"].shape)
+        vc = _bits(st.d["vc"][l]).reshape(W["vc"].shape)
+        assert bf16_close(v["x1"], orc.rmsnorm_bf16(h.astype(np.float64)), orc)
+        _dense_check(orc, 4, W["qkv"], st.nqkv, st.H, v["x1"], v["qkv"])
+        kvb = orc.f64_array_to_bf16(v["qkv"][:, st.nq:].astype(np.float64))
+        for r in range(R):
+            a = int(np.searchsorted(ars_o, r, side="right") - 1)
+            pos = st.lens[a] + r - ars_o[a]
+            assert np.array_equal(kc[a, :, pos].reshape(-1), kvb[r, :st.nkv])
+            assert np.array_equal(vc[a, :, pos].reshape(-1), kvb[r, st.nkv:])
+        Qb = orc.f64_array_to_bf16(v["qkv"][:, :st.nq].astype(np.float64)).reshape(R, st.n_qh, 128)
+        O_ref, B = orc.decode_attn(Qb, kc, vc, st.lens, ars_o, st.n_qh, st.n_kvh, 128, st.cap)
+        o = orc.bf16_array_to_f64(v["attn"]).reshape(O_ref.shape)
+        rel = np.where(np.arange(R)[:, None, None] < M, 2e-3, 2.0 ** -8)
+        assert (np.abs(o - O_ref) <= rel * B + np.abs(O_ref) * 2.0 ** -8 + 1e-30).all()
+        _dense_check(orc, 4, W["o"], st.H, st.nq, v["attn"], v["hmid"], base=h.astype(np.float64))
+        assert bf16_close(v["x2"], orc.rmsnorm_bf16(v["hmid"].astype(np.float64)), orc)
+        _dense_check(orc, 4, W["gu"], 2 * st.I, st.H, v["x2"], v["gu"])
+        gu = v["gu"].astype(np.float64)
+        assert bf16_close(v["act"], orc.silu_mul_bf16(gu[:, :st.I], gu[:, st.I:]), orc, frac=5e-3)
+        _dense_check(orc, 6, W["down"], st.H, st.I, v["act"], v["hout"], base=v["hmid"].astype(np.float64))
+        h = v["hout"]
+    assert np.array_equal(h, Hd.cpu().numpy())
+    assert q.dense_status() == 0 and q.device_status() == 0
+
+
+def test_mixed_step_rejects_bad_arguments(q):
+    st = Stack(q, 1, 256, 512, 4, 2, [2, 0], [3, 5], seed=3, extra_cap=8)
+    X = torch.zeros(2 + 8, 256, dtype=torch.bfloat16, device="cuda")
+    H = torch.empty(10, 256, dtype=torch.float32, device="cuda")
+    ws = q.alloc_ws(st.model.mixed_ws_bytes(2, 8))
+    with pytest.raises(q.QadError):  # chunk runs past the cache
+        st.model.mixed_step(X, 2, st.arsd, st.A, 2, st.lensd, 1, st.cap - 4, 8, H, ws)
+    with pytest.raises(q.QadError):  # no such agent
+        st.model.mixed_step(X, 2, st.arsd, st.A, 2, st.lensd, st.A, 0, 8, H, ws)
+    with pytest.raises(q.QadError):  # workspace too small
+        st.model.mixed_step(X, 2, st.arsd, st.A, 2, st.lensd, 1, 5, 8, H, ws[:1024])
