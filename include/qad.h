@@ -380,6 +380,59 @@ int qad_mixed_step(qad_model *model, const uint16_t *X, int M, const int *agent_
                    int max_rows_per_agent, const int *lens, int chunk_agent, int chunk_len, int C, float *H_out,
                    void *ws, size_t ws_bytes, void *stream);
 
+/* ---------------------------------------------------------------- step scheduler (host only)
+ * OpenJet page: the agents' tokens and drafts share one weight stream
+ * (section 只搬一次权重), a long prompt is fed in pieces so it does not stall
+ * the others (section 真正重要的是少互相堵车), and an agent's cached context is
+ * reused by its next request (time to first token). Plain host code, no CUDA.
+ *
+ * Policy: chunk_tokens prompt rows per chunk; in QAD_SCHED_INTERLEAVE mode a
+ * chunk rides along with the decode rows on every (decode_steps_per_chunk+1)-th
+ * step (every step when nobody decodes); QAD_SCHED_PREFILL_FIRST runs a
+ * pending prompt's chunks alone, holding the decoding agents back (the
+ * behaviour without chunked prefill, kept as the comparison). Decode rows:
+ * one per decoding agent, then up to n_draft drafts each, within
+ * max_decode_rows (<= 16); a round-robin start (step mod n_agents) rotates who
+ * goes first when the budget is short. */
+#define QAD_SCHED_INTERLEAVE 0
+#define QAD_SCHED_PREFILL_FIRST 1
+typedef struct {
+    int chunk_tokens;
+    int decode_steps_per_chunk;
+    int max_decode_rows;
+    int n_draft;
+    int mode;
+} qad_sched_policy;
+
+/* One agent's host-side state (caller-owned). */
+typedef struct {
+    int len;          /* tokens in its KV cache */
+    int prompt_left;  /* prompt tokens still to prefill (0: decoding) */
+    int active;       /* 0: paused (e.g. waiting on a tool call) */
+    int drafts;       /* draft tokens ready for its next decode step */
+} qad_sched_agent;
+
+/* Plan step number `step`: decode_rows[a] (host int [n_agents]) rows per
+ * agent, the chunk's agent (-1: none) and row count. Returns M (the decode
+ * rows) or a negative QAD_ERR_* code. */
+int qad_sched_plan(const qad_sched_policy *policy, const qad_sched_agent *agents, int n_agents, long long step,
+                   int *decode_rows, int *chunk_agent, int *chunk_rows);
+/* Apply a planned step: a decoding agent with k accepted drafts (n_accept,
+ * host int [n_agents] or NULL for none; clamped to its rows - 1) grows by
+ * k + 1 and its drafts are spent; the chunk's agent grows by the chunk and its
+ * prompt_left shrinks by it. Returns 0 or QAD_ERR_INVALID for a plan that does
+ * not fit the states. */
+int qad_sched_commit(qad_sched_agent *agents, int n_agents, const int *decode_rows, int chunk_agent,
+                     int chunk_rows, const int *n_accept);
+/* Prompt-lookup drafting: for n = max_ngram down to min_ngram, find the latest
+ * earlier occurrence of the last n tokens of tokens[0..n_tokens) (one that is
+ * followed by at least one token) and copy up to n_draft of the tokens that
+ * followed it into drafts. Returns the number written (0 if no n-gram recurs). */
+int qad_prompt_lookup(const int *tokens, int n_tokens, int min_ngram, int max_ngram, int n_draft, int *drafts);
+/* Length of the common prefix of two token sequences: how much of an agent's
+ * cached context a new request can keep (set len to it; the rest is prompt). */
+int qad_common_prefix(const int *a, int na, const int *b, int nb);
+
 /* Number of kernel launches one qad_decode_step issues (for accounting). */
 int qad_decode_step_launches(const qad_model *model);
 

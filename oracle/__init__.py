@@ -300,3 +300,20 @@ def decode_layer(Wqkv, Wo, Wgu, Wdown, H, I, n_qh, n_kvh, hd, h, ars, lens, Kc, 
         lib().orc_decode_layer(*W, *common, Kc.reshape(-1), Vc.reshape(-1), cap, nthreads or max_threads(),
                                *ptrs)
     return inter
+
+
+def prompt_lookup(tokens, min_ngram, max_ngram, n_draft):
+    """Prompt-lookup drafts, written out: for n from max_ngram down to min_ngram,
+    every earlier position j whose n tokens equal the context's last n tokens
+    and that is followed by at least one token is a match; the latest match
+    wins and its following tokens (up to n_draft) are the drafts."""
+    T = list(tokens)
+    for n in range(max_ngram, min_ngram - 1, -1):
+        if n >= len(T):
+            continue
+        suffix = T[len(T) - n:]
+        matches = [j for j in range(0, len(T) - n) if T[j:j + n] == suffix]
+        if matches:
+            j = max(matches)
+            return T[j + n:j + n + n_draft]
+    return []

@@ -34,6 +34,16 @@ class ModelDesc(C.Structure):
 
 
 KV_BF16, KV_Q8_0 = 0, 8
+SCHED_INTERLEAVE, SCHED_PREFILL_FIRST = 0, 1
+
+
+class SchedPolicy(C.Structure):
+    _fields_ = [("chunk_tokens", C.c_int), ("decode_steps_per_chunk", C.c_int), ("max_decode_rows", C.c_int),
+                ("n_draft", C.c_int), ("mode", C.c_int)]
+
+
+class SchedAgent(C.Structure):
+    _fields_ = [("len", C.c_int), ("prompt_left", C.c_int), ("active", C.c_int), ("drafts", C.c_int)]
 
 
 class AgentRows(C.Structure):
@@ -77,6 +87,12 @@ SIGNATURES = {
     "qad_pack_rows": (C.c_int, [C.POINTER(AgentRows), C.c_int, C.c_int, C.c_int, C.c_void_p, C.c_void_p,
                                 C.c_void_p, C.c_void_p]),
     "qad_model_create": (C.c_int, [C.POINTER(ModelDesc), C.POINTER(C.c_void_p)]),
+    "qad_sched_plan": (C.c_int, [C.POINTER(SchedPolicy), C.POINTER(SchedAgent), C.c_int, C.c_longlong,
+                                 C.POINTER(C.c_int), C.POINTER(C.c_int), C.POINTER(C.c_int)]),
+    "qad_sched_commit": (C.c_int, [C.POINTER(SchedAgent), C.c_int, C.POINTER(C.c_int), C.c_int, C.c_int,
+                                   C.POINTER(C.c_int)]),
+    "qad_prompt_lookup": (C.c_int, [C.POINTER(C.c_int), C.c_int, C.c_int, C.c_int, C.c_int, C.POINTER(C.c_int)]),
+    "qad_common_prefix": (C.c_int, [C.POINTER(C.c_int), C.c_int, C.POINTER(C.c_int), C.c_int]),
     "qad_mixed_step_ws_bytes": (C.c_size_t, [C.c_void_p, C.c_int, C.c_int]),
     "qad_mixed_step_debug_bytes": (C.c_size_t, [C.c_void_p, C.c_int, C.c_int]),
     "qad_mixed_step": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int, C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_int,
@@ -370,6 +386,50 @@ def decode_attn_q8(Q, Kq, Kd, Vq, Vd, lens, agent_row_start, n_agents, max_rows_
                                     _dev(ws, "ws"), ws.numel() * ws.element_size(), _stream(stream)),
            "qad_decode_attn_q8")
     return O
+
+
+# ------------------------------------------------------------------ scheduler (host)
+
+def _ints(xs):
+    xs = list(xs)
+    return (C.c_int * max(len(xs), 1))(*xs)
+
+
+class Scheduler:
+    """Host-side step planner over per-agent states (the C scheduler's state lives here)."""
+
+    def __init__(self, n_agents, chunk_tokens=2048, decode_steps_per_chunk=0, max_decode_rows=12, n_draft=2,
+                 mode=SCHED_INTERLEAVE):
+        self.policy = SchedPolicy(chunk_tokens, decode_steps_per_chunk, max_decode_rows, n_draft, mode)
+        self.agents = (SchedAgent * n_agents)()
+        self.n = n_agents
+        self.step = 0
+
+    def plan(self):
+        """(decode_rows list, chunk_agent or -1, chunk_rows) for the next step."""
+        rows = (C.c_int * self.n)()
+        ca, cr = C.c_int(), C.c_int()
+        _check(lib().qad_sched_plan(C.byref(self.policy), self.agents, self.n, self.step, rows, C.byref(ca),
+                                    C.byref(cr)), "qad_sched_plan")
+        return list(rows), ca.value, cr.value
+
+    def commit(self, rows, chunk_agent, chunk_rows, n_accept=None):
+        acc = _ints(n_accept) if n_accept is not None else None
+        _check(lib().qad_sched_commit(self.agents, self.n, _ints(rows), chunk_agent, chunk_rows, acc),
+               "qad_sched_commit")
+        self.step += 1
+
+
+def prompt_lookup(tokens, n_draft=2, min_ngram=1, max_ngram=3):
+    """Drafts from the latest earlier occurrence of the context's last n-gram (list, possibly empty)."""
+    out = (C.c_int * max(n_draft, 1))()
+    k = _check(lib().qad_prompt_lookup(_ints(tokens), len(tokens), min_ngram, max_ngram, n_draft, out),
+               "qad_prompt_lookup")
+    return list(out)[:k]
+
+
+def common_prefix(a, b) -> int:
+    return _check(lib().qad_common_prefix(_ints(a), len(a), _ints(b), len(b)), "qad_common_prefix")
 
 
 # ------------------------------------------------------------------ model / decode step

@@ -8,7 +8,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libqad.so")
-SOURCES = ["host_api.cu", "codec.cu", "gemm.cu", "attn.cu", "attn_q8.cu", "step.cu", "dense.cu", "prefill_attn.cu", "verify.cu"]
+SOURCES = ["host_api.cu", "codec.cu", "gemm.cu", "attn.cu", "attn_q8.cu", "step.cu", "dense.cu", "prefill_attn.cu", "verify.cu", "sched.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "--expt-relaxed-constexpr", "-Xcompiler", "-fPIC,-O2",
          "-Xptxas", "-warn-spills"]
