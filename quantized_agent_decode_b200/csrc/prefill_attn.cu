@@ -28,6 +28,7 @@ constexpr int QV = 64;      // query vectors per CTA
 constexpr int KT = 64;      // keys per tile
 constexpr int STAGES = 2;
 constexpr int TILE = KT * 128 * 2;  // 16 KB per K (or V) tile
+constexpr float M_SLACK = 8.f;      // scores may pass the reference maximum by 2^8
 }  // namespace pf
 
 struct PrefillArgs {
@@ -117,11 +118,14 @@ __global__ void __launch_bounds__(128) k_prefill_attn(PrefillArgs p)
                 mma_bf16(s[nt], qf[ks + 1][0], qf[ks + 1][1], qf[ks + 1][2], qf[ks + 1][3], b2, b3);
             }
         }
-        // online softmax; rows r = 0 (vector g) and 1 (vector g + 8)
+        // Online softmax; rows r = 0 (vector g) and 1 (vector g + 8). The reference
+        // maximum m moves (cross-lane reduction, rescale of o and l) only when a score
+        // passes it by more than M_SLACK log2 units, so P <= 2^8 (well inside bf16's
+        // range) and most tiles skip the reduction and the rescale.
         const bool need_mask = kb + KT - 1 > p.len + (wv / p.G) || kb + KT > kend;
+        bool over = false;
 #pragma unroll
-        for (int r = 0; r < 2; ++r) {
-            float mx = -INFINITY;
+        for (int r = 0; r < 2; ++r)
 #pragma unroll
             for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
@@ -130,28 +134,41 @@ __global__ void __launch_bounds__(128) k_prefill_attn(PrefillArgs p)
                     if (need_mask && kb + 8 * nt + 2 * c + e > lim[r])
                         x = -INFINITY;
                     s[nt][2 * r + e] = x;
-                    mx = fmaxf(mx, x);
+                    over |= x > m[r] + M_SLACK;
                 }
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-            const float mn = fmaxf(m[r], mx);
-            const float corr = mn == -INFINITY ? 1.f : exp2f(m[r] - mn);
+        if (__any_sync(0xffffffffu, over)) {
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                float mx = -INFINITY;
+#pragma unroll
+                for (int nt = 0; nt < 8; ++nt)
+                    mx = fmaxf(mx, fmaxf(s[nt][2 * r], s[nt][2 * r + 1]));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+                const float mn = fmaxf(m[r], mx);
+                const float corr = mn == -INFINITY ? 1.f : ex2_approx(m[r] - mn);
+                m[r] = mn;
+                l[r] *= corr;
+#pragma unroll
+                for (int nd = 0; nd < 16; ++nd) {
+                    o[nd][2 * r] *= corr;
+                    o[nd][2 * r + 1] *= corr;
+                }
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const bool none = m[r] == -INFINITY;
             float sum = 0.f;
 #pragma unroll
             for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
-                    const float pv = mn == -INFINITY ? 0.f : exp2f(s[nt][2 * r + e] - mn);
+                    const float pv = none ? 0.f : ex2_approx(s[nt][2 * r + e] - m[r]);
                     s[nt][2 * r + e] = pv;
                     sum += pv;
                 }
-            m[r] = mn;
-            l[r] = l[r] * corr + sum;
-#pragma unroll
-            for (int nd = 0; nd < 16; ++nd) {
-                o[nd][2 * r] *= corr;
-                o[nd][2 * r + 1] *= corr;
-            }
+            l[r] += sum;
         }
         // O += P V: P (bf16) straight from the S registers, V^T via ldmatrix.trans
 #pragma unroll
