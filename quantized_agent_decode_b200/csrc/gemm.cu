@@ -749,6 +749,135 @@ __global__ void __launch_bounds__(Cfg<FMT>::THREADS, 1) k_qgemm(const __grid_con
     trace_end(a.trace);
 }
 
+// Q4_K form without a producer warp: 4 consumer groups of 4 warps (16 warps,
+// so each SM sub-partition runs 4 consumers at the same register budget as 3
+// consumers + the producer). Group grp consumes units grp, grp+4, ... through
+// its own two ring slots (grp and grp+4 of 8) and refills a slot itself: after
+// the group's 4 warps release unit i (one arrival each on the slot's empty
+// barrier), lane 0 of the group's first warp issues unit i+8 into it. Before
+// the wait on the previous kernel each group requests the weights of its first
+// two units; every wait is bounded and reports through g_gemm_status.
+#ifndef QAD_Q4_SELF_REFILL
+#define QAD_Q4_SELF_REFILL 1
+#endif
+namespace sr {
+constexpr int CG = 4, GW = 4, S = 8, THREADS = 32 * CG * GW;
+}
+template <int NT>
+constexpr size_t gemm_sr_smem_bytes()
+{
+    return (size_t)sr::S * Stage<4, NT>::BYTES + 2 * sr::S * sizeof(uint64_t);
+}
+
+template <int NT>
+__global__ void __launch_bounds__(sr::THREADS, 1) k_qgemm_sr(const __grid_constant__ WeightMaps maps, GemmArgs a)
+{
+    extern __shared__ __align__(128) uint8_t smem[];
+    using St = Stage<4, NT>;
+    constexpr int S = sr::S, GW = sr::GW, CG = sr::CG, TILE = Cfg<4>::TILE;
+    static_assert(S % CG == 0 && TILE == RW * GW, "each group owns S / CG slots; a unit is GW warps of RW rows");
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + (size_t)S * St::BYTES);
+    uint64_t *empty = full + S;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int grp = warp / GW, wi = warp % GW;
+    const int u0 = (int)((long long)blockIdx.x * a.units / gridDim.x);
+    const int u1 = (int)((long long)(blockIdx.x + 1) * a.units / gridDim.x);
+    const int n_units = u1 - u0;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < S; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], GW);
+        }
+        mbar_fence_init();
+    }
+    __syncthreads();
+    trace_start(a.trace);
+    pdl_trigger();
+    const bool leader = wi == 0 && lane == 0;
+    auto issue = [&](int i, bool weights, bool frags) {
+        const int u = u0 + i, t = u / a.nblk, b = u - t * a.nblk;
+        uint8_t *st = smem + (size_t)(i % S) * St::BYTES;
+        uint64_t *bar = &full[i % S];
+        if (weights) {
+            mbar_arrive_expect_tx(bar, (uint32_t)St::COPY_BYTES);
+            tma_load_2d(st, &maps.w, b * 144, t * TILE, bar);
+        }
+        if (frags)
+            bulk_g2s(st + St::W_BYTES, a.rec + (size_t)b * St::R_BYTES, St::R_BYTES, bar);
+    };
+    int issued = -1;  // highest unit this group's leader has requested
+    if (leader)
+        for (int i = grp; i < n_units && i < S; i += CG) {
+            issue(i, true, false);  // weights do not depend on the previous kernel
+            issued = i;
+        }
+    pdl_wait();
+    if (leader)
+        for (int i = grp; i < n_units && i < S; i += CG)
+            issue(i, false, true);
+    trace_ready(a.trace);
+
+    const int g = lane >> 2, c = lane & 3;
+    const int jj = 2 * (c & 1);
+    const uint32_t selT = (uint32_t)(jj | ((jj + 1) << 4) | ((jj + 4) << 8) | ((jj + 5) << 12));
+    const bool hib = c >= 2;
+    float tot[2][NT][4];
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                tot[mt][nt][e] = 0.f;
+    int t = 0, b = 0;
+    if (grp < n_units) {
+        t = (u0 + grp) / a.nblk;
+        b = (u0 + grp) - t * a.nblk;
+    }
+    int done = grp - CG;  // last unit this warp consumed
+    for (int i = grp; i < n_units; i += CG) {
+        const uint8_t *st = smem + (size_t)(i % S) * St::BYTES;
+        if (!mbar_wait(&full[i % S], (i / S) & 1)) {
+            if (lane == 0)
+                atomicExch(&g_gemm_status, ERR_FULL_TIMEOUT);
+            break;
+        }
+        const uint8_t *XS = st + St::W_BYTES;
+        const uint8_t *RS = XS + St::R_BYTES - 64;
+        q4_block<NT>(st + (size_t)(RW * wi) * 144, XS, XS + St::X_BYTES, RS, g, c, selT, hib, tot);
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(&empty[i % S]);
+        done = i;
+        if (leader && i + S < n_units) {
+            // the slot's next user is unit i + S of this group: refill it once all GW warps released it
+            if (!mbar_wait(&empty[i % S], (i / S) & 1)) {
+                atomicExch(&g_gemm_status, ERR_EMPTY_TIMEOUT);
+            } else {
+                issue(i + S, true, true);
+                issued = i + S;
+            }
+        }
+        int tn = t, bn = b + CG;
+        while (bn >= a.nblk) {
+            bn -= a.nblk;
+            ++tn;
+        }
+        if (tn != t || i + CG >= n_units) {
+            flush_rows<NT>(tot[0], a, t * TILE + RW * wi, g, c);
+            flush_rows<NT>(tot[1], a, t * TILE + RW * wi + 16, g, c);
+        }
+        t = tn;
+        b = bn;
+    }
+    // after an error exit, copies this group requested but did not consume land before the CTA exits
+    if (leader)
+        for (int k = done + CG; k <= issued; k += CG)
+            if (!mbar_wait(&full[k % S], (k / S) & 1, 20000))
+                atomicExch(&g_gemm_status, ERR_FULL_TIMEOUT);
+    trace_end(a.trace);
+}
+
 // Q6_K-like GGUF blocks -> packed device layout (plane A: first 208 bytes of
 // each block; plane D: d, rows padded to a multiple of 8 blocks with zeros).
 __global__ void k_q6k_pack(const uint8_t *__restrict__ W, int N, int nblk, uint8_t *__restrict__ P)
@@ -840,7 +969,12 @@ int launch_gemm(int fmt, const WeightMapsBlob &maps_blob, int N, int K, int M, c
     a.trace = trace;
     void (*kern)(const WeightMaps, GemmArgs);
     size_t smem;
-    if (fmt == 4) {
+    int threads = fmt == 4 ? Cfg<4>::THREADS : Cfg<6>::THREADS;
+    if (fmt == 4 && QAD_Q4_SELF_REFILL) {
+        kern = nt == 1 ? k_qgemm_sr<1> : k_qgemm_sr<2>;
+        smem = nt == 1 ? gemm_sr_smem_bytes<1>() : gemm_sr_smem_bytes<2>();
+        threads = sr::THREADS;
+    } else if (fmt == 4) {
         kern = nt == 1 ? k_qgemm<4, 1> : k_qgemm<4, 2>;
         smem = nt == 1 ? gemm_smem_bytes<4, 1>() : gemm_smem_bytes<4, 2>();
     } else {
@@ -859,7 +993,6 @@ int launch_gemm(int fmt, const WeightMapsBlob &maps_blob, int N, int K, int M, c
             done[dev][v] = true;
     }
     const int grid = num_sms();
-    const int threads = fmt == 4 ? Cfg<4>::THREADS : Cfg<6>::THREADS;
     cudaError_t e = pdl ? launch_pdl(kern, dim3(grid), dim3(threads), smem, s, maps, a)
                         : (kern<<<grid, threads, smem, s>>>(maps, a), cudaGetLastError());
     return cuda_check(e, "gemm launch");
