@@ -260,11 +260,17 @@ int qad_verify_step(const float *H, int M, int hidden, float rms_eps, const void
  *   Q       device bf16 [C][n_qh][128]
  *   Kc, Vc  device bf16 [n_kvh][kv_cap][128] (this agent's cache); len + C <= kv_cap
  *   O       device bf16 [C][n_qh][128], written
- * Tensor-core products with fp32 softmax; the probabilities enter the PV
- * product rounded to bf16 (relative error <= 2^-9). hd must be 128. Q, caches
- * and O 16-byte aligned. Returns 0 or a negative QAD_ERR_* code. */
+ * Tensor-core products (tcgen05, S and O in TMEM) with fp32 softmax; the
+ * probabilities enter the PV product rounded to bf16 (relative error <= 2^-9).
+ * hd must be 128. Q, caches and O 16-byte aligned. Returns 0 or a negative
+ * QAD_ERR_* code. */
 int qad_prefill_attn(const uint16_t *Q, const uint16_t *Kc, const uint16_t *Vc, int len, int C, int kv_cap,
                      int n_qh, int n_kvh, int hd, float scale, uint16_t *O, void *stream);
+/* Status of the prefill attention's bounded pipeline waits since the last
+ * reset: 0 = none timed out, > 0 = the stage that timed out (the launch then
+ * skips its remaining work). reset != 0 clears it. Negative QAD_ERR_* on a
+ * CUDA error. */
+int qad_prefill_status(int reset);
 
 /* ---------------------------------------------------------------- row packer
  * Host-only. Stacks every agent's rows (next token + drafts) agent-major into

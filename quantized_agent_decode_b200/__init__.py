@@ -73,6 +73,7 @@ SIGNATURES = {
     "qad_q6k_gemm_dense": (C.c_int, [C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p,
                                      C.c_size_t, C.c_void_p]),
     "qad_dense_status": (C.c_int, [C.c_int]),
+    "qad_prefill_status": (C.c_int, [C.c_int]),
     "qad_verify_ws_bytes": (C.c_size_t, [C.c_int, C.c_int, C.c_int]),
     "qad_verify_step": (C.c_int, [C.c_void_p, C.c_int, C.c_int, C.c_float, C.c_void_p, C.c_int, C.c_void_p, C.c_int]
                         + [C.c_void_p] * 7 + [C.c_size_t, C.c_void_p]),
@@ -231,6 +232,11 @@ def q4k_gemm_noalloc(W, N, K, X, M, Y, accumulate=False, stream=None):
 
 def dense_gemm_ws_bytes(K: int, M: int) -> int:
     return int(lib().qad_dense_gemm_ws_bytes(K, M))
+
+
+def prefill_status(reset: bool = True) -> int:
+    """0 if every prefill-attention pipeline wait completed since the last reset."""
+    return _check(lib().qad_prefill_status(int(reset)), "qad_prefill_status")
 
 
 def dense_status(reset: bool = True) -> int:

@@ -212,16 +212,6 @@ __device__ __forceinline__ void dequant_q6(const uint8_t *blk, float d, int kk, 
     }
 }
 
-__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-
-__device__ __forceinline__ void umma_f16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                            uint32_t accumulate)
-{
-    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-                 "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-                 ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-                 : "memory");
-}
 
 template <int FMT>
 __global__ void __launch_bounds__(dn::THREADS, 1) k_dense_gemm(const __grid_constant__ WeightMapsBlob mapsb, DenseArgs a)

@@ -19,6 +19,8 @@
 //  * Online softmax in fp32 (exp2 with the scale folded in); P is rounded to
 //    bf16 once and used straight from the S accumulator registers as the A
 //    operand of the PV product.
+#include <cuda.h>
+
 #include "attn.cuh"
 
 namespace qad {
@@ -208,8 +210,362 @@ __global__ void __launch_bounds__(128) k_prefill_attn(PrefillArgs p)
     }
 }
 
+int launch_prefill_attn_mma(const uint16_t *Q, const uint16_t *Kc, const uint16_t *Vc, int len, int C, int kv_cap,
+                            int n_qh, int n_kvh, float scale, uint16_t *O, cudaStream_t s);
+
+// ------------------------------------------------------------- tcgen05 form
+//
+// CTA = 128 query vectors of one kv-head (the MMA's M), heavy (late) row
+// blocks first. Six warps: four softmax warps (thread = query vector = TMEM
+// lane), a producer warp (TMA) and an MMA warp (one thread issues tcgen05.mma).
+//  * K and V arrive by TMA in 128-key tiles, double-buffered, as 16 boxes of
+//    8 dims x 128 keys: [dim chunk][key][8 dims], which is exactly the
+//    K-major no-swizzle operand layout (8-row x 16-byte core matrices) of B
+//    in S = Q K^T. Q is loaded once in the same layout.
+//  * S (128 x 128 fp32) and O (128 x 128 fp32) live in TMEM (256 columns).
+//  * A softmax thread reads its S row from TMEM, masks, keeps a running
+//    reference maximum that moves (with a rescale of its O row in TMEM) only
+//    when a score passes it by more than 2^8, and writes P = 2^(s - m) as bf16
+//    into shared memory in the A-operand layout [key chunk][row][8 keys]; the
+//    four warps also transpose the V tile with ldmatrix.trans into the K-major
+//    B layout [key chunk][dim][8 keys] (zeroing keys past the causal end).
+//  * O += P V^T-tile by tcgen05.mma; the last tile's completion releases the
+//    epilogue, which divides by the row sum and stores bf16.
+// Every mbarrier wait is bounded; on a timeout the CTA records a status,
+// stops issuing, waits for its own copies and MMAs, frees TMEM and exits.
+namespace pt {
+constexpr int ROWS = 128, KT = 128, TB = KT * 128 * 2;  // 32 KB operand tiles
+constexpr int SW = 4;                                   // softmax warps
+constexpr int THREADS = 32 * (SW + 2);
+constexpr float M_SLACK = 8.f;
+constexpr size_t SMEM = 1024 + 7 * (size_t)TB + 256;  // Q, K[2], V[2], Vt, P, barriers
+enum { ST_KV = 1, ST_S = 2, ST_P = 3, ST_PV = 4, ST_DONE = 5 };
+}  // namespace pt
+
+__device__ int g_prefill_status;
+
+struct PfMaps {
+    CUtensorMap k, v;  // [n_kvh * kv_cap][128] bf16, boxes of 8 dims x 128 keys
+};
+
+__global__ void __launch_bounds__(pt::THREADS, 1) k_prefill_attn_tc(const __grid_constant__ PfMaps maps, PrefillArgs p)
+{
+    using namespace pt;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    uint8_t *QS = smem, *KS = QS + TB, *VS = KS + 2 * TB, *VT = VS + 2 * TB, *PS = VT + TB;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(PS + TB);
+    uint64_t *kv_full = bar, *kv_free = bar + 2, *s_full = bar + 4, *s_free = bar + 5, *p_full = bar + 6,
+             *pv_done = bar + 7, *done = bar + 8;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + 9);
+    __shared__ int s_bad;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int kvh = blockIdx.y;
+    const int R = p.C * p.G;
+    const int nrb = (R + ROWS - 1) / ROWS;
+    const int v0 = (nrb - 1 - (int)blockIdx.x) * ROWS;  // late row blocks (more keys) first
+    const int j_last = min(p.C - 1, (v0 + ROWS - 1) / p.G);
+    const int kend = p.len + j_last + 1;
+    const int ntiles = (kend + KT - 1) / KT;
+
+    if (threadIdx.x == 0) {
+        s_bad = 0;
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&kv_full[i], 1);
+            mbar_init(&kv_free[i], 1);
+        }
+        mbar_init(s_full, 1);
+        mbar_init(s_free, SW * 32);
+        mbar_init(p_full, SW * 32);
+        mbar_init(pv_done, 1);
+        mbar_init(done, 1);
+        mbar_fence_init();
+    }
+    // Q tile (zero past the chunk) in the A-operand layout [dim chunk][row][8 dims]
+    if (warp < SW) {
+        const int r = threadIdx.x, v = v0 + r;
+        const bool ok = v < R;
+        const int j = ok ? v / p.G : 0, hl = ok ? v - j * p.G : 0;
+        const uint16_t *qrow = p.Q + ((size_t)j * p.n_qh + kvh * p.G + hl) * 128;
+#pragma unroll
+        for (int dc = 0; dc < 16; ++dc)
+            cp_async16_zfill(QS + dc * 2048 + r * 16, qrow + 8 * dc, ok);
+        cp_async_commit();
+        cp_async_wait<0>();
+        fence_proxy_async();
+    }
+    if (warp == SW + 1) {
+        tmem_alloc(tmem_slot, 256);  // S: columns 0..127, O: 128..255
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot, tS = tmem, tO = tmem + 128;
+    auto fail = [&](int code) {
+        atomicExch(&g_prefill_status, code);
+        atomicExch(&s_bad, 1);
+    };
+    auto bad = [&]() { return *(volatile int *)&s_bad != 0; };
+
+    if (warp == SW) {
+        // ------------------------------------------------ producer: K and V tiles by TMA
+        if (lane == 0) {
+            int j = 0;
+            for (; j < ntiles && !bad(); ++j) {
+                const int s = j & 1;
+                if (j >= 2 && !mbar_wait(&kv_free[s], ((j >> 1) - 1) & 1)) {
+                    fail(ST_KV);
+                    break;
+                }
+                mbar_arrive_expect_tx(&kv_full[s], 2 * TB);
+                const int y = kvh * p.kv_cap + j * KT;
+                for (int dc = 0; dc < 16; ++dc) {
+                    tma_load_2d(KS + s * TB + dc * 2048, &maps.k, 8 * dc, y, &kv_full[s]);
+                    tma_load_2d(VS + s * TB + dc * 2048, &maps.v, 8 * dc, y, &kv_full[s]);
+                }
+            }
+            for (int k = max(0, j - 2); k < j; ++k)  // every issued copy lands before teardown
+                if (!mbar_wait(&kv_full[k & 1], (k >> 1) & 1, 20000))
+                    fail(ST_KV);
+        }
+    } else if (warp == SW + 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = umma_idesc_bf16(ROWS, KT);  // both products are 128 x 128
+            bool issued = false;
+            // S_{j+1} is issued as soon as the softmax warps have read S_j, so it runs while they
+            // work on tile j; PV_j follows once they have written P_j and the transposed V_j.
+            auto issue_s = [&](int j) {
+                const uint32_t qb = smem_u32(QS), kb = smem_u32(KS + (j & 1) * TB);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    umma_f16_ss(tS, umma_desc_k_noswz(qb + ks * 4096, 2048, 128),
+                                umma_desc_k_noswz(kb + ks * 4096, 2048, 128), idesc, ks > 0);
+                umma_commit(s_full);
+                issued = true;
+            };
+            if (mbar_wait(&kv_full[0], 0)) {
+                tc_fence_after();
+                issue_s(0);
+            } else {
+                fail(ST_S);
+            }
+            for (int j = 0; j < ntiles && !bad(); ++j) {
+                if (j + 1 < ntiles) {
+                    if (!mbar_wait(&kv_full[(j + 1) & 1], ((j + 1) >> 1) & 1) || !mbar_wait(s_free, j & 1)) {
+                        fail(ST_S);
+                        break;
+                    }
+                    tc_fence_after();
+                    issue_s(j + 1);
+                }
+                if (!mbar_wait(p_full, j & 1)) {
+                    fail(ST_P);
+                    break;
+                }
+                tc_fence_after();
+                mbar_arrive(&kv_free[j & 1]);  // S_j is done and the V tile has been transposed
+                const uint32_t pb = smem_u32(PS), vb = smem_u32(VT);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    umma_f16_ss(tO, umma_desc_k_noswz(pb + ks * 4096, 2048, 128),
+                                umma_desc_k_noswz(vb + ks * 4096, 2048, 128), idesc, (j | ks) != 0);
+                umma_commit(pv_done);
+            }
+            if (issued) {  // every MMA this thread issued completes before TMEM is freed
+                umma_commit(done);
+                if (!mbar_wait(done, 0, 20000))
+                    fail(ST_DONE);
+            }
+        }
+    } else {
+        // ------------------------------------------------ softmax warps: thread = query vector = TMEM lane
+        const int r = threadIdx.x, v = v0 + r;
+        const bool live = v < R;
+        const int jrow = live ? v / p.G : 0;
+        const int lim = live ? p.len + jrow : -1;  // last visible key
+        const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+        float m = -INFINITY, l = 0.f;
+        for (int j = 0; j < ntiles && !bad(); ++j) {
+            if (!__all_sync(0xffffffffu, mbar_wait(s_full, j & 1))) {
+                fail(ST_S);
+                break;
+            }
+            tc_fence_after();
+            float x[KT];
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc)
+                tmem_ld_x32(tS + lane_off + 32 * cc, reinterpret_cast<uint32_t *>(x + 32 * cc));
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(s_free);
+            const int kb = j * KT;
+            bool over = false;
+#pragma unroll
+            for (int i = 0; i < KT; ++i) {
+                const int key = kb + i;
+                x[i] = (key < kend && key <= lim) ? x[i] * p.scale_log2 : -INFINITY;
+                over |= x[i] > m + M_SLACK;
+            }
+            // the new reference maximum and P in registers first: this overlaps the
+            // previous tile's PV product, which only the writes below must wait for
+            const bool resc = __any_sync(0xffffffffu, over);
+            float corr = 1.f;
+            if (resc) {
+                float mx = -INFINITY;
+#pragma unroll
+                for (int i = 0; i < KT; ++i)
+                    mx = fmaxf(mx, x[i]);
+                const float mn = fmaxf(m, mx);
+                corr = mn == -INFINITY ? 1.f : ex2_approx(m - mn);
+                m = mn;
+            }
+            const bool none = m == -INFINITY;
+            uint32_t pw[KT / 2];
+            float psum = 0.f;
+#pragma unroll
+            for (int i = 0; i < KT / 2; ++i) {
+                const float p0 = none ? 0.f : ex2_approx(x[2 * i] - m);
+                const float p1 = none ? 0.f : ex2_approx(x[2 * i + 1] - m);
+                psum += p0 + p1;
+                pw[i] = pack_bf162(p0, p1);
+            }
+            l = l * corr + psum;
+            // the previous PV product must be done before O is rescaled or P / Vt rewritten
+            if (j > 0 && !__all_sync(0xffffffffu, mbar_wait(pv_done, (j - 1) & 1))) {
+                fail(ST_PV);
+                break;
+            }
+            tc_fence_after();
+            if (resc && j > 0) {  // O holds earlier tiles: scale this row
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    uint32_t ov[32];
+                    tmem_ld_x32(tO + lane_off + 32 * cc, ov);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        ov[i] = __float_as_uint(__uint_as_float(ov[i]) * corr);
+                    tmem_st_x32(tO + lane_off + 32 * cc, ov);
+                }
+                tmem_wait_st();
+            }
+            // P as bf16 into [key chunk][row][8 keys]
+#pragma unroll
+            for (int kc = 0; kc < 16; ++kc)
+                *reinterpret_cast<uint4 *>(PS + kc * 2048 + r * 16) =
+                    make_uint4(pw[4 * kc], pw[4 * kc + 1], pw[4 * kc + 2], pw[4 * kc + 3]);
+            // V tile -> Vt [key chunk][dim][8 keys]: this warp's dim chunks 4w .. 4w+3, 32 keys per ldmatrix
+            const int s = j & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(&kv_full[s], (j >> 1) & 1))) {
+                fail(ST_KV);
+                break;
+            }
+            const uint8_t *Vs = VS + s * TB;
+#pragma unroll
+            for (int dd = 0; dd < 4; ++dd) {
+                const int dc = 4 * warp + dd;
+#pragma unroll
+                for (int kg = 0; kg < 4; ++kg) {
+                    uint32_t t4[4];
+                    ldsm_x4_t(t4[0], t4[1], t4[2], t4[3], Vs + dc * 2048 + (32 * kg + lane) * 16);
+#pragma unroll
+                    for (int mi = 0; mi < 4; ++mi) {
+                        const int kc = 4 * kg + mi, key = kb + 8 * kc + 2 * (lane & 3);
+                        uint32_t val = t4[mi];
+                        if (key >= kend)
+                            val = 0u;
+                        else if (key + 1 >= kend)
+                            val &= 0xFFFFu;
+                        *reinterpret_cast<uint32_t *>(VT + kc * 2048 + (8 * dc + (lane >> 2)) * 16 + (lane & 3) * 4) =
+                            val;
+                    }
+                }
+            }
+            fence_proxy_async();
+            tc_fence_before();
+            mbar_arrive(p_full);
+        }
+        // epilogue: O / l -> bf16
+        if (!bad() && __all_sync(0xffffffffu, mbar_wait(pv_done, (ntiles - 1) & 1))) {
+            tc_fence_after();
+            const int hl = live ? v - jrow * p.G : 0;
+            uint16_t *orow = p.O + ((size_t)jrow * p.n_qh + kvh * p.G + hl) * 128;
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                uint32_t ov[32];
+                tmem_ld_x32(tO + lane_off + 32 * cc, ov);
+                tmem_wait_ld();
+                if (live)
+#pragma unroll
+                    for (int i = 0; i < 32; i += 8)
+                        *reinterpret_cast<uint4 *>(orow + 32 * cc + i) = make_uint4(
+                            pack_bf162(__uint_as_float(ov[i]) * inv, __uint_as_float(ov[i + 1]) * inv),
+                            pack_bf162(__uint_as_float(ov[i + 2]) * inv, __uint_as_float(ov[i + 3]) * inv),
+                            pack_bf162(__uint_as_float(ov[i + 4]) * inv, __uint_as_float(ov[i + 5]) * inv),
+                            pack_bf162(__uint_as_float(ov[i + 6]) * inv, __uint_as_float(ov[i + 7]) * inv));
+            }
+        } else if (!bad()) {
+            fail(ST_PV);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == SW + 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
+#ifndef QAD_PREFILL_TC
+#define QAD_PREFILL_TC 1
+#endif
+
 int launch_prefill_attn(const uint16_t *Q, const uint16_t *Kc, const uint16_t *Vc, int len, int C, int kv_cap,
                         int n_qh, int n_kvh, float scale, uint16_t *O, cudaStream_t s)
+{
+    if (QAD_PREFILL_TC) {
+        PrefillArgs a;
+        a.Q = Q;
+        a.Kc = Kc;
+        a.Vc = Vc;
+        a.O = O;
+        a.len = len;
+        a.C = C;
+        a.kv_cap = kv_cap;
+        a.n_qh = n_qh;
+        a.n_kvh = n_kvh;
+        a.G = n_qh / n_kvh;
+        a.scale_log2 = scale * 1.4426950408889634f;
+        PfMaps maps;
+        int rc = encode_tmap_2d(&maps.k, Kc, 2, 128, (uint64_t)n_kvh * kv_cap, 256, 8, pt::KT);
+        if (!rc)
+            rc = encode_tmap_2d(&maps.v, Vc, 2, 128, (uint64_t)n_kvh * kv_cap, 256, 8, pt::KT);
+        if (rc)
+            return rc;
+        static bool done[64] = {};
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (dev < 0 || dev >= 64 || !done[dev]) {
+            rc = cuda_check(cudaFuncSetAttribute(k_prefill_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)pt::SMEM),
+                            "cudaFuncSetAttribute(prefill attn tc)");
+            if (rc)
+                return rc;
+            if (dev >= 0 && dev < 64)
+                done[dev] = true;
+        }
+        dim3 grid((C * a.G + pt::ROWS - 1) / pt::ROWS, n_kvh);
+        k_prefill_attn_tc<<<grid, pt::THREADS, pt::SMEM, s>>>(maps, a);
+        return cuda_check(cudaGetLastError(), "prefill attn launch");
+    }
+    return launch_prefill_attn_mma(Q, Kc, Vc, len, C, kv_cap, n_qh, n_kvh, scale, O, s);
+}
+
+int launch_prefill_attn_mma(const uint16_t *Q, const uint16_t *Kc, const uint16_t *Vc, int len, int C, int kv_cap,
+                            int n_qh, int n_kvh, float scale, uint16_t *O, cudaStream_t s)
 {
     PrefillArgs a;
     a.Q = Q;
@@ -257,4 +613,19 @@ extern "C" int qad_prefill_attn(const uint16_t *Q, const uint16_t *Kc, const uin
     if (((uintptr_t)Q | (uintptr_t)Kc | (uintptr_t)Vc | (uintptr_t)O) & 15)
         return qad::fail(QAD_ERR_INVALID, "qad_prefill_attn: Q, caches and O must be 16-byte aligned");
     return qad::launch_prefill_attn(Q, Kc, Vc, len, C, kv_cap, n_qh, n_kvh, scale, O, (cudaStream_t)stream);
+}
+
+extern "C" int qad_prefill_status(int reset)
+{
+    int v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, qad::g_prefill_status, sizeof(int));
+    if (e != cudaSuccess)
+        return qad::cuda_check(e, "qad_prefill_status");
+    if (reset && v) {
+        const int z = 0;
+        e = cudaMemcpyToSymbol(qad::g_prefill_status, &z, sizeof(int));
+        if (e != cudaSuccess)
+            return qad::cuda_check(e, "qad_prefill_status reset");
+    }
+    return v;
 }

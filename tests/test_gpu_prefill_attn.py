@@ -53,13 +53,18 @@ CASES = [  # (len, C, n_qh, n_kvh)
 
 @pytest.mark.parametrize("len_,C,n_qh,n_kvh", CASES)
 def test_prefill_attn_parity(q, orc, len_, C, n_qh, n_kvh):
-    cap = len_ + C + 3
+    """Cache slots past the chunk hold NaN: a kernel must neither read them into
+    a visible product nor let them leak through a zero probability."""
+    cap = len_ + C + 131
     Q = synth.bf16_normal_np(SEED, 700 + C, (C, n_qh, 128))
     Kc = synth.bf16_normal_np(SEED, 701 + C, (n_kvh, cap, 128))
     Vc = synth.bf16_normal_np(SEED, 702 + C, (n_kvh, cap, 128))
+    Kc[:, len_ + C:] = 0x7FC0
+    Vc[:, len_ + C:] = 0x7FC0
     O = torch.zeros(C, n_qh, 128, dtype=torch.bfloat16, device="cuda")
     q.prefill_attn(_dev(Q), _dev(Kc), _dev(Vc), len_, C, cap, n_qh, n_kvh, 128, O)
     torch.cuda.synchronize()
+    assert q.prefill_status() == 0
     O_ref, B = orc.decode_attn(Q, Kc[None], Vc[None], np.array([len_], np.int32), np.array([0, C], np.int32),
                                n_qh, n_kvh, 128, cap)
     _check(orc, _bits(O), O_ref, B)
@@ -77,6 +82,7 @@ def test_prefill_attn_chunk_after_23k_tokens(q, orc):
     O = torch.zeros(C, n_qh, 128, dtype=torch.bfloat16, device="cuda")
     q.prefill_attn(Qd, Kd, Vd, len_, C, cap, n_qh, n_kvh, 128, O)
     torch.cuda.synchronize()
+    assert q.prefill_status() == 0
     Q, Kc, Vc, Ob = _bits(Qd), _bits(Kd), _bits(Vd), _bits(O)
     for j in (0, 1, 63, 64, 1023, 2046, 2047):
         O_ref, B = orc.decode_attn(Q[j:j + 1], Kc[None], Vc[None], np.array([len_ + j], np.int32),
