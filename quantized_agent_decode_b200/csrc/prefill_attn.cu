@@ -401,33 +401,42 @@ __global__ void __launch_bounds__(pt::THREADS, 1) k_prefill_attn_tc(const __grid
             tc_fence_before();
             mbar_arrive(s_free);
             const int kb = j * KT;
-            bool over = false;
-#pragma unroll
-            for (int i = 0; i < KT; ++i) {
-                const int key = kb + i;
-                x[i] = (key < kend && key <= lim) ? x[i] * p.scale_log2 : -INFINITY;
-                over |= x[i] > m + M_SLACK;
-            }
-            // the new reference maximum and P in registers first: this overlaps the
-            // previous tile's PV product, which only the writes below must wait for
-            const bool resc = __any_sync(0xffffffffu, over);
-            float corr = 1.f;
-            if (resc) {
-                float mx = -INFINITY;
+            // Tiles wholly below every row's causal limit (the CTA's first row sees the
+            // fewest keys) need no mask: the row maximum is taken on the raw scores and
+            // the scale folds into one fused multiply-add per probability.
+            const bool interior = kb + KT - 1 <= p.len + v0 / p.G;
+            float mx = -INFINITY;
+            if (interior) {
 #pragma unroll
                 for (int i = 0; i < KT; ++i)
                     mx = fmaxf(mx, x[i]);
+                mx *= p.scale_log2;
+            } else {
+#pragma unroll
+                for (int i = 0; i < KT; ++i) {
+                    const int key = kb + i;
+                    x[i] = (key < kend && key <= lim) ? x[i] * p.scale_log2 : -INFINITY;
+                    mx = fmaxf(mx, x[i]);
+                }
+            }
+            // the new reference maximum and P in registers first: this overlaps the
+            // previous tile's PV product, which only the writes below must wait for
+            const bool resc = __any_sync(0xffffffffu, mx > m + M_SLACK);
+            float corr = 1.f;
+            if (resc) {
                 const float mn = fmaxf(m, mx);
                 corr = mn == -INFINITY ? 1.f : ex2_approx(m - mn);
                 m = mn;
             }
             const bool none = m == -INFINITY;
+            const float sc = interior ? p.scale_log2 : 1.f;  // scores still unscaled on interior tiles
+            const float nm = none ? 0.f : -m;
             uint32_t pw[KT / 2];
             float psum = 0.f;
 #pragma unroll
             for (int i = 0; i < KT / 2; ++i) {
-                const float p0 = none ? 0.f : ex2_approx(x[2 * i] - m);
-                const float p1 = none ? 0.f : ex2_approx(x[2 * i + 1] - m);
+                const float p0 = none ? 0.f : ex2_approx(fmaf(x[2 * i], sc, nm));
+                const float p1 = none ? 0.f : ex2_approx(fmaf(x[2 * i + 1], sc, nm));
                 psum += p0 + p1;
                 pw[i] = pack_bf162(p0, p1);
             }
