@@ -129,3 +129,23 @@ def test_compute_calls_fail_loudly_without_gpu(qlib):
     with pytest.raises(qlib.QadError):
         qlib.q4k_gemm(torch.zeros(1, 144, dtype=torch.uint8), 1, 256, torch.zeros(1, 256, dtype=torch.bfloat16),
                       1, torch.zeros(1, 1))
+
+
+def test_q8_and_mixed_argument_checks_and_cache_sizes(qlib):
+    """Host-side checks of the q8_0 and mixed-step entry points (no launch reached),
+    and the cache sizes they expect."""
+    L = qlib.lib()
+    fake = C.c_void_p(0x10000)  # aligned, never dereferenced: every call below fails its checks first
+    assert L.qad_q8_0_quantize(fake, 0, 48, fake, fake, None) == -2          # n % 32
+    assert L.qad_q8_0_quantize(None, 0, 64, fake, fake, None) == -1
+    assert L.qad_q8_0_quantize(C.c_void_p(0x10004), 0, 64, fake, fake, None) == -1  # x not 16-byte aligned
+    args = [fake] * 7 + [4, 3, 100, 48, 8]
+    assert L.qad_decode_attn_q8(*args, 64, 0.1, fake, fake, 1 << 20, None) == -2  # hd != 128
+    assert L.qad_decode_attn_q8(*args, 128, 0.1, fake, fake, 16, None) == -3     # workspace
+    assert L.qad_mixed_step(None, fake, 2, fake, 1, 2, fake, 0, 0, 8, fake, fake, 1 << 20, None) == -1
+    # bf16: 2 bytes per value; q8_0: 1 byte per value, then fp16 scales per 32 at a 256-byte boundary
+    A, kvh, cap = 4, 8, 1027
+    assert qlib.kv_cache_bytes(qlib.KV_BF16, A, kvh, cap) == A * kvh * cap * 128 * 2
+    codes = A * kvh * cap * 128
+    assert qlib.kv_cache_bytes(qlib.KV_Q8_0, A, kvh, cap) == (codes + 255) // 256 * 256 + A * kvh * cap * 4 * 2
+    assert qlib.kv_cache_bytes(7, A, kvh, cap) == 0 and qlib.kv_cache_bytes(qlib.KV_Q8_0, A, kvh, cap, hd=64) == 0
