@@ -26,6 +26,11 @@
 #define QAD_ATTN_MIN_SPLIT_KEYS 256
 #endif
 
+// CTAs per SM the short-cache plan aims for (build-time tunable).
+#ifndef QAD_ATTN_SHORT_CTAS_PER_SM
+#define QAD_ATTN_SHORT_CTAS_PER_SM 1
+#endif
+
 namespace qad {
 
 constexpr int QG = ATT_QG;      // query vectors per CTA
@@ -428,14 +433,16 @@ AttnPlan attn_plan(int n_agents, int n_qh, int n_kvh, int kv_cap, int max_rows_p
     // warp's tiles (16 keys each, 4 warps) all fit its 6-stage ring, so every
     // cached key is in flight before the kernel waits for its queries.
     {
-        int sp = num_sms() / pairs;
+        int sp = QAD_ATTN_SHORT_CTAS_PER_SM * num_sms() / pairs;
         if (sp < 1)
             sp = 1;
         int ch = (kv_cap + sp - 1) / sp;
         ch = ((ch + 63) / 64) * 64;
-        if ((ch / KT + ATT_WARPS - 1) / ATT_WARPS <= ATT_STAGES_SHORT - 1) {
+        // two CTAs per SM only fit with the 3-deep ring
+        const int st = QAD_ATTN_SHORT_CTAS_PER_SM > 1 ? ATT_STAGES_LONG : ATT_STAGES_SHORT;
+        if ((ch / KT + ATT_WARPS - 1) / ATT_WARPS <= st - 1) {
             pl.CH = ch;
-            pl.stages = ATT_STAGES_SHORT;
+            pl.stages = st;
             pl.max_splits = (kv_cap + ch - 1) / ch;
             pl.part_bytes = (size_t)n_agents * n_kvh * pl.n_rg * pl.max_splits * PART_FLOATS * sizeof(float);
             return pl;
