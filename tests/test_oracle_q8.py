@@ -141,3 +141,28 @@ def test_q8_decode_layer_appends_and_attends(orc):
     o = o.reshape(M, nq).numpy()
     got = orc.bf16_array_to_f64(i8["attn"])
     assert np.abs(got - o).max() <= 2.0 ** -8 * np.abs(o).max()
+
+
+def test_q8_attention_matches_numpy_restatement(orc):
+    """The q8_0 attention against numpy on tiny random caches: dequantise
+    (fp16 scale x int8 code), scores, max-subtracted softmax, weighted sum."""
+    A, n_kvh, n_qh, hd, cap = 2, 1, 3, 128, 12
+    lens, ars = np.array([4, 9], np.int32), np.array([0, 2, 3], np.int32)
+    rng = np.random.default_rng(16)
+    Kq = rng.integers(-127, 128, (A, n_kvh, cap, hd)).astype(np.int8)
+    Vq = rng.integers(-127, 128, (A, n_kvh, cap, hd)).astype(np.int8)
+    Kd = (rng.random((A, n_kvh, cap, hd // 32)) * 0.02 + 0.001).astype(np.float16).view(np.uint16)
+    Vd = (rng.random((A, n_kvh, cap, hd // 32)) * 0.02 + 0.001).astype(np.float16).view(np.uint16)
+    Q = synth.bf16_normal_np(SEED, 31, (3, n_qh, hd))
+    O, _ = orc.decode_attn_q8(Q, Kq, Kd, Vq, Vd, lens, ars, n_qh, n_kvh, hd, cap)
+    K = np.repeat(Kd.view(np.float16).astype(np.float64), 32, axis=3) * Kq
+    V = np.repeat(Vd.view(np.float16).astype(np.float64), 32, axis=3) * Vq
+    q = orc.bf16_array_to_f64(Q)
+    for r in range(3):
+        a = 0 if r < 2 else 1
+        nk = lens[a] + (r - ars[a]) + 1
+        for h in range(n_qh):
+            s = K[a, 0, :nk] @ q[r, h] / np.sqrt(hd)
+            p = np.exp(s - s.max())
+            ref = (p / p.sum()) @ V[a, 0, :nk]
+            assert np.allclose(O[r, h], ref, rtol=1e-12, atol=1e-12)
