@@ -25,6 +25,10 @@ int num_sms();
 // to a 128-byte, 64-byte aligned CUtensorMap.
 int encode_tmap_2d(void *map, const void *base, int elem_bytes, uint64_t cols, uint64_t rows, uint64_t row_stride_bytes,
                    uint32_t box_cols, uint32_t box_rows);
+// 3-D view of a [rows][128] bf16 matrix whose box {8 values, box_rows rows, 16
+// chunks} lands in shared memory as [chunk][row][8 values] (the tcgen05 K-major
+// no-swizzle operand layout): coordinates (0, first row, 0).
+int encode_tmap_kmajor_bf16(void *map, const void *base, uint64_t rows, uint32_t box_rows);
 // Launch with programmatic dependent launch (the kernel may start while the
 // previous kernel in the stream drains; it waits in griddepcontrol.wait).
 template <typename... KArgs, typename... Args>
@@ -319,6 +323,14 @@ __device__ __forceinline__ void tma_load_2d(void *smem_dst, const void *tmap, in
                  ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y),
                  "r"(smem_u32(bar))
                  : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(void *smem_dst, const void *tmap, int x, int y, int z, uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
+        ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+        : "memory");
 }
 
 // ----------------------------------------------------------------- 5th-gen tensor core (tcgen05) + TMEM

@@ -48,6 +48,42 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t
                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+static EncodeTiledFn encode_fn();
+
+int encode_tmap_kmajor_bf16(void *map, const void *base, uint64_t rows, uint32_t box_rows)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn)
+        return fail(QAD_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    // [rows][128] bf16 viewed as (8 values, row, 16-value chunk): a box lands as
+    // [chunk][row][8 values], the K-major no-swizzle core-matrix layout
+    const cuuint64_t dims[3] = {8, rows, 16};
+    const cuuint64_t strides[2] = {256, 16};
+    const cuuint32_t box[3] = {8, box_rows, 16};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(reinterpret_cast<CUtensorMap *>(map), CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<void *>(base),
+                    dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return fail(QAD_ERR_CUDA, "cuTensorMapEncodeTiled (3-D chunk view) failed (%d): rows %llu box %u", (int)r,
+                    (unsigned long long)rows, box_rows);
+    return QAD_OK;
+}
+
+static EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
 int encode_tmap_2d(void *map, const void *base, int elem_bytes, uint64_t cols, uint64_t rows, uint64_t row_stride_bytes,
                    uint32_t box_cols, uint32_t box_rows)
 {

@@ -218,10 +218,11 @@ int launch_prefill_attn_mma(const uint16_t *Q, const uint16_t *Kc, const uint16_
 // CTA = 128 query vectors of one kv-head (the MMA's M), heavy (late) row
 // blocks first. Six warps: four softmax warps (thread = query vector = TMEM
 // lane), a producer warp (TMA) and an MMA warp (one thread issues tcgen05.mma).
-//  * K and V arrive by TMA in 128-key tiles, double-buffered, as 16 boxes of
-//    8 dims x 128 keys: [dim chunk][key][8 dims], which is exactly the
-//    K-major no-swizzle operand layout (8-row x 16-byte core matrices) of B
-//    in S = Q K^T. Q is loaded once in the same layout.
+//  * K and V arrive by TMA in 128-key tiles, double-buffered, one box each
+//    through a 3-D view of the cache (8 dims, key, 16-dim chunk) that lands as
+//    [dim chunk][key][8 dims], exactly the K-major no-swizzle operand layout
+//    (8-row x 16-byte core matrices) of B in S = Q K^T. Q is loaded once in
+//    the same layout.
 //  * S (128 x 128 fp32) and O (128 x 128 fp32) live in TMEM (256 columns).
 //  * A softmax thread reads its S row from TMEM, masks, keeps a running
 //    reference maximum that moves (with a rescale of its O row in TMEM) only
@@ -245,7 +246,7 @@ enum { ST_KV = 1, ST_S = 2, ST_P = 3, ST_PV = 4, ST_DONE = 5 };
 __device__ int g_prefill_status;
 
 struct PfMaps {
-    CUtensorMap k, v;  // [n_kvh * kv_cap][128] bf16, boxes of 8 dims x 128 keys
+    CUtensorMap k, v;  // [n_kvh * kv_cap][128] bf16 as (8 dims, key, dim chunk), boxes of 128 keys
 };
 
 __global__ void __launch_bounds__(pt::THREADS, 1) k_prefill_attn_tc(const __grid_constant__ PfMaps maps, PrefillArgs p)
@@ -320,10 +321,8 @@ __global__ void __launch_bounds__(pt::THREADS, 1) k_prefill_attn_tc(const __grid
                 }
                 mbar_arrive_expect_tx(&kv_full[s], 2 * TB);
                 const int y = kvh * p.kv_cap + j * KT;
-                for (int dc = 0; dc < 16; ++dc) {
-                    tma_load_2d(KS + s * TB + dc * 2048, &maps.k, 8 * dc, y, &kv_full[s]);
-                    tma_load_2d(VS + s * TB + dc * 2048, &maps.v, 8 * dc, y, &kv_full[s]);
-                }
+                tma_load_3d(KS + s * TB, &maps.k, 0, y, 0, &kv_full[s]);  // one box: all 16 dim chunks
+                tma_load_3d(VS + s * TB, &maps.v, 0, y, 0, &kv_full[s]);
             }
             for (int k = max(0, j - 2); k < j; ++k)  // every issued copy lands before teardown
                 if (!mbar_wait(&kv_full[k & 1], (k >> 1) & 1, 20000))
@@ -549,9 +548,9 @@ int launch_prefill_attn(const uint16_t *Q, const uint16_t *Kc, const uint16_t *V
         a.G = n_qh / n_kvh;
         a.scale_log2 = scale * 1.4426950408889634f;
         PfMaps maps;
-        int rc = encode_tmap_2d(&maps.k, Kc, 2, 128, (uint64_t)n_kvh * kv_cap, 256, 8, pt::KT);
+        int rc = encode_tmap_kmajor_bf16(&maps.k, Kc, (uint64_t)n_kvh * kv_cap, pt::KT);
         if (!rc)
-            rc = encode_tmap_2d(&maps.v, Vc, 2, 128, (uint64_t)n_kvh * kv_cap, 256, 8, pt::KT);
+            rc = encode_tmap_kmajor_bf16(&maps.v, Vc, (uint64_t)n_kvh * kv_cap, pt::KT);
         if (rc)
             return rc;
         static bool done[64] = {};
