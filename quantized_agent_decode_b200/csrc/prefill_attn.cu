@@ -215,162 +215,188 @@ int launch_prefill_attn_mma(const uint16_t *Q, const uint16_t *Kc, const uint16_
 
 // ------------------------------------------------------------- tcgen05 form
 //
-// CTA = 128 query vectors of one kv-head (the MMA's M), heavy (late) row
-// blocks first. Six warps: four softmax warps (thread = query vector = TMEM
-// lane), a producer warp (TMA) and an MMA warp (one thread issues tcgen05.mma).
-//  * K and V arrive by TMA in 128-key tiles, double-buffered, one box each
-//    through a 3-D view of the cache (8 dims, key, 16-dim chunk) that lands as
-//    [dim chunk][key][8 dims], exactly the K-major no-swizzle operand layout
-//    (8-row x 16-byte core matrices) of B in S = Q K^T. Q is loaded once in
-//    the same layout.
-//  * S (128 x 128 fp32) and O (128 x 128 fp32) live in TMEM (256 columns).
-//  * A softmax thread reads its S row from TMEM, masks, keeps a running
-//    reference maximum that moves (with a rescale of its O row in TMEM) only
-//    when a score passes it by more than 2^8, and writes P = 2^(s - m) as bf16
-//    into shared memory in the A-operand layout [key chunk][row][8 keys]; the
-//    four warps also transpose the V tile with ldmatrix.trans into the K-major
-//    B layout [key chunk][dim][8 keys] (zeroing keys past the causal end).
-//  * O += P V^T-tile by tcgen05.mma; the last tile's completion releases the
-//    epilogue, which divides by the row sum and stores bf16.
-// Every mbarrier wait is bounded; on a timeout the CTA records a status,
-// stops issuing, waits for its own copies and MMAs, frees TMEM and exits.
+// CTA = two blocks of 128 query vectors (A and B, adjacent rows) of one
+// kv-head, so every K/V tile brought into shared memory serves 256 query
+// vectors (the kernel is bound by re-reading each kv-head's K/V prefix through
+// L2 once per CTA); heavy (late) pairs first. Ten warps: softmax warps 0-3 own
+// block A and 4-7 block B (thread = query vector = TMEM lane; warp w reaches
+// lanes 32 (w & 3)..), a producer warp (TMA) and an MMA warp (one thread
+// issues tcgen05.mma). Keys go in 64-key tiles through a 3-deep ring:
+//  * K and V arrive as one TMA box each through a 3-D view of the cache (8
+//    dims, key, 16-dim chunk) that lands as [dim chunk][key][8 dims], the
+//    K-major no-swizzle operand layout (8-row x 16-byte core matrices) of B in
+//    S = Q K^T. Q is loaded once in the same layout.
+//  * TMEM: S_A, S_B (64 columns each), O_A, O_B (128 each).
+//  * The MMA thread alternates the blocks: S_X(j+1) as soon as block X's
+//    softmax has read S_X(j), then PV_X(j) once it has written P_X(j), so the
+//    tensor core works on one block while the other block's softmax runs.
+//  * A softmax thread keeps a reference maximum that moves (with a rescale of
+//    its O row in TMEM) only when a score passes it by more than 2^8, skips the
+//    masks on tiles below every row's causal limit, and writes P = 2^(s - m) as
+//    bf16 in the A-operand layout [key chunk][row][8 keys]. All eight warps
+//    transpose each V tile with ldmatrix.trans into the K-major B layout [key
+//    chunk][dim][8 keys] (double-buffered; keys past the causal end are zeroed,
+//    so cache slots beyond the chunk never reach a product).
+// Every mbarrier wait is bounded; on a timeout the CTA records a status, stops
+// issuing, waits for its own copies and MMAs, frees TMEM and exits.
 namespace pt {
-constexpr int ROWS = 128, KT = 128, TB = KT * 128 * 2;  // 32 KB operand tiles
-constexpr int SW = 4;                                   // softmax warps
-constexpr int THREADS = 32 * (SW + 2);
+constexpr int ROWS = 128, KT = 64, NS = 3;  // rows per block, keys per tile, K/V ring depth
+constexpr int QB = ROWS * 128 * 2;          // 32 KB: one block's Q
+constexpr int KB = KT * 128 * 2;            // 16 KB: one K or V tile, one Vt, one P
+constexpr int THREADS = 32 * 10;
 constexpr float M_SLACK = 8.f;
-constexpr size_t SMEM = 1024 + 7 * (size_t)TB + 256;  // Q, K[2], V[2], Vt, P, barriers
-enum { ST_KV = 1, ST_S = 2, ST_P = 3, ST_PV = 4, ST_DONE = 5 };
+constexpr size_t SMEM = 128 + 2 * (size_t)QB + (2 * NS + 4) * (size_t)KB + 256;  // Q[2], K/V[NS], Vt[2], P[2]
+enum { ST_KV = 1, ST_S = 2, ST_P = 3, ST_PV = 4, ST_DONE = 5, ST_VT = 6 };
 }  // namespace pt
 
 __device__ int g_prefill_status;
 
 struct PfMaps {
-    CUtensorMap k, v;  // [n_kvh * kv_cap][128] bf16 as (8 dims, key, dim chunk), boxes of 128 keys
+    CUtensorMap k, v;  // [n_kvh * kv_cap][128] bf16 as (8 dims, key, dim chunk), boxes of 64 keys
 };
 
 __global__ void __launch_bounds__(pt::THREADS, 1) k_prefill_attn_tc(const __grid_constant__ PfMaps maps, PrefillArgs p)
 {
     using namespace pt;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    uint8_t *QS = smem, *KS = QS + TB, *VS = KS + 2 * TB, *VT = VS + 2 * TB, *PS = VT + TB;
-    uint64_t *bar = reinterpret_cast<uint64_t *>(PS + TB);
-    uint64_t *kv_full = bar, *kv_free = bar + 2, *s_full = bar + 4, *s_free = bar + 5, *p_full = bar + 6,
-             *pv_done = bar + 7, *done = bar + 8;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + 9);
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~(uintptr_t)127);
+    uint8_t *QS = smem, *KS = QS + 2 * QB, *VS = KS + NS * KB, *VT = VS + NS * KB, *PS = VT + 2 * KB;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(PS + 2 * KB);
+    uint64_t *kv_full = bar, *kv_free = bar + NS, *s_full = bar + 2 * NS, *s_free = s_full + 2, *p_full = s_free + 2,
+             *pv_done = p_full + 2, *vt_full = pv_done + 2, *vt_free = vt_full + 2, *done = vt_free + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 1);
     __shared__ int s_bad;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int kvh = blockIdx.y;
     const int R = p.C * p.G;
-    const int nrb = (R + ROWS - 1) / ROWS;
-    const int v0 = (nrb - 1 - (int)blockIdx.x) * ROWS;  // late row blocks (more keys) first
-    const int j_last = min(p.C - 1, (v0 + ROWS - 1) / p.G);
+    const int npair = (R + 2 * ROWS - 1) / (2 * ROWS);
+    const int v0 = (npair - 1 - (int)blockIdx.x) * 2 * ROWS;  // late pairs (more keys) first
+    const int j_last = min(p.C - 1, (v0 + 2 * ROWS - 1) / p.G);
     const int kend = p.len + j_last + 1;
     const int ntiles = (kend + KT - 1) / KT;
 
     if (threadIdx.x == 0) {
         s_bad = 0;
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < NS; ++i) {
             mbar_init(&kv_full[i], 1);
             mbar_init(&kv_free[i], 1);
         }
-        mbar_init(s_full, 1);
-        mbar_init(s_free, SW * 32);
-        mbar_init(p_full, SW * 32);
-        mbar_init(pv_done, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s_full[i], 1);
+            mbar_init(&s_free[i], 128);
+            mbar_init(&p_full[i], 128);
+            mbar_init(&pv_done[i], 1);
+            mbar_init(&vt_full[i], 256);
+            mbar_init(&vt_free[i], 1);
+        }
         mbar_init(done, 1);
         mbar_fence_init();
     }
-    // Q tile (zero past the chunk) in the A-operand layout [dim chunk][row][8 dims]
-    if (warp < SW) {
+    // Q of both blocks (zero past the chunk), [block][dim chunk][row][8 dims]
+    if (warp < 8) {
         const int r = threadIdx.x, v = v0 + r;
         const bool ok = v < R;
         const int j = ok ? v / p.G : 0, hl = ok ? v - j * p.G : 0;
         const uint16_t *qrow = p.Q + ((size_t)j * p.n_qh + kvh * p.G + hl) * 128;
+        uint8_t *qb = QS + (r >> 7) * QB + (r & 127) * 16;
 #pragma unroll
         for (int dc = 0; dc < 16; ++dc)
-            cp_async16_zfill(QS + dc * 2048 + r * 16, qrow + 8 * dc, ok);
+            cp_async16_zfill(qb + dc * 2048, qrow + 8 * dc, ok);
         cp_async_commit();
         cp_async_wait<0>();
         fence_proxy_async();
     }
-    if (warp == SW + 1) {
-        tmem_alloc(tmem_slot, 256);  // S: columns 0..127, O: 128..255
+    if (warp == 9) {
+        tmem_alloc(tmem_slot, 512);  // S_A 0..63, S_B 64..127, O_A 128..255, O_B 256..383
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = *tmem_slot, tS = tmem, tO = tmem + 128;
+    const uint32_t tmem = *tmem_slot;
     auto fail = [&](int code) {
         atomicExch(&g_prefill_status, code);
         atomicExch(&s_bad, 1);
     };
     auto bad = [&]() { return *(volatile int *)&s_bad != 0; };
 
-    if (warp == SW) {
+    if (warp == 8) {
         // ------------------------------------------------ producer: K and V tiles by TMA
         if (lane == 0) {
             int j = 0;
             for (; j < ntiles && !bad(); ++j) {
-                const int s = j & 1;
-                if (j >= 2 && !mbar_wait(&kv_free[s], ((j >> 1) - 1) & 1)) {
+                const int s = j % NS;
+                if (j >= NS && !mbar_wait(&kv_free[s], ((j / NS) - 1) & 1)) {
                     fail(ST_KV);
                     break;
                 }
-                mbar_arrive_expect_tx(&kv_full[s], 2 * TB);
+                mbar_arrive_expect_tx(&kv_full[s], 2 * KB);
                 const int y = kvh * p.kv_cap + j * KT;
-                tma_load_3d(KS + s * TB, &maps.k, 0, y, 0, &kv_full[s]);  // one box: all 16 dim chunks
-                tma_load_3d(VS + s * TB, &maps.v, 0, y, 0, &kv_full[s]);
+                tma_load_3d(KS + s * KB, &maps.k, 0, y, 0, &kv_full[s]);
+                tma_load_3d(VS + s * KB, &maps.v, 0, y, 0, &kv_full[s]);
             }
-            for (int k = max(0, j - 2); k < j; ++k)  // every issued copy lands before teardown
-                if (!mbar_wait(&kv_full[k & 1], (k >> 1) & 1, 20000))
+            for (int k = max(0, j - NS); k < j; ++k)  // every issued copy lands before teardown
+                if (!mbar_wait(&kv_full[k % NS], (k / NS) & 1, 20000))
                     fail(ST_KV);
         }
-    } else if (warp == SW + 1) {
+    } else if (warp == 9) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc = umma_idesc_bf16(ROWS, KT);  // both products are 128 x 128
+            constexpr uint32_t idesc_s = umma_idesc_bf16(ROWS, KT), idesc_o = umma_idesc_bf16(ROWS, 128);
             bool issued = false;
-            // S_{j+1} is issued as soon as the softmax warps have read S_j, so it runs while they
-            // work on tile j; PV_j follows once they have written P_j and the transposed V_j.
-            auto issue_s = [&](int j) {
-                const uint32_t qb = smem_u32(QS), kb = smem_u32(KS + (j & 1) * TB);
+            auto issue_s = [&](int X, int j) {
+                const uint32_t qb = smem_u32(QS + X * QB), kb = smem_u32(KS + (j % NS) * KB);
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
-                    umma_f16_ss(tS, umma_desc_k_noswz(qb + ks * 4096, 2048, 128),
-                                umma_desc_k_noswz(kb + ks * 4096, 2048, 128), idesc, ks > 0);
-                umma_commit(s_full);
+                    umma_f16_ss(tmem + 64 * X, umma_desc_k_noswz(qb + ks * 4096, 2048, 128),
+                                umma_desc_k_noswz(kb + ks * 2048, 1024, 128), idesc_s, ks > 0);
+                umma_commit(&s_full[X]);
                 issued = true;
+            };
+            auto issue_pv = [&](int X, int j) {
+                const uint32_t pb = smem_u32(PS + X * KB), vb = smem_u32(VT + (j & 1) * KB);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    umma_f16_ss(tmem + 128 + 128 * X, umma_desc_k_noswz(pb + ks * 4096, 2048, 128),
+                                umma_desc_k_noswz(vb + ks * 4096, 2048, 128), idesc_o, (j | ks) != 0);
+                umma_commit(&pv_done[X]);
             };
             if (mbar_wait(&kv_full[0], 0)) {
                 tc_fence_after();
-                issue_s(0);
+                issue_s(0, 0);
+                issue_s(1, 0);
             } else {
                 fail(ST_S);
             }
             for (int j = 0; j < ntiles && !bad(); ++j) {
-                if (j + 1 < ntiles) {
-                    if (!mbar_wait(&kv_full[(j + 1) & 1], ((j + 1) >> 1) & 1) || !mbar_wait(s_free, j & 1)) {
-                        fail(ST_S);
+                const bool more = j + 1 < ntiles;
+                if (more && !mbar_wait(&kv_full[(j + 1) % NS], ((j + 1) / NS) & 1)) {
+                    fail(ST_KV);
+                    break;
+                }
+                bool ok = true;
+                for (int X = 0; X < 2 && ok; ++X) {
+                    if (more) {  // the next S of this block once its softmax has read the current one
+                        if (!mbar_wait(&s_free[X], j & 1)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        issue_s(X, j + 1);
+                    }
+                    if (!mbar_wait(&p_full[X], j & 1) || (X == 0 && !mbar_wait(&vt_full[j & 1], (j >> 1) & 1))) {
+                        ok = false;
                         break;
                     }
                     tc_fence_after();
-                    issue_s(j + 1);
+                    issue_pv(X, j);
                 }
-                if (!mbar_wait(p_full, j & 1)) {
+                if (!ok) {
                     fail(ST_P);
                     break;
                 }
-                tc_fence_after();
-                mbar_arrive(&kv_free[j & 1]);  // S_j is done and the V tile has been transposed
-                const uint32_t pb = smem_u32(PS), vb = smem_u32(VT);
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks)
-                    umma_f16_ss(tO, umma_desc_k_noswz(pb + ks * 4096, 2048, 128),
-                                umma_desc_k_noswz(vb + ks * 4096, 2048, 128), idesc, (j | ks) != 0);
-                umma_commit(pv_done);
+                umma_commit(&vt_free[j & 1]);   // both PV products of tile j read Vt[j & 1]
+                mbar_arrive(&kv_free[j % NS]);  // S_A(j), S_B(j) were read and V_j transposed
             }
             if (issued) {  // every MMA this thread issued completes before TMEM is freed
                 umma_commit(done);
@@ -379,31 +405,64 @@ __global__ void __launch_bounds__(pt::THREADS, 1) k_prefill_attn_tc(const __grid
             }
         }
     } else {
-        // ------------------------------------------------ softmax warps: thread = query vector = TMEM lane
-        const int r = threadIdx.x, v = v0 + r;
+        // ------------------------------------------------ softmax warps
+        const int X = warp >> 2, quarter = warp & 3;
+        const int r = 32 * quarter + lane, v = v0 + X * ROWS + r;
         const bool live = v < R;
         const int jrow = live ? v / p.G : 0;
-        const int lim = live ? p.len + jrow : -1;  // last visible key
-        const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+        const int lim = live ? p.len + jrow : -1;            // last visible key
+        const int lim_blk = min(p.len + (v0 + X * ROWS) / p.G, kend - 1);  // the block's smallest limit
+        const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
+        const uint32_t tS = tmem + 64 * X + lane_off, tO = tmem + 128 + 128 * X + lane_off;
+        uint8_t *PX = PS + X * KB;
         float m = -INFINITY, l = 0.f;
         for (int j = 0; j < ntiles && !bad(); ++j) {
-            if (!__all_sync(0xffffffffu, mbar_wait(s_full, j & 1))) {
+            const int s = j % NS, kb = j * KT;
+            // this warp's share of the V transpose: dim chunks 2w, 2w+1, both 32-key groups
+            if (!__all_sync(0xffffffffu, mbar_wait(&kv_full[s], (j / NS) & 1)) ||
+                (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&vt_free[j & 1], ((j >> 1) - 1) & 1)))) {
+                fail(ST_VT);
+                break;
+            }
+            const uint8_t *Vs = VS + s * KB;
+            uint8_t *Vt = VT + (j & 1) * KB;
+#pragma unroll
+            for (int dd = 0; dd < 2; ++dd) {
+                const int dc = 2 * warp + dd;
+#pragma unroll
+                for (int kg = 0; kg < 2; ++kg) {
+                    uint32_t t4[4];
+                    ldsm_x4_t(t4[0], t4[1], t4[2], t4[3], Vs + dc * 1024 + (32 * kg + lane) * 16);
+#pragma unroll
+                    for (int mi = 0; mi < 4; ++mi) {
+                        const int kc = 4 * kg + mi, key = kb + 8 * kc + 2 * (lane & 3);
+                        uint32_t val = t4[mi];
+                        if (key >= kend)
+                            val = 0u;
+                        else if (key + 1 >= kend)
+                            val &= 0xFFFFu;
+                        *reinterpret_cast<uint32_t *>(Vt + kc * 2048 + (8 * dc + (lane >> 2)) * 16 + (lane & 3) * 4) =
+                            val;
+                    }
+                }
+            }
+            fence_proxy_async();
+            mbar_arrive(&vt_full[j & 1]);
+            // the S row of this block
+            if (!__all_sync(0xffffffffu, mbar_wait(&s_full[X], j & 1))) {
                 fail(ST_S);
                 break;
             }
             tc_fence_after();
             float x[KT];
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc)
-                tmem_ld_x32(tS + lane_off + 32 * cc, reinterpret_cast<uint32_t *>(x + 32 * cc));
+            for (int cc = 0; cc < 2; ++cc)
+                tmem_ld_x32(tS + 32 * cc, reinterpret_cast<uint32_t *>(x + 32 * cc));
             tmem_wait_ld();
             tc_fence_before();
-            mbar_arrive(s_free);
-            const int kb = j * KT;
-            // Tiles wholly below every row's causal limit (the CTA's first row sees the
-            // fewest keys) need no mask: the row maximum is taken on the raw scores and
-            // the scale folds into one fused multiply-add per probability.
-            const bool interior = kb + KT - 1 <= p.len + v0 / p.G;
+            mbar_arrive(&s_free[X]);
+            // tiles below every row's causal limit: no mask, maximum on raw scores
+            const bool interior = kb + KT - 1 <= lim_blk;
             float mx = -INFINITY;
             if (interior) {
 #pragma unroll
@@ -418,8 +477,6 @@ __global__ void __launch_bounds__(pt::THREADS, 1) k_prefill_attn_tc(const __grid
                     mx = fmaxf(mx, x[i]);
                 }
             }
-            // the new reference maximum and P in registers first: this overlaps the
-            // previous tile's PV product, which only the writes below must wait for
             const bool resc = __any_sync(0xffffffffu, mx > m + M_SLACK);
             float corr = 1.f;
             if (resc) {
@@ -428,7 +485,7 @@ __global__ void __launch_bounds__(pt::THREADS, 1) k_prefill_attn_tc(const __grid
                 m = mn;
             }
             const bool none = m == -INFINITY;
-            const float sc = interior ? p.scale_log2 : 1.f;  // scores still unscaled on interior tiles
+            const float sc = interior ? p.scale_log2 : 1.f;
             const float nm = none ? 0.f : -m;
             uint32_t pw[KT / 2];
             float psum = 0.f;
@@ -440,63 +497,35 @@ __global__ void __launch_bounds__(pt::THREADS, 1) k_prefill_attn_tc(const __grid
                 pw[i] = pack_bf162(p0, p1);
             }
             l = l * corr + psum;
-            // the previous PV product must be done before O is rescaled or P / Vt rewritten
-            if (j > 0 && !__all_sync(0xffffffffu, mbar_wait(pv_done, (j - 1) & 1))) {
+            // this block's previous PV product must be done before O is rescaled or P rewritten
+            if (j > 0 && !__all_sync(0xffffffffu, mbar_wait(&pv_done[X], (j - 1) & 1))) {
                 fail(ST_PV);
                 break;
             }
             tc_fence_after();
-            if (resc && j > 0) {  // O holds earlier tiles: scale this row
+            if (resc && j > 0) {
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc) {
                     uint32_t ov[32];
-                    tmem_ld_x32(tO + lane_off + 32 * cc, ov);
+                    tmem_ld_x32(tO + 32 * cc, ov);
                     tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 32; ++i)
                         ov[i] = __float_as_uint(__uint_as_float(ov[i]) * corr);
-                    tmem_st_x32(tO + lane_off + 32 * cc, ov);
+                    tmem_st_x32(tO + 32 * cc, ov);
                 }
                 tmem_wait_st();
             }
-            // P as bf16 into [key chunk][row][8 keys]
 #pragma unroll
-            for (int kc = 0; kc < 16; ++kc)
-                *reinterpret_cast<uint4 *>(PS + kc * 2048 + r * 16) =
+            for (int kc = 0; kc < 8; ++kc)
+                *reinterpret_cast<uint4 *>(PX + kc * 2048 + r * 16) =
                     make_uint4(pw[4 * kc], pw[4 * kc + 1], pw[4 * kc + 2], pw[4 * kc + 3]);
-            // V tile -> Vt [key chunk][dim][8 keys]: this warp's dim chunks 4w .. 4w+3, 32 keys per ldmatrix
-            const int s = j & 1;
-            if (!__all_sync(0xffffffffu, mbar_wait(&kv_full[s], (j >> 1) & 1))) {
-                fail(ST_KV);
-                break;
-            }
-            const uint8_t *Vs = VS + s * TB;
-#pragma unroll
-            for (int dd = 0; dd < 4; ++dd) {
-                const int dc = 4 * warp + dd;
-#pragma unroll
-                for (int kg = 0; kg < 4; ++kg) {
-                    uint32_t t4[4];
-                    ldsm_x4_t(t4[0], t4[1], t4[2], t4[3], Vs + dc * 2048 + (32 * kg + lane) * 16);
-#pragma unroll
-                    for (int mi = 0; mi < 4; ++mi) {
-                        const int kc = 4 * kg + mi, key = kb + 8 * kc + 2 * (lane & 3);
-                        uint32_t val = t4[mi];
-                        if (key >= kend)
-                            val = 0u;
-                        else if (key + 1 >= kend)
-                            val &= 0xFFFFu;
-                        *reinterpret_cast<uint32_t *>(VT + kc * 2048 + (8 * dc + (lane >> 2)) * 16 + (lane & 3) * 4) =
-                            val;
-                    }
-                }
-            }
             fence_proxy_async();
             tc_fence_before();
-            mbar_arrive(p_full);
+            mbar_arrive(&p_full[X]);
         }
         // epilogue: O / l -> bf16
-        if (!bad() && __all_sync(0xffffffffu, mbar_wait(pv_done, (ntiles - 1) & 1))) {
+        if (!bad() && __all_sync(0xffffffffu, mbar_wait(&pv_done[X], (ntiles - 1) & 1))) {
             tc_fence_after();
             const int hl = live ? v - jrow * p.G : 0;
             uint16_t *orow = p.O + ((size_t)jrow * p.n_qh + kvh * p.G + hl) * 128;
@@ -504,7 +533,7 @@ __global__ void __launch_bounds__(pt::THREADS, 1) k_prefill_attn_tc(const __grid
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc) {
                 uint32_t ov[32];
-                tmem_ld_x32(tO + lane_off + 32 * cc, ov);
+                tmem_ld_x32(tO + 32 * cc, ov);
                 tmem_wait_ld();
                 if (live)
 #pragma unroll
@@ -521,9 +550,9 @@ __global__ void __launch_bounds__(pt::THREADS, 1) k_prefill_attn_tc(const __grid
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == SW + 1) {
+    if (warp == 9) {
         tc_fence_after();
-        tmem_dealloc(tmem, 256);
+        tmem_dealloc(tmem, 512);
     }
 }
 
@@ -565,7 +594,7 @@ int launch_prefill_attn(const uint16_t *Q, const uint16_t *Kc, const uint16_t *V
             if (dev >= 0 && dev < 64)
                 done[dev] = true;
         }
-        dim3 grid((C * a.G + pt::ROWS - 1) / pt::ROWS, n_kvh);
+        dim3 grid((C * a.G + 2 * pt::ROWS - 1) / (2 * pt::ROWS), n_kvh);
         k_prefill_attn_tc<<<grid, pt::THREADS, pt::SMEM, s>>>(maps, a);
         return cuda_check(cudaGetLastError(), "prefill attn launch");
     }
