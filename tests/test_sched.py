@@ -115,3 +115,32 @@ def test_commit_accepts_drafts_and_rejects_bad_plans(q):
     assert s.agents[1].len == 300 and s.agents[1].prompt_left == 0
     with pytest.raises(q.QadError):
         s.commit([0, 1], 0, 1)   # agent 0 has no prompt left to chunk
+
+
+def test_prompt_lookup_drafts_pay_off_on_repetitive_streams(q, orc):
+    """A toy agent whose true continuation repeats its context (as code edits
+    often do): prompt-lookup drafts are accepted by the greedy rule (oracle),
+    so each scheduled step commits more than one token."""
+    rng = np.random.default_rng(7)
+    base = rng.integers(0, 1000, 40).tolist()
+    truth = base * 6                       # the stream the agent will produce
+    ctx = truth[:50]                       # already cached (prompt + earlier output)
+    s = q.Scheduler(1, n_draft=2, max_decode_rows=3)
+    s.agents[0].len, s.agents[0].prompt_left, s.agents[0].active = len(ctx), 0, 1
+    steps = 0
+    while len(ctx) < 200:
+        drafts = q.prompt_lookup(ctx, n_draft=2)
+        s.agents[0].drafts = len(drafts)
+        rows, ca, cr = s.plan()
+        n = rows[0]
+        row_tokens = [ctx[-1]] + drafts[:n - 1]           # inputs of the agent's rows
+        pos = len(ctx)
+        row_argmax = [truth[pos + k] for k in range(n)]   # what the model predicts after each row
+        ars = np.array([0, n], np.int32)
+        lens2, out, acc = orc.accept_greedy(row_argmax, row_tokens, ars, [s.agents[0].len])
+        s.commit(rows, ca, cr, n_accept=[int(acc[0])])
+        ctx += [int(t) for t in out if t >= 0]
+        assert s.agents[0].len == len(ctx) == int(lens2[0])
+        steps += 1
+    assert ctx[:200] == truth[:len(ctx)][:200]
+    assert (len(ctx) - 50) / steps > 2.5  # close to 3 tokens per step once the pattern repeats
