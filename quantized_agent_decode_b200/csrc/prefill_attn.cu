@@ -8,7 +8,10 @@
 // the agent's own KV cache. It is the decode attention's definition with
 // C ~ 2048 rows instead of 3.
 //
-// Design (sm_100a warp MMAs, flash-attention style):
+// Two kernels. The default (k_prefill_attn_tc, described before it) runs the
+// products on tcgen05 with S and O in TMEM. The warp-MMA form below
+// (k_prefill_attn, selected at build time with QAD_PREFILL_TC=0) is the
+// flash-attention-style predecessor:
 //  * CTA = 64 query vectors of one kv-head (vector v = row j * G + local head,
 //    so the G heads sharing a kv-head are adjacent and one causal limit covers
 //    whole rows), 4 warps of 16 vectors. Q stays in registers as the A
@@ -16,9 +19,10 @@
 //  * K and V stream through a double-buffered shared-memory ring in 64-key
 //    tiles (cp.async, 16-byte chunks XOR-swizzled so ldmatrix is conflict
 //    free); K feeds S via ldmatrix, V feeds O += P V via ldmatrix.trans.
-//  * Online softmax in fp32 (exp2 with the scale folded in); P is rounded to
-//    bf16 once and used straight from the S accumulator registers as the A
-//    operand of the PV product.
+//  * Online softmax in fp32 (exp2 with the scale folded in) against a
+//    reference maximum that moves only when a score passes it by more than
+//    2^8; P is rounded to bf16 once and used straight from the S accumulator
+//    registers as the A operand of the PV product.
 #include <cuda.h>
 
 #include "attn.cuh"
