@@ -157,6 +157,49 @@ __device__ __forceinline__ uint32_t pack_bf162(float lo, float hi)
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
     return r;
 }
+// Packed fp32 pairs (sm_100 f32x2 instructions): d = a * b + c, d = a + b, d = a * b, per lane of the pair.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c)
+{
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b)
+{
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b)
+{
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+// Byte i (0..3) of v as the fp32 value 2^23 + byte (the byte lands in the low
+// mantissa bits of 0x4B000000); subtracting 2^23 gives the byte exactly.
+__device__ __forceinline__ float byte_f23(uint32_t v, int i)
+{
+    return __uint_as_float(prmt(v, 0x4B000000u, 0x7440u | (uint32_t)i));
+}
+// A bf16 pair as an fp16 pair (round to nearest; exact for values in fp16's
+// normal range, since bf16 carries 8 significant bits and fp16 11).
+__device__ __forceinline__ uint32_t bf162_to_h2(uint32_t v)
+{
+    return pack_half2(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
+}
 __device__ __forceinline__ float half_lo(uint32_t v) { return __half2float(__ushort_as_half((unsigned short)(v & 0xFFFF))); }
 __device__ __forceinline__ float half_hi(uint32_t v) { return __half2float(__ushort_as_half((unsigned short)(v >> 16))); }
 __device__ __forceinline__ float bf16_to_f(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
@@ -281,6 +324,19 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32
     for (uint32_t i = 0; i < limit; ++i)
         if (mbar_try_wait(bar, parity))
             return true;
+    return false;
+}
+// Bounded wait that sleeps ~sleep_ns between polls, so a waiting warp gives its
+// issue slots to the warps doing the work (a try_wait that returns at once
+// would otherwise be re-issued in a tight loop). Gives up after ~2 s.
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t sleep_ns)
+{
+    const uint32_t limit = 2000000000u / (sleep_ns ? sleep_ns : 1u);
+    for (uint32_t i = 0; i < limit; ++i) {
+        if (mbar_try_wait(bar, parity, 0))
+            return true;
+        __nanosleep(sleep_ns);
+    }
     return false;
 }
 // global -> shared bulk copy completing on an mbarrier (bytes % 16 == 0, both addresses 16-byte aligned)
@@ -428,6 +484,28 @@ __device__ __forceinline__ void umma_f16_ss(uint32_t d_tmem, uint64_t a_desc, ui
     asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
                  "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
                  ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+                 : "memory");
+}
+// The same two products issued from a whole warp: every lane runs the issue loop
+// with the same (warp-uniform) operands and one lane, chosen by elect.sync,
+// issues. Keeping the warp converged lets the operands live in uniform
+// registers, so a stream of MMAs issues at a fraction of the instructions.
+__device__ __forceinline__ void umma_f16_ts_warp(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                                 uint32_t accumulate)
+{
+    const uint32_t z = 0;
+    asm volatile("{\n\t.reg .pred p, e;\n\t.reg .b32 r;\n\telect.sync r|e, 0xffffffff;\n\t"
+                 "setp.ne.b32 p, %4, 0;\n\t"
+                 "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %5, %5, %5}, p;\n\t}"
+                 ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(z)
+                 : "memory");
+}
+// tcgen05.commit from a whole warp (one elected lane commits).
+__device__ __forceinline__ void umma_commit_warp(uint64_t *bar)
+{
+    asm volatile("{\n\t.reg .pred e;\n\t.reg .b32 r;\n\telect.sync r|e, 0xffffffff;\n\t"
+                 "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}"
+                 ::"r"(smem_u32(bar))
                  : "memory");
 }
 // Generic-proxy writes to shared memory made visible to the async proxy (tensor core, TMA).

@@ -18,9 +18,9 @@
 //    x 64 k fp16, already in core-matrix order) by one bulk copy per k-step.
 //  * Eight dequant warps turn each 64-wide k-step of the raw blocks into fp16
 //    weights in core-matrix order (one weight row per thread, one 32-wide half
-//    of the k-step per warp): w = fp16(d*sc) * q - fp16(dmin*m) for Q4_K (q
-//    exact in fp16, one fused multiply-add per pair), w = fp16(d*sc) * (q - 32)
-//    for Q6_K.
+//    of the k-step per warp). Each weight (d*sc*q - dmin*m for Q4_K,
+//    d*sc*(q-32) for Q6_K) is formed in fp32 with packed f32x2 operations and
+//    rounded to fp16 once, so an operand is within 2^-11 of its weight.
 //  * Two accumulators (512 TMEM columns): four epilogue warps read tile t out
 //    of TMEM, apply the activation row scales and store Y while the MMAs of
 //    tile t + 1 run.
@@ -132,16 +132,13 @@ __global__ void __launch_bounds__(256) k_prep_dense(const uint16_t *__restrict__
     }
 }
 
-// fp16 pair (v, v)
-__device__ __forceinline__ uint32_t h2dup(float v)
-{
-    const uint32_t h = __half_as_ushort(__float2half_rn(v));
-    return h | (h << 16);
-}
-
 // 32 fp16 weights of row n for k-step kk (0..3) of a Q4_K block: half 0 = the
 // low nibbles (k 0..31 of the step, chunks 0..3), half 1 = the high nibbles
 // (k 32..63, chunks 4..7); chunk c of the A stage sits at c * 2048 + n * 16.
+// Each weight w = d*sc*q - dmin*m is formed in fp32 by one fused multiply-add
+// (q, d*sc and dmin*m are exact there, so it rounds once, by at most 2^-24 |w|)
+// and rounded to fp16 once: the operand differs from w by at most
+// (2^-11 + 2^-24) |w|, or 2^-25 in fp16's subnormal range.
 __device__ __forceinline__ void dequant_q4(const uint8_t *blk, int kk, int half, uint8_t *A, int n)
 {
     const uint4 h = lds_v4(blk);
@@ -157,9 +154,9 @@ __device__ __forceinline__ void dequant_q4(const uint8_t *blk, int kk, int half,
         sc = (float)((byte(j + 4) & 0xF) | ((byte(j - 4) >> 6) << 4));
         mn = (float)((byte(j + 4) >> 4) | ((byte(j) >> 6) << 4));
     }
-    // the high nibble enters as 16 q, so its scale is d*sc/16
-    const uint32_t av = h2dup(half ? d * sc * 0.0625f : d * sc), bv = h2dup(-dmin * mn);
-    const uint32_t mask = half ? 0x00F000F0u : 0x000F000Fu;
+    const float ds = d * sc, dm = -dmin * mn;  // exact in fp32 (at most 17 significant bits)
+    const float2 DS = make_float2(ds, ds), DM = make_float2(dm, dm);
+    const float2 OFF = make_float2(-8388608.f, -8388608.f);  // -2^23
     const uint4 q0 = lds_v4(blk + 16 + 32 * kk), q1 = lds_v4(blk + 32 + 32 * kk);
     const uint32_t qw[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
 #pragma unroll
@@ -168,28 +165,35 @@ __device__ __forceinline__ void dequant_q4(const uint8_t *blk, int kk, int half,
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
             const uint32_t w = qw[2 * c + u];
-            const uint32_t t01 = prmt(w, w, 0x1100u), t23 = prmt(w, w, 0x3322u);
-            // (1024 + q) -> q exact -> a*q + b
-            o[2 * u] = hfma2(hsub2(and_or(t01, mask, H2_1024), H2_1024), av, bv);
-            o[2 * u + 1] = hfma2(hsub2(and_or(t23, mask, H2_1024), H2_1024), av, bv);
+            const uint32_t v = (half ? (w >> 4) : w) & 0x0F0F0F0Fu;  // four 4-bit quants as bytes
+#pragma unroll
+            for (int pr = 0; pr < 2; ++pr) {
+                const float2 q = fadd2(make_float2(byte_f23(v, 2 * pr), byte_f23(v, 2 * pr + 1)), OFF);
+                const float2 wv = ffma2(q, DS, DM);
+                o[2 * u + pr] = pack_half2(wv.x, wv.y);
+            }
         }
         *reinterpret_cast<uint4 *>(A + (4 * half + c) * 2048 + n * 16) = make_uint4(o[0], o[1], o[2], o[3]);
     }
 }
 
-constexpr uint32_t H2_1056D = 0x64206420u;  // 1056.0
-
 // Q6_K-like (packed plane A, d from the D tile): k-step kk = half h, group sel;
 // `part` 0 writes k 0..31 of the step (chunks 0..3), part 1 k 32..63.
+// w = d*sc*(q-32) is exact in fp32 (at most 18 + 5 significant bits) and is
+// rounded to fp16 once (at most 2^-11 |w|, or 2^-25 in the subnormal range).
 __device__ __forceinline__ void dequant_q6(const uint8_t *blk, float d, int kk, int part, uint8_t *A, int n)
 {
     const int h = kk >> 1, sel = kk & 1;
     const uint2 sw = lds_v2(blk + 192 + 8 * h);
-    const int8_t *scb = reinterpret_cast<const int8_t *>(&sw);
-    uint32_t a[2];
+    float2 DS[2];
 #pragma unroll
-    for (int g = 0; g < 2; ++g)  // 16-weight groups of the part: scales 4 sel + 2 part + g
-        a[g] = h2dup(d * (float)scb[4 * sel + 2 * part + g]);
+    for (int g = 0; g < 2; ++g) {  // 16-weight groups of the part: scales 4 sel + 2 part + g
+        const int i = 2 * part + g;  // byte i of word sel (int8)
+        const int scv = (int)(int8_t)(uint8_t)((sel ? sw.y : sw.x) >> (8 * i));
+        const float ds = d * (float)scv;  // exact (at most 18 significant bits)
+        DS[g] = make_float2(ds, ds);
+    }
+    const float2 OFF = make_float2(-8388640.f, -8388640.f);  // -(2^23 + 32): byte_f23(q) + OFF = q - 32
     {  // part 0: k 0..31 (ql[l], qh bits 4sel); part 1: k 32..63 (ql[l+32], qh bits 4sel+2)
         const uint8_t *ql = blk + 64 * h + 32 * part;
         const uint8_t *qh = blk + 128 + 32 * h;
@@ -202,10 +206,12 @@ __device__ __forceinline__ void dequant_q6(const uint8_t *blk, float d, int kk, 
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
                 const uint32_t q = ((lw[u] >> (4 * sel)) & 0x0F0F0F0Fu) | (((hw[u] >> sh) & 0x03030303u) << 4);
-                const uint32_t t01 = prmt(q, q, 0x1100u), t23 = prmt(q, q, 0x3322u);
-                const uint32_t sc = a[c2 >> 1];
-                o[2 * u] = hmul2(hsub2(and_or(t01, 0x003F003Fu, H2_1024), H2_1056D), sc);
-                o[2 * u + 1] = hmul2(hsub2(and_or(t23, 0x003F003Fu, H2_1024), H2_1056D), sc);
+#pragma unroll
+                for (int pr = 0; pr < 2; ++pr) {
+                    const float2 qm = fadd2(make_float2(byte_f23(q, 2 * pr), byte_f23(q, 2 * pr + 1)), OFF);
+                    const float2 wv = fmul2(qm, DS[c2 >> 1]);
+                    o[2 * u + pr] = pack_half2(wv.x, wv.y);
+                }
             }
             *reinterpret_cast<uint4 *>(A + (4 * part + c2) * 2048 + n * 16) = make_uint4(o[0], o[1], o[2], o[3]);
         }

@@ -10,31 +10,29 @@
 // multiply-accumulate hidden under it.
 //
 // Design (sm_100a):
-//  * A producer warp streams each unit (a tile of weight rows x one 256-wide
-//    block) into a ring of shared-memory stages with one 2-D tensor-map load
-//    (TMA), plus one bulk copy of that block's activation record; each stage
-//    completes on an mbarrier. Every quantized byte leaves HBM exactly once.
-//  * The block is decoded in registers into fp16 tensor-core operands that are
-//    EXACT: for Q4_K, A = sc_j * q (<= 945) and the mins enter through a second
-//    small MMA against per-sub-block activation sums; for Q6_K, A = sc * (q-32)
-//    (|.| <= 4096). The fp16 values come from the "1024 + q" exponent trick (OR
-//    of the nibble into the mantissa of 1024.0) followed by one fused
-//    multiply-add that applies the scale.
-//  * M = 12 rows need ~16 multiply-adds per weight, four times what the FP32
-//    pipes deliver at the HBM rate, so the product runs on the tensor cores as
-//    m16n8k16 warp MMAs (weights = A, the 16 padded activation rows = B). Each
-//    consumer warp owns 32 weight rows (two m16 tiles), so every activation
-//    fragment read from shared memory feeds four MMAs.
-//  * The activations are prepared once per GEMM (k_prep) into fp16 B
-//    fragments in exactly the register order each lane consumes, with a
-//    power-of-two scale per (row, block) so fp16's range always holds them.
+//  * A prep kernel forms the activation rows exactly as the step defines them
+//    (the bf16 input, RMSNorm of the residual, silu(gate)*up or the merged
+//    attention output) and writes, per 256-wide block, a record holding them as
+//    fp16 of x * 2^e(r,b) in the tensor core's operand layout, with a power of
+//    two per (row, block) so every bf16 value converts exactly.
+//  * The GEMM (k_qgemm_tc, below) streams each unit (128 weight rows x one
+//    block) by TMA into a ring of shared-memory stages; every quantized byte
+//    leaves HBM exactly once. Sixteen decode warps turn a unit into EXACT fp16
+//    operands in tensor memory: for Q4_K, A = sc_j * q (<= 945) with the mins
+//    entering through one more small product against per-sub-block activation
+//    sums; for Q6_K, A = sc * (q - 32). The fp16 values come from the
+//    "1024 + q" exponent trick (OR of the nibble into the mantissa of 1024.0)
+//    and one fused multiply-add that applies the scale.
+//  * One thread issues tcgen05.mma (M = 128 weight rows, N = 16 activation
+//    rows, K = 16) with A in tensor memory and the record in shared memory, so
+//    the multiply costs the decoding warps no instructions; four epilogue warps
+//    apply the block's d, dmin and the row scales.
 //  * Work is split stream-K style over a persistent grid (one CTA per SM):
-//    each CTA takes a contiguous run of units, its consumer groups take them
-//    round-robin and accumulate in registers, adding partial tile sums into Y
-//    with fp32 atomics when a group's run leaves a tile.
-//  * Programmatic dependent launch: the first units' weights are requested
-//    before griddepcontrol.wait, so the weight stream starts while the
-//    producer of the activations is still finishing.
+//    each CTA takes a contiguous run of units and adds a tile's partial sums
+//    into Y with fp32 atomics when its run leaves the tile.
+//  * Programmatic dependent launch: the weights are requested before
+//    griddepcontrol.wait, so the weight stream starts while the producer of the
+//    activations is still finishing.
 #include <cuda.h>
 
 #include <mutex>
@@ -48,23 +46,12 @@ namespace qad {
 // read and cleared by qad_device_status().
 __device__ int g_gemm_status;
 
-// ------------------------------------------------------------- fragment layout
-// Activation rows r = 8*nt + g (nt < NT, g < 8); blocks b < nblk; k-steps
-// s < 16; lane quad c < 4. One record per block (rec_bytes), so a GEMM unit
-// fetches its block's operand with one bulk copy and a warp's 32 lanes read 32
-// consecutive entries.
-//   X (uint2 units): [s][g][c][nt] = {b0, b1}: the two B registers of the
-//       m16n8k16 fragment: b0 = (x[k0], x[k0+2]), b1 = (x[k0+1], x[k0+3]) with
-//       k0 = 256 b + frag_k0(s, c), as fp16 of x * 2^e(r,b).
-//   S (uint2 units): [g][c][nt] = {(Shi_2c, Shi_2c+1), (Slo_2c, Slo_2c+1)}
-//       with S_j the sum of the 32 fp16 activations of Q4_K sub-block j split
-//       into two fp16 parts (Q4_K only).
-//   RS: 16 floats, 2^-e(r,b) (0 for rows >= M).
+// ------------------------------------------------------------- operand records
 // e(r,b) puts the block's largest |x| in [512, 1024): fp16 holds every bf16
 // value of the block exactly unless it is 2^24 times smaller than that max.
 static inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-size_t frag_bytes(int K, int nt) { return align256((size_t)(K / 256) * rec_bytes(4, nt)); }
+size_t frag_bytes(int K, int) { return align256((size_t)(K / 256) * REC_BYTES); }
 
 FragBuf frag_carve(void *ws, int, int)
 {
@@ -72,35 +59,6 @@ FragBuf frag_carve(void *ws, int, int)
     f.rec = (uint8_t *)ws;
     return f;
 }
-
-// Which activation column feeds logical k-slot (s, c). The weight-side decode
-// below produces, for lane quad c and k-step s, the weights at within-block
-// positions k0, k0+2 (first B register) and k0+1, k0+3 (second).
-__host__ __device__ constexpr int frag_k0(int fmt, int s, int c)
-{
-    // Q4_K: quant bytes 32c..32c+31: word s>>1, low (s even) or high (s odd) nibbles.
-    // Q6_K: half c>>1, l-range 16*(c&1); word s>>2; s&3 selects the 32-weight quarter.
-    return fmt == 4 ? 64 * c + 4 * (s >> 1) + 32 * (s & 1) : 128 * (c >> 1) + 16 * (c & 1) + 4 * (s >> 2) + 32 * (s & 3);
-}
-
-// The inverse: the slot (s, c) whose k0 is 4t (t < 64), so thread t of a block
-// reads columns 4t..4t+3 and its loads coalesce. For Q4_K, t >> 3 is the
-// sub-block 2c + (s & 1).
-__host__ __device__ constexpr int slot_s(int fmt, int t)
-{
-    return fmt == 4 ? 2 * (t & 7) + ((t >> 3) & 1) : 4 * (t & 3) + ((t & 31) >> 3);
-}
-__host__ __device__ constexpr int slot_c(int fmt, int t) { return fmt == 4 ? t >> 4 : 2 * (t >> 5) + ((t >> 2) & 1); }
-
-constexpr bool slot_maps_consistent()
-{
-    for (int fmt = 4; fmt <= 6; fmt += 2)
-        for (int t = 0; t < 64; ++t)
-            if (frag_k0(fmt, slot_s(fmt, t), slot_c(fmt, t)) != 4 * t || slot_s(fmt, t) > 15 || slot_c(fmt, t) > 3)
-                return false;
-    return true;
-}
-static_assert(slot_maps_consistent(), "fragment slot maps must invert frag_k0");
 
 // ------------------------------------------------------------- prep kernel
 
@@ -145,12 +103,12 @@ __device__ __forceinline__ void zero_next_output(const PrepSrc &S)
     }
 }
 
-// Grid (ceil(nblk / 4), 8*NT): CTA (x, r) forms row r's blocks 4x..4x+3, one
+// Grid (ceil(nblk / 4), 16): CTA (x, r) forms row r's blocks 4x..4x+3, one
 // 64-thread quarter per block, thread t of a quarter owning columns 4t..4t+3.
 // The values are formed exactly as the GEMM must see them (bf16: the input
 // itself, RMSNorm of the fp32 residual, silu(gate)*up, or the merged
-// attention output), then scaled per (row, block) into fp16 fragments.
-template <int FMT, int NT>
+// attention output), then scaled per (row, block) into the fp16 record.
+template <int FMT>
 __global__ void __launch_bounds__(256) k_prep(PrepArgs a)
 {
     __shared__ float red[8];
@@ -289,12 +247,11 @@ __global__ void __launch_bounds__(256) k_prep(PrepArgs a)
         return;
     }
     const float sc = ldexpf(1.f, e);
-    uint8_t *rec = a.fb.rec + (size_t)b * rec_bytes(FMT, NT);
-    const int g = r & 7, nt = r >> 3;
-    const int s = slot_s(FMT, t), c = slot_c(FMT, t);
+    uint8_t *rec = a.fb.rec + (size_t)b * REC_BYTES;
     const float h0 = round_half(x[0] * sc), h1 = round_half(x[1] * sc), h2 = round_half(x[2] * sc),
                 h3 = round_half(x[3] * sc);
-    reinterpret_cast<uint2 *>(rec)[((s * 8 + g) * 4 + c) * NT + nt] =
+    // MMA positions 4t .. 4t+3 (k chunk t / 2, half t & 1 of the row's 16 bytes) hold columns 4t + {0,2,1,3}
+    *reinterpret_cast<uint2 *>(rec + (t >> 1) * 256 + r * 16 + (t & 1) * 8) =
         make_uint2(pack_half2(h0, h2), pack_half2(h1, h3));
     if (FMT == 4) {
         // sub-block j = t >> 3 is the 8 lanes t & ~7 .. +7 (fp32 sum of its fp16 values)
@@ -304,78 +261,86 @@ __global__ void __launch_bounds__(256) k_prep(PrepArgs a)
         sj += __shfl_xor_sync(0xffffffffu, sj, 4);
         const float sj1 = __shfl_down_sync(0xffffffffu, sj, 8);  // sub-block j + 1
         if ((t & 15) == 0) {
+            const int j = t >> 3;  // even
             const float hi0 = round_half(sj), hi1 = round_half(sj1);
-            reinterpret_cast<uint2 *>(rec + 4096 * NT)[(g * 4 + c) * NT + nt] =
-                make_uint2(pack_half2(hi0, hi1), pack_half2(sj - hi0, sj1 - hi1));
+            *reinterpret_cast<uint32_t *>(rec + REC_S_OFF + r * 16 + 2 * j) = pack_half2(hi0, hi1);
+            *reinterpret_cast<uint32_t *>(rec + REC_S_OFF + 256 + r * 16 + 2 * j) = pack_half2(sj - hi0, sj1 - hi1);
         }
     }
     if (t == 0)
-        reinterpret_cast<float *>(rec + rec_bytes(FMT, NT) - 64)[r] = live ? ldexpf(1.f, -e) : 0.f;
+        reinterpret_cast<float *>(rec + REC_RS_OFF)[r] = live ? ldexpf(1.f, -e) : 0.f;
     zero_next_output(S);  // last: the next GEMM's output is not read by this kernel
     trace_end(a.trace);
 }
 
-// ------------------------------------------------------------- GEMM kernels
+// ------------------------------------------------------------- GEMM kernel (tcgen05)
 //
-// One CTA per SM: 8 consumer warps + 1 producer warp. A CTA unit is a tile of
-// 128 weight rows x one 256-wide block. Units are numbered tile-major with the
-// block fastest, and each CTA takes a contiguous run of them (stream-K). For
-// each unit the producer issues ONE 2-D tensor-map load (TMA) of the 128
-// row-blocks (plus the d plane for Q6_K) and one bulk copy of the block's
-// activation fragments into a ring of shared-memory stages, completing on a
-// "full" mbarrier; the consumer warps (16 rows each) decode their rows from
-// shared memory, run the MMAs and release the stage on an "empty" mbarrier.
-// Every wait is bounded: on timeout the warp records a status code and returns.
+// One CTA per SM, persistent over a contiguous run of units (stream-K); a unit
+// is a tile of 128 weight rows x one 256-wide block. The weights of a unit are
+// decoded once, in registers, into exact fp16 tensor-core operands that go
+// straight to tensor memory, and the 5th-generation tensor core multiplies
+// them with the block's 16-row activation operand:
 //
-// Q6_K-like weights use the packed device layout of qad_q6k_pack(): plane A
-// [N][nblk][208] (ql, qh, int8 scales: the first 208 bytes of each GGUF block,
-// so every field is 16-byte aligned) followed by plane D [N][ceil8(nblk)] fp16
-// d. 210-byte GGUF blocks cannot be addressed by TMA (16-byte start rule).
+//   weight producer (1 thread)  TMA: 128 rows x one block -> raw stage   [SR-deep ring]
+//   record producer (1 thread)  bulk copy: the block's operand record    [SB-deep ring]
+//   16 decode warps             raw stage -> A = sc*q (Q4_K) or sc*(q-32) (Q6_K) as fp16
+//                               in TMEM: two groups of 8 take alternate units; warp w
+//                               covers lane quarter w & 3 (thread = weight row = TMEM
+//                               lane) and k half (w >> 2) & 1       [2 A buffers x 2 halves]
+//   2 MMA warps                 per unit 16 x tcgen05.mma M=128 N=16 K=16 (A from TMEM,
+//                               B from shared memory) into the unit's accumulator, plus
+//                               for Q4_K one more for the mins (A = m_j, B = sub-block
+//                               sums); warp k takes the units of decode group k, the
+//                               whole warp runs the loop and one elected lane issues
+//   4 epilogue warps            y = d * acc - dmin * acc_mins (per row), times the
+//                               activation row scales, summed over the tile's blocks
+//                               in registers, added into Y with fp32 atomics when the
+//                               run leaves the tile                       [NACC slots]
+//
+// A decode warp does 128 weights of each of its 32 rows per unit: per-unit
+// synchronisation (one raw-stage wait, one A-half wait, a few arrivals) costs
+// several hundred cycles, so a warp's share of a unit must be large, and two
+// groups keep two units in flight in the two A buffers TMEM has room for.
+// The k order inside the operands: A column c of a block holds the weights at
+// k = 4 (c / 2) + (c & 1) + {0, 2} (the pair a nibble mask gives without
+// shifting), so MMA position 4 t + {0, 1, 2, 3} carries block position
+// 4 t + {0, 2, 1, 3}; the record builder writes the activations in that order.
+// Every mbarrier wait is bounded: on a timeout the CTA records a status, stops
+// issuing, waits for its own copies and MMAs, frees its tensor memory and
+// exits.
 
-constexpr int RW = 32;               // weight rows per consumer warp (two m16 tiles)
-constexpr int Q6A_BYTES = 208;       // plane A bytes per Q6_K block
-
-// CG consumer groups of GW warps take units round-robin; each warp owns RW
-// weight rows of the unit. Stages are reused every S units and S is a multiple
-// of CG, so unit i and unit i + S (the next use of a stage) belong to the same
-// group: a group never waits on a stage phase whose predecessor it has not
-// itself seen complete (parity waits cannot tell phase u from phase u - 2).
-// Consumer groups per CTA (build-time tunables).
-#ifndef QAD_Q4_GROUPS
-#define QAD_Q4_GROUPS 3
-#endif
-#ifndef QAD_Q6_GROUPS
-#define QAD_Q6_GROUPS 2
-#endif
+namespace tg {
+constexpr int TILE = 128;                      // weight rows per unit (MMA M, TMEM lanes)
+constexpr int NCOL = 16;                       // activation rows (MMA N)
+constexpr int DW = 16;                         // decode warps: 2 groups x 2 k halves x 4 lane quarters
+constexpr int EW = 4;                          // epilogue warps
+constexpr int NG = 2;                          // decode groups = MMA warps = A buffers
+constexpr int W_PROD = DW + EW, W_REC = W_PROD + 1, W_MMA = W_REC + 1;
+constexpr int THREADS = 32 * (W_MMA + NG);
+constexpr int NACC = 4;                        // TMEM accumulator slots
+constexpr int SB = 4;                          // operand-record stages
+constexpr int ND = 8;                          // ring of per-unit d, dmin (decode -> epilogue)
+static_assert(NACC % NG == 0 && SB % NG == 0, "a group's units use fixed slots and stages");
+static_assert(ND >= NG + NACC, "a d slot is rewritten only after its epilogue has read it");
+constexpr uint32_t COL_A = 0;                  // A buffers: 128 columns each (256 fp16 per row)
+constexpr uint32_t COL_MA = 128 * NG;          // mins operand: 8 columns per A buffer
+constexpr uint32_t COL_ACC = 288;              // accumulator slots: 16 (product) + 16 (mins) columns
+static_assert(COL_MA + 8 * NG <= COL_ACC && COL_ACC + 32 * NACC <= 512, "TMEM map");
+constexpr int Q6A = 208;                       // plane A bytes per Q6_K block
 template <int FMT>
-struct Cfg {
-    static constexpr int GW = 4;                       // warps per consumer group
-    static constexpr int CG = FMT == 4 ? QAD_Q4_GROUPS : QAD_Q6_GROUPS;  // consumer groups
-    static constexpr int TILE = RW * GW;               // weight rows per unit
-    static constexpr int S = 6;                        // pipeline stages
-    static constexpr int THREADS = 32 * (CG * GW + 1);
-    static constexpr int ROW_BYTES = FMT == 4 ? 144 : Q6A_BYTES;
-    static_assert(S % CG == 0, "stage reuse must stay within one consumer group");
+struct Stg {
+    static constexpr int SR = FMT == 4 ? 8 : 6;             // raw weight stages (even: a stage keeps one group)
+    static constexpr int ROW = FMT == 4 ? 144 : Q6A;
+    static constexpr int W = TILE * ROW;                    // weight bytes per unit
+    static constexpr int D = FMT == 4 ? 0 : TILE * 16;      // Q6_K: 8 fp16 d per row (aligned group of 8 blocks)
+    static constexpr int RAW = (W + D + 127) / 128 * 128;
+    static constexpr int NBAR = 2 * SR + 2 * SB + 4 * NG + 2 * NACC + ND + NG;
+    static constexpr size_t SMEM = 128 + (size_t)SR * RAW + (size_t)SB * REC_BYTES + (size_t)ND * TILE * 8 + 8 * NBAR + 16;
+    static_assert(SR % NG == 0, "raw stages alternate between the decode groups");
+    static_assert(SMEM <= 232448, "shared memory per CTA");
 };
-
-template <int FMT, int NT>
-struct Stage {
-    static constexpr int W_BYTES = Cfg<FMT>::TILE * Cfg<FMT>::ROW_BYTES;
-    static constexpr int D_BYTES = FMT == 4 ? 0 : Cfg<FMT>::TILE * 16;  // 8 fp16 d per row (aligned group of 8 blocks)
-    static constexpr int X_BYTES = 4096 * NT;                          // the block's operand record:
-    static constexpr int S_BYTES = FMT == 4 ? 256 * NT : 0;            //   X, S, then 16 row scales
-    static constexpr int R_BYTES = rec_bytes(FMT, NT);
-    static constexpr int COPY_BYTES = W_BYTES + D_BYTES + R_BYTES;     // what lands per unit
-    // every stage starts on a 128-byte boundary (tensor-map copy destinations)
-    static constexpr int BYTES = (COPY_BYTES + 127) / 128 * 128;
-    static_assert(W_BYTES % 128 == 0 && D_BYTES % 128 == 0 && R_BYTES % 16 == 0, "stage field alignment");
-};
-
-template <int FMT, int NT>
-constexpr size_t gemm_smem_bytes()
-{
-    return (size_t)Cfg<FMT>::S * Stage<FMT, NT>::BYTES + 2 * Cfg<FMT>::S * sizeof(uint64_t);
-}
+enum { ST_RAW = 1, ST_REC = 2, ST_A = 3, ST_ACC = 4, ST_DONE = 5 };
+}  // namespace tg
 
 struct WeightMaps {
     CUtensorMap w;  // Q4_K matrix, or Q6_K plane A
@@ -384,498 +349,384 @@ struct WeightMaps {
 
 struct GemmArgs {
     int N, nblk, M, ldy, units;
-    const uint8_t *rec;  // operand records, rec_bytes(FMT, NT) apart
+    const uint8_t *rec;  // operand records, REC_BYTES apart
     float *Y;
     unsigned long long *trace;
 };
 
-enum { ERR_FULL_TIMEOUT = 1, ERR_EMPTY_TIMEOUT = 2 };
-
-// Add a warp's partial sums of 16 weight rows (n0 + g, n0 + g + 8) to Y.
-template <int NT>
-__device__ __forceinline__ void flush_rows(float (&tot)[NT][4], const GemmArgs &a, int n0, int g, int c)
+// (v, v) as fp16 pair from byte i of w (an integer 0..255): 1024 + v built in the
+// mantissa, 1024 subtracted exactly.
+__device__ __forceinline__ uint32_t byte_h2(uint32_t w, uint32_t i)
 {
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int n = n0 + g + 8 * (e >> 1);
-            const int r = 8 * nt + 2 * c + (e & 1);
-            if (n < a.N && r < a.M)
-                atomicAdd(a.Y + (size_t)r * a.ldy + n, tot[nt][e]);
-            tot[nt][e] = 0.f;
-        }
+    return hsub2(prmt(w, 0x64u, 0x4040u | i | (i << 8)), H2_1024);
 }
 
-template <int NT>
-__device__ __forceinline__ void lds_b(const uint8_t *p, uint32_t (&b)[NT][2])
+// Q4_K: 64 weights of this thread's row (k part p = quant bytes 32p .. 32p + 31,
+// sub-blocks 2p (low nibbles) and 2p + 1 (high nibbles)) as 32 exact fp16 pairs
+// sc_j * q in column order (16 h + 2 i + s: h = high nibble, i = quant word,
+// s = the word shifted by one byte).
+__device__ __forceinline__ void decode_q4(const uint8_t *blk, int p, uint32_t (&out)[32])
 {
-    if (NT == 2) {
-        const uint4 v = lds_v4(p);
-        b[0][0] = v.x;
-        b[0][1] = v.y;
-        b[NT - 1][0] = v.z;
-        b[NT - 1][1] = v.w;
-    } else {
-        const uint2 v = lds_v2(p);
-        b[0][0] = v.x;
-        b[0][1] = v.y;
+    const uint4 h = lds_v4(blk);
+    const uint32_t scA = h.y & 0x3F3F3F3Fu;                                    // sc_0..3
+    const uint32_t scB = (h.w & 0x0F0F0F0Fu) | ((h.y >> 2) & 0x30303030u);     // sc_4..7
+    const uint32_t scw = p < 2 ? scA : scB;
+    const uint32_t bo = 2u * (uint32_t)(p & 1);
+    const uint32_t SC0 = byte_h2(scw, bo);                                     // (sc_2p, sc_2p)
+    const uint32_t NG0 = hmul2(SC0, H2_NEG1024);
+    // the high nibble enters as 1024 + 16 q: scale sc / 16, offset -64 sc
+    const uint32_t SC1 = hfma2(prmt(scw, 0x64u, 0x4040u | (bo + 1) | ((bo + 1) << 8)), H2_SIXTEENTH, H2_NEG64);
+    const uint32_t NG1 = hmul2(SC1, H2_NEG1024);
+    const uint4 qa = lds_v4(blk + 16 + 32 * p), qb = lds_v4(blk + 32 + 32 * p);
+    const uint32_t w8[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const uint32_t w = w8[i], ws = w >> 8;
+        out[2 * i] = hfma2(and_or(w, 0x000F000Fu, H2_1024), SC0, NG0);
+        out[2 * i + 1] = hfma2(and_or(ws, 0x000F000Fu, H2_1024), SC0, NG0);
+        out[16 + 2 * i] = hfma2(and_or(w, 0x00F000F0u, H2_1024), SC1, NG1);
+        out[16 + 2 * i + 1] = hfma2(and_or(ws, 0x00F000F0u, H2_1024), SC1, NG1);
     }
 }
 
-__device__ __forceinline__ uint32_t u4w(const uint4 &v, int i)
+// Q4_K mins operand of this thread's row: (m_0, m_1) .. (m_6, m_7) twice (K = 16:
+// the first 8 meet the high parts of the sub-block sums, the last 8 the low parts).
+__device__ __forceinline__ void decode_q4_mins(const uint8_t *blk, uint32_t (&mm)[8])
 {
-    return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+    const uint4 h = lds_v4(blk);
+    const uint32_t mA = h.z & 0x3F3F3F3Fu;                                     // m_0..3
+    const uint32_t mB = ((h.w >> 4) & 0x0F0F0F0Fu) | ((h.z >> 2) & 0x30303030u);  // m_4..7
+    mm[0] = hsub2(prmt(mA, 0x64u, 0x4140u), H2_1024);
+    mm[1] = hsub2(prmt(mA, 0x64u, 0x4342u), H2_1024);
+    mm[2] = hsub2(prmt(mB, 0x64u, 0x4140u), H2_1024);
+    mm[3] = hsub2(prmt(mB, 0x64u, 0x4342u), H2_1024);
+    mm[4] = mm[0];
+    mm[5] = mm[1];
+    mm[6] = mm[2];
+    mm[7] = mm[3];
 }
 
-// Row scales 2^-e(r,b) of the activation rows this lane's accumulators hold.
-template <int NT>
-__device__ __forceinline__ void lds_rs(const uint8_t *RS, int c, float (&rs)[NT][2])
+// Q6_K-like: this thread's k part p (half hh = p >> 1, l range 16 (p & 1) ..
+// + 15) gives 64 weights in four sub-blocks sb = 8 hh + 2 m + (p & 1), m = 0..3
+// (quants at k = 128 hh + 32 m + l); out[8 m + 2 i + s] = sc_sb * (q - 32) as
+// fp16 pairs, i = quant word, s = shifted pair. Exact when |sc (q - 32)| <= 2048
+// (always for scales in -64..64), else within half an fp16 ulp (2^-11 relative).
+__device__ __forceinline__ void decode_q6(const uint8_t *blk, int p, uint32_t (&out)[32])
 {
+    const int hh = p >> 1, lh = p & 1;
+    const uint2 sw = lds_v2(blk + 192 + 8 * hh);  // scales 8 hh .. 8 hh + 7
+    const uint32_t sv[2] = {sw.x ^ 0x80808080u, sw.y ^ 0x80808080u};  // biased: sc + 128
+    uint32_t SC[4];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-        const float2 v = lds_v2f(RS + 4 * (8 * nt + 2 * c));
-        rs[nt][0] = v.x;
-        rs[nt][1] = v.y;
+    for (int m = 0; m < 4; ++m) {  // scale index 2 m + lh inside the 8: word m >> 1, byte 2 (m & 1) + lh
+        const uint32_t bi = 2u * (uint32_t)(m & 1) + (uint32_t)lh;
+        SC[m] = hsub2(prmt(sv[m >> 1], 0x64u, 0x4040u | bi | (bi << 8)), H2_1152);  // (1024 + sc + 128) - 1152
     }
-}
-
-// One Q4_K block of this warp's 32 weight rows (tiles mt = 0, 1; this lane
-// decodes rows 16 mt + g and 16 mt + g + 8, indexed q = 2 mt + rh) against
-// all activation rows. W: the warp's first row in the stage; XS/SS/RS: the
-// block's operand record.
-template <int NT>
-__device__ __forceinline__ void q4_block(const uint8_t *W, const uint8_t *XS, const uint8_t *SS, const uint8_t *RS,
-                                         int g, int c, uint32_t selT, bool hib, float (&tot)[2][NT][4])
-{
-    uint32_t SCl[4], NGl[4], SCh[4], NGh[4], AM[4];
-    float dd[4], dm[4];
+    const uint4 L0 = lds_v4(blk + 64 * hh + 16 * lh), L1 = lds_v4(blk + 64 * hh + 32 + 16 * lh);
+    const uint4 HH = lds_v4(blk + 128 + 32 * hh + 16 * lh);
+    const uint32_t l0[4] = {L0.x, L0.y, L0.z, L0.w}, l1[4] = {L1.x, L1.y, L1.z, L1.w};
+    const uint32_t hw[4] = {HH.x, HH.y, HH.z, HH.w};
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const uint4 h = lds_v4(W + (16 * (q >> 1) + g + 8 * (q & 1)) * 144);
-        // scales/mins of sub-blocks 2c and 2c+1 (bytes (2c)&3, +1 of the packed words)
-        const uint32_t scA = h.y & 0x3F3F3F3Fu, mA = h.z & 0x3F3F3F3Fu;
-        const uint32_t scB = (h.w & 0x0F0F0F0Fu) | ((h.y >> 2) & 0x30303030u);
-        const uint32_t mB = ((h.w >> 4) & 0x0F0F0F0Fu) | ((h.z >> 2) & 0x30303030u);
-        const uint32_t T = prmt(hib ? scB : scA, hib ? mB : mA, selT);  // [sc_lo, sc_hi, m_lo, m_hi]
-        const uint32_t Tl = prmt(T, 0x64u, 0x4040u);                     // 1024 + sc_lo (x2)
-        const uint32_t Th = prmt(T, 0x64u, 0x4141u);                     // 1024 + sc_hi (x2)
-        const uint32_t Tm = prmt(T, 0x64u, 0x4342u);                     // 1024 + (m_lo, m_hi)
-        SCl[q] = hsub2(Tl, H2_1024);                                     // sc_lo
-        NGl[q] = hmul2(SCl[q], H2_NEG1024);                              // -1024 sc_lo
-        SCh[q] = hfma2(Th, H2_SIXTEENTH, H2_NEG64);                      // sc_hi / 16
-        NGh[q] = hmul2(SCh[q], H2_NEG1024);                              // -64 sc_hi
-        AM[q] = hsub2(Tm, H2_1024);                                      // (m_lo, m_hi)
-        dd[q] = half_lo(h.x);
-        dm[q] = half_hi(h.x);
-    }
-    float acc[2][NT][4];
-    const uint8_t *xl = XS + (g * 4 + c) * 8 * NT;
+    for (int i = 0; i < 4; ++i) {
+        uint32_t qt[4];
+        qt[0] = (l0[i] & 0x0F0F0F0Fu) | ((hw[i] << 4) & 0x30303030u);
+        qt[1] = (l1[i] & 0x0F0F0F0Fu) | ((hw[i] << 2) & 0x30303030u);
+        qt[2] = ((l0[i] >> 4) & 0x0F0F0F0Fu) | (hw[i] & 0x30303030u);
+        qt[3] = ((l1[i] >> 4) & 0x0F0F0F0Fu) | ((hw[i] >> 2) & 0x30303030u);
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-        uint4 qw[4];  // quant words 4 half .. 4 half + 3 of this lane's 32 bytes, per row
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-            qw[q] = lds_v4(W + (16 * (q >> 1) + g + 8 * (q & 1)) * 144 + 16 + 32 * c + 16 * half);
-#pragma unroll
-        for (int ii = 0; ii < 4; ++ii) {
-            const int i = 4 * half + ii;
-            uint32_t blo[NT][2], bhi[NT][2];
-            lds_b<NT>(xl + (2 * i) * 256 * NT, blo);
-            lds_b<NT>(xl + (2 * i + 1) * 256 * NT, bhi);
-#pragma unroll
-            for (int mt = 0; mt < 2; ++mt) {
-                const int q0 = 2 * mt, q1 = 2 * mt + 1;
-                const uint32_t w0 = u4w(qw[q0], ii), w1 = u4w(qw[q1], ii);
-                const uint32_t w0s = w0 >> 8, w1s = w1 >> 8;
-                // low nibbles: sub-block 2c, k-step 2i
-                const uint32_t a0 = hfma2(and_or(w0, 0x000F000Fu, H2_1024), SCl[q0], NGl[q0]);
-                const uint32_t a1 = hfma2(and_or(w1, 0x000F000Fu, H2_1024), SCl[q1], NGl[q1]);
-                const uint32_t a2 = hfma2(and_or(w0s, 0x000F000Fu, H2_1024), SCl[q0], NGl[q0]);
-                const uint32_t a3 = hfma2(and_or(w1s, 0x000F000Fu, H2_1024), SCl[q1], NGl[q1]);
-                // high nibbles: sub-block 2c+1, k-step 2i+1
-                const uint32_t c0 = hfma2(and_or(w0, 0x00F000F0u, H2_1024), SCh[q0], NGh[q0]);
-                const uint32_t c1 = hfma2(and_or(w1, 0x00F000F0u, H2_1024), SCh[q1], NGh[q1]);
-                const uint32_t c2 = hfma2(and_or(w0s, 0x00F000F0u, H2_1024), SCh[q0], NGh[q0]);
-                const uint32_t c3 = hfma2(and_or(w1s, 0x00F000F0u, H2_1024), SCh[q1], NGh[q1]);
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    if (i == 0)
-                        mma_f16_zero(acc[mt][nt], a0, a1, a2, a3, blo[nt][0], blo[nt][1]);
-                    else
-                        mma_f16(acc[mt][nt], a0, a1, a2, a3, blo[nt][0], blo[nt][1]);
-                    mma_f16(acc[mt][nt], c0, c1, c2, c3, bhi[nt][0], bhi[nt][1]);
-                }
-            }
+        for (int m = 0; m < 4; ++m) {
+            out[8 * m + 2 * i] = hmul2(hsub2(prmt(qt[m], 0x64u, 0x4240u), H2_1056), SC[m]);
+            out[8 * m + 2 * i + 1] = hmul2(hsub2(prmt(qt[m], 0x64u, 0x4341u), H2_1056), SC[m]);
         }
     }
-    // mins: sum_j m_j * S_j, S split into two fp16 parts along k
-    uint32_t sb[NT][2];
-    lds_b<NT>(SS + (g * 4 + c) * 8 * NT, sb);
-    float rs[NT][2];
-    lds_rs<NT>(RS, c, rs);
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            float accm[4];
-            mma_f16_zero(accm, AM[2 * mt], AM[2 * mt + 1], AM[2 * mt], AM[2 * mt + 1], sb[nt][0], sb[nt][1]);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int q = 2 * mt + (e >> 1);
-                const float y = fmaf(dd[q], acc[mt][nt][e], -dm[q] * accm[e]);
-                tot[mt][nt][e] = fmaf(rs[nt][e & 1], y, tot[mt][nt][e]);
-            }
-        }
 }
 
+// Pipeline waits: poll with a short sleep between tries so a waiting warp
+// leaves its issue slots to the warps doing the work; the decode <-> MMA
+// hand-offs (on the critical path) sleep least.
+#define QAD_TG_WAIT(bar, par) mbar_wait_sleep(bar, par, 32)
+#define QAD_TG_WAIT_SLOW(bar, par) mbar_wait_sleep(bar, par, 256)
 
-// One Q6_K-like block (packed layout) of this warp's 32 weight rows. A: the
-// warp's first row in plane A of the stage; D: its first row of the d tile.
-template <int NT>
-__device__ __forceinline__ void q6_block(const uint8_t *A, const uint8_t *D, int bsub, const uint8_t *XS,
-                                         const uint8_t *RS, int g, int c, float (&tot)[2][NT][4])
+template <int FMT>
+__global__ void __launch_bounds__(tg::THREADS, 1) k_qgemm_tc(const __grid_constant__ WeightMaps maps, GemmArgs a)
 {
-    uint32_t SC[4][4];
-    float dd[4];
-    const int h = c >> 1, lq = 16 * (c & 1);
-    const uint32_t j = (uint32_t)(c & 1);
-    const uint32_t sel0 = j | 0x40u | (j << 8) | 0x4000u, sel1 = (j + 2) | 0x40u | ((j + 2) << 8) | 0x4000u;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const int row = 16 * (q >> 1) + g + 8 * (q & 1);
-        const uint8_t *blk = A + row * Q6A_BYTES;
-        // int8 scales of sub-blocks 8h + 2t + (c&1): bytes (c&1) + 2t of the 8 scale bytes
-        const uint2 sw = lds_v2(blk + 192 + 8 * h);
-        const uint32_t s0 = sw.x ^ 0x80808080u, s1 = sw.y ^ 0x80808080u;
-        // (sc + 128) + 1024 - 1152 = sc, exact in fp16
-        SC[q][0] = hsub2(prmt(s0, 0x64u, sel0), H2_1152);
-        SC[q][1] = hsub2(prmt(s0, 0x64u, sel1), H2_1152);
-        SC[q][2] = hsub2(prmt(s1, 0x64u, sel0), H2_1152);
-        SC[q][3] = hsub2(prmt(s1, 0x64u, sel1), H2_1152);
-        const uint32_t dw = lds_u32(D + row * 16 + (bsub & 6) * 2);
-        dd[q] = __half2float(__ushort_as_half((unsigned short)(dw >> ((bsub & 1) * 16))));
-    }
-    float acc[2][NT][4];
-    const uint8_t *xl = XS + (g * 4 + c) * 8 * NT;
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-        uint2 L0[4], L1[4], HH[4];  // words 2 half, 2 half + 1 of ql (two quarters) and qh, per row
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const uint8_t *blk = A + (16 * (q >> 1) + g + 8 * (q & 1)) * Q6A_BYTES;
-            L0[q] = lds_v2(blk + 64 * h + lq + 8 * half);
-            L1[q] = lds_v2(blk + 64 * h + 32 + lq + 8 * half);
-            HH[q] = lds_v2(blk + 128 + 32 * h + lq + 8 * half);
-        }
-#pragma unroll
-        for (int ii = 0; ii < 2; ++ii) {
-            const int i = 2 * half + ii;
-            uint32_t qt[4][4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const uint32_t l0 = ii ? L0[q].y : L0[q].x, l1 = ii ? L1[q].y : L1[q].x;
-                const uint32_t hh = ii ? HH[q].y : HH[q].x;
-                qt[q][0] = (l0 & 0x0F0F0F0Fu) | ((hh << 4) & 0x30303030u);
-                qt[q][1] = (l1 & 0x0F0F0F0Fu) | ((hh << 2) & 0x30303030u);
-                qt[q][2] = ((l0 >> 4) & 0x0F0F0F0Fu) | (hh & 0x30303030u);
-                qt[q][3] = ((l1 >> 4) & 0x0F0F0F0Fu) | ((hh >> 2) & 0x30303030u);
-            }
-#pragma unroll
-            for (int t = 0; t < 4; ++t) {
-                const int s = 4 * i + t;
-                uint32_t bf[NT][2];
-                lds_b<NT>(xl + s * 256 * NT, bf);
-#pragma unroll
-                for (int mt = 0; mt < 2; ++mt) {
-                    const int q0 = 2 * mt, q1 = 2 * mt + 1;
-                    // pairs (bytes 0,2) and (bytes 1,3) -> 1024 + q -> q - 32 -> sc*(q-32)
-                    const uint32_t a0 = hmul2(hsub2(prmt(qt[q0][t], 0x64u, 0x4240u), H2_1056), SC[q0][t]);
-                    const uint32_t a1 = hmul2(hsub2(prmt(qt[q1][t], 0x64u, 0x4240u), H2_1056), SC[q1][t]);
-                    const uint32_t a2 = hmul2(hsub2(prmt(qt[q0][t], 0x64u, 0x4341u), H2_1056), SC[q0][t]);
-                    const uint32_t a3 = hmul2(hsub2(prmt(qt[q1][t], 0x64u, 0x4341u), H2_1056), SC[q1][t]);
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        if (s == 0)
-                            mma_f16_zero(acc[mt][nt], a0, a1, a2, a3, bf[nt][0], bf[nt][1]);
-                        else
-                            mma_f16(acc[mt][nt], a0, a1, a2, a3, bf[nt][0], bf[nt][1]);
-                    }
-                }
-            }
-        }
-    }
-    float rs[NT][2];
-    lds_rs<NT>(RS, c, rs);
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-                tot[mt][nt][e] = fmaf(dd[2 * mt + (e >> 1)] * rs[nt][e & 1], acc[mt][nt][e], tot[mt][nt][e]);
-}
-
-template <int FMT, int NT>
-__global__ void __launch_bounds__(Cfg<FMT>::THREADS, 1) k_qgemm(const __grid_constant__ WeightMaps maps, GemmArgs a)
-{
-    extern __shared__ __align__(128) uint8_t smem[];
-    using St = Stage<FMT, NT>;
-    using Cf = Cfg<FMT>;
-    constexpr int S = Cf::S, GW = Cf::GW, CG = Cf::CG, TILE = Cf::TILE;
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + (size_t)S * St::BYTES);
-    uint64_t *empty = full + S;
+    using namespace tg;
+    using G = Stg<FMT>;
+    constexpr int SR = G::SR;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~(uintptr_t)127);
+    uint8_t *RAW = smem;
+    uint8_t *RECS = RAW + (size_t)SR * G::RAW;
+    float2 *DD = reinterpret_cast<float2 *>(RECS + (size_t)SB * REC_BYTES);  // [ND][TILE] (d, dmin) per unit
+    uint64_t *bar = reinterpret_cast<uint64_t *>(DD + ND * TILE);
+    uint64_t *raw_full = bar, *raw_empty = bar + SR, *b_full = bar + 2 * SR, *b_empty = b_full + SB;
+    uint64_t *a_full = b_empty + SB, *a_empty = a_full + 2 * NG;  // [buffer][k half]
+    uint64_t *acc_full = a_empty + 2 * NG, *acc_empty = acc_full + NACC, *dd_full = acc_empty + NACC;
+    uint64_t *done = dd_full + ND;  // one per MMA warp
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + NG);
+    __shared__ int s_bad;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int u0 = (int)((long long)blockIdx.x * a.units / gridDim.x);
     const int u1 = (int)((long long)(blockIdx.x + 1) * a.units / gridDim.x);
     const int n_units = u1 - u0;
     if (threadIdx.x == 0) {
-        for (int i = 0; i < S; ++i) {
-            mbar_init(&full[i], 1);
-            mbar_init(&empty[i], GW);  // the warps of the consumer group that used the stage
+        s_bad = 0;
+        for (int i = 0; i < SR; ++i) {
+            mbar_init(&raw_full[i], 1);
+            mbar_init(&raw_empty[i], DW / NG);  // the 8 warps of the stage's group
         }
+        for (int i = 0; i < SB; ++i) {
+            mbar_init(&b_full[i], 1);
+            mbar_init(&b_empty[i], EW);
+        }
+        for (int i = 0; i < 2 * NG; ++i) {
+            mbar_init(&a_full[i], 4);  // the four lane-quarter warps of one k half
+            mbar_init(&a_empty[i], 1);
+        }
+        for (int i = 0; i < NACC; ++i) {
+            mbar_init(&acc_full[i], 1);
+            mbar_init(&acc_empty[i], EW);
+        }
+        for (int i = 0; i < ND; ++i)
+            mbar_init(&dd_full[i], 4);  // the k-half-0 warps of the unit's group
+        for (int i = 0; i < NG; ++i)
+            mbar_init(&done[i], 1);
         mbar_fence_init();
     }
+    if (warp == W_MMA) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
     __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
     trace_start(a.trace);
     pdl_trigger();
+    auto fail = [&](int code) {
+        atomicExch(&g_gemm_status, code);
+        atomicExch(&s_bad, 1);
+    };
+    auto bad = [&]() { return *(volatile int *)&s_bad != 0; };
 
-    if (warp == CG * GW) {
-        // ------------------------------------------------ producer warp (lane 0 issues)
-        if (lane != 0) {
-            pdl_wait();
-            return;
-        }
-        auto issue = [&](int i, int t, int b, bool weights, bool frags) {
-            uint8_t *st = smem + (size_t)(i % S) * St::BYTES;
-            uint64_t *bar = &full[i % S];
-            if (weights) {
-                mbar_arrive_expect_tx(bar, (uint32_t)St::COPY_BYTES);
-                tma_load_2d(st, &maps.w, b * Cf::ROW_BYTES, t * TILE, bar);
+    if (warp == W_PROD) {
+        // ------------------------------------------------ weights by TMA (independent of the previous kernel)
+        if (lane == 0) {
+            int i = 0;
+            for (; i < n_units && !bad(); ++i) {
+                if (i >= SR && !QAD_TG_WAIT_SLOW(&raw_empty[i % SR], ((i / SR) - 1) & 1)) {
+                    fail(ST_RAW);
+                    break;
+                }
+                const int u = u0 + i, t = u / a.nblk, b = u - t * a.nblk;
+                uint8_t *st = RAW + (size_t)(i % SR) * G::RAW;
+                uint64_t *bb = &raw_full[i % SR];
+                mbar_arrive_expect_tx(bb, (uint32_t)(G::W + G::D));
+                tma_load_2d(st, &maps.w, b * G::ROW, t * TILE, bb);
                 if (FMT == 6)
-                    tma_load_2d(st + St::W_BYTES, &maps.d, b & ~7, t * TILE, bar);
+                    tma_load_2d(st + G::W, &maps.d, b & ~7, t * TILE, bb);
             }
-            if (frags)
-                bulk_g2s(st + St::W_BYTES + St::D_BYTES, a.rec + (size_t)b * St::R_BYTES, St::R_BYTES, bar);
-        };
-        const int pre = min(S, n_units);
-        int t = n_units > 0 ? u0 / a.nblk : 0, b = u0 - t * a.nblk;
-        for (int i = 0, tt = t, bb = b; i < pre; ++i) {
-            issue(i, tt, bb, true, false);  // weights do not depend on the previous kernel
-            if (++bb == a.nblk) {
-                bb = 0;
-                ++tt;
-            }
+            for (int k = max(0, i - SR); k < i; ++k)  // every issued copy lands before teardown
+                if (!mbar_wait(&raw_full[k % SR], (k / SR) & 1, 20000))
+                    fail(ST_RAW);
         }
+    } else if (warp == W_REC) {
+        // ------------------------------------------------ operand records (written by the previous kernel)
         pdl_wait();
-        int i = 0;
-        for (; i < pre; ++i) {
-            issue(i, t, b, false, true);
-            if (++b == a.nblk) {
-                b = 0;
-                ++t;
+        if (a.trace && lane == 0)
+            atomicMin(a.trace + 1, gtimer());  // past the dependency wait
+        if (lane == 0) {
+            int i = 0;
+            for (; i < n_units && !bad(); ++i) {
+                const int b = (u0 + i) % a.nblk, bs = i % SB;
+                if (i >= SB && !QAD_TG_WAIT_SLOW(&b_empty[bs], ((i / SB) - 1) & 1)) {
+                    fail(ST_REC);
+                    break;
+                }
+                mbar_arrive_expect_tx(&b_full[bs], (uint32_t)REC_BYTES);
+                bulk_g2s(RECS + (size_t)bs * REC_BYTES, a.rec + (size_t)b * REC_BYTES, REC_BYTES, &b_full[bs]);
             }
+            for (int k = max(0, i - SB); k < i; ++k)
+                if (!mbar_wait(&b_full[k % SB], (k / SB) & 1, 20000))
+                    fail(ST_REC);
         }
-        for (; i < n_units; ++i) {
-            if (!mbar_wait(&empty[i % S], ((i / S) - 1) & 1)) {
-                atomicExch(&g_gemm_status, ERR_EMPTY_TIMEOUT);
+    } else if (warp >= W_MMA) {
+        // ------------------------------------------------ MMA warps: warp g multiplies the units of decode group g;
+        // the whole warp runs the loop with warp-uniform operands, one elected lane issues
+        constexpr uint32_t idesc = umma_idesc_f16(TILE, NCOL);
+        const int g = warp - W_MMA;
+        const uint32_t at = tmem + COL_A + 128 * g;
+        bool issued = false;
+        for (int i = g; i < n_units; i += NG) {
+            const int bs = i % SB, c = i % NACC;
+            bool ok = __all_sync(0xffffffffu, QAD_TG_WAIT(&b_full[bs], (i / SB) & 1)) &&
+                      (i < NACC || __all_sync(0xffffffffu, QAD_TG_WAIT(&acc_empty[c], ((i / NACC) - 1) & 1)));
+            const uint32_t rb = smem_u32(RECS + (size_t)bs * REC_BYTES);
+            const uint64_t bdesc = umma_desc_k_noswz(rb, 256, 128);  // + 32 per 512-byte k step (16-byte units)
+            const uint32_t acc = tmem + COL_ACC + 32 * c;
+#pragma unroll
+            for (int h = 0; h < 2 && ok; ++h) {  // k half h (k steps 8h .. 8h+7) once its four warps wrote it
+                if (!__all_sync(0xffffffffu, QAD_TG_WAIT(&a_full[2 * g + h], (i / NG) & 1))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (FMT == 4 && h == 0)
+                    umma_f16_ts_warp(acc + 16, tmem + COL_MA + 8 * g, bdesc + (REC_S_OFF >> 4), idesc, 0);
+#pragma unroll
+                for (int m = 0; m < 8; ++m) {
+                    const int k = 8 * h + m;
+                    umma_f16_ts_warp(acc, at + 8 * k, bdesc + 32 * k, idesc, k != 0);
+                }
+                issued = true;
+                umma_commit_warp(&a_empty[2 * g + h]);
+            }
+            if (!ok) {
+                fail(ST_A);
                 break;
             }
-            issue(i, t, b, true, true);
-            if (++b == a.nblk) {
+            umma_commit_warp(&acc_full[c]);
+        }
+        if (issued) {  // every MMA this warp issued completes before TMEM is freed
+            umma_commit_warp(&done[g]);
+            if (!__all_sync(0xffffffffu, mbar_wait(&done[g], 0, 20000)))
+                fail(ST_DONE);
+        }
+    } else if (warp < DW) {
+        // ------------------------------------------------ decode: group g, k half h, lane quarter q
+        const int g = warp >> 3, h = (warp >> 2) & 1, q = warp & 3;
+        const int row = 32 * q + lane;
+        const uint32_t lanes = (uint32_t)(32 * q) << 16;
+        const uint32_t abase = tmem + lanes + COL_A + 128 * g;
+        int b = n_units > g ? (u0 + g) % a.nblk : 0;
+        for (int i = g; i < n_units; i += NG) {
+            const int s = i % SR;
+            if (!__all_sync(0xffffffffu, QAD_TG_WAIT(&raw_full[s], (i / SR) & 1)) ||
+                (i >= NG && !__all_sync(0xffffffffu, QAD_TG_WAIT(&a_empty[2 * g + h], ((i / NG) - 1) & 1)))) {
+                fail(ST_RAW);
+                break;
+            }
+            tc_fence_after();
+            const uint8_t *st = RAW + (size_t)s * G::RAW;
+            const uint8_t *blk = st + (size_t)row * G::ROW;
+#pragma unroll
+            for (int pp = 0; pp < 2; ++pp) {  // the half's two k parts (64 weights each)
+                const int p = 2 * h + pp;
+                uint32_t out[32];
+                if (FMT == 4) {
+                    decode_q4(blk, p, out);
+                    tmem_st_x32(abase + 32 * p, out);
+                } else {
+                    decode_q6(blk, p, out);
+                    const uint32_t base = abase + 8 * (8 * (p >> 1) + (p & 1));
+#pragma unroll
+                    for (int m = 0; m < 4; ++m)  // sub-block 8 hh + 2 m + lh: columns 8 sb .. 8 sb + 7
+                        tmem_st_x8(base + 16 * m, out + 8 * m);
+                }
+            }
+            if (h == 0) {  // the mins operand and the block's d (and dmin) of this row for the epilogue
+                float2 dv;
+                if (FMT == 4) {
+                    uint32_t mm[8];
+                    decode_q4_mins(blk, mm);
+                    tmem_st_x8(tmem + lanes + COL_MA + 8 * g, mm);
+                    const uint32_t hd = lds_u32(blk);
+                    dv = make_float2(half_lo(hd), half_hi(hd));
+                } else {
+                    const uint32_t dw = lds_u32(st + G::W + row * 16 + (b & 6) * 2);
+                    dv = make_float2((b & 1) ? half_hi(dw) : half_lo(dw), 0.f);
+                }
+                DD[(i % ND) * TILE + row] = dv;
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&a_full[2 * g + h]);
+                mbar_arrive(&raw_empty[s]);
+                if (h == 0)
+                    mbar_arrive(&dd_full[i % ND]);
+            }
+            b += NG;
+            if (b >= a.nblk)
+                b -= a.nblk;
+        }
+    } else {
+        // ------------------------------------------------ epilogue: per-block scales, sum over the tile's blocks
+        pdl_wait();  // Y was prepared (zeroed) by the previous kernel
+        const int q = warp - DW, row = 32 * q + lane;
+        const uint32_t lanes = (uint32_t)(32 * q) << 16;
+        float tot[NCOL];
+#pragma unroll
+        for (int r = 0; r < NCOL; ++r)
+            tot[r] = 0.f;
+        int t = n_units > 0 ? u0 / a.nblk : 0, b = u0 - t * a.nblk;
+        for (int i = 0; i < n_units; ++i) {
+            const int bs = i % SB, c = i % NACC;
+            // d (and dmin) of this row for unit i: published by the unit's k-half-0 decode warps.
+            // The slot is rewritten for unit i + ND only after the MMAs of unit i + ND - NG started,
+            // which needs this warp's release of unit i + ND - NG - NACC >= i.
+            if (!__all_sync(0xffffffffu, QAD_TG_WAIT_SLOW(&dd_full[i % ND], (i / ND) & 1))) {
+                fail(ST_RAW);
+                break;
+            }
+            const float2 dv = DD[(i % ND) * TILE + row];
+            const float d = dv.x, dmin = dv.y;
+            if (!__all_sync(0xffffffffu, QAD_TG_WAIT_SLOW(&acc_full[c], (i / NACC) & 1)) ||
+                !__all_sync(0xffffffffu, QAD_TG_WAIT_SLOW(&b_full[bs], (i / SB) & 1))) {
+                fail(ST_ACC);
+                break;
+            }
+            tc_fence_after();
+            uint32_t acc[16], accm[16];
+            tmem_ld_x16(tmem + lanes + COL_ACC + 32 * c, acc);
+            if (FMT == 4)
+                tmem_ld_x16(tmem + lanes + COL_ACC + 32 * c + 16, accm);
+            tmem_wait_ld();
+            tc_fence_before();
+            const float *RS = reinterpret_cast<const float *>(RECS + (size_t)bs * REC_BYTES + REC_RS_OFF);
+            float rs[NCOL];
+#pragma unroll
+            for (int r = 0; r < NCOL; r += 4) {
+                const uint4 v = lds_v4(RS + r);
+                rs[r] = __uint_as_float(v.x);
+                rs[r + 1] = __uint_as_float(v.y);
+                rs[r + 2] = __uint_as_float(v.z);
+                rs[r + 3] = __uint_as_float(v.w);
+            }
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&acc_empty[c]);
+                mbar_arrive(&b_empty[bs]);
+            }
+#pragma unroll
+            for (int r = 0; r < NCOL; ++r) {
+                const float y = FMT == 4 ? fmaf(d, __uint_as_float(acc[r]), -dmin * __uint_as_float(accm[r]))
+                                         : d * __uint_as_float(acc[r]);
+                tot[r] = fmaf(rs[r], y, tot[r]);
+            }
+            if (++b == a.nblk || i + 1 == n_units) {
+                const int n = t * TILE + row;
+                if (n < a.N)
+#pragma unroll
+                    for (int r = 0; r < NCOL; ++r)
+                        if (r < a.M)
+                            atomicAdd(a.Y + (size_t)r * a.ldy + n, tot[r]);
+#pragma unroll
+                for (int r = 0; r < NCOL; ++r)
+                    tot[r] = 0.f;
                 b = 0;
                 ++t;
             }
         }
-        // every issued copy lands before this CTA may exit
-        for (int k = max(0, i - S); k < i; ++k)
-            if (!mbar_wait(&full[k % S], (k / S) & 1, 20000))
-                atomicExch(&g_gemm_status, ERR_FULL_TIMEOUT);
-        trace_end(a.trace);
-        return;
-    }
-
-    // ---------------------------------------------------- consumer groups (round-robin units)
-    const int grp = warp / GW, wi = warp % GW;
-    const int g = lane >> 2, c = lane & 3;
-    const int jj = 2 * (c & 1);
-    const uint32_t selT = (uint32_t)(jj | ((jj + 1) << 4) | ((jj + 4) << 8) | ((jj + 5) << 12));
-    const bool hib = c >= 2;
-    pdl_wait();
-    trace_ready(a.trace);
-    float tot[2][NT][4];
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-                tot[mt][nt][e] = 0.f;
-    int t = 0, b = 0;
-    if (grp < n_units) {
-        t = (u0 + grp) / a.nblk;
-        b = (u0 + grp) - t * a.nblk;
-    }
-    for (int i = grp; i < n_units; i += CG) {
-        const uint8_t *st = smem + (size_t)(i % S) * St::BYTES;
-        if (!mbar_wait(&full[i % S], (i / S) & 1)) {
-            if (lane == 0)
-                atomicExch(&g_gemm_status, ERR_FULL_TIMEOUT);
-            return;
-        }
-        const uint8_t *XS = st + St::W_BYTES + St::D_BYTES;
-        const uint8_t *RS = XS + St::R_BYTES - 64;
-        if (FMT == 4)
-            q4_block<NT>(st + (size_t)(RW * wi) * 144, XS, XS + St::X_BYTES, RS, g, c, selT, hib, tot);
-        else
-            q6_block<NT>(st + (size_t)(RW * wi) * Q6A_BYTES, st + St::W_BYTES + (size_t)(RW * wi) * 16, b & 7, XS, RS,
-                         g, c, tot);
-        __syncwarp();
-        if (lane == 0)
-            mbar_arrive(&empty[i % S]);
-        // next unit of this group: CG blocks further along
-        int tn = t, bn = b + CG;
-        while (bn >= a.nblk) {
-            bn -= a.nblk;
-            ++tn;
-        }
-        if (tn != t || i + CG >= n_units) {
-            flush_rows<NT>(tot[0], a, t * TILE + RW * wi, g, c);
-            flush_rows<NT>(tot[1], a, t * TILE + RW * wi + 16, g, c);
-        }
-        t = tn;
-        b = bn;
     }
     trace_end(a.trace);
-}
-
-// Q4_K form without a producer warp: 4 consumer groups of 4 warps (16 warps,
-// so each SM sub-partition runs 4 consumers at the same register budget as 3
-// consumers + the producer). Group grp consumes units grp, grp+4, ... through
-// its own two ring slots (grp and grp+4 of 8) and refills a slot itself: after
-// the group's 4 warps release unit i (one arrival each on the slot's empty
-// barrier), lane 0 of the group's first warp issues unit i+8 into it. Before
-// the wait on the previous kernel each group requests the weights of its first
-// two units; every wait is bounded and reports through g_gemm_status.
-#ifndef QAD_Q4_SELF_REFILL
-#define QAD_Q4_SELF_REFILL 1
-#endif
-namespace sr {
-constexpr int CG = 4, GW = 4, S = 8, THREADS = 32 * CG * GW;
-}
-template <int NT>
-constexpr size_t gemm_sr_smem_bytes()
-{
-    return (size_t)sr::S * Stage<4, NT>::BYTES + 2 * sr::S * sizeof(uint64_t);
-}
-
-template <int NT>
-__global__ void __launch_bounds__(sr::THREADS, 1) k_qgemm_sr(const __grid_constant__ WeightMaps maps, GemmArgs a)
-{
-    extern __shared__ __align__(128) uint8_t smem[];
-    using St = Stage<4, NT>;
-    constexpr int S = sr::S, GW = sr::GW, CG = sr::CG, TILE = Cfg<4>::TILE;
-    static_assert(S % CG == 0 && TILE == RW * GW, "each group owns S / CG slots; a unit is GW warps of RW rows");
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + (size_t)S * St::BYTES);
-    uint64_t *empty = full + S;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int grp = warp / GW, wi = warp % GW;
-    const int u0 = (int)((long long)blockIdx.x * a.units / gridDim.x);
-    const int u1 = (int)((long long)(blockIdx.x + 1) * a.units / gridDim.x);
-    const int n_units = u1 - u0;
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < S; ++i) {
-            mbar_init(&full[i], 1);
-            mbar_init(&empty[i], GW);
-        }
-        mbar_fence_init();
-    }
+    tc_fence_before();
     __syncthreads();
-    trace_start(a.trace);
-    pdl_trigger();
-    const bool leader = wi == 0 && lane == 0;
-    auto issue = [&](int i, bool weights, bool frags) {
-        const int u = u0 + i, t = u / a.nblk, b = u - t * a.nblk;
-        uint8_t *st = smem + (size_t)(i % S) * St::BYTES;
-        uint64_t *bar = &full[i % S];
-        if (weights) {
-            mbar_arrive_expect_tx(bar, (uint32_t)St::COPY_BYTES);
-            tma_load_2d(st, &maps.w, b * 144, t * TILE, bar);
-        }
-        if (frags)
-            bulk_g2s(st + St::W_BYTES, a.rec + (size_t)b * St::R_BYTES, St::R_BYTES, bar);
-    };
-    int issued = -1;  // highest unit this group's leader has requested
-    if (leader)
-        for (int i = grp; i < n_units && i < S; i += CG) {
-            issue(i, true, false);  // weights do not depend on the previous kernel
-            issued = i;
-        }
-    pdl_wait();
-    if (leader)
-        for (int i = grp; i < n_units && i < S; i += CG)
-            issue(i, false, true);
-    trace_ready(a.trace);
-
-    const int g = lane >> 2, c = lane & 3;
-    const int jj = 2 * (c & 1);
-    const uint32_t selT = (uint32_t)(jj | ((jj + 1) << 4) | ((jj + 4) << 8) | ((jj + 5) << 12));
-    const bool hib = c >= 2;
-    float tot[2][NT][4];
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-                tot[mt][nt][e] = 0.f;
-    int t = 0, b = 0;
-    if (grp < n_units) {
-        t = (u0 + grp) / a.nblk;
-        b = (u0 + grp) - t * a.nblk;
+    if (warp == W_MMA) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
     }
-    int done = grp - CG;  // last unit this warp consumed
-    for (int i = grp; i < n_units; i += CG) {
-        const uint8_t *st = smem + (size_t)(i % S) * St::BYTES;
-        if (!mbar_wait(&full[i % S], (i / S) & 1)) {
-            if (lane == 0)
-                atomicExch(&g_gemm_status, ERR_FULL_TIMEOUT);
-            break;
-        }
-        const uint8_t *XS = st + St::W_BYTES;
-        const uint8_t *RS = XS + St::R_BYTES - 64;
-        q4_block<NT>(st + (size_t)(RW * wi) * 144, XS, XS + St::X_BYTES, RS, g, c, selT, hib, tot);
-        __syncwarp();
-        if (lane == 0)
-            mbar_arrive(&empty[i % S]);
-        done = i;
-        if (leader && i + S < n_units) {
-            // the slot's next user is unit i + S of this group: refill it once all GW warps released it
-            if (!mbar_wait(&empty[i % S], (i / S) & 1)) {
-                atomicExch(&g_gemm_status, ERR_EMPTY_TIMEOUT);
-            } else {
-                issue(i + S, true, true);
-                issued = i + S;
-            }
-        }
-        int tn = t, bn = b + CG;
-        while (bn >= a.nblk) {
-            bn -= a.nblk;
-            ++tn;
-        }
-        if (tn != t || i + CG >= n_units) {
-            flush_rows<NT>(tot[0], a, t * TILE + RW * wi, g, c);
-            flush_rows<NT>(tot[1], a, t * TILE + RW * wi + 16, g, c);
-        }
-        t = tn;
-        b = bn;
-    }
-    // after an error exit, copies this group requested but did not consume land before the CTA exits
-    if (leader)
-        for (int k = done + CG; k <= issued; k += CG)
-            if (!mbar_wait(&full[k % S], (k / S) & 1, 20000))
-                atomicExch(&g_gemm_status, ERR_FULL_TIMEOUT);
-    trace_end(a.trace);
 }
 
 // Q6_K-like GGUF blocks -> packed device layout (plane A: first 208 bytes of
@@ -884,13 +735,13 @@ __global__ void k_q6k_pack(const uint8_t *__restrict__ W, int N, int nblk, uint8
 {
     const int nblk8 = (nblk + 7) & ~7;
     uint8_t *A = P;
-    uint16_t *D = reinterpret_cast<uint16_t *>(P + (size_t)N * nblk * Q6A_BYTES);
+    uint16_t *D = reinterpret_cast<uint16_t *>(P + (size_t)N * nblk * tg::Q6A);
     const long long total = (long long)N * nblk;
     for (long long blk = blockIdx.x * (long long)(blockDim.x / 32) + threadIdx.x / 32; blk < total;
          blk += (long long)gridDim.x * (blockDim.x / 32)) {
         const uint8_t *src = W + blk * 210;
-        uint8_t *dst = A + blk * Q6A_BYTES;
-        for (int i = threadIdx.x & 31; i < Q6A_BYTES; i += 32)
+        uint8_t *dst = A + blk * tg::Q6A;
+        for (int i = threadIdx.x & 31; i < tg::Q6A; i += 32)
             dst[i] = src[i];
         if ((threadIdx.x & 31) == 0) {
             const long long n = blk / nblk, b = blk - n * nblk;
@@ -905,7 +756,7 @@ __global__ void k_q6k_pack(const uint8_t *__restrict__ W, int N, int nblk, uint8
 size_t q6k_packed_bytes(long long N, int K)
 {
     const int nblk = K / 256, nblk8 = (nblk + 7) & ~7;
-    return (size_t)N * nblk * Q6A_BYTES + (size_t)N * nblk8 * 2;
+    return (size_t)N * nblk * tg::Q6A + (size_t)N * nblk8 * 2;
 }
 
 // ------------------------------------------------------------- launchers
@@ -917,19 +768,14 @@ static int set_smem(K kernel, size_t bytes)
                       "cudaFuncSetAttribute");
 }
 
-int frag_nt(int M) { return M <= 8 ? 1 : 2; }
+int frag_nt(int) { return 2; }
 
 int launch_prep(int fmt, int K, int M, const PrepSrc &src, const FragBuf &fb, cudaStream_t s, bool pdl,
                 unsigned long long *trace)
 {
-    const int nt = frag_nt(M);
     PrepArgs a{src, K, M, fb, trace};
-    void (*kern)(PrepArgs);
-    if (fmt == 4)
-        kern = nt == 1 ? k_prep<4, 1> : k_prep<4, 2>;
-    else
-        kern = nt == 1 ? k_prep<6, 1> : k_prep<6, 2>;
-    const dim3 grid((K / 256 + 3) / 4, 8 * nt);
+    void (*kern)(PrepArgs) = fmt == 4 ? k_prep<4> : k_prep<6>;
+    const dim3 grid((K / 256 + 3) / 4, QAD_MAX_ROWS);
     cudaError_t e = pdl ? launch_pdl(kern, grid, dim3(256), 0, s, a)
                         : (kern<<<grid, 256, 0, s>>>(a), cudaGetLastError());
     return cuda_check(e, "prep launch");
@@ -941,50 +787,35 @@ int make_weight_maps(int fmt, const void *W, int N, int K, WeightMapsBlob *out)
     WeightMaps *m = reinterpret_cast<WeightMaps *>(out);
     const int nblk = K / 256;
     if (fmt == 4)
-        return encode_tmap_2d(&m->w, W, 1, (uint64_t)nblk * 144, (uint64_t)N, (uint64_t)nblk * 144, 144,
-                              Cfg<4>::TILE);
-    int rc = encode_tmap_2d(&m->w, W, 1, (uint64_t)nblk * Q6A_BYTES, (uint64_t)N, (uint64_t)nblk * Q6A_BYTES,
-                            Q6A_BYTES, Cfg<6>::TILE);
+        return encode_tmap_2d(&m->w, W, 1, (uint64_t)nblk * 144, (uint64_t)N, (uint64_t)nblk * 144, 144, tg::TILE);
+    int rc = encode_tmap_2d(&m->w, W, 1, (uint64_t)nblk * tg::Q6A, (uint64_t)N, (uint64_t)nblk * tg::Q6A, tg::Q6A,
+                            tg::TILE);
     if (rc)
         return rc;
     const int nblk8 = (nblk + 7) & ~7;
-    const uint8_t *D = (const uint8_t *)W + (size_t)N * nblk * Q6A_BYTES;
-    return encode_tmap_2d(&m->d, D, 2, (uint64_t)nblk8, (uint64_t)N, (uint64_t)nblk8 * 2, 8, Cfg<6>::TILE);
+    const uint8_t *D = (const uint8_t *)W + (size_t)N * nblk * tg::Q6A;
+    return encode_tmap_2d(&m->d, D, 2, (uint64_t)nblk8, (uint64_t)N, (uint64_t)nblk8 * 2, 8, tg::TILE);
 }
 
 int launch_gemm(int fmt, const WeightMapsBlob &maps_blob, int N, int K, int M, const FragBuf &fb, float *Y, int ldy,
                 cudaStream_t s, bool pdl, unsigned long long *trace)
 {
-    const int nt = frag_nt(M);
     const WeightMaps &maps = reinterpret_cast<const WeightMaps &>(maps_blob);
     GemmArgs a;
     a.N = N;
     a.nblk = K / 256;
     a.M = M;
     a.ldy = ldy;
-    const int tile = fmt == 4 ? Cfg<4>::TILE : Cfg<6>::TILE;
-    a.units = ((N + tile - 1) / tile) * a.nblk;
+    a.units = ((N + tg::TILE - 1) / tg::TILE) * a.nblk;
     a.rec = fb.rec;
     a.Y = Y;
     a.trace = trace;
-    void (*kern)(const WeightMaps, GemmArgs);
-    size_t smem;
-    int threads = fmt == 4 ? Cfg<4>::THREADS : Cfg<6>::THREADS;
-    if (fmt == 4 && QAD_Q4_SELF_REFILL) {
-        kern = nt == 1 ? k_qgemm_sr<1> : k_qgemm_sr<2>;
-        smem = nt == 1 ? gemm_sr_smem_bytes<1>() : gemm_sr_smem_bytes<2>();
-        threads = sr::THREADS;
-    } else if (fmt == 4) {
-        kern = nt == 1 ? k_qgemm<4, 1> : k_qgemm<4, 2>;
-        smem = nt == 1 ? gemm_smem_bytes<4, 1>() : gemm_smem_bytes<4, 2>();
-    } else {
-        kern = nt == 1 ? k_qgemm<6, 1> : k_qgemm<6, 2>;
-        smem = nt == 1 ? gemm_smem_bytes<6, 1>() : gemm_smem_bytes<6, 2>();
-    }
-    static bool done[64][4] = {};
+    void (*kern)(const WeightMaps, GemmArgs) = fmt == 4 ? k_qgemm_tc<4> : k_qgemm_tc<6>;
+    const size_t smem = fmt == 4 ? tg::Stg<4>::SMEM : tg::Stg<6>::SMEM;
+    static bool done[64][2] = {};
     int dev = 0;
     cudaGetDevice(&dev);
-    const int v = (fmt == 4 ? 0 : 2) + (nt - 1);
+    const int v = fmt == 4 ? 0 : 1;
     if (dev < 0 || dev >= 64 || !done[dev][v]) {
         int rc = set_smem(kern, smem);
         if (rc)
@@ -993,8 +824,8 @@ int launch_gemm(int fmt, const WeightMapsBlob &maps_blob, int N, int K, int M, c
             done[dev][v] = true;
     }
     const int grid = num_sms();
-    cudaError_t e = pdl ? launch_pdl(kern, dim3(grid), dim3(threads), smem, s, maps, a)
-                        : (kern<<<grid, threads, smem, s>>>(maps, a), cudaGetLastError());
+    cudaError_t e = pdl ? launch_pdl(kern, dim3(grid), dim3(tg::THREADS), smem, s, maps, a)
+                        : (kern<<<grid, tg::THREADS, smem, s>>>(maps, a), cudaGetLastError());
     return cuda_check(e, "gemm launch");
 }
 

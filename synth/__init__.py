@@ -14,8 +14,9 @@ Distributions (the workloads named for the multi-agent decode step):
   "quants uniform in 0..15, scales and mins uniform in 0..63".
 * Q6_K-like blocks (210 bytes = 256 weights): the 128 low-nibble bytes and the
   64 high-bit bytes are uniform random bytes (every 6-bit quant uniform in
-  0..63), the 16 int8 sub-block scales are uniform in 0..63 and ``d`` is
-  fp16(|N(0,1)| * 0.01).
+  0..63), the 16 int8 sub-block scales are uniform in 0..63 (or, with
+  ``signed=True``, uniform over the whole int8 range -128..127, as quantisers
+  of real checkpoints produce) and ``d`` is fp16(|N(0,1)| * 0.01).
 * Activations, queries, keys and values: bf16(N(0,1)) (round to nearest even).
 
 Two back ends draw the same distributions: numpy on the host (small cases the
@@ -75,13 +76,13 @@ def q4k_matrix_np(seed: int, tag: int, n_rows: int, k: int) -> np.ndarray:
     return blk.reshape(n_rows, (k // QK) * Q4K_BLOCK_BYTES)
 
 
-def q6k_matrix_np(seed: int, tag: int, n_rows: int, k: int) -> np.ndarray:
+def q6k_matrix_np(seed: int, tag: int, n_rows: int, k: int, signed: bool = False) -> np.ndarray:
     """uint8 [n_rows, k/256*210]: row n's blocks are contiguous."""
     assert k % QK == 0
     nb = n_rows * (k // QK)
     g = np_rng(seed, 6, tag)
     blk = g.integers(0, 256, size=(nb, Q6K_BLOCK_BYTES), dtype=np.uint8)
-    blk[:, Q6K_SCALES_OFF:Q6K_SCALES_OFF + 16] = g.integers(0, 64, size=(nb, 16), dtype=np.uint8)
+    blk[:, Q6K_SCALES_OFF:Q6K_SCALES_OFF + 16] = g.integers(0, 256 if signed else 64, size=(nb, 16), dtype=np.uint8)
     d = _fp16_bits_np(np.abs(g.standard_normal(nb)) * 0.01)
     blk[:, Q6K_D_OFF:Q6K_D_OFF + 2] = d.view(np.uint8).reshape(nb, 2)
     return blk.reshape(n_rows, (k // QK) * Q6K_BLOCK_BYTES)
@@ -106,13 +107,13 @@ def q4k_matrix_torch(gen: torch.Generator, n_rows: int, k: int, device) -> torch
     return blk.view(n_rows, (k // QK) * Q4K_BLOCK_BYTES)
 
 
-def q6k_matrix_torch(gen: torch.Generator, n_rows: int, k: int, device) -> torch.Tensor:
+def q6k_matrix_torch(gen: torch.Generator, n_rows: int, k: int, device, signed: bool = False) -> torch.Tensor:
     """uint8 [n_rows, k/256*210] drawn in ``device`` memory."""
     assert k % QK == 0
     nb = n_rows * (k // QK)
     blk = torch.randint(0, 256, (nb, Q6K_BLOCK_BYTES), dtype=torch.uint8, device=device, generator=gen)
     blk[:, Q6K_SCALES_OFF:Q6K_SCALES_OFF + 16] = torch.randint(
-        0, 64, (nb, 16), dtype=torch.uint8, device=device, generator=gen)
+        0, 256 if signed else 64, (nb, 16), dtype=torch.uint8, device=device, generator=gen)
     v = (torch.randn(nb, device=device, generator=gen).abs_() * 0.01).to(torch.float16)
     blk[:, Q6K_D_OFF:Q6K_D_OFF + 2] = v.view(torch.uint8).view(nb, 2)
     return blk.view(n_rows, (k // QK) * Q6K_BLOCK_BYTES)

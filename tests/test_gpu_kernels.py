@@ -163,6 +163,22 @@ def test_q6k_gemm_one_hot_reads_weights(q, orc):
         assert (np.abs(Y[r] - w[:, k]) <= 2.0 ** -24 * np.abs(w[:, k])).all()
 
 
+def test_q6k_gemm_one_hot_signed_scales(q, orc):
+    """Signed int8 scales over the whole range: the operand sc*(q-32) is exact in
+    fp16 up to 2048 in magnitude and within half an ulp (2^-11 relative) above it,
+    so |y - w| <= (2^-11 + 2^-24) |w|."""
+    N, K = 48, 768
+    W = synth.q6k_matrix_np(SEED, 96, N, K, signed=True)
+    ks = [0, 15, 16, 64, 127, 128, 255, 256, 511, 767]
+    X = np.zeros((len(ks), K), np.uint16)
+    for r, k in enumerate(ks):
+        X[r, k] = 0x3F80
+    Y = _gemm(q, 6, W, N, K, X, len(ks))
+    w = orc.dequant(6, W, N, K)
+    for r, k in enumerate(ks):
+        assert (np.abs(Y[r] - w[:, k]) <= (2.0 ** -11 + 2.0 ** -24) * np.abs(w[:, k])).all()
+
+
 def test_gemm_rows_are_independent(q, orc):
     """Row r of a 12-row product equals the 1-row product on row r (within tolerance)."""
     N, K = 200, 2048
@@ -196,6 +212,22 @@ def test_gemm_full_size_down_projection(q, orc):
     N, K, M = 5120, 17408, 12
     g = synth.torch_gen(SEED, "cuda", 3)
     Wg = synth.q6k_matrix_torch(g, N, K, "cuda")
+    Xd = synth.bf16_normal_torch(g, (M, K), "cuda")
+    Y = torch.zeros(M, N, device="cuda")
+    q.q6k_gemm(q.q6k_pack(Wg, N, K), N, K, Xd, M, Y)
+    torch.cuda.synchronize()
+    Yr, A = orc.gemm(6, Wg.cpu().numpy(), N, K, _bits(Xd))
+    ratio = np.abs(Y.cpu().double().numpy() - Yr) / (1e-3 * A)
+    assert ratio.max() <= 1.0, ratio.max()
+    assert q.device_status() == 0
+
+
+def test_gemm_full_size_down_projection_signed_scales(q, orc):
+    """The down projection with signed int8 sub-block scales over the whole range
+    (-128..127, as real Q6_K checkpoints carry them): N=5120, K=17408, 12 rows."""
+    N, K, M = 5120, 17408, 12
+    g = synth.torch_gen(SEED, "cuda", 4)
+    Wg = synth.q6k_matrix_torch(g, N, K, "cuda", signed=True)
     Xd = synth.bf16_normal_torch(g, (M, K), "cuda")
     Y = torch.zeros(M, N, device="cuda")
     q.q6k_gemm(q.q6k_pack(Wg, N, K), N, K, Xd, M, Y)

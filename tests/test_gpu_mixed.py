@@ -3,11 +3,11 @@ the dense tensor-core GEMMs) against the fp64 oracle, teacher-forced per layer.
 
 The oracle's layer is the same definition with the chunk agent holding C rows
 at positions chunk_len .. chunk_len + C - 1 (causal, like draft rows).
-Tolerances: dense GEMM 2^-10 * B + 1e-3 * A (fp16 weight tiles, see the dense
-GEMM tests); decode-row attention 2e-3 * sum p|v|, chunk-row attention
-2^-8 * sum p|v| (bf16 probabilities), both plus half a bf16 ulp (2^-8
-relative) of the output; bf16 rounding points equal except for rare one-ulp
-flips at rounding ties.
+Tolerances: every GEMM output 1e-3 * sum |w x| (each weight enters the dense
+tensor-core product within 2^-11 of its value, see the dense GEMM tests);
+attention, decode and chunk rows alike, 2e-3 * sum p|v| plus half a bf16 ulp
+(2^-8 relative) of the output; bf16 rounding points equal except for rare
+one-ulp flips at rounding ties.
 """
 import numpy as np
 import pytest
@@ -15,7 +15,6 @@ import torch
 
 import synth
 from conftest import SEED
-from test_gpu_dense import _bound
 from test_gpu_step import Stack, _bits, bf16_close, dbg_views
 
 pytestmark = pytest.mark.gpu
@@ -32,10 +31,9 @@ def q():
 
 def _dense_check(orc, fmt, W, N, K, Xb, Y_gpu, base=None):
     Yr, A = orc.gemm(fmt, W, N, K, Xb)
-    B = _bound(orc, fmt, W, N, K, Xb)
     ref = Yr if base is None else base + Yr
     slack = 0 if base is None else 8 * 2.0 ** -24 * (np.abs(base) + np.abs(Yr))
-    ratio = np.abs(Y_gpu.astype(np.float64) - ref) / (2.0 ** -10 * B + 1e-3 * A + slack + 1e-30)
+    ratio = np.abs(Y_gpu.astype(np.float64) - ref) / (1e-3 * A + slack + 1e-30)
     assert ratio.max() <= 1.0, ratio.max()
 
 
@@ -75,8 +73,7 @@ def test_mixed_step_teacher_forced(q, orc, n_rows, lens, C):
         Qb = orc.f64_array_to_bf16(v["qkv"][:, :st.nq].astype(np.float64)).reshape(R, st.n_qh, 128)
         O_ref, B = orc.decode_attn(Qb, kc, vc, st.lens, ars_o, st.n_qh, st.n_kvh, 128, st.cap)
         o = orc.bf16_array_to_f64(v["attn"]).reshape(O_ref.shape)
-        rel = np.where(np.arange(R)[:, None, None] < M, 2e-3, 2.0 ** -8)
-        assert (np.abs(o - O_ref) <= rel * B + np.abs(O_ref) * 2.0 ** -8 + 1e-30).all()
+        assert (np.abs(o - O_ref) <= 2e-3 * B + np.abs(O_ref) * 2.0 ** -8 + 1e-30).all()
         _dense_check(orc, 4, W["o"], st.H, st.nq, v["attn"], v["hmid"], base=h.astype(np.float64))
         assert bf16_close(v["x2"], orc.rmsnorm_bf16(v["hmid"].astype(np.float64)), orc)
         _dense_check(orc, 4, W["gu"], 2 * st.I, st.H, v["x2"], v["gu"])

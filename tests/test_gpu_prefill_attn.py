@@ -2,9 +2,10 @@
 
 Row j of the chunk (position len + j) attends keys 0 .. len + j: the oracle's
 decode attention with one agent whose rows are the whole chunk. The GPU path
-rounds the probabilities to bf16 once before the PV product (relative error
-<= 2^-9), so per element
-    |o - o_ref| <= 2^-8 * B + half a bf16 ulp of o_ref,
+forms S = Q K^T from exact bf16 products, rounds each probability once to fp16
+(relative error <= 2^-11) and converts V to fp16 exactly, so per element the
+decode attention's bound holds:
+    |o - o_ref| <= 2e-3 * B + half a bf16 ulp of o_ref (2^-9 |o_ref|),
 with B = sum_t p_t |v_t| from the oracle.
 """
 import numpy as np
@@ -36,7 +37,7 @@ def _bits(t):
 
 def _check(orc, o_bits, O_ref, B):
     o = orc.bf16_array_to_f64(o_bits).reshape(O_ref.shape)
-    tol = 2.0 ** -8 * B + np.abs(O_ref) * 2.0 ** -9 + 1e-30
+    tol = 2e-3 * B + np.abs(O_ref) * 2.0 ** -9 + 1e-30
     ratio = np.abs(o - O_ref) / tol
     assert ratio.max() <= 1.0, f"max err / tol = {ratio.max():.3g}"
 
