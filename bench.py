@@ -111,8 +111,9 @@ class Workload:
         self.lens = torch.full((na,), cl, dtype=torch.int32, device=device)
         self.H_out = torch.empty(self.M, H, dtype=torch.float32, device=device)
         self.ws = q.alloc_ws(self.model.ws_bytes(self.M), device)
-        self.weight_bytes = sum(t.numel() for ts in (self.w_qkv, self.w_o, self.w_gu, self.w_down) for t in ts)
-        # (the packed down projection carries each block's 210 bytes plus up to 14 bytes of row padding)
+        # quantized weight bytes streamed per step: the GGUF blocks of the listed matrices (144 B per Q4_K
+        # block, 210 B per Q6_K block); the d-plane row padding of the packed down projection is not counted
+        self.weight_bytes = sh.weight_bytes_per_layer() * L
         # keys and values read per step (incl. new rows): bf16, or q8_0 codes + one fp16 scale per 32
         self.kv_bytes = 2 * L * na * sh.n_kvh * (cl + rpa) * (hd + hd // 16 if self.kv_q8 else hd * 2)
         self.act_bytes = L * self.M * (2 * H * 4 + 2 * I * 4 + (nq + 2 * nkv) * 4)  # fp32 outputs/residual
@@ -139,30 +140,65 @@ class Workload:
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
-    """nvidia-smi samples during the timed region (SM clock, throttle reasons)."""
+    """SM clock and clock-event (throttle) reasons sampled during the timed region:
+    NVML every 2 ms from a background thread (nvidia-smi every 100 ms if NVML is
+    unavailable), so even a sub-second timed region holds many samples."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown"}
 
     def __init__(self, index: int):
-        self.index, self.rows, self.proc = index, [], None
+        self.index, self.rows, self.proc, self.nv, self.stop = index, [], None, None, False
+        self.source = None
 
     def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_sm = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.t = threading.Thread(target=self._poll_nvml, daemon=True)
+            self.t.start()
+            self.source = "nvml 2 ms"
+            return self
+        except Exception:
+            self.nv = None
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
                                           "--format=csv,noheader,nounits", "-lms", "100"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
+            self.source = "nvidia-smi 100 ms"
         except FileNotFoundError:
             self.proc = None
         return self
+
+    def _poll_nvml(self):
+        nv, h = self.nv, self.h
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        while not self.stop:
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                bits = get_reasons(h)
+            except Exception:
+                break
+            reasons = [name for bit, name in self.REASONS.items() if bits & bit]
+            self.rows.append((time.perf_counter(), ("nvml", sm, self.max_sm, reasons)))
+            time.sleep(0.002)
 
     def _read(self):
         for line in self.proc.stdout:
             self.rows.append((time.perf_counter(), [x.strip() for x in line.split(",")]))
 
     def __exit__(self, *a):
+        self.stop = True
+        if self.nv is not None:
+            self.t.join(timeout=1)
         if self.proc:
             self.proc.terminate()
             try:
@@ -175,13 +211,18 @@ class ClockSampler:
         rows = [r for t, r in self.rows if (t0 is None or t >= t0) and (t1 is None or t <= t1)]
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        sm = [float(r[1]) for r in rows if len(r) > 2 and r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if len(r) > 2 and r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4)
-                          if len(r) > 5 + i and r[5 + i].lower() == "active"})
+        if rows[0][0] == "nvml":
+            sm = [float(r[1]) for r in rows]
+            mx = [float(r[2]) for r in rows]
+            reasons = sorted({x for r in rows for x in r[3]})
+        else:
+            sm = [float(r[1]) for r in rows if len(r) > 2 and r[1].replace(".", "").isdigit()]
+            mx = [float(r[2]) for r in rows if len(r) > 2 and r[2].replace(".", "").isdigit()]
+            names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+            reasons = sorted({names[i] for r in rows for i in range(4)
+                              if len(r) > 5 + i and r[5 + i].lower() == "active"})
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+                "reasons": reasons, "samples": len(rows), "source": self.source}
 
 
 # ------------------------------------------------------------------ helpers
@@ -406,17 +447,29 @@ def run_gpu(args, ws, rank, local):
     ms_step = max_over_ranks(e0.elapsed_time(e1) / args.steps, ws)
     status = q.device_status(reset=True)
 
-    # end to end through the host-buffer entry point (pinned host in/out, copies timed)
-    Xh = w.X.cpu().pin_memory()
-    arsh = w.ars.cpu().pin_memory()
+    # end to end through the public API: each step packs the agents' rows on the host
+    # (qad_pack_rows), copies them from pinned host memory, runs the step
+    # (qad_decode_step_host: H2D, graph replay, D2H of the final hidden rows) and
+    # waits for the result
+    agent_rows = [w.X[a * w.rows_per_agent:(a + 1) * w.rows_per_agent].cpu() for a in range(w.n_agents)]
+    lens_list = w.lens.cpu().tolist()
+    Xh = torch.empty(w.M, w.shape.hidden, dtype=torch.bfloat16).pin_memory()
+    arsh = torch.empty(w.n_agents + 1, dtype=torch.int32).pin_memory()
     lensh = w.lens.cpu().pin_memory()
     Hh = torch.empty(w.M, w.shape.hidden, dtype=torch.float32).pin_memory()
-    for _ in range(max(1, args.warmup)):
+
+    def e2e_step():
+        Xp, _, _, ars_p = q.pack_rows(agent_rows, lens_list, w.shape.hidden)
+        Xh.copy_(Xp)
+        arsh.copy_(ars_p)
         w.model.decode_step_host(Xh, w.M, arsh, w.n_agents, w.rows_per_agent, lensh, Hh, w.ws, stream)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
     barrier(ws)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        w.model.decode_step_host(Xh, w.M, arsh, w.n_agents, w.rows_per_agent, lensh, Hh, w.ws, stream)
+        e2e_step()
     e2e_ms = max_over_ranks((time.perf_counter() - t0) * 1e3 / args.steps, ws)
     h2d = Xh.numel() * 2 + arsh.numel() * 4 + lensh.numel() * 4
     d2h = Hh.numel() * 4
@@ -719,7 +772,7 @@ def run_sched(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--steps", type=int, default=400)  # ~2.4 s timed at ~6 ms per step
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="stack12_ctx1k", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -737,8 +790,20 @@ def main():
         return run_kernel(args)
     if args.trace:
         return run_trace(args)
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        # one process per GPU: re-launch under torch.distributed.run on this node
+        import socket
+        with socket.socket() as sk:
+            sk.bind(("127.0.0.1", 0))
+            port = sk.getsockname()[1]
+        cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={args.gpus}",
+               "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__), *sys.argv[1:]]
+        return subprocess.call(cmd)
     ws, rank, local = (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
                        int(os.environ.get("LOCAL_RANK", "0")))
+    if ws != args.gpus:
+        print(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={ws}", file=sys.stderr)
+        return 2
     if args.impl == "reference":
         return run_reference(args, ws, rank)
     ws, rank, local = dist_setup()

@@ -115,12 +115,14 @@ int qad_q6k_pack(const void *W, int N, int K, void *W_packed, void *stream);
  * streams are decoding, and plain C integrations that only hold pointers to
  * buffers owned elsewhere. Arguments and result are those of qad_q4k_gemm
  * without the workspace: the scratch is a fixed array of
- * qad_q4k_gemm_noalloc_scratch_bytes() bytes (1 MiB; enough for K <= 30464 at
- * 16 rows) in device memory that every GPU loading this library holds until
- * the process exits. Calls that need more scratch fail with
- * QAD_ERR_UNSUPPORTED before any launch. The first call on each device looks
- * up the array's device address (cudaGetSymbolAddress); make that first call
- * before any stream capture. All calls on a device share the one array, and
+ * qad_q4k_gemm_noalloc_scratch_bytes() bytes (1 MiB; enough for K <= 30464,
+ * for every row count M from 1 to 16) in device memory that every GPU loading
+ * this library holds until the process exits. Calls that need more scratch
+ * fail with QAD_ERR_UNSUPPORTED before any launch. Outside stream capture each
+ * call looks up the array's device address (cudaGetSymbolAddress), so a device
+ * reset in between is harmless; a call whose stream is being captured reuses
+ * the address an earlier call found on that device, so make one call before
+ * any stream capture (a first call during capture fails with QAD_ERR_INVALID). All calls on a device share the one array, and
  * each call rewrites the parts it reads, so calls that overlap on the GPU
  * (different streams, or different host threads without ordering) race and
  * must be serialised by the caller. Nothing here calls cudaMalloc, cudaFree
@@ -291,6 +293,12 @@ int qad_pack_rows(const qad_agent_rows *agents, int n_agents, int hidden, int ma
                   int *row_agent, int *row_pos, int *agent_row_start);
 
 /* ---------------------------------------------------------------- decode step
+ * [OpenJet page], section 只搬一次权重 (move the weights once): one model
+ * serves several coding agents; its quantized weights are read from memory once
+ * per step for the stacked rows of all active agents, and each agent keeps its
+ * own KV cache. The page ships it as one persistent kernel over a Q4_K_M model
+ * (intro: Qwen3.8-27B Q4_K_M); here the model is the stack of decoder layers
+ * below, Q4_K matrices with a Q6_K-like down projection.
  * A model is a stack of decoder layers whose weights and KV caches the caller
  * owns. Per layer (device pointers):
  *   w_qkv  Q4_K [(n_qh + 2 n_kvh) hd][hidden]   rows: q heads, k heads, v heads
@@ -322,7 +330,11 @@ typedef struct qad_model qad_model;
 int qad_model_create(const qad_model_desc *desc, qad_model **out);
 void qad_model_destroy(qad_model *model);
 
-/* One decode-and-verify forward step for the packed batch, per layer:
+/* One decode-and-verify forward step for the packed batch ([OpenJet page],
+ * section 只搬一次权重: every agent's next token and its drafts form the rows
+ * of one batch, each weight read once is used for every row, the drafts are
+ * checked in the same pass, and each agent's rows attend over that agent's own
+ * cache), per layer:
  *   x1 = bf16(rmsnorm(h)); qkv = x1 Wqkv^T; Q = bf16(q); append bf16 k, v of
  *   every row at its position; o = attention; h += bf16(o) Wo^T;
  *   x2 = bf16(rmsnorm(h)); gu = x2 Wgu^T; h += bf16(silu(gate)*up) Wdown^T.

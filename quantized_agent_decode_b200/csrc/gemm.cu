@@ -942,12 +942,17 @@ extern "C" int qad_q6k_gemm(const void *W, int N, int K, const uint16_t *X, int 
 // For them the activation-fragment scratch lives in a fixed array of device
 // memory that every GPU loading this library keeps until the process exits.
 
-static constexpr size_t NOALLOC_SCRATCH_BYTES = (size_t)1 << 20;  // 1 MiB: K <= 30720 at 16 rows
+// 1 MiB holds the operand records of K <= 30464 (119 blocks of 8,768 bytes) for
+// every row count from 1 to 16: the record layout does not depend on M.
+static constexpr size_t NOALLOC_SCRATCH_BYTES = (size_t)1 << 20;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[NOALLOC_SCRATCH_BYTES];
 
-// The array's host-side name is not a device address: resolve it once per
-// device (with that device current) and reuse the address.
-static void *noalloc_scratch_address(int *rc)
+// The array's host-side name is not a device address: resolve it with the
+// device current. Outside stream capture the address is looked up on every call
+// (a device reset reloads the module and may move the array); a call made while
+// its stream is being captured reuses the address found by an earlier call on
+// that device, and fails if there is none.
+static void *noalloc_scratch_address(cudaStream_t stream, int *rc)
 {
     static void *addr[64] = {};
     static std::mutex mu;
@@ -961,8 +966,14 @@ static void *noalloc_scratch_address(int *rc)
         *rc = qad::fail(QAD_ERR_UNSUPPORTED, "qad_q4k_gemm_noalloc: device ordinal %d >= 64", dev);
         return nullptr;
     }
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    e = cudaStreamIsCapturing(stream, &cap);
+    if (e != cudaSuccess) {
+        *rc = qad::cuda_check(e, "qad_q4k_gemm_noalloc: cudaStreamIsCapturing");
+        return nullptr;
+    }
     std::lock_guard<std::mutex> lock(mu);
-    if (!addr[dev]) {
+    if (cap == cudaStreamCaptureStatusNone) {
         void *p = nullptr;
         e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
         if (e != cudaSuccess) {
@@ -970,6 +981,12 @@ static void *noalloc_scratch_address(int *rc)
             return nullptr;
         }
         addr[dev] = p;
+    } else if (!addr[dev]) {
+        *rc = qad::fail(QAD_ERR_INVALID,
+                        "qad_q4k_gemm_noalloc: first call on device %d made during stream capture; make one call "
+                        "before capturing",
+                        dev);
+        return nullptr;
     }
     *rc = QAD_OK;
     return addr[dev];
@@ -992,7 +1009,7 @@ extern "C" int qad_q4k_gemm_noalloc(const void *W, int N, int K, const uint16_t 
                          "(use qad_q4k_gemm with a workspace)",
                          K, M, need, NOALLOC_SCRATCH_BYTES);
     int rc = QAD_OK;
-    void *scratch = noalloc_scratch_address(&rc);
+    void *scratch = noalloc_scratch_address((cudaStream_t)stream, &rc);
     if (!scratch)
         return rc;
     return gemm_entry(4, W, N, K, X, M, Y, accumulate, scratch, NOALLOC_SCRATCH_BYTES, stream);
