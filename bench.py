@@ -769,6 +769,77 @@ def run_sched(args):
     return 0
 
 
+def run_ttft(args):
+    """Next-request time to first token with and without KV reuse: agents 0-2 keep
+    decoding (1024 cached tokens, 1 token + 2 drafts each) while agent 3, whose
+    cache holds its previous 23000-token context, sends a request that appends 512
+    new tokens. With reuse (qad_common_prefix of the old and new token sequences)
+    only the suffix is prefilled; without it the whole 23512-token prompt is fed
+    from an empty cache in 2048-row chunks. Each chunk rides with the decode rows
+    in one mixed step; the first token is the argmax of the vocabulary head over
+    the prompt's last row. Device time by CUDA events around the whole sequence."""
+    import quantized_agent_decode_b200 as q
+    from quantized_agent_decode_b200 import build
+    build.build()
+    PREV, NEW, CHUNK, A, VOCAB = 23000, 512, 2048, 4, 151936
+    w = Workload("stack12_ctx1k", ctx=PREV + NEW + 16)
+    H = w.shape.hidden
+    g = synth.torch_gen(SEED, "cuda", 93)
+    X = synth.bf16_normal_torch(g, (9 + CHUNK, H), "cuda")
+    W_head = synth.q4k_matrix_torch(g, VOCAB, H, "cuda")
+    Hout = torch.empty(9 + CHUNK, H, dtype=torch.float32, device="cuda")
+    ws_mix = q.alloc_ws(w.model.mixed_ws_bytes(9, CHUNK))
+    ars_d = torch.tensor([0, 3, 6, 9, 9], dtype=torch.int32, device="cuda")
+    lens_d = torch.zeros(A, dtype=torch.int32, device="cuda")
+    head_ars = torch.tensor([0, 1], dtype=torch.int32, device="cuda")
+    head_tok = torch.zeros(1, dtype=torch.int32, device="cuda")
+    head_len = torch.zeros(1, dtype=torch.int32, device="cuda")
+    first_tok = torch.zeros(1, dtype=torch.int32, device="cuda")
+    n_acc = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws_head = q.alloc_ws(q.verify_ws_bytes(H, VOCAB, 1))
+    rng = np.random.default_rng(SEED)
+    old_tokens = rng.integers(0, VOCAB, PREV).tolist()
+    new_tokens = old_tokens + rng.integers(0, VOCAB, NEW).tolist()
+
+    def request(start):
+        """Prefill new_tokens[start:] of agent 3 in chunks beside the decode rows, then the head."""
+        pos = start
+        while pos < len(new_tokens):
+            C = min(CHUNK, len(new_tokens) - pos)
+            lens_d.copy_(torch.tensor([1024, 1024, 1024, pos], dtype=torch.int32))
+            w.model.mixed_step(X[:9 + C], 9, ars_d, A, 3, lens_d, 3, pos, C, Hout, ws_mix)
+            pos += C
+        q.verify_step(Hout[8 + C:9 + C], 1, H, W_head, VOCAB, head_ars, 1, head_tok, head_len, first_tok, n_acc,
+                      ws=ws_head)
+        return pos
+
+    def timed(start):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record()
+        request(start)
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1)
+
+    reuse = q.common_prefix(old_tokens, new_tokens)
+    timed(reuse)  # warm-up of both shapes
+    timed(PREV + NEW - CHUNK)
+    t_reuse = statistics.median(timed(reuse) for _ in range(5))
+    t_full = statistics.median(timed(0) for _ in range(2))
+    out = {"workload": "64-layer stack; agents 0-2 decoding at 1024 cached tokens (3 rows each) while agent 3 "
+                       f"sends a request of {NEW} new tokens after a {PREV}-token context",
+           "reused_prefix_tokens": reuse, "chunk_rows": CHUNK,
+           "ttft_ms_with_kv_reuse": round(t_reuse, 2),
+           "ttft_ms_without_reuse": round(t_full, 2),
+           "speedup": round(t_full / t_reuse, 1),
+           "mixed_steps": {"with_reuse": -(-NEW // CHUNK), "without": -(-(PREV + NEW) // CHUNK)},
+           "head": f"Q4_K vocabulary head {VOCAB} x {H}, argmax of the prompt's last row",
+           "device_status": q.device_status(), "dense_status": q.dense_status()}
+    print(json.dumps(out), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -781,11 +852,15 @@ def main():
                     help="time one kernel of the step instead (profiler captures)")
     ap.add_argument("--rows", type=int, default=12)
     ap.add_argument("--trace", action="store_true", help="print the per-launch device timeline of one step")
+    ap.add_argument("--ttft", action="store_true",
+                    help="next-request time to first token with and without KV reuse (23000-token context)")
     ap.add_argument("--sched", action="store_true",
                     help="decode rate of three agents while a 20480-token prompt is chunked in (scheduler policies)")
     args = ap.parse_args()
     if args.sched:
         return run_sched(args)
+    if args.ttft:
+        return run_ttft(args)
     if args.kernel:
         return run_kernel(args)
     if args.trace:
