@@ -273,14 +273,19 @@ __global__ void __launch_bounds__(pt::THREADS, 1) k_prefill_attn_tc(const __grid
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(&s_free[X]);
-            // tiles below every row's causal limit: no mask, maximum on raw scores
+            // scores in the log2 domain, rounded once: the maximum and every exponent below use the same
+            // values, so s - m is exact where it matters and P <= 2^15 holds whatever the scores' size
+            // (computing the maximum and the exponents with different roundings lets s - m exceed the slack
+            // by the scores' rounding error, which is large once |s| is large). Tiles below every row's
+            // causal limit skip the mask.
             const bool interior = kb + KT - 1 <= lim_blk;
             float mx = -INFINITY;
             if (interior) {
 #pragma unroll
-                for (int i = 0; i < KT; ++i)
+                for (int i = 0; i < KT; ++i) {
+                    x[i] *= p.scale_log2;
                     mx = fmaxf(mx, x[i]);
-                mx *= p.scale_log2;
+                }
             } else {
 #pragma unroll
                 for (int i = 0; i < KT; ++i) {
@@ -297,14 +302,12 @@ __global__ void __launch_bounds__(pt::THREADS, 1) k_prefill_attn_tc(const __grid
                 m = mn;
             }
             const bool none = m == -INFINITY;
-            const float sc = interior ? p.scale_log2 : 1.f;
-            const float nm = none ? 0.f : P_LOG2_SCALE - m;
             uint32_t pw[KT / 2];
             float psum = 0.f;
 #pragma unroll
             for (int i = 0; i < KT / 2; ++i) {
-                const float p0 = none ? 0.f : ex2_approx(fmaf(x[2 * i], sc, nm));
-                const float p1 = none ? 0.f : ex2_approx(fmaf(x[2 * i + 1], sc, nm));
+                const float p0 = none ? 0.f : ex2_approx((x[2 * i] - m) + P_LOG2_SCALE);
+                const float p1 = none ? 0.f : ex2_approx((x[2 * i + 1] - m) + P_LOG2_SCALE);
                 psum += p0 + p1;
                 pw[i] = pack_half2(p0, p1);
             }

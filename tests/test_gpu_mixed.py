@@ -96,3 +96,83 @@ def test_mixed_step_rejects_bad_arguments(q):
         st.model.mixed_step(X, 2, st.arsd, st.A, 2, st.lensd, st.A, 0, 8, H, ws)
     with pytest.raises(q.QadError):  # workspace too small
         st.model.mixed_step(X, 2, st.arsd, st.A, 2, st.lensd, 1, 5, 8, H, ws[:1024])
+
+
+def test_mixed_step_full_stack_2048_chunk_sampled(q, orc):
+    """The mixed step at full size: the 64-layer bench stack, agents 0-2 decoding
+    3 rows each at 23000 cached tokens and agent 3's 2048-row prompt chunk at
+    positions 23000 .. 25047. Layer 0 and the deepest layer whose input is still
+    finite (at least layer 32) teacher-forced from the step's own
+    intermediates: every x1, x2 and act row, 96 sampled output columns of each
+    GEMM, the k/v append of every row, the attention of every decode row and of
+    24 sampled chunk rows (one oracle call per row, at its own position)."""
+    import bench
+    from test_gpu_step import bf16_close, dbg_views
+    CTX, C, rpa = 23000, 2048, 3
+    w = bench.Workload("stack12_ctx23k", ctx=CTX + C + 4)
+    sh = w.shape
+    H, I = sh.hidden, sh.inter
+    nq, nkv = sh.n_qh * 128, sh.n_kvh * 128
+    nqkv = nq + 2 * nkv
+    A, M = 4, 3 * rpa
+    R = M + C
+    rng = np.random.default_rng(7)
+    X = synth.bf16_normal_np(SEED, 9300, (R, H))
+    Xd = torch.from_numpy(X.view(np.int16)).view(torch.bfloat16).cuda()
+    ars = np.array([0, 3, 6, 9, 9], np.int32)
+    lens = np.array([CTX] * A, np.int32)
+    ars_d, lens_d = torch.from_numpy(ars).cuda(), torch.from_numpy(lens).cuda()
+    Hd = torch.empty(R, H, dtype=torch.float32, device="cuda")
+    ws = q.alloc_ws(w.model.mixed_ws_bytes(M, C))
+    dbg = w.model.set_debug_mixed(M, C)
+    w.model.mixed_step(Xd, M, ars_d, A, rpa, lens_d, 3, CTX, C, Hd, ws)
+    torch.cuda.synchronize()
+    assert q.device_status() == 0 and q.dense_status() == 0
+    ars_o = np.array([0, 3, 6, 9, R], np.int32)  # agent 3 holds the chunk rows
+    cols = lambda N: np.sort(rng.choice(N, size=96, replace=False))  # noqa: E731
+
+    def dense(fmt, Wm, N, K, Xb, Y, base=None):
+        sel = cols(N)
+        Yr, Aabs = orc.gemm_rows(fmt, Wm, K, sel, Xb)
+        ref = Yr if base is None else base[:, sel] + Yr
+        slack = 0 if base is None else 8 * 2.0 ** -24 * (np.abs(base[:, sel]) + np.abs(Yr))
+        ratio = np.abs(Y[:, sel].astype(np.float64) - ref) / (1e-3 * Aabs + slack + 1e-30)
+        assert ratio.max() <= 1.0, ratio.max()
+
+    # The synthetic stack's residual grows layer by layer (random weights); the chunk rows overflow fp32
+    # near the last layers. The deep layer checked is the deepest whose input is still finite.
+    deep = next(l for l in range(sh.n_layers - 1, 0, -1)
+                if np.isfinite(dbg_views(dbg, l - 1, R, H, I, nq, nqkv)["hout"]).all())
+    assert deep >= sh.n_layers // 2, deep
+    for l in (0, deep):
+        v = dbg_views(dbg, l, R, H, I, nq, nqkv)
+        if l == 0:
+            h_in = orc.bf16_array_to_f64(X).astype(np.float32)
+        else:
+            h_in = dbg_views(dbg, l - 1, R, H, I, nq, nqkv)["hout"]
+        assert bf16_close(v["x1"], orc.rmsnorm_bf16(h_in.astype(np.float64)), orc)
+        dense(4, w.w_qkv[l].cpu().numpy(), nqkv, H, v["x1"], v["qkv"])
+        kc = _bits(w.kc[l]).reshape(w.kc[l].shape)
+        vc = _bits(w.vc[l]).reshape(w.vc[l].shape)
+        kvb = orc.f64_array_to_bf16(v["qkv"][:, nq:].astype(np.float64))
+        pos = np.concatenate([lens[a] + np.arange(ars_o[a + 1] - ars_o[a]) for a in range(A)])
+        agent = np.repeat(np.arange(A), np.diff(ars_o))
+        assert np.array_equal(kc[agent, :, pos].reshape(R, -1), kvb[:, :nkv])
+        assert np.array_equal(vc[agent, :, pos].reshape(R, -1), kvb[:, nkv:])
+        Qb = orc.f64_array_to_bf16(v["qkv"][:, :nq].astype(np.float64)).reshape(R, sh.n_qh, 128)
+        o = orc.bf16_array_to_f64(v["attn"]).reshape(R, sh.n_qh, 128)
+        O_ref, B = orc.decode_attn(Qb[:M], kc[:3], vc[:3], lens[:3], ars[:4], sh.n_qh, sh.n_kvh, 128, w.kv_cap)
+        assert (np.abs(o[:M] - O_ref) <= 2e-3 * B + np.abs(O_ref) * 2.0 ** -8 + 1e-30).all()
+        for j in np.sort(rng.choice(C, size=24, replace=False)):
+            r = M + int(j)
+            O1, B1 = orc.decode_attn(Qb[r:r + 1], kc[3:4], vc[3:4], [CTX + int(j)], [0, 1], sh.n_qh, sh.n_kvh, 128,
+                                     w.kv_cap)
+            assert (np.abs(o[r:r + 1] - O1) <= 2e-3 * B1 + np.abs(O1) * 2.0 ** -8 + 1e-30).all(), j
+        dense(4, w.w_o[l].cpu().numpy(), H, nq, v["attn"], v["hmid"], base=h_in.astype(np.float64))
+        assert bf16_close(v["x2"], orc.rmsnorm_bf16(v["hmid"].astype(np.float64)), orc)
+        dense(4, w.w_gu[l].cpu().numpy(), 2 * I, H, v["x2"], v["gu"])
+        gu = v["gu"].astype(np.float64)
+        assert bf16_close(v["act"], orc.silu_mul_bf16(gu[:, :I], gu[:, I:]), orc, frac=5e-3)
+        dense(6, w.down_gguf(l).cpu().numpy(), H, I, v["act"], v["hout"], base=v["hmid"].astype(np.float64))
+    last = dbg_views(dbg, sh.n_layers - 1, R, H, I, nq, nqkv)["hout"]
+    assert np.array_equal(last, Hd.cpu().numpy(), equal_nan=True)

@@ -71,6 +71,33 @@ def test_prefill_attn_parity(q, orc, len_, C, n_qh, n_kvh):
     _check(orc, _bits(O), O_ref, B)
 
 
+def _scaled(bits, f):
+    """bf16 bits of f times the values (N(0,1) draws scaled to large magnitudes)."""
+    import oracle as o
+    return o.f64_array_to_bf16(o.bf16_array_to_f64(bits) * f)
+
+
+@pytest.mark.parametrize("len_,C,scale", [(300, 200, 1.5e4), (0, 130, 3e3), (1000, 64, 5e2)])
+def test_prefill_attn_large_scores(q, orc, len_, C, scale):
+    """q, k, v of order 1e3..1e4 (as a deep synthetic stack produces): scaled
+    scores reach ~1e9 in the log2 domain, where fp32 spacing is ~100; the
+    softmax must stay finite and equal to the oracle's (close to a hard max)."""
+    n_qh, n_kvh = 16, 4
+    cap = len_ + C + 3
+    Q = _scaled(synth.bf16_normal_np(SEED, 720 + C, (C, n_qh, 128)), scale)
+    Kc = _scaled(synth.bf16_normal_np(SEED, 721 + C, (n_kvh, cap, 128)), scale)
+    Vc = _scaled(synth.bf16_normal_np(SEED, 722 + C, (n_kvh, cap, 128)), min(scale, 1e4))
+    O = torch.zeros(C, n_qh, 128, dtype=torch.bfloat16, device="cuda")
+    q.prefill_attn(_dev(Q), _dev(Kc), _dev(Vc), len_, C, cap, n_qh, n_kvh, 128, O)
+    torch.cuda.synchronize()
+    assert q.prefill_status() == 0
+    o = _bits(O)
+    assert np.isfinite(orc.bf16_array_to_f64(o)).all()
+    O_ref, B = orc.decode_attn(Q, Kc[None], Vc[None], np.array([len_], np.int32), np.array([0, C], np.int32),
+                               n_qh, n_kvh, 128, cap)
+    _check(orc, o, O_ref, B)
+
+
 def test_prefill_attn_chunk_after_23k_tokens(q, orc):
     """A 2048-row chunk after 23000 cached tokens (48/8 heads), sampled rows against the
     oracle row by row (row j is a one-row agent with len + j cached tokens)."""
