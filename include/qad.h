@@ -137,6 +137,21 @@ int qad_q4k_gemm_noalloc(const void *W, int N, int K, const uint16_t *X, int M, 
  * incomplete). Synchronous (reads device memory); reset != 0 clears it.
  * Returns the status (>= 0) or a negative QAD_ERR_* code. */
 int qad_device_status(int reset);
+
+/* Test hook for the bounded waits (no counterpart on the pages): makes the
+ * producer of CTA 0 of the next launches of one pipeline stop issuing copies,
+ * so that CTA's waits on them run out and the kernel takes its early exit
+ * (records a status, waits for the copies and tensor-core work it already
+ * issued, frees its tensor memory, returns) instead of completing.
+ *   kernel = 0: the skinny GEMM (qad_q4k_gemm, qad_q6k_gemm and the decode
+ *               step); no operand-record copy from CTA 0's unit `at` on
+ *               (its status: qad_device_status);
+ *   kernel = 1: the dense GEMM (qad_q4k_gemm_dense, qad_q6k_gemm_dense);
+ *               no copy from CTA 0's activation k-step `at` on (qad_dense_status).
+ * at < 0 switches the hook off. The outputs of an affected launch are
+ * incomplete. Each timed-out wait takes about 2 s. Synchronous (writes device
+ * memory). Returns QAD_OK, or QAD_ERR_INVALID for an unknown kernel. */
+int qad_debug_stall(int kernel, int at);
 int qad_q4k_gemm(const void *W, int N, int K, const uint16_t *X, int M, float *Y, int accumulate,
                  void *ws, size_t ws_bytes, void *stream);
 int qad_q6k_gemm(const void *W, int N, int K, const uint16_t *X, int M, float *Y, int accumulate,

@@ -58,6 +58,7 @@ SIGNATURES = {
     "qad_q6k_unpack": (C.c_int, [C.c_void_p, C.c_longlong] + [C.c_void_p] * 3 + [C.c_void_p]),
     "qad_gemm_ws_bytes": (C.c_size_t, [C.c_int, C.c_int]),
     "qad_device_status": (C.c_int, [C.c_int]),
+    "qad_debug_stall": (C.c_int, [C.c_int, C.c_int]),
     "qad_q6k_packed_bytes": (C.c_size_t, [C.c_longlong, C.c_int]),
     "qad_q6k_pack": (C.c_int, [C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_void_p]),
     "qad_q4k_gemm_noalloc_scratch_bytes": (C.c_size_t, []),
@@ -168,6 +169,12 @@ def alloc_ws(nbytes: int, device="cuda") -> torch.Tensor:
 def device_status(reset: bool = True) -> int:
     """0 if every GEMM pipeline wait on this device completed since the last reset."""
     return _check(lib().qad_device_status(int(reset)), "qad_device_status")
+
+
+def debug_stall(kernel: int, at: int) -> None:
+    """Test hook: CTA 0 of the skinny (kernel 0) or dense (kernel 1) GEMM stops
+    issuing copies from its step `at` on (at < 0: off), so its waits run out."""
+    _check(lib().qad_debug_stall(int(kernel), int(at)), "qad_debug_stall")
 
 
 # ------------------------------------------------------------------ codecs

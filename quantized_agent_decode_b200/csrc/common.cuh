@@ -328,14 +328,22 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32
 }
 // Bounded wait that sleeps ~sleep_ns between polls, so a waiting warp gives its
 // issue slots to the warps doing the work (a try_wait that returns at once
-// would otherwise be re-issued in a tight loop). Gives up after ~2 s.
+// would otherwise be re-issued in a tight loop). Gives up once 2 s have passed
+// on the global timer (checked every 256 polls), or after 2e9 / sleep_ns polls
+// whatever the timer says.
+constexpr unsigned long long MBAR_WAIT_LIMIT_NS = 2000000000ull;
 __device__ __forceinline__ bool mbar_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t sleep_ns)
 {
+    if (mbar_try_wait(bar, parity, 0))
+        return true;
+    const unsigned long long t0 = gtimer();
     const uint32_t limit = 2000000000u / (sleep_ns ? sleep_ns : 1u);
     for (uint32_t i = 0; i < limit; ++i) {
+        __nanosleep(sleep_ns);
         if (mbar_try_wait(bar, parity, 0))
             return true;
-        __nanosleep(sleep_ns);
+        if ((i & 255) == 255 && gtimer() - t0 > MBAR_WAIT_LIMIT_NS)
+            return false;
     }
     return false;
 }

@@ -38,6 +38,9 @@
 namespace qad {
 
 __device__ int g_dense_status;
+// Test hook (qad_debug_stall): v > 0 makes the producer of CTA 0 issue no copy
+// from its activation step v - 1 on, so that CTA's pipeline waits run out.
+__device__ int g_dense_stall;
 
 namespace dn {
 constexpr int TN = 128;            // weight rows per tile (MMA M)
@@ -279,10 +282,11 @@ __global__ void __launch_bounds__(dn::THREADS, 1) k_dense_gemm(const __grid_cons
     if (warp == 0) {
         // ------------------------------------------------ producer
         if (lane == 0) {
+            const int stall = blockIdx.x == 0 ? *(volatile int *)&g_dense_stall - 1 : -1;
             int bk = 0, ks = 0;
-            for (int t = blockIdx.x; t < tiles && !bad(); t += gridDim.x) {
+            for (int t = blockIdx.x; t < tiles && !bad() && ks != stall; t += gridDim.x) {
                 const int nt = t / a.mt, mt = t % a.mt;
-                for (int blk = 0; blk < a.nblk && !bad(); ++blk) {
+                for (int blk = 0; blk < a.nblk && !bad() && ks != stall; ++blk) {
                     const int s = bk % SR;
                     if (bk >= SR && !mbar_wait(&raw_empty[s], ((bk / SR) - 1) & 1)) {
                         fail(ST_RAW);
@@ -294,7 +298,7 @@ __global__ void __launch_bounds__(dn::THREADS, 1) k_dense_gemm(const __grid_cons
                     if (FMT == 6)
                         tma_load_2d(st + R::W, md, blk & ~7, nt * TN, &raw_full[s]);
                     ++bk;
-                    for (int kk = 0; kk < 4; ++kk) {
+                    for (int kk = 0; kk < 4 && ks != stall; ++kk) {
                         const int sb = ks % SB;
                         if (ks >= SB && !mbar_wait(&b_empty[sb], ((ks / SB) - 1) & 1)) {
                             fail(ST_B);
@@ -529,6 +533,14 @@ extern "C" size_t qad_dense_gemm_ws_bytes(int K, int M)
         return 0;
     return qad::dense_ws_bytes(K, M);
 }
+
+namespace qad {
+int dense_set_stall(int at)
+{
+    const int v = at < 0 ? 0 : at + 1;
+    return cuda_check(cudaMemcpyToSymbol(g_dense_stall, &v, sizeof(int)), "dense stall hook");
+}
+}  // namespace qad
 
 extern "C" int qad_dense_status(int reset)
 {

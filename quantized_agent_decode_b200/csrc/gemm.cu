@@ -37,6 +37,7 @@
 
 #include <mutex>
 
+#include "dense.cuh"
 #include "gemm.cuh"
 
 
@@ -45,6 +46,9 @@ namespace qad {
 // Set by a GEMM whose pipeline wait timed out (1: a consumer, 2: the producer);
 // read and cleared by qad_device_status().
 __device__ int g_gemm_status;
+// Test hook (qad_debug_stall): v > 0 makes the record producer of CTA 0 issue no
+// operand copy from its unit v - 1 on, so that CTA's pipeline waits run out.
+__device__ int g_gemm_stall;
 
 // ------------------------------------------------------------- operand records
 // e(r,b) puts the block's largest |x| in [512, 1024): fp16 holds every bf16
@@ -536,8 +540,9 @@ __global__ void __launch_bounds__(tg::THREADS, 1) k_qgemm_tc(const __grid_consta
         if (a.trace && lane == 0)
             atomicMin(a.trace + 1, gtimer());  // past the dependency wait
         if (lane == 0) {
+            const int stall = blockIdx.x == 0 ? *(volatile int *)&g_gemm_stall - 1 : -1;
             int i = 0;
-            for (; i < n_units && !bad(); ++i) {
+            for (; i < n_units && !bad() && i != stall; ++i) {
                 const int b = (u0 + i) % a.nblk, bs = i % SB;
                 if (i >= SB && !QAD_TG_WAIT_SLOW(&b_empty[bs], ((i / SB) - 1) & 1)) {
                     fail(ST_REC);
@@ -856,6 +861,23 @@ extern "C" int qad_device_status(int reset)
             return qad::cuda_check(e, "qad_device_status reset");
     }
     return v;
+}
+
+namespace qad {
+int gemm_set_stall(int at)
+{
+    const int v = at < 0 ? 0 : at + 1;
+    return cuda_check(cudaMemcpyToSymbol(g_gemm_stall, &v, sizeof(int)), "gemm stall hook");
+}
+}  // namespace qad
+
+extern "C" int qad_debug_stall(int kernel, int at)
+{
+    if (kernel == 0)
+        return qad::gemm_set_stall(at);
+    if (kernel == 1)
+        return qad::dense_set_stall(at);
+    return qad::fail(QAD_ERR_INVALID, "qad_debug_stall: unknown kernel %d", kernel);
 }
 
 extern "C" size_t qad_gemm_ws_bytes(int K, int M)

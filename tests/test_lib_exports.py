@@ -149,3 +149,11 @@ def test_q8_and_mixed_argument_checks_and_cache_sizes(qlib):
     codes = A * kvh * cap * 128
     assert qlib.kv_cache_bytes(qlib.KV_Q8_0, A, kvh, cap) == (codes + 255) // 256 * 256 + A * kvh * cap * 4 * 2
     assert qlib.kv_cache_bytes(7, A, kvh, cap) == 0 and qlib.kv_cache_bytes(qlib.KV_Q8_0, A, kvh, cap, hd=64) == 0
+
+
+def test_debug_stall_rejects_unknown_kernel(qlib):
+    """The wait-timeout test hook validates its kernel index before any CUDA call."""
+    with pytest.raises(qlib.QadError):
+        qlib.debug_stall(7, 0)
+    with pytest.raises(qlib.QadError):
+        qlib.debug_stall(-1, 0)
