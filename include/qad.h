@@ -147,7 +147,9 @@ int qad_device_status(int reset);
  *               step); no operand-record copy from CTA 0's unit `at` on
  *               (its status: qad_device_status);
  *   kernel = 1: the dense GEMM (qad_q4k_gemm_dense, qad_q6k_gemm_dense);
- *               no copy from CTA 0's activation k-step `at` on (qad_dense_status).
+ *               no copy from CTA 0's activation k-step `at` on (qad_dense_status);
+ *   kernel = 2: the prefill attention (qad_prefill_attn and the mixed step);
+ *               no K/V tile from CTA (0, 0)'s tile `at` on (qad_prefill_status).
  * at < 0 switches the hook off. The outputs of an affected launch are
  * incomplete. Each timed-out wait takes about 2 s. Synchronous (writes device
  * memory). Returns QAD_OK, or QAD_ERR_INVALID for an unknown kernel. */

@@ -172,8 +172,9 @@ def device_status(reset: bool = True) -> int:
 
 
 def debug_stall(kernel: int, at: int) -> None:
-    """Test hook: CTA 0 of the skinny (kernel 0) or dense (kernel 1) GEMM stops
-    issuing copies from its step `at` on (at < 0: off), so its waits run out."""
+    """Test hook: CTA 0 of the skinny GEMM (kernel 0), the dense GEMM (1) or the
+    prefill attention (2) stops issuing copies from its step `at` on (at < 0:
+    off), so its waits run out."""
     _check(lib().qad_debug_stall(int(kernel), int(at)), "qad_debug_stall")
 
 

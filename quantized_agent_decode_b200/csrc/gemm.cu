@@ -877,6 +877,8 @@ extern "C" int qad_debug_stall(int kernel, int at)
         return qad::gemm_set_stall(at);
     if (kernel == 1)
         return qad::dense_set_stall(at);
+    if (kernel == 2)
+        return qad::prefill_set_stall(at);
     return qad::fail(QAD_ERR_INVALID, "qad_debug_stall: unknown kernel %d", kernel);
 }
 

@@ -62,6 +62,9 @@ enum { ST_KV = 1, ST_S = 2, ST_P = 3, ST_PV = 4, ST_DONE = 5, ST_VT = 6 };
 }  // namespace pt
 
 __device__ int g_prefill_status;
+// Test hook (qad_debug_stall): v > 0 makes the producer of CTA (0, 0) issue no
+// K/V tile from its tile v - 1 on, so that CTA's pipeline waits run out.
+__device__ int g_prefill_stall;
 
 struct PfMaps {
     CUtensorMap k, v;  // [n_kvh * kv_cap][128] bf16 as (8 dims, key, dim chunk), boxes of 64 keys
@@ -135,8 +138,9 @@ __global__ void __launch_bounds__(pt::THREADS, 1) k_prefill_attn_tc(const __grid
     if (warp == 8) {
         // ------------------------------------------------ producer: K and V tiles by TMA
         if (lane == 0) {
+            const int stall = blockIdx.x == 0 && blockIdx.y == 0 ? *(volatile int *)&g_prefill_stall - 1 : -1;
             int j = 0;
-            for (; j < ntiles && !bad(); ++j) {
+            for (; j < ntiles && !bad() && j != stall; ++j) {
                 const int s = j % NS;
                 if (j >= NS && !mbar_wait(&kv_free[s], ((j / NS) - 1) & 1)) {
                     fail(ST_KV);
@@ -427,6 +431,14 @@ extern "C" int qad_prefill_attn(const uint16_t *Q, const uint16_t *Kc, const uin
         return qad::fail(QAD_ERR_INVALID, "qad_prefill_attn: Q, caches and O must be 16-byte aligned");
     return qad::launch_prefill_attn(Q, Kc, Vc, len, C, kv_cap, n_qh, n_kvh, scale, O, (cudaStream_t)stream);
 }
+
+namespace qad {
+int prefill_set_stall(int at)
+{
+    const int v = at < 0 ? 0 : at + 1;
+    return cuda_check(cudaMemcpyToSymbol(g_prefill_stall, &v, sizeof(int)), "prefill stall hook");
+}
+}  // namespace qad
 
 extern "C" int qad_prefill_status(int reset)
 {

@@ -8,11 +8,12 @@ qad_debug_stall makes the producer of CTA 0 stop issuing copies part-way, so
 that CTA's consumers wait for data nothing will deliver (no fault, no trap:
 the wait simply never completes).
 
-Checked for the skinny and the dense GEMM: the call returns within seconds,
-the status word reports the timed-out wait, and the device is still usable:
-the same GEMM right after, with the hook off, matches the oracle and reports
-no timeout. That second launch also allocates all of tensor memory on every
-SM, which it could not if the aborted CTA had kept its columns.
+Checked for the skinny and the dense GEMM and the prefill attention: the call
+returns within seconds, the status word reports the timed-out wait, and the
+device is still usable: the same launch right after, with the hook off,
+matches the oracle and reports no timeout. That second launch also allocates
+tensor memory again, which it could not if the aborted CTA had kept its
+columns.
 """
 import time
 
@@ -91,4 +92,30 @@ def test_dense_gemm_wait_timeout_then_recovers(q, orc):
     assert q.dense_status() == 0
     Yr, A = orc.gemm(4, W, N, K, X)
     ratio = np.abs(Y.cpu().double().numpy() - Yr) / (1e-3 * A + 1e-30)
+    assert ratio.max() <= 1.0, f"max err / tol = {ratio.max():.3g}"
+
+
+def test_prefill_attention_wait_timeout_then_recovers(q, orc):
+    # 130 rows x 4 query heads per kv-head = 520 query vectors: 3 CTA pairs per kv-head;
+    # CTA (0, 0) takes the last pair, whose keys end at 300 + 130: 7 tiles of 64 keys
+    len_, C, n_qh, n_kvh = 300, 130, 16, 4
+    cap = len_ + C + 3
+    Q = synth.bf16_normal_np(SEED, 1320, (C, n_qh, 128))
+    Kc = synth.bf16_normal_np(SEED, 1321, (n_kvh, cap, 128))
+    Vc = synth.bf16_normal_np(SEED, 1322, (n_kvh, cap, 128))
+    Qd, Kd, Vd = _bf16(Q), _bf16(Kc), _bf16(Vc)
+    O = torch.zeros(C, n_qh, 128, dtype=torch.bfloat16, device="cuda")
+    q.prefill_status(reset=True)
+    took = _stalled(q, 2, 3, lambda: q.prefill_attn(Qd, Kd, Vd, len_, C, cap, n_qh, n_kvh, 128, O))
+    status = q.prefill_status(reset=True)
+    assert status != 0, "a wait on a tile that was never loaded did not time out"
+    assert took < 30.0, f"the stalled attention took {took:.1f} s to return"
+    O.zero_()
+    q.prefill_attn(Qd, Kd, Vd, len_, C, cap, n_qh, n_kvh, 128, O)
+    torch.cuda.synchronize()
+    assert q.prefill_status() == 0
+    O_ref, B = orc.decode_attn(Q, Kc[None], Vc[None], np.array([len_], np.int32), np.array([0, C], np.int32),
+                               n_qh, n_kvh, 128, cap)
+    o = orc.bf16_array_to_f64(O.cpu().view(torch.int16).numpy().view(np.uint16)).reshape(O_ref.shape)
+    ratio = np.abs(o - O_ref) / (2e-3 * B + np.abs(O_ref) * 2.0 ** -9 + 1e-30)
     assert ratio.max() <= 1.0, f"max err / tol = {ratio.max():.3g}"
