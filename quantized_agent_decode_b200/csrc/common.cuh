@@ -317,32 +317,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity, ui
         : "memory");
     return done != 0;
 }
-// Bounded wait on an mbarrier phase: gives up after `limit` polls of at most
-// ~20 us each (about 2 s in all) and reports false.
+// Bounded wait on an mbarrier phase. Each poll may suspend the thread until the
+// phase completes (the hardware wakes it; a waiting warp issues nothing) or
+// ~20 us pass. Gives up and reports false once 2 s have passed on the global
+// timer (checked every 64 polls), or after `limit` polls whatever the timer says.
+constexpr unsigned long long MBAR_WAIT_LIMIT_NS = 2000000000ull;
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t limit = 100000)
 {
-    for (uint32_t i = 0; i < limit; ++i)
-        if (mbar_try_wait(bar, parity))
-            return true;
-    return false;
-}
-// Bounded wait that sleeps ~sleep_ns between polls, so a waiting warp gives its
-// issue slots to the warps doing the work (a try_wait that returns at once
-// would otherwise be re-issued in a tight loop). Gives up once 2 s have passed
-// on the global timer (checked every 256 polls), or after 2e9 / sleep_ns polls
-// whatever the timer says.
-constexpr unsigned long long MBAR_WAIT_LIMIT_NS = 2000000000ull;
-__device__ __forceinline__ bool mbar_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t sleep_ns)
-{
-    if (mbar_try_wait(bar, parity, 0))
+    if (mbar_try_wait(bar, parity))
         return true;
     const unsigned long long t0 = gtimer();
-    const uint32_t limit = 2000000000u / (sleep_ns ? sleep_ns : 1u);
-    for (uint32_t i = 0; i < limit; ++i) {
-        __nanosleep(sleep_ns);
-        if (mbar_try_wait(bar, parity, 0))
+    for (uint32_t i = 1; i < limit; ++i) {
+        if (mbar_try_wait(bar, parity))
             return true;
-        if ((i & 255) == 255 && gtimer() - t0 > MBAR_WAIT_LIMIT_NS)
+        if ((i & 63) == 0 && gtimer() - t0 > MBAR_WAIT_LIMIT_NS)
             return false;
     }
     return false;
