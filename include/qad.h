@@ -132,14 +132,14 @@ int qad_q4k_gemm_noalloc(const void *W, int N, int K, const uint16_t *X, int M, 
                          void *stream);
 
 /* Device status word of the GEMM pipelines on the current device: 0 if every
- * shared-memory pipeline wait completed; non-zero if a wait gave up after its
- * bounded number of polls (the kernel then returned early and its outputs are
- * incomplete). Synchronous (reads device memory); reset != 0 clears it.
+ * shared-memory pipeline wait completed; non-zero if a wait gave up (after
+ * about 2 s; the kernel then returned early and its outputs are incomplete). Synchronous (reads device memory); reset != 0 clears it.
  * Returns the status (>= 0) or a negative QAD_ERR_* code. */
 int qad_device_status(int reset);
 
 /* Test hook for the bounded waits (no counterpart on the pages): makes the
- * producer of CTA 0 of the next launches of one pipeline stop issuing copies,
+ * producer of CTA 0 of the next launches of one pipeline on the current
+ * device stop issuing copies,
  * so that CTA's waits on them run out and the kernel takes its early exit
  * (records a status, waits for the copies and tensor-core work it already
  * issued, frees its tensor memory, returns) instead of completing.

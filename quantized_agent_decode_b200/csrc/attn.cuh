@@ -50,8 +50,8 @@ int launch_attn_q8_fused(const AttnPlan &pl, const float *qkv, int ldqkv, int8_t
 int launch_attn_q8(const AttnPlan &pl, const uint16_t *Q, const int8_t *Kq, const uint16_t *Kd, const int8_t *Vq,
                    const uint16_t *Vd, const int *lens, const int *ars, int n_agents, int kv_cap, int n_qh, int n_kvh,
                    float scale, uint16_t *O, float *part, cudaStream_t s, bool pdl);
-// Causal attention of a C-row prompt chunk of one agent (bf16 caches of that agent).
 int prefill_set_stall(int at);  // test hook behind qad_debug_stall (kernel 2)
+// Causal attention of a C-row prompt chunk of one agent (bf16 caches of that agent).
 int launch_prefill_attn(const uint16_t *Q, const uint16_t *Kc, const uint16_t *Vc, int len, int C, int kv_cap, int n_qh,
                         int n_kvh, float scale, uint16_t *O, cudaStream_t s);
 // Byte offset of the scale plane inside one q8_0 cache allocation.
