@@ -528,6 +528,7 @@ def run_gpu(args, ws, rank, local):
 
 DENSE_KERNELS = {  # prefill chunk (2048 prompt rows + 12 decode rows) through one matrix: (format, N, K, M)
     "pf_gate_up": (4, 34816, 5120, 2060), "pf_down": (6, 5120, 17408, 2060), "pf_qkv": (4, 8192, 5120, 2060),
+    "pf_o": (4, 5120, 6144, 2060),
 }
 
 STEP_LAUNCHES = ["prep_rms_attn", "gemm_qkv", "attn", "prep_merge", "gemm_o", "prep_rms_mlp", "gemm_gate_up",

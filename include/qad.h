@@ -165,12 +165,15 @@ int qad_q6k_gemm(const void *W, int N, int K, const uint16_t *X, int M, float *Y
  * same quantized weights; at that M the product is compute-bound.
  *
  * Y[m][n] = sum_k w[n][k] * x[m][k] for M >= 1 rows on the 5th-generation
- * tensor cores (tcgen05, fp16 operands, fp32 accumulate in TMEM). The weights
- * are dequantized in shared memory to fp16: w = fp16(d*sc)*q - fp16(dmin*m)
- * (Q4_K) or fp16(d*sc)*(q - 32) (Q6_K-like), so each weight carries a
- * relative rounding error <= 2^-11 on top of the exact definition; x enters as
- * fp16 of x * 2^e_m with a per-row power of two (exact for bf16 rows whose
- * dynamic range is below 2^38).
+ * tensor cores (tcgen05, fp16 operands, fp32 accumulate in TMEM). Each weight
+ * is formed in fp32 (d*sc*q - dmin*m for Q4_K, d*sc*(q - 32) for Q6_K-like)
+ * and rounded to fp16 once in shared memory, so it is within (2^-11 + 2^-24)
+ * of its exact value relative to |w|; x enters as fp16 of x * 2^e_m with a
+ * per-row power of two (exact for bf16 rows whose dynamic range is below
+ * 2^38). When the last round of 128 x 256 output tiles would leave many SMs
+ * idle, its tiles are split between CTAs along K and their parts are added
+ * into Y with fp32 atomics; such launches are not bit-reproducible run to run
+ * (the rest of Y is).
  *   W   device: Q4_K [N][K/256][144] (qad_q4k_gemm_dense) or the packed
  *       Q6_K-like layout of qad_q6k_pack (qad_q6k_gemm_dense); 16-byte aligned
  *   X   device bf16 [M][K], 16-byte aligned;  Y  device fp32 [M][N], overwritten

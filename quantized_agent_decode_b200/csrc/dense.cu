@@ -8,7 +8,12 @@
 // the product is compute-bound (~2 FLOP per weight per row), so it belongs
 // on the 5th-generation tensor cores.
 //
-// Design (sm_100a, one CTA per SM, persistent over output tiles):
+// Design (sm_100a, one CTA per SM, persistent): rounds of output tiles go one
+// tile per CTA (tile c + r * grid: the CTAs of a round work on neighbouring
+// tiles and share their weights and activations in L2). When the last round
+// is partial and would leave many CTAs idle for many blocks, its tiles are cut
+// into (tile, 256-k block) units and split evenly over all CTAs instead
+// (stream-K); see dense_schedule:
 //  * Output tile = 128 weight rows x 256 activation rows. The accumulator
 //    D[128][256] fp32 lives in TMEM (256 columns); one elected thread issues
 //    tcgen05.mma kind::f16 (M=128, N=256, K=16) with both operands in shared
@@ -21,9 +26,11 @@
 //    of the k-step per warp). Each weight (d*sc*q - dmin*m for Q4_K,
 //    d*sc*(q-32) for Q6_K) is formed in fp32 with packed f32x2 operations and
 //    rounded to fp16 once, so an operand is within 2^-11 of its weight.
-//  * Two accumulators (512 TMEM columns): four epilogue warps read tile t out
-//    of TMEM, apply the activation row scales and store Y while the MMAs of
-//    tile t + 1 run.
+//  * Two accumulators (512 TMEM columns): four epilogue warps read one tile
+//    segment (the run's part of a tile) out of TMEM, apply the activation row
+//    scales and store Y while the MMAs of the next segment run. A tile whose
+//    blocks are split between CTAs was zeroed by the prep kernel and each of
+//    its segments is added into Y (fp32 atomics); a whole tile is stored.
 //  * Activations enter as fp16 of x * 2^e_m (per-row power of two putting the
 //    row's max |x| in [2^14, 2^15)); a prep kernel writes them straight into
 //    the tile order the bulk copies want, zero-padding M to whole tiles.
@@ -73,22 +80,92 @@ enum { ST_RAW = 1, ST_B = 2, ST_A = 3, ST_ACC = 4, ST_DONE = 5 };
 
 struct DenseArgs {
     int N, K, M, mt, nt, nblk;
+    int tiles;            // mt * nt
+    int rounds;           // rounds of tiles (tile c + r * grid < tiles, r < rounds)
+    int sk_units;         // units of the last round split over all CTAs (0: none)
     const uint16_t *x16;  // activation tiles (dense_x16 layout)
     const float *rs;      // per activation row 2^-e (0 past M)
     float *Y;
     int ldy;
 };
 
+// Segment i of this CTA's work: blocks b0 .. b1-1 of tile t. Rounds first (whole
+// tiles), then (SK) the CTA's share [u0, u1) of the last round's units, cut at
+// tile boundaries. False when there is no segment i. The kernel is compiled
+// twice: without SK it holds none of the split-tile code.
+template <bool SK>
+__device__ __forceinline__ bool dense_segment(const DenseArgs &a, int i, int &t, int &b0, int &b1)
+{
+    if (!SK || i < a.rounds) {
+        t = (int)blockIdx.x + i * (int)gridDim.x;
+        b0 = 0;
+        b1 = a.nblk;
+        return t < a.tiles && (SK || i < a.rounds);
+    }
+    const int j = i - a.rounds;
+    const int u0 = (int)((long long)blockIdx.x * a.sk_units / gridDim.x);
+    const int u1 = (int)((long long)(blockIdx.x + 1) * a.sk_units / gridDim.x);
+    const int u = j == 0 ? u0 : (u0 / a.nblk + j) * a.nblk;
+    if (u >= u1)
+        return false;
+    t = a.rounds * (int)gridDim.x + u / a.nblk;
+    b0 = u % a.nblk;
+    b1 = min(a.nblk, b0 + (u1 - u));
+    return true;
+}
+
+// Epilogue of one tile segment for this thread's weight column ng: the 256
+// accumulator columns (activation rows) times their row scales, stored into Y
+// (a whole tile) or added into it (ADD: a segment of a zeroed, split tile).
+template <bool ADD>
+__device__ __forceinline__ void dense_store_tile(const DenseArgs &a, uint32_t tacc, const float (&rsv)[dn::TM / 32],
+                                                 int mt, int ng, int lane)
+{
+    const bool col_ok = ng < a.N;
+#pragma unroll
+    for (int j = 0; j < dn::TM / 16; ++j) {
+        uint32_t v[16];
+        tmem_ld_x16(tacc + 16 * j, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int mm = 16 * j + i, m = mt * dn::TM + mm;
+            const float r = __shfl_sync(0xffffffffu, rsv[mm / 32], mm % 32);
+            if (m < a.M && col_ok) {
+                if (ADD)
+                    atomicAdd(a.Y + (size_t)m * a.ldy + ng, __uint_as_float(v[i]) * r);
+                else
+                    a.Y[(size_t)m * a.ldy + ng] = __uint_as_float(v[i]) * r;
+            }
+        }
+    }
+}
+
 // Activation tile layout: [m_tile][k-step][k-chunk 8][256 rows][8 fp16]; one
 // (m_tile, k-step) is 32 KB contiguous, i.e. exactly the B operand of one
 // k-step in core-matrix order (chunk stride 4096 B, 8-row stride 128 B).
+// It also zeroes, in row r of Y, the last-round tiles whose units the GEMM's
+// CTAs split (a CTA boundary c * sk_units / grid inside the tile): their
+// segments are added into Y. Tile t = (n-tile t / n_mt, m-tile t % n_mt).
 __global__ void __launch_bounds__(256) k_prep_dense(const uint16_t *__restrict__ X, int ldx, int M, int K,
-                                                    uint16_t *__restrict__ x16, float *__restrict__ rs)
+                                                    uint16_t *__restrict__ x16, float *__restrict__ rs,
+                                                    float *__restrict__ Y, int N, int n_mt, int t_sk, int sk_units,
+                                                    int grid)
 {
     __shared__ float red[8];
     const int r = blockIdx.x, tid = threadIdx.x;
     const int mt = r / dn::TM, rr = r % dn::TM, ksteps = K / dn::KS;
     const bool live = r < M;
+    const int nblk = K / 256;
+    if (live && sk_units > 0)
+        for (int c = 1 + tid; c < grid; c += 256) {
+            const int u = (int)((long long)c * sk_units / grid), t = t_sk + u / nblk;
+            if (u % nblk == 0 || t % n_mt != mt)
+                continue;
+            const int n0 = (t / n_mt) * dn::TN, n1 = min(N, n0 + dn::TN);
+            for (int n = n0; n < n1; ++n)
+                Y[(size_t)r * N + n] = 0.f;
+        }
     float mx = 0.f;
     if (live)
         for (int q = tid; q < K / 8; q += 256) {
@@ -222,7 +299,7 @@ __device__ __forceinline__ void dequant_q6(const uint8_t *blk, float d, int kk, 
 }
 
 
-template <int FMT>
+template <int FMT, bool SK>
 __global__ void __launch_bounds__(dn::THREADS, 1) k_dense_gemm(const __grid_constant__ WeightMapsBlob mapsb, DenseArgs a)
 {
     using namespace dn;
@@ -241,8 +318,6 @@ __global__ void __launch_bounds__(dn::THREADS, 1) k_dense_gemm(const __grid_cons
     const CUtensorMap *mw = reinterpret_cast<const CUtensorMap *>(mapsb.bytes);
     const CUtensorMap *md = mw + 1;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int tiles = a.mt * a.nt;
-    const int ksteps = a.K / KS;
 
     if (threadIdx.x == 0) {
         s_bad = 0;
@@ -283,10 +358,10 @@ __global__ void __launch_bounds__(dn::THREADS, 1) k_dense_gemm(const __grid_cons
         // ------------------------------------------------ producer
         if (lane == 0) {
             const int stall = blockIdx.x == 0 ? *(volatile int *)&g_dense_stall - 1 : -1;
-            int bk = 0, ks = 0;
-            for (int t = blockIdx.x; t < tiles && !bad() && ks != stall; t += gridDim.x) {
+            int bk = 0, ks = 0, t, b0, b1;
+            for (int sg = 0; !bad() && ks != stall && dense_segment<SK>(a, sg, t, b0, b1); ++sg) {
                 const int nt = t / a.mt, mt = t % a.mt;
-                for (int blk = 0; blk < a.nblk && !bad() && ks != stall; ++blk) {
+                for (int blk = b0; blk < b1 && !bad() && ks != stall; ++blk) {
                     const int s = bk % SR;
                     if (bk >= SR && !mbar_wait(&raw_empty[s], ((bk / SR) - 1) & 1)) {
                         fail(ST_RAW);
@@ -305,7 +380,7 @@ __global__ void __launch_bounds__(dn::THREADS, 1) k_dense_gemm(const __grid_cons
                             break;
                         }
                         mbar_arrive_expect_tx(&b_full[sb], (uint32_t)B_BYTES);
-                        bulk_g2s(BS + sb * B_BYTES, a.x16 + ((size_t)mt * ksteps + 4 * blk + kk) * (B_BYTES / 2),
+                        bulk_g2s(BS + sb * B_BYTES, a.x16 + ((size_t)mt * (4 * a.nblk) + 4 * blk + kk) * (B_BYTES / 2),
                                  B_BYTES, &b_full[sb]);
                         ++ks;
                     }
@@ -323,18 +398,18 @@ __global__ void __launch_bounds__(dn::THREADS, 1) k_dense_gemm(const __grid_cons
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc = umma_idesc_f16(TN, TM);
-            int ks = 0, tc = 0;
+            int ks = 0, tc = 0, t, b0, b1;
             bool issued = false;
-            for (int t = blockIdx.x; t < tiles && !bad(); t += gridDim.x, ++tc) {
+            for (; !bad() && dense_segment<SK>(a, tc, t, b0, b1); ++tc) {
                 const int acc = tc & 1;
-                if (tc >= 2) {  // the epilogue has drained this accumulator's previous tile
+                if (tc >= 2) {  // the epilogue has drained this accumulator's previous segment
                     if (!mbar_wait(&acc_empty[acc], ((tc >> 1) - 1) & 1)) {
                         fail(ST_ACC);
                         break;
                     }
                     tc_fence_after();
                 }
-                for (int k = 0; k < ksteps; ++k, ++ks) {
+                for (int k = 4 * b0; k < 4 * b1; ++k, ++ks) {
                     const int sa = ks % SA, sb = ks % SB;
                     if (!mbar_wait(&a_full[sa], (ks / SA) & 1) || !mbar_wait(&b_full[sb], (ks / SB) & 1)) {
                         fail(ST_A);
@@ -346,7 +421,7 @@ __global__ void __launch_bounds__(dn::THREADS, 1) k_dense_gemm(const __grid_cons
                     for (int j = 0; j < 4; ++j) {
                         const uint64_t ad = umma_desc_k_noswz(abase + j * 2 * (TN * 16), TN * 16, 128);
                         const uint64_t bd = umma_desc_k_noswz(bbase + j * 2 * (TM * 16), TM * 16, 128);
-                        umma_f16_ss(tmem + 256 * acc, ad, bd, idesc, (k | j) != 0);
+                        umma_f16_ss(tmem + 256 * acc, ad, bd, idesc, k != 4 * b0 || j != 0);
                     }
                     issued = true;
                     umma_commit(&a_empty[sa]);
@@ -367,9 +442,9 @@ __global__ void __launch_bounds__(dn::THREADS, 1) k_dense_gemm(const __grid_cons
         // ------------------------------------------------ dequant (weight row n, one k half)
         const int dw = warp - 2, quarter = dw & 3, half = dw >> 2;
         const int n = 32 * quarter + lane;
-        int bk = 0, ks = 0;
-        for (int t = blockIdx.x; t < tiles && !bad(); t += gridDim.x) {
-            for (int blk = 0; blk < a.nblk && !bad(); ++blk, ++bk) {
+        int bk = 0, ks = 0, t, b0, b1;
+        for (int sg = 0; !bad() && dense_segment<SK>(a, sg, t, b0, b1); ++sg) {
+            for (int blk = b0; blk < b1 && !bad(); ++blk, ++bk) {
                 const int s = bk % SR;
                 if (!__all_sync(0xffffffffu, mbar_wait(&raw_full[s], (bk / SR) & 1))) {
                     fail(ST_RAW);
@@ -406,8 +481,9 @@ __global__ void __launch_bounds__(dn::THREADS, 1) k_dense_gemm(const __grid_cons
         // ------------------------------------------------ epilogue: D[n][m] * 2^-e_m -> Y[m][n]
         const int quarter = warp & 3;  // TMEM lanes 32 quarter .. + 31 (this warp's access window)
         const int n = 32 * quarter + lane;
-        int tc = 0;
-        for (int t = blockIdx.x; t < tiles && !bad(); t += gridDim.x, ++tc) {
+        int tc = 0, t, b0, b1;
+        for (; !bad() && dense_segment<SK>(a, tc, t, b0, b1); ++tc) {
+            const bool whole = !SK || (b0 == 0 && b1 == a.nblk);  // else the tile was zeroed: add the segment
             const int nt = t / a.mt, mt = t % a.mt, acc = tc & 1;
             float rsv[TM / 32];  // row scales of this tile's 256 activation rows, 8 per lane
 #pragma unroll
@@ -418,21 +494,11 @@ __global__ void __launch_bounds__(dn::THREADS, 1) k_dense_gemm(const __grid_cons
                 break;
             }
             tc_fence_after();
-            const int ng = nt * TN + n;
-            const bool col_ok = ng < a.N;
-#pragma unroll
-            for (int j = 0; j < TM / 16; ++j) {
-                uint32_t v[16];
-                tmem_ld_x16(tmem + 256 * acc + ((uint32_t)(32 * quarter) << 16) + 16 * j, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int mm = 16 * j + i, m = mt * TM + mm;
-                    const float r = __shfl_sync(0xffffffffu, rsv[mm / 32], mm % 32);
-                    if (m < a.M && col_ok)
-                        a.Y[(size_t)m * a.ldy + ng] = __uint_as_float(v[i]) * r;
-                }
-            }
+            const uint32_t tacc = tmem + 256 * acc + ((uint32_t)(32 * quarter) << 16);
+            if (whole)
+                dense_store_tile<false>(a, tacc, rsv, mt, nt * TN + n, lane);
+            else if (SK)
+                dense_store_tile<true>(a, tacc, rsv, mt, nt * TN + n, lane);
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
@@ -473,8 +539,31 @@ size_t dense_ws_bytes(int K, int M)
     return mpad * (size_t)K * 2 + ((mpad * 4 + 255) & ~(size_t)255);
 }
 
-template <int FMT>
-static int launch_dense_t(const WeightMapsBlob &maps, const DenseArgs &a, cudaStream_t s)
+// The schedule. Rounds of one tile per CTA; if the last round is partial, its
+// tiles are split over all CTAs (stream-K) only when the CTAs it would leave
+// idle, times its blocks, come to more than DENSE_SK_MIN_IDLE units per CTA:
+// the split tiles' fp32 atomic additions cost about that much. Measured at
+// M = 2060 (two rounds plus 64 of 148 tiles): the split took the Q6_K down
+// projection (68 blocks) from 580 to 508 us, but cost gate|up (20 blocks, 80
+// of 148) 783 -> 838 us, q|k|v 206 -> 242 and o (24 blocks) 185 -> 194.
+constexpr int DENSE_SK_MIN_IDLE = 20;
+struct DenseSchedule {
+    int grid, rounds, sk_units;
+};
+static DenseSchedule dense_schedule(int tiles, int nblk)
+{
+    const int sms = num_sms();
+    const long long units = (long long)tiles * nblk;
+    const int g_sk = units < sms ? (int)units : sms;
+    const int rem = tiles % g_sk;
+    if (rem > 0 && (long long)(g_sk - rem) * nblk > (long long)DENSE_SK_MIN_IDLE * g_sk)
+        return {g_sk, tiles / g_sk, rem * nblk};
+    const int g = tiles < sms ? tiles : sms;
+    return {g, (tiles + g - 1) / g, 0};
+}
+
+template <int FMT, bool SK>
+static int launch_dense_t(const WeightMapsBlob &maps, const DenseArgs &a, int grid, cudaStream_t s)
 {
     const size_t smem = dn::smem_bytes<FMT>();
     static bool done[64] = {};
@@ -482,16 +571,14 @@ static int launch_dense_t(const WeightMapsBlob &maps, const DenseArgs &a, cudaSt
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64 || !done[dev]) {
         int rc = cuda_check(
-            cudaFuncSetAttribute(k_dense_gemm<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem),
+            cudaFuncSetAttribute(k_dense_gemm<FMT, SK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem),
             "cudaFuncSetAttribute(dense)");
         if (rc)
             return rc;
         if (dev >= 0 && dev < 64)
             done[dev] = true;
     }
-    const int tiles = a.mt * a.nt;
-    const int grid = tiles < num_sms() ? tiles : num_sms();
-    k_dense_gemm<FMT><<<grid, dn::THREADS, smem, s>>>(maps, a);
+    k_dense_gemm<FMT, SK><<<grid, dn::THREADS, smem, s>>>(maps, a);
     return cuda_check(cudaGetLastError(), "dense gemm launch");
 }
 
@@ -502,10 +589,12 @@ int launch_dense(int fmt, const void *W, int N, int K, const uint16_t *X, int M,
     int rc = make_dense_maps(fmt, W, N, K, &maps);
     if (rc)
         return rc;
-    const int mt = (M + dn::TM - 1) / dn::TM;
+    const int mt = (M + dn::TM - 1) / dn::TM, ntl = (N + dn::TN - 1) / dn::TN, tiles = mt * ntl;
+    const DenseSchedule sch = dense_schedule(tiles, K / 256);
     uint16_t *x16 = (uint16_t *)ws;
     float *rs = (float *)((char *)ws + (size_t)mt * dn::TM * K * 2);
-    k_prep_dense<<<mt * dn::TM, 256, 0, s>>>(X, K, M, K, x16, rs);
+    k_prep_dense<<<mt * dn::TM, 256, 0, s>>>(X, K, M, K, x16, rs, Y, N, mt, sch.rounds * sch.grid, sch.sk_units,
+                                             sch.grid);
     rc = cuda_check(cudaGetLastError(), "dense prep launch");
     if (rc)
         return rc;
@@ -514,13 +603,18 @@ int launch_dense(int fmt, const void *W, int N, int K, const uint16_t *X, int M,
     a.K = K;
     a.M = M;
     a.mt = mt;
-    a.nt = (N + dn::TN - 1) / dn::TN;
+    a.nt = ntl;
     a.nblk = K / 256;
+    a.tiles = tiles;
+    a.rounds = sch.rounds;
+    a.sk_units = sch.sk_units;
     a.x16 = x16;
     a.rs = rs;
     a.Y = Y;
     a.ldy = N;
-    return fmt == 4 ? launch_dense_t<4>(maps, a, s) : launch_dense_t<6>(maps, a, s);
+    if (sch.sk_units > 0)
+        return fmt == 4 ? launch_dense_t<4, true>(maps, a, sch.grid, s) : launch_dense_t<6, true>(maps, a, sch.grid, s);
+    return fmt == 4 ? launch_dense_t<4, false>(maps, a, sch.grid, s) : launch_dense_t<6, false>(maps, a, sch.grid, s);
 }
 
 }  // namespace qad

@@ -49,6 +49,10 @@ DENSE_CASES = [
     (6, 384, 1024, 513, False),
     (6, 256, 1024, 300, True),    # signed int8 sub-block scales
     (6, 136, 4352, 17, True),
+    # 32 tiles of 26 blocks on a 148-SM part: the schedule splits them over all CTAs
+    # (stream-K, ~5.6 units per CTA, 3-5 CTAs per tile added into a zeroed output)
+    (6, 2048, 6656, 300, True),
+    (4, 2048, 6656, 300, False),
 ]
 
 

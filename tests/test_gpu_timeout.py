@@ -75,14 +75,15 @@ def test_skinny_gemm_wait_timeout_then_recovers(q, orc):
 
 
 def test_dense_gemm_wait_timeout_then_recovers(q, orc):
-    # 2 weight tiles x 2 activation tiles: CTA 0 owns tile 0, k-steps 0 .. 7
+    # 2 weight tiles x 2 activation tiles x 2 blocks = 8 units over 8 CTAs (stream-K):
+    # CTA 0 owns the first block of tile 0, k-steps 0 .. 3
     N, K, M = 256, 512, 300
     W = synth.q4k_matrix_np(SEED, 1310, N, K)
     X = synth.bf16_normal_np(SEED, 1311, (M, K))
     Wd, Xd = torch.from_numpy(W).cuda(), _bf16(X)
     Y = torch.zeros(M, N, device="cuda")
     q.dense_status(reset=True)
-    took = _stalled(q, 1, 5, lambda: q.q4k_gemm_dense(Wd, N, K, Xd, M, Y))
+    took = _stalled(q, 1, 2, lambda: q.q4k_gemm_dense(Wd, N, K, Xd, M, Y))
     status = q.dense_status(reset=True)
     assert status != 0, "a wait on a copy that was never issued did not time out"
     assert took < 30.0, f"the stalled GEMM took {took:.1f} s to return"
