@@ -65,7 +65,8 @@ def test_skinny_gemm_writes_stay_inside(q, fmt, N, K, M):
     assert q.device_status() == 0
 
 
-@pytest.mark.parametrize("fmt,N,K,M", [(4, 300, 1280, 77), (6, 260, 2304, 130)])
+@pytest.mark.parametrize("fmt,N,K,M", [(4, 300, 1280, 77), (6, 260, 2304, 130),
+                                       (6, 2000, 6656, 290)])  # last round split (zeroing + atomic adds)
 def test_dense_gemm_writes_stay_inside(q, fmt, N, K, M):
     g = synth.torch_gen(SEED, "cuda", 600 + N)
     W = (synth.q4k_matrix_torch if fmt == 4 else synth.q6k_matrix_torch)(g, N, K, "cuda")
