@@ -144,9 +144,10 @@ __device__ __forceinline__ void dense_store_tile(const DenseArgs &a, uint32_t ta
 // Activation tile layout: [m_tile][k-step][k-chunk 8][256 rows][8 fp16]; one
 // (m_tile, k-step) is 32 KB contiguous, i.e. exactly the B operand of one
 // k-step in core-matrix order (chunk stride 4096 B, 8-row stride 128 B).
-// It also zeroes, in row r of Y, the last-round tiles whose units the GEMM's
-// CTAs split (a CTA boundary c * sk_units / grid inside the tile): their
-// segments are added into Y. Tile t = (n-tile t / n_mt, m-tile t % n_mt).
+// The prep kernel (one CTA per activation row r) writes row r into those tiles
+// and zeroes, in row r of Y, the last-round tiles whose units the GEMM's CTAs
+// split (a CTA boundary c * sk_units / grid inside the tile): their segments
+// are added into Y. Tile t = (n-tile t / n_mt, m-tile t % n_mt).
 __global__ void __launch_bounds__(256) k_prep_dense(const uint16_t *__restrict__ X, int ldx, int M, int K,
                                                     uint16_t *__restrict__ x16, float *__restrict__ rs,
                                                     float *__restrict__ Y, int N, int n_mt, int t_sk, int sk_units,
